@@ -1,0 +1,33 @@
+"""Oracle: the calibration Hessian H = 2·XᵀX (test infrastructure only).
+
+Sources
+  * hncyxsy.com/news/243429 §3.1 step 1: from the layer's input activations X, form
+    H = 2XXᵀ + λI (the "+" is lost in the page's text; λ is the damping term, applied later
+    in ``factor.damp``). The page writes X with tokens as columns; here X is stored
+    tokens × channels, so the same matrix reads 2·XᵀX.
+  * gtnt.cn/news/115337 §4: collect each layer's Hessian from calibration forward passes.
+
+The sum runs over all tokens, unnormalised (GPTQ's result is invariant to a positive scale of
+H because the damping is relative to mean(diag H)). Accumulation is additive over calls.
+"""
+
+import numpy as np
+
+
+def hessian(X, chunk=8192):
+    """H = 2·Σ_t x_t x_tᵀ in fp64 for X of shape [n_tokens, d_in] (any float dtype)."""
+    X = np.asarray(X)
+    n, d = X.shape
+    H = np.zeros((d, d), dtype=np.float64)
+    for t0 in range(0, n, chunk):
+        Xc = X[t0:t0 + chunk].astype(np.float64)
+        H += Xc.T @ Xc
+    return 2.0 * H
+
+
+def hessian_entries(X, rows, cols):
+    """H[rows][:, cols] only, for sampled parity checks of large Hessians."""
+    X = np.asarray(X)
+    Xr = X[:, rows].astype(np.float64)
+    Xc = X[:, cols].astype(np.float64)
+    return 2.0 * (Xr.T @ Xc)

@@ -1,0 +1,61 @@
+"""Oracle: the asymmetric per-group min-max quantizer (test infrastructure only).
+
+Sources
+  * 0539edu.com/news/6111416 §2.1: q = round(x/scale) + zero_point; the worked example maps the
+    range [-2.5, 3.7] onto the 256 INT8 levels with scale = (max - min)/(qmax - qmin) ≈ 0.0243.
+  * 0539edu.com/news/6111416 §4.2: one fp16 scale and one fp16 zero point per group.
+  * hncyxsy.com/news/243429 §3.1 step 3: per column, pick the quantization scale, round, keep
+    the error.
+
+Readings taken where the pages are silent:
+  * Codes use the unsigned range [0, maxq], maxq = 2**bits - 1 (the INT8 example's signed range
+    differs only by an offset of 2**(bits-1)).
+  * The range is the literal min and max of the group.
+  * scale = (xmax - xmin)/maxq rounded UP to fp16, so that the stored scale is what the codes
+    are computed with and |w - ŵ| <= scale/2 holds exactly for every entry.
+  * zero = rint(-xmin/scale), round half to even; an integer, stored as an fp16 value.
+  * A group with xmax == xmin gets scale 1.
+  * q = clamp(rint(w/scale) + zero, 0, maxq), round half to even; ŵ = scale·(q - zero).
+"""
+
+import numpy as np
+
+
+def fp16_round_up(x):
+    """Smallest fp16 value >= x, element-wise, returned as fp64.
+
+    ``np.float16`` converts fp64 with one round-to-nearest-even step; where that landed below
+    x, the next fp16 value up is taken. Values above the fp16 range become +inf.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    h = x.astype(np.float16)
+    below = h.astype(np.float64) < x
+    h = np.where(below, np.nextafter(h, np.float16(np.inf)), h)
+    return h.astype(np.float64)
+
+
+def group_params(xmin, xmax, maxq):
+    """(scale, zero) for groups with the given minima and maxima (fp64 arrays).
+
+    scale is fp16-representable (held in fp64), zero is integer-valued (held in fp64).
+    """
+    xmin = np.asarray(xmin, dtype=np.float64)
+    xmax = np.asarray(xmax, dtype=np.float64)
+    span = xmax - xmin
+    with np.errstate(divide="ignore", invalid="ignore"):
+        scale = fp16_round_up(span / maxq)
+        scale = np.where(span == 0.0, 1.0, scale)
+        zero = np.rint(-xmin / scale)
+    return scale, zero
+
+
+def quantize(w, scale, zero, maxq):
+    """Integer codes q = clamp(rint(w/scale) + zero, 0, maxq) (fp64 in, int64 out)."""
+    w = np.asarray(w, dtype=np.float64)
+    q = np.rint(w / scale) + zero
+    return np.clip(q, 0, maxq).astype(np.int64)
+
+
+def dequantize(q, scale, zero):
+    """ŵ = scale·(q - zero) in fp64."""
+    return np.asarray(scale, np.float64) * (np.asarray(q, np.float64) - zero)
