@@ -1,0 +1,533 @@
+"""Benchmark: GPTQ layer-wise quantization of one 7B-shaped linear layer per GPU.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+One step = the whole hot path over one layer with its inputs resident in HBM:
+  Hessian 2·XᵀX over the calibration tokens (tensor cores) -> damping -> act_order (if on) ->
+  Cholesky + triangular inverse (U) -> blocked column loop with OBS compensation + lazy batch
+  updates -> output assembly -> reconstruction loss -> group min-max RTN baseline of the same W.
+Default workload ``mlp_up_7b``: W 11008x4096 fp16, X 262144x4096 fp16, INT4 g128 B128,
+percdamp 0.01. value = weights quantized per second over all ranks (each rank quantizes its
+own layer: weak scaling, no data-path collective).
+
+Prints one JSON line on rank 0. ``--impl reference`` times the fp64 CPU checker on a bounded
+sample of the same workload instead (rank 0 only).
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from post_weight_quantization_24_b200 import workloads  # noqa: E402
+
+METRIC = "GPTQ weights quantized/s & calib tokens/s per layer; % roofline per stage"
+UNIT = "weights/s"
+PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "sm_max_mhz": 1965.0}
+N_SM, FP32_LANES_PER_SM = 148, 128
+
+
+def load_peaks():
+    try:
+        with open(PEAKS_PATH) as f:
+            p = json.load(f)
+        p["source"] = "measured"
+        return p
+    except (OSError, ValueError):
+        p = dict(FALLBACK_PEAKS)
+        p["source"] = "fallback"
+        return p
+
+
+# ------------------------------------------------------------------------------------------
+# distributed plumbing (one process per GPU)
+# ------------------------------------------------------------------------------------------
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world, local, backend="nccl"):
+    import datetime
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return world > 1
+
+
+def max_over_ranks(x: float, distributed: bool, device) -> float:
+    if not distributed:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(distributed: bool):
+    if distributed:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ------------------------------------------------------------------------------------------
+# clocks during the timed region
+# ------------------------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.path = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            sel = ["-i", "GPU-" + uuid if not uuid.startswith("GPU-") else uuid]
+        except Exception:
+            sel = []
+        self.sel = sel
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", *self.sel], stdout=open(self.path, "w"),
+                stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(parts[1]), smax=float(parts[2]), power=float(parts[3]),
+                                 hw=parts[5], hwt=parts[6], swt=parts[7], swp=parts[8]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        busy = [r for r in rows if r["power"] > 250.0] or rows
+        reasons = set()
+        for r in rows:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("swp", "sw_power_cap")):
+                if r[key].lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in busy),
+                "sm_max_mhz": max(r["smax"] for r in rows),
+                "power_w_max": max(r["power"] for r in rows),
+                "samples": len(rows), "samples_under_load": len(busy),
+                "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------------------------------------
+# the committed ncu summary of the dominant kernel (traffic is null if the kernel changed)
+# ------------------------------------------------------------------------------------------
+def ncu_traffic(summary_name: str, source_file: str):
+    path = os.path.join(ROOT, "profiles", summary_name)
+    try:
+        text = open(path).read()
+    except OSError:
+        return None, None
+    m_h = re.search(r"kernel_source_sha256:\s*([0-9a-f]{64})", text)
+    m_b = re.search(r"dram_bytes_per_launch_full_size:\s*([0-9.eE+]+)", text)
+    if not (m_h and m_b):
+        return None, path
+    src = os.path.join(ROOT, "post_weight_quantization_24_b200", "csrc", source_file)
+    cur = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    if cur != m_h.group(1):
+        return None, path
+    return float(m_b.group(1)), path
+
+
+def source_sha(source_file: str) -> str:
+    src = os.path.join(ROOT, "post_weight_quantization_24_b200", "csrc", source_file)
+    return hashlib.sha256(open(src, "rb").read()).hexdigest()
+
+
+# ------------------------------------------------------------------------------------------
+# our arm
+# ------------------------------------------------------------------------------------------
+class LayerStep:
+    """All device buffers for one layer and the step that quantizes it."""
+
+    def __init__(self, gptq, wl: workloads.LayerWorkload, device):
+        self.gptq, self.wl, self.device = gptq, wl, device
+        self.W = workloads.make_weights(wl, device=device)
+        self.X = workloads.make_activations(wl, device=device)
+        self.h = gptq.Hessian(wl.d_in)
+        self.Hraw = self.h.raw()
+        ng = wl.d_in // wl.group_size
+        self.out = dict(codes=torch.empty(wl.d_out, wl.d_in, dtype=torch.uint8, device=device),
+                        scales=torch.empty(wl.d_out, ng, dtype=torch.float16, device=device),
+                        zeros=torch.empty(wl.d_out, ng, dtype=torch.float16, device=device),
+                        g_idx=torch.empty(wl.d_in, dtype=torch.int32, device=device),
+                        perm=torch.empty(wl.d_in, dtype=torch.int32, device=device))
+        self.rtn_out = (torch.empty(wl.d_out, wl.d_in // 2 if wl.bits == 4 else wl.d_in,
+                                    dtype=torch.uint8, device=device),
+                        torch.empty(wl.d_out, ng, dtype=torch.float16, device=device),
+                        torch.empty(wl.d_out, ng, dtype=torch.float16, device=device))
+        nbytes = gptq.quantize_layer_workspace(wl.d_out, wl.d_in, wl.block_size)
+        self.ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        self.ev = {k: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for k in ("hessian", "gptq", "rtn")}
+        self.loss = None
+
+    def run(self, timed=False):
+        g, wl = self.gptq, self.wl
+        e = self.ev
+        if timed:
+            e["hessian"][0].record()
+        self.h.reset()
+        self.h.accumulate(self.X)
+        if timed:
+            e["hessian"][1].record()
+            e["gptq"][0].record()
+        res = g.quantize_layer(self.W, self.Hraw, bits=wl.bits, group_size=wl.group_size,
+                               block_size=wl.block_size, percdamp=wl.percdamp,
+                               act_order=wl.act_order, compute_loss=True, workspace=self.ws,
+                               out=self.out)
+        self.loss = res["loss"]
+        if timed:
+            e["gptq"][1].record()
+            e["rtn"][0].record()
+        g.rtn_minmax_quantize(self.W, wl.bits, wl.group_size, out=self.rtn_out)
+        if timed:
+            e["rtn"][1].record()
+
+    def stage_ms(self):
+        return {k: a.elapsed_time(b) for k, (a, b) in self.ev.items()}
+
+
+def run_ours(args):
+    world, rank, local = dist_env()
+    distributed = init_dist(world, local)
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    from post_weight_quantization_24_b200 import gptq
+    gptq.lib()
+    peaks = load_peaks()
+
+    # each rank quantizes its own layer (different seed): independent units, no collective
+    wl = workloads.WORKLOADS[args.workload].replace(seed=workloads.WORKLOADS[args.workload].seed + rank)
+    step = LayerStep(gptq, wl, device)
+    flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=device)   # > L2 (126 MB)
+
+    gptq.profile_enable(True)
+    for _ in range(args.warmup):
+        step.run()
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(local)
+    stage_tot = {k: 0.0 for k in ("hessian", "gptq", "rtn")}
+    lib_stage_tot = {k: 0.0 for k in gptq.STAGES}
+    total_ms = 0.0
+    barrier(distributed)
+    torch.cuda.synchronize()
+    sampler.start()
+    launches0 = gptq.launch_count()
+    t_wall0 = time.perf_counter()
+    for _ in range(args.steps):
+        flush.zero_()                                   # L2 flush, outside the timed events
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record()
+        step.run(timed=True)
+        t1.record()
+        torch.cuda.synchronize()
+        total_ms += t0.elapsed_time(t1)
+        for k, v in step.stage_ms().items():
+            stage_tot[k] += v
+        for k, v in gptq.profile_read().items():
+            lib_stage_tot[k] += v
+    torch.cuda.synchronize()
+    wall_s = time.perf_counter() - t_wall0
+    launches = gptq.launch_count() - launches0
+    clocks = sampler.stop()
+    barrier(distributed)
+
+    K = args.steps
+    total_ms_max = max_over_ranks(total_ms, distributed, device)
+    ms_per_step = total_ms_max / K
+    weights_per_step = wl.d_out * wl.d_in
+    value = world * K * weights_per_step / (total_ms_max / 1e3)
+
+    hess_ms = stage_tot["hessian"] / K
+    gptq_ms = stage_tot["gptq"] / K
+    rtn_ms = stage_tot["rtn"] / K
+    lib_ms = {k: v / K for k, v in lib_stage_tot.items()}
+    d, n, d_out = wl.d_in, wl.n_tokens, wl.d_out
+
+    # ---- per-stage roofline ----
+    clock_mhz = (clocks or {}).get("sm_mhz") or peaks.get("clocks_under_load", {}).get("sm_mhz_median", 1312.0)
+    fp32_peak_tf = N_SM * FP32_LANES_PER_SM * 2 * clock_mhz * 1e6 / 1e12
+    fp32_peak_max_tf = N_SM * FP32_LANES_PER_SM * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+    hess_flops = float(n) * d * (d + 1)                          # symmetric 2·XᵀX
+    hess_tf = hess_flops / (hess_ms / 1e3) / 1e12
+    tc_peak = peaks["bf16_tflops"]                               # fp16 MMA rate = bf16 rate
+    chol_flops = d ** 3 / 3.0
+    trtri_flops = d ** 3 / 3.0
+    col_flops = 2.0 * d_out * d * wl.block_size / 2.0
+    lazy_flops = 2.0 * d_out * sum(wl.block_size * max(0, d - j0 - wl.block_size)
+                                   for j0 in range(0, d, wl.block_size))
+    loss_flops = 2.0 * 2.0 * d_out * d * d
+    rtn_bytes = d_out * d * (2 + (0.5 if wl.bits == 4 else 1.0)) + d_out * (d // wl.group_size) * 4
+
+    def tf(fl, ms):
+        return fl / (ms / 1e3) / 1e12 if ms > 0 else None
+
+    stages = {
+        "hessian": {"ms": hess_ms, "bound": "tensor", "tflops": hess_tf,
+                    "frac": hess_tf / tc_peak, "calib_tokens_per_s": n / (hess_ms / 1e3)},
+        "prepare": {"ms": lib_ms["prepare"]},
+        "cholesky": {"ms": lib_ms["cholesky"], "bound": "alu",
+                     "tflops": tf(chol_flops, lib_ms["cholesky"])},
+        "trtri": {"ms": lib_ms["trtri"], "bound": "alu", "tflops": tf(trtri_flops, lib_ms["trtri"])},
+        "column_loop": {"ms": lib_ms["column_loop"], "bound": "alu",
+                        "tflops": tf(col_flops, lib_ms["column_loop"])},
+        "lazy_update": {"ms": lib_ms["lazy_update"], "bound": "alu",
+                        "tflops": tf(lazy_flops, lib_ms["lazy_update"])},
+        "assemble": {"ms": lib_ms["assemble"]},
+        "loss": {"ms": lib_ms["loss"], "bound": "alu", "tflops": tf(loss_flops, lib_ms["loss"])},
+        "rtn": {"ms": rtn_ms, "bound": "hbm", "gbs": rtn_bytes / (rtn_ms / 1e3) / 1e9,
+                "frac": rtn_bytes / (rtn_ms / 1e3) / 1e9 / peaks["hbm_gbs"]},
+    }
+    for k in ("cholesky", "trtri", "column_loop", "lazy_update", "loss"):
+        if stages[k].get("tflops") is not None:
+            stages[k]["frac"] = stages[k]["tflops"] / fp32_peak_tf
+
+    # dominant kernel by time share
+    dom = max(("hessian", "lazy_update", "loss", "cholesky", "trtri", "column_loop"),
+              key=lambda k: stages[k]["ms"])
+    if dom == "hessian":
+        traffic, _ = ncu_traffic("hessian_tc_kernel_mlp_up_7b.md", "hessian.cu")
+        roof = {"kernel": "hessian_tc_kernel", "bound": "tensor", "achieved": hess_tf,
+                "peak": tc_peak, "unit": "TFLOP/s", "frac": hess_tf / tc_peak,
+                "traffic": traffic,
+                "peak_note": "measured bf16 dense burst (fp16 MMA runs at the bf16 rate); of measured"
+                if peaks["source"] == "measured" else "fallback"}
+    else:
+        traffic, _ = ncu_traffic("sgemm_kernel_mlp_up_7b.md", "sgemm.cuh")
+        roof = {"kernel": dom, "bound": "alu", "achieved": stages[dom]["tflops"],
+                "peak": fp32_peak_tf, "unit": "TFLOP/s",
+                "frac": stages[dom]["tflops"] / fp32_peak_tf, "traffic": traffic,
+                "peak_note": f"FFMA peak 148 SM x 128 lanes x 2 flop at the sampled "
+                             f"{clock_mhz:.0f} MHz ({fp32_peak_max_tf:.1f} TF at max clock)"}
+
+    # ---- end to end through the public API with host buffers ----
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(step, gptq, args, distributed, device, world)
+
+    res = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": f"{wl.name}: W {d_out}x{d} {wl.w_dtype}, X {n}x{d} fp16 "
+                               f"(lognormal channel scales, outliers), INT{wl.bits} g{wl.group_size} "
+                               f"B{wl.block_size} percdamp {wl.percdamp} act_order {wl.act_order}",
+                   "per_rank": "one independent layer per GPU (seed = rank)",
+                   "l2": "X (2.1 GB) larger than L2, plus a 512 MB L2 flush between steps",
+                   "arithmetic": "Hessian fp16 x fp16 -> fp32 on tcgen05; factorisation, column "
+                                 "loop, lazy update, loss in fp32 FFMA; group scalars fp64"},
+        "calib_tokens_per_s": world * n / (hess_ms / 1e3),
+        "layer_loss": step.loss,
+        "stages": stages,
+        "roofline": roof,
+        "clocks": clocks,
+        "gpu_launches": launches,
+        "wall_s_timed": wall_s,
+        "e2e": e2e,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(step, wl)
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    if distributed:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def run_e2e(step, gptq, args, distributed, device, world):
+    """Same step, with the inputs copied in from pinned host memory and the results copied
+    back inside the timed region."""
+    wl = step.wl
+    X_h = step.X.cpu().pin_memory()
+    W_h = step.W.cpu().pin_memory()
+    outs_h = {k: torch.empty_like(v, device="cpu").pin_memory() for k, v in step.out.items()}
+    rtn_h = tuple(torch.empty_like(t, device="cpu").pin_memory() for t in step.rtn_out)
+    h2d = X_h.numel() * X_h.element_size() + W_h.numel() * W_h.element_size()
+    d2h = sum(t.numel() * t.element_size() for t in outs_h.values()) + \
+        sum(t.numel() * t.element_size() for t in rtn_h) + 4   # + the loss (float)
+
+    def one():
+        step.X.copy_(X_h, non_blocking=True)
+        step.W.copy_(W_h, non_blocking=True)
+        step.run()
+        for k, t in step.out.items():
+            outs_h[k].copy_(t, non_blocking=True)
+        for hst, dev in zip(rtn_h, step.rtn_out):
+            hst.copy_(dev, non_blocking=True)
+
+    for _ in range(2):
+        one()
+    torch.cuda.synchronize()
+    barrier(distributed)
+    total = 0.0
+    K = max(1, min(args.steps, 10))
+    for _ in range(K):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        one()
+        b.record()
+        torch.cuda.synchronize()
+        total += a.elapsed_time(b)
+    total = max_over_ranks(total, distributed, device)
+    return {"value": world * K * wl.d_out * wl.d_in / (total / 1e3), "unit": UNIT,
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "ms_per_step": total / K, "steps": K}
+
+
+# ------------------------------------------------------------------------------------------
+# CPU checker timings (the fp64 oracle as it stands, on a bounded sample)
+# ------------------------------------------------------------------------------------------
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        n = [i.get("num_threads") for i in info if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+def oracle_sample(W_np, X_np, wl, n_tok, n_rows, n_rtn_rows, seed=0):
+    """Time the oracle's stages on a sample; return (extrapolated full-step seconds, detail)."""
+    from oracle import gptq as ogptq
+    from oracle import hessian as ohess
+    from oracle import loss as oloss
+    from oracle import rtn as ortn
+    rng = np.random.default_rng(seed)
+    d, d_out, n = wl.d_in, wl.d_out, wl.n_tokens
+    t = time.perf_counter()
+    Hs = ohess.hessian(X_np[:n_tok])
+    t_h = time.perf_counter() - t
+    t = time.perf_counter()
+    perm, U = ogptq.prepare_u(Hs, wl.percdamp, wl.act_order)
+    t_u = time.perf_counter() - t
+    rows = np.sort(rng.choice(d_out, n_rows, replace=False))
+    Wn = W_np.astype(np.float64)
+    t = time.perf_counter()
+    out = ogptq.gptq_blocked_ref(Wn, Hs, wl.bits, wl.group_size, wl.block_size, wl.percdamp,
+                                 wl.act_order, rows=rows, U=U)
+    t_g = time.perf_counter() - t
+    t = time.perf_counter()
+    oloss.recon_loss(Wn[rows], out["What"], Hs)
+    t_l = time.perf_counter() - t
+    t = time.perf_counter()
+    ortn.rtn_minmax(Wn[:n_rtn_rows], wl.bits, wl.group_size)
+    t_r = time.perf_counter() - t
+    full = (t_h * n / n_tok + t_u + (t_g + t_l) * d_out / n_rows + t_r * d_out / n_rtn_rows)
+    measured = t_h + t_u + t_g + t_l + t_r
+    detail = (f"oracle fp64 on a sample: Hessian over {n_tok} of {n} tokens (x{n / n_tok:.0f}), "
+              f"U for the full d={d}, GPTQ + loss on {n_rows} of {d_out} rows "
+              f"(x{d_out / n_rows:.1f}), RTN on {n_rtn_rows} rows (x{d_out / n_rtn_rows:.1f}); "
+              f"sample took {measured:.1f} s, extrapolated full step {full:.1f} s")
+    return full, measured, detail
+
+
+def cpu_baseline(step, wl):
+    X_np = step.X[:8192].cpu().numpy()
+    W_np = step.W.float().cpu().numpy()
+    full, measured, detail = oracle_sample(W_np, X_np, wl, n_tok=8192, n_rows=128,
+                                           n_rtn_rows=2048)
+    return {"value": wl.d_out * wl.d_in / full, "unit": UNIT, "cores": _blas_threads(),
+            "kind": "oracle", "sample": detail}
+
+
+def run_reference(args):
+    world, rank, local = dist_env()
+    if rank != 0:
+        return
+    wl = workloads.WORKLOADS[args.workload]
+    # the same generator recipe on the CPU (bounded: only what the sample touches)
+    W = workloads.make_weights(wl, device="cpu").float().numpy()
+    X = workloads.make_activations(wl, device="cpu", n_tokens=2048).numpy()
+    fulls, measured = [], 0.0
+    for i in range(args.warmup + args.steps):
+        full, m, detail = oracle_sample(W, X, wl, n_tok=2048, n_rows=32, n_rtn_rows=512, seed=i)
+        if i >= args.warmup:
+            fulls.append(full)
+            measured += m
+    full = statistics.mean(fulls)
+    value = wl.d_out * wl.d_in / full
+    cores = _blas_threads()
+    res = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": full * 1e3, "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "impl": "reference",
+           "config": {"workload": f"{wl.name}: W {wl.d_out}x{wl.d_in} {wl.w_dtype}, "
+                                  f"X {wl.n_tokens}x{wl.d_in} fp16, INT{wl.bits} g{wl.group_size} "
+                                  f"B{wl.block_size} percdamp {wl.percdamp}"},
+           "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                            "sample": detail + f"; {args.steps} timed samples"},
+           "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(res), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default="mlp_up_7b", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

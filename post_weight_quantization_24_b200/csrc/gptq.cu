@@ -1,0 +1,261 @@
+// GPTQ column loop, lazy batch update, output assembly and reconstruction loss.
+//
+// GPTQ deep-dive (hncyxsy.com/news/243429):
+//   §2.2  quantizing column q moves the not-yet-quantized columns by
+//         delta = -(w_q - quant(w_q)) / [H_F^-1]_qq * (H_F^-1)_{q,.}; with U^T U = H_d^-1 the
+//         same update reads  e = (w_q - What_q) / U_qq,  w_c -= e * U_qc  for c > q;
+//   §2.4  fixed column order; lazy batch updates: errors of a block are accumulated and the
+//         later columns are updated once per block (a GEMM);
+//   §3.1  step 3: per block of 128 columns, column by column: pick the scale, round, record
+//         the error; then update the remaining columns.
+// gtnt.cn/news/115337 §4: block_size is a multiple of group_size, so groups never straddle
+// blocks. Rows of W are independent given U, which is what the kernels parallelise over.
+#include <algorithm>
+
+#include "internal.cuh"
+#include "quant.cuh"
+#include "sgemm.cuh"
+
+namespace gq {
+
+namespace gb {
+constexpr int MAXB = 128;            // widest block handled in one launch
+constexpr int LANES_PER_ROW = 16;    // 8 columns per lane, two rows per warp
+constexpr int WARPS = 8;
+constexpr int THREADS = WARPS * 32;
+constexpr int SMEM = (MAXB * MAXB + MAXB) * 4;
+}  // namespace gb
+
+// In-block column loop. The block's U[j0:j0+bw, j0:j0+bw] (zero below the diagonal) and the
+// reciprocals of its diagonal sit in shared memory. Each half-warp owns one row and holds its
+// bw (<= 128) block weights in registers, 8 per lane. Column i is owned by lane i/8: it is
+// broadcast with a shuffle, every lane of the row computes the same code and error, and each
+// lane applies the rank-1 update to its 8 columns with one row of U (entries left of column
+// i are zero, so no masking is needed). Group scale/zero come from a half-warp min/max
+// reduction over the group's current weights at the group's first column.
+__global__ void __launch_bounds__(gb::THREADS) gptq_block_kernel(
+    float* __restrict__ Wk, int d_out, int d_in, int j0, int bw, const float* __restrict__ U,
+    int g, int bits, uint8_t* __restrict__ codes_p, uint16_t* __restrict__ scales,
+    uint16_t* __restrict__ zeros, float* __restrict__ Err, int err_ld, const int* status) {
+    if (status_bad(status)) return;
+    extern __shared__ float smem[];
+    float* Us = smem;                      // [MAXB][MAXB]
+    float* dinv = smem + gb::MAXB * gb::MAXB;
+    const int maxq = (1 << bits) - 1;
+    const int n_groups_row = d_in / g;
+
+    for (int e = threadIdx.x; e < gb::MAXB * gb::MAXB / 4; e += blockDim.x) {
+        const int i = e / (gb::MAXB / 4), c4 = (e % (gb::MAXB / 4)) * 4;
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (i < bw && c4 < bw) {
+            v = *reinterpret_cast<const float4*>(U + static_cast<int64_t>(j0 + i) * d_in + j0 + c4);
+            if (c4 + 0 < i) v.x = 0.f;
+            if (c4 + 1 < i) v.y = 0.f;
+            if (c4 + 2 < i) v.z = 0.f;
+            if (c4 + 3 < i) v.w = 0.f;
+        }
+        *reinterpret_cast<float4*>(Us + i * gb::MAXB + c4) = v;
+    }
+    for (int i = threadIdx.x; i < gb::MAXB; i += blockDim.x)
+        dinv[i] = i < bw ? 1.0f / U[static_cast<int64_t>(j0 + i) * d_in + j0 + i] : 0.0f;
+    __syncthreads();
+
+    const int lane = lane_id(), half = lane >> 4, hl = lane & 15;
+    const int c0 = hl * 8;                           // this lane's first block column
+    const unsigned full = 0xffffffffu;
+    const int warps_total = gridDim.x * gb::WARPS;
+    const int n_pairs = (d_out + 1) / 2;
+    for (int pair = blockIdx.x * gb::WARPS + warp_id(); pair < n_pairs; pair += warps_total) {
+        const int r = pair * 2 + half;
+        const bool row_ok = r < d_out;
+        float w[8];
+        float* wrow = Wk + static_cast<int64_t>(r) * d_in + j0;
+        if (row_ok && c0 < bw) {
+            const float4 a = *reinterpret_cast<const float4*>(wrow + c0);
+            const float4 b = *reinterpret_cast<const float4*>(wrow + c0 + 4);
+            w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
+            w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+        } else {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) w[k] = 0.f;
+        }
+        float e[8];
+        uint32_t qlo = 0, qhi = 0;
+        QParams P;
+        P.scale = 1.f; P.zero = 0.f; P.inv_scale = 1.f;
+#pragma unroll 1
+        for (int i0 = 0; i0 < bw; i0 += 8) {
+            const int owner = (half << 4) | (i0 >> 3);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const int i = i0 + c;
+                if (i >= bw) break;
+                if ((j0 + i) % g == 0) {
+                    // group [i, i+g) of the block: min/max of its current weights in this row
+                    float mn = INFINITY, mx = -INFINITY;
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const int col = c0 + k;
+                        if (col >= i && col < i + g && col < bw) {
+                            mn = fminf(mn, w[k]);
+                            mx = fmaxf(mx, w[k]);
+                        }
+                    }
+#pragma unroll
+                    for (int off = 8; off > 0; off >>= 1) {
+                        mn = fminf(mn, __shfl_xor_sync(full, mn, off));
+                        mx = fmaxf(mx, __shfl_xor_sync(full, mx, off));
+                    }
+                    P = group_params(mn, mx, maxq);
+                    if (hl == 0 && row_ok) {
+                        const int64_t gi = static_cast<int64_t>(r) * n_groups_row + (j0 + i) / g;
+                        scales[gi] = half_bits(P.scale);
+                        zeros[gi] = half_bits(P.zero);
+                    }
+                }
+                const float wi = __shfl_sync(full, w[c], owner);
+                const int qi = quant_code(wi, P, maxq);
+                const float err = (wi - dequant(qi, P)) * dinv[i];
+                if (hl == (i0 >> 3)) {
+                    e[c] = err;
+                    if (c < 4) qlo |= static_cast<uint32_t>(qi) << (8 * c);
+                    else qhi |= static_cast<uint32_t>(qi) << (8 * (c - 4));
+                }
+                const float4 u0 = *reinterpret_cast<const float4*>(Us + i * gb::MAXB + c0);
+                const float4 u1 = *reinterpret_cast<const float4*>(Us + i * gb::MAXB + c0 + 4);
+                w[0] = fmaf(-err, u0.x, w[0]);
+                w[1] = fmaf(-err, u0.y, w[1]);
+                w[2] = fmaf(-err, u0.z, w[2]);
+                w[3] = fmaf(-err, u0.w, w[3]);
+                w[4] = fmaf(-err, u1.x, w[4]);
+                w[5] = fmaf(-err, u1.y, w[5]);
+                w[6] = fmaf(-err, u1.z, w[6]);
+                w[7] = fmaf(-err, u1.w, w[7]);
+            }
+        }
+        if (row_ok && c0 < bw) {
+            uint2 qv;
+            qv.x = qlo;
+            qv.y = qhi;
+            *reinterpret_cast<uint2*>(codes_p + static_cast<int64_t>(r) * d_in + j0 + c0) = qv;
+            float* er = Err + static_cast<int64_t>(r) * err_ld + c0;
+            *reinterpret_cast<float4*>(er) = make_float4(e[0], e[1], e[2], e[3]);
+            *reinterpret_cast<float4*>(er + 4) = make_float4(e[4], e[5], e[6], e[7]);
+        }
+    }
+}
+
+static bool g_block_attr_set = false;
+
+gptq_status gptq_block_launch(float* Wk, int d_out, int d_in, int j0, int bw, const float* U,
+                              int group_size, int bits, uint8_t* codes_p, uint16_t* scales,
+                              uint16_t* zeros, float* Err, int err_ld, const int* status,
+                              cudaStream_t s) {
+    if (!g_block_attr_set) {
+        GPTQ_CUDA_TRY(cudaFuncSetAttribute(gptq_block_kernel,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, gb::SMEM));
+        g_block_attr_set = true;
+    }
+    const int n_pairs = (d_out + 1) / 2;
+    const int need = (n_pairs + gb::WARPS - 1) / gb::WARPS;
+    const int grid = std::max(1, std::min(need, num_sms() * 3));
+    gptq_block_kernel<<<grid, gb::THREADS, gb::SMEM, s>>>(Wk, d_out, d_in, j0, bw, U, group_size,
+                                                          bits, codes_p, scales, zeros, Err,
+                                                          err_ld, status);
+    GPTQ_LAUNCHED();
+    return GPTQ_OK;
+}
+
+// W[:, j1:] -= Err_block * U[j0:j1, j1:]
+gptq_status lazy_update_launch(float* Wk, int d_out, int d_in, int j0, int bw, const float* U,
+                               const float* Err, int err_ld, const int* status, cudaStream_t s) {
+    const int j1 = j0 + bw;
+    if (j1 >= d_in) return GPTQ_OK;
+    SgemmArgs a{};
+    a.M = d_out; a.N = d_in - j1; a.K = bw; a.alpha = -1.f; a.beta = 1.f;
+    a.A = Err; a.lda = err_ld;
+    a.B = U + static_cast<int64_t>(j0) * d_in + j1; a.ldb = d_in;
+    a.C = Wk + j1; a.ldc = d_in; a.abort_flag = status;
+    return sgemm_launch(a, false, EPI_STORE, s);
+}
+
+// codes[r][c] = codes_p[r][invperm[c]]; g_idx[c] = invperm[c] / g; perm_out = perm
+__global__ void assemble_kernel(const uint8_t* __restrict__ codes_p, int d_out, int d_in,
+                                const int* __restrict__ perm, const int* __restrict__ invperm,
+                                int g, int act_order, uint8_t* __restrict__ codes,
+                                int32_t* __restrict__ g_idx, int32_t* __restrict__ perm_out) {
+    const int64_t n = static_cast<int64_t>(d_out) * d_in;
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    const int64_t t0 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    for (int64_t c = t0; c < d_in; c += stride) {
+        g_idx[c] = invperm[c] / g;
+        if (perm_out) perm_out[c] = perm[c];
+    }
+    if (!act_order) return;
+    for (int64_t e = t0; e < n; e += stride) {
+        const int64_t r = e / d_in;
+        const int c = static_cast<int>(e - r * d_in);
+        codes[e] = codes_p[r * d_in + invperm[c]];
+    }
+}
+
+gptq_status assemble_launch(const uint8_t* codes_p, int d_out, int d_in, const int* perm,
+                            const int* invperm, int group_size, int act_order, uint8_t* codes,
+                            int32_t* g_idx, int32_t* perm_out, cudaStream_t s) {
+    const int64_t n = act_order ? static_cast<int64_t>(d_out) * d_in : d_in;
+    const int blocks = static_cast<int>(std::min<int64_t>((n + 255) / 256, num_sms() * 16));
+    assemble_kernel<<<std::max(blocks, 1), 256, 0, s>>>(codes_p, d_out, d_in, perm, invperm,
+                                                       group_size, act_order, codes, g_idx,
+                                                       perm_out);
+    GPTQ_LAUNCHED();
+    return GPTQ_OK;
+}
+
+// Dp[r][p] = W[r][perm[p]] - What[r][p] (processing order), What from codes, scales, zeros
+template <typename T>
+__global__ void delta_kernel(const T* __restrict__ W, int d_out, int d_in,
+                             const int* __restrict__ perm, const uint8_t* __restrict__ codes_p,
+                             const uint16_t* __restrict__ scales,
+                             const uint16_t* __restrict__ zeros, int g, float* __restrict__ Dp) {
+    const int64_t n = static_cast<int64_t>(d_out) * d_in;
+    const int ng = d_in / g;
+    for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < n;
+         e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t r = e / d_in;
+        const int p = static_cast<int>(e - r * d_in);
+        const int64_t gi = r * ng + p / g;
+        const float s = __half2float(__ushort_as_half(scales[gi]));
+        const float z = __half2float(__ushort_as_half(zeros[gi]));
+        const float wh = s * (static_cast<float>(codes_p[e]) - z);
+        Dp[e] = static_cast<float>(W[r * d_in + perm[p]]) - wh;
+    }
+}
+
+// tr(D H D^T) and tr(W H W^T) in the processing order (a common permutation of rows and
+// columns leaves both traces unchanged), each as a GEMM whose epilogue dots with its A operand.
+gptq_status loss_launch(const void* W, int w_dtype, int d_out, int d_in, const float* H,
+                        const int* perm, const uint8_t* codes_p, const uint16_t* scales,
+                        const uint16_t* zeros, int group_size, float* Wk, float* Hp,
+                        DevState* st, cudaStream_t s) {
+    GPTQ_TRY(gather_h_launch(H, d_in, perm, st, 0, Hp, &st->status, s));
+    const int64_t n = static_cast<int64_t>(d_out) * d_in;
+    const int blocks = static_cast<int>(std::min<int64_t>((n + 255) / 256, num_sms() * 32));
+    if (w_dtype == GPTQ_DTYPE_F16)
+        delta_kernel<__half><<<blocks, 256, 0, s>>>(static_cast<const __half*>(W), d_out, d_in,
+                                                    perm, codes_p, scales, zeros, group_size, Wk);
+    else
+        delta_kernel<float><<<blocks, 256, 0, s>>>(static_cast<const float*>(W), d_out, d_in,
+                                                   perm, codes_p, scales, zeros, group_size, Wk);
+    GPTQ_LAUNCHED();
+    SgemmArgs a{};
+    a.M = d_out; a.N = d_in; a.K = d_in; a.alpha = 1.f; a.beta = 0.f;
+    a.A = Wk; a.lda = d_in; a.B = Hp; a.ldb = d_in; a.D = Wk; a.ldd = d_in;
+    a.dot = &st->loss_num; a.abort_flag = &st->status;
+    GPTQ_TRY(sgemm_launch(a, false, EPI_DOT, s));
+    GPTQ_TRY(gather_w_launch(W, w_dtype, d_out, d_in, perm, Wk, &st->status, s));
+    a.dot = &st->loss_den;
+    GPTQ_TRY(sgemm_launch(a, false, EPI_DOT, s));
+    return GPTQ_OK;
+}
+
+}  // namespace gq

@@ -1,0 +1,63 @@
+// Declarations shared between the library's translation units.
+#pragma once
+
+#include "common.cuh"
+
+namespace gq {
+
+// Per-call device state at the head of the quantizer workspace (zeroed at the start of a call).
+struct DevState {
+    int status;        // first error code recorded by any kernel (0 = none)
+    int pad;
+    double lam;        // damping term percdamp * mean(diag H)
+    double diag_sum;
+    double loss_num;   // tr(D H D^T)
+    double loss_den;   // tr(W H W^T)
+};
+
+constexpr int kCholBlock = 128;   // panel width of the blocked Cholesky / triangular inverse
+
+// rtn.cu
+gptq_status rtn_launch(const void* W, int w_dtype, int d_out, int d_in, int bits,
+                       int group_size, uint8_t* out, uint16_t* scales, uint16_t* zeros,
+                       cudaStream_t s);
+
+// hessian.cu
+gptq_status hessian_launch(float* H, int d, const void* X, int64_t n, int unit_tokens,
+                           int* status, cudaStream_t s);
+gptq_status mirror_upper_launch(const float* H, float* out, int d, cudaStream_t s);
+
+// factor.cu
+gptq_status diag_stats_launch(const float* H, int d, double percdamp, DevState* st,
+                              cudaStream_t s);
+gptq_status act_order_launch(const float* H, int d, int act_order, int* perm, int* invperm,
+                             cudaStream_t s);
+// reversed = 1: A[i][j] = Hsym[perm[d-1-i]][perm[d-1-j]] + lambda*delta_ij (damped, reversed)
+// reversed = 0: A[i][j] = Hsym[perm[i]][perm[j]] (undamped)
+gptq_status gather_h_launch(const float* H, int d, const int* perm, const DevState* st,
+                            int reversed, float* A, int* status, cudaStream_t s);
+gptq_status gather_w_launch(const void* W, int w_dtype, int d_out, int d_in, const int* perm,
+                            float* Wk, int* status, cudaStream_t s);
+// In-place lower Cholesky of A (lda = d); writes the inverses of the diagonal blocks to Dinv
+// (ceil(d/nb) blocks of nb x nb, row-major, zero above the diagonal). P: d*nb floats scratch.
+gptq_status cholesky_launch(float* A, int d, float* Dinv, float* P, int* status, cudaStream_t s);
+// X = L^-1 (lower) from the factor in A and Dinv; then U = reverse(X) in place in X.
+gptq_status trtri_reverse_launch(const float* A, int d, const float* Dinv, float* X, float* P,
+                                 int* status, cudaStream_t s);
+
+// gptq.cu
+gptq_status gptq_block_launch(float* Wk, int d_out, int d_in, int j0, int bw, const float* U,
+                              int group_size, int bits, uint8_t* codes_p, uint16_t* scales,
+                              uint16_t* zeros, float* Err, int err_ld, const int* status,
+                              cudaStream_t s);
+gptq_status lazy_update_launch(float* Wk, int d_out, int d_in, int j0, int bw, const float* U,
+                               const float* Err, int err_ld, const int* status, cudaStream_t s);
+gptq_status assemble_launch(const uint8_t* codes_p, int d_out, int d_in, const int* perm,
+                            const int* invperm, int group_size, int act_order, uint8_t* codes,
+                            int32_t* g_idx, int32_t* perm_out, cudaStream_t s);
+gptq_status loss_launch(const void* W, int w_dtype, int d_out, int d_in, const float* H,
+                        const int* perm, const uint8_t* codes_p, const uint16_t* scales,
+                        const uint16_t* zeros, int group_size, float* Wk, float* Hp,
+                        DevState* st, cudaStream_t s);
+
+}  // namespace gq

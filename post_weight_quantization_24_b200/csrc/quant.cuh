@@ -1,0 +1,82 @@
+// The asymmetric per-group min-max quantizer, shared by RTN and the GPTQ column loop.
+//
+// 0539edu.com/news/6111416 §2.1: q = round(x/scale) + zero_point, scale = (max-min)/(qmax-qmin).
+// §4.2: one fp16 scale and one fp16 zero point per group.
+//
+// Group scalars are computed in fp64:  scale = smallest fp16 >= (xmax - xmin)/maxq (1 when the
+// group is constant), zero = rint(-xmin/scale) (half to even). Per-element codes
+// q = clamp(rint(w/scale) + zero, 0, maxq) are decided EXACTLY in fp32: an approximate
+// quotient gives a candidate k, and the sign of w - (k +- 1/2)*scale, computed with a single
+// fused multiply-add (one rounding of the exact value, so its sign is exact), moves k by one
+// where needed and resolves exact halves to even. The result equals rint of the exact
+// quotient for any fp16/fp32 w and fp16 scale.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+namespace gq {
+
+// Smallest fp16 value >= x for x >= 0 (finite), returned as an fp64 holding that value.
+// fp16 values near x are spaced 2^(e-10) for x in [2^e, 2^(e+1)), e >= -14, and 2^-24 below
+// 2^-14 (subnormals); dividing and multiplying by a power of two is exact, so
+// ceil(x / spacing) * spacing is the answer. Above 65504 the result is +inf.
+__device__ __forceinline__ double fp16_ceil(double x) {
+    if (!(x > 0.0)) return x;
+    if (x > 65504.0) return __longlong_as_double(0x7FF0000000000000LL);
+    const long long bits = __double_as_longlong(x);
+    int e = static_cast<int>((bits >> 52) & 0x7FF) - 1023;   // floor(log2 x) for normal x
+    if (e < -14) e = -14;
+    const double spacing = __longlong_as_double(static_cast<long long>(e - 10 + 1023) << 52);
+    return ceil(x / spacing) * spacing;
+}
+
+struct QParams {
+    float scale;      // fp16-representable
+    float zero;       // integer-valued
+    float inv_scale;  // approximate 1/scale, only used to form the candidate code
+};
+
+__device__ __forceinline__ QParams group_params(float xmin, float xmax, int maxq) {
+    const double span = static_cast<double>(xmax) - static_cast<double>(xmin);
+    const double s = (span == 0.0) ? 1.0 : fp16_ceil(span / static_cast<double>(maxq));
+    const double z = rint(-static_cast<double>(xmin) / s);
+    QParams p;
+    p.scale = static_cast<float>(s);
+    p.zero = static_cast<float>(z);
+    p.inv_scale = static_cast<float>(1.0 / s);
+    return p;
+}
+
+// rint(w / scale) with the exact tie-to-even decision described above.
+__device__ __forceinline__ float round_quotient(float w, float scale, float inv_scale) {
+    float k = rintf(w * inv_scale);
+    if (fabsf(k) >= 4194304.0f) {  // 2^22: k +- 1/2 would not be exact in fp32
+        return static_cast<float>(rint(static_cast<double>(w) / static_cast<double>(scale)));
+    }
+    const float up = fmaf(-(k + 0.5f), scale, w);   // sign of w - (k + 1/2) * scale
+    const float dn = fmaf(-(k - 0.5f), scale, w);   // sign of w - (k - 1/2) * scale
+    const bool k_odd = (static_cast<int>(k) & 1) != 0;
+    if (up > 0.0f || (up == 0.0f && k_odd)) {
+        k += 1.0f;
+    } else if (dn < 0.0f || (dn == 0.0f && k_odd)) {
+        k -= 1.0f;
+    }
+    return k;
+}
+
+__device__ __forceinline__ int quant_code(float w, const QParams& p, int maxq) {
+    float q = round_quotient(w, p.scale, p.inv_scale) + p.zero;
+    q = fminf(fmaxf(q, 0.0f), static_cast<float>(maxq));
+    return static_cast<int>(q);
+}
+
+__device__ __forceinline__ float dequant(int q, const QParams& p) {
+    return p.scale * (static_cast<float>(q) - p.zero);
+}
+
+__device__ __forceinline__ uint16_t half_bits(float v) {
+    return __half_as_ushort(__float2half_rn(v));  // exact for fp16-representable v
+}
+
+}  // namespace gq

@@ -1,0 +1,240 @@
+"""GPTQ on the GPU against the fp64 oracle.
+
+Tolerances: codes agree on >= 99 % of entries and every mismatch is one level; the layer
+reconstruction loss is within 1 % (relative) of the oracle's. With H = c·I the GPU must
+reproduce RTN bit for bit. The oracle always starts from X (its own fp64 Hessian); the GPU
+path starts from the same X through its tensor-core Hessian.
+"""
+
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import factor as ofac
+from oracle import gptq as ogptq
+from oracle import hessian as ohess
+from oracle import loss as oloss
+from oracle import rtn as ortn
+from post_weight_quantization_24_b200 import workloads
+
+pytestmark = pytest.mark.gpu
+
+
+def gpu_hessian(lib, X):
+    h = lib.Hessian(X.shape[1])
+    h.accumulate(X)
+    return h.get()
+
+
+def log_parity(**rec):
+    """Append parity statistics to $GPTQ_PARITY_LOG (a JSON-lines file) when it is set."""
+    path = os.environ.get("GPTQ_PARITY_LOG")
+    if path:
+        rec["test"] = os.environ.get("PYTEST_CURRENT_TEST", "").split(" ")[0]
+        with open(path, "a") as f:
+            f.write(json.dumps(rec) + "\n")
+
+
+def compare_codes(got, ref, frac=0.99, max_diff=1):
+    diff = got.astype(np.int64) - ref.astype(np.int64)
+    agree = float(np.mean(diff == 0))
+    hist = {int(k): int(v) for k, v in zip(*np.unique(diff, return_counts=True))}
+    log_parity(agree=agree, diff_hist=hist)
+    assert agree >= frac, f"codes agree on {agree:.5f}, differences {hist}"
+    if max_diff is not None:
+        assert np.max(np.abs(diff)) <= max_diff, f"code differences {hist}"
+    return agree
+
+
+def self_consistency(W0p, Whp, codes_p, scales, zeros, Hd, g, bits, tie_tol=0.05):
+    """Check every GPU decision against exact arithmetic given the GPU's own earlier decisions.
+
+    With the first q columns (processing order) fixed at the GPU's quantized values, the
+    compensated weights of the rest are the least-squares re-solve
+        w_R = w_R0 - H_RR^-1 H_RQ (What_Q - w_Q0)
+    (fp64, damped H). Column q's code must be the rounding of its re-solved value with the
+    GPU's group scale and zero, unless that value lies within `tie_tol` of a rounding boundary;
+    group scales must match the re-solved group range to within one fp16 step.
+    Returns (non-tie mismatches, near-tie cases, scale mismatches).
+    """
+    from oracle import quantizer
+    maxq = 2 ** bits - 1
+    d = W0p.shape[1]
+    bad = near = sbad = 0
+    for q in range(d):
+        if q == 0:
+            wR = W0p
+        else:
+            rhs = Hd[q:, :q] @ (Whp[:, :q] - W0p[:, :q]).T
+            wR = W0p[:, q:] - np.linalg.solve(Hd[q:, q:], rhs).T
+        if q % g == 0:
+            grp = wR[:, :g]
+            s_exact, _ = quantizer.group_params(grp.min(1), grp.max(1), maxq)
+            s_gpu = scales[:, q // g]
+            up = np.nextafter(s_exact.astype(np.float16), np.float16(np.inf)).astype(np.float64)
+            dn = np.nextafter(s_exact.astype(np.float16), np.float16(-np.inf)).astype(np.float64)
+            sbad += int(np.sum((s_gpu != s_exact) & (s_gpu != up) & (s_gpu != dn)))
+        s, z = scales[:, q // g], zeros[:, q // g]
+        t = wR[:, 0] / s
+        want = np.clip(np.rint(t) + z, 0, maxq)
+        dist = np.abs(np.abs(t - np.floor(t)) - 0.5)
+        mism = want != codes_p[:, q]
+        tie = dist < tie_tol
+        bad += int(np.sum(mism & ~tie))
+        near += int(np.sum(mism & tie))
+    return bad, near, sbad
+
+
+def run_case(lib, W, X, bits, g, B, act_order, percdamp=0.01, rows=None):
+    H = gpu_hessian(lib, X)
+    out = lib.quantize_layer(W, H, bits=bits, group_size=g, block_size=B, percdamp=percdamp,
+                             act_order=act_order, compute_loss=True)
+    torch.cuda.synchronize()
+    Wn = W.float().cpu().numpy().astype(np.float64)
+    Href = ohess.hessian(X.cpu().numpy())
+    ref = ogptq.gptq_blocked_ref(Wn, Href, bits, g, block_size=B, percdamp=percdamp,
+                                 act_order=act_order, rows=rows)
+    return out, ref, Wn, Href
+
+
+def check_outputs(out, ref, Wn, Href, g, perm_must_match=True, max_diff=1):
+    perm_gpu = out["perm"].cpu().numpy()
+    if perm_must_match:
+        assert np.array_equal(perm_gpu, ref["perm"])
+    assert np.array_equal(out["g_idx"].cpu().numpy(), ref["g_idx"])
+    codes = out["codes"].cpu().numpy()
+    agree = compare_codes(codes, ref["codes"], max_diff=max_diff)
+    # the GPU's reconstruction, scored with the oracle's loss on the oracle's Hessian
+    s = out["scales"].float().cpu().numpy().astype(np.float64)
+    z = out["zeros"].float().cpu().numpy().astype(np.float64)
+    gi = out["g_idx"].cpu().numpy()
+    What = s[:, gi] * (codes - z[:, gi])
+    l_gpu = oloss.recon_loss(Wn, What, Href)
+    l_ref = oloss.recon_loss(Wn, ref["What"], Href)
+    assert abs(l_gpu - l_ref) <= 0.01 * l_ref, (l_gpu, l_ref)
+    # the loss the library reports for itself
+    log_parity(agree=agree, loss_gpu=l_gpu, loss_lib=out["loss"], loss_ref=l_ref)
+    assert abs(out["loss"] - l_ref) <= 0.01 * l_ref, (out["loss"], l_ref)
+    return agree, l_gpu, l_ref
+
+
+@pytest.mark.parametrize("bits,g,B,act_order", [
+    (4, 128, 128, False), (4, 128, 128, True), (3, 128, 128, True), (4, 64, 128, False),
+    (4, 32, 64, True), (2, 128, 128, False), (8, 128, 128, True), (4, 8, 16, False)])
+def test_linear_512(cuda_lib, bits, g, B, act_order):
+    wl = workloads.WORKLOADS["linear_512"]
+    W = workloads.make_weights(wl, device="cuda")
+    X = workloads.make_activations(wl, device="cuda")
+    out, ref, Wn, Href = run_case(cuda_lib, W, X, bits, g, B, act_order)
+    check_outputs(out, ref, Wn, Href, g)
+
+
+@pytest.mark.parametrize("d_out,d_in,n,g,B,act_order", [
+    (77, 384, 1500, 64, 128, True), (31, 200, 800, 8, 64, False), (64, 264, 900, 8, 128, True),
+    (5, 136, 300, 8, 64, False), (129, 1024, 3000, 128, 128, True)])
+def test_ragged_shapes(cuda_lib, d_out, d_in, n, g, B, act_order):
+    wl = workloads.WORKLOADS["mlp_up_7b"].replace(d_out=d_out, d_in=d_in, n_tokens=n, seed=d_in)
+    W = workloads.make_weights(wl, device="cuda")
+    X = workloads.make_activations(wl, device="cuda")
+    out, ref, Wn, Href = run_case(cuda_lib, W, X, 4, g, B, act_order)
+    check_outputs(out, ref, Wn, Href, g)
+
+
+@pytest.mark.parametrize("dtype", [torch.float16, torch.float32])
+@pytest.mark.parametrize("act_order", [False, True])
+def test_identity_hessian_is_rtn_bit_exact(cuda_lib, dtype, act_order):
+    wl = workloads.WORKLOADS["mlp_up_7b"].replace(d_out=300, d_in=768)
+    W = workloads.make_weights(wl, device="cuda").to(dtype)
+    H = 5.0 * torch.eye(768, device="cuda")
+    out = cuda_lib.quantize_layer(W, H, bits=4, group_size=128, act_order=act_order)
+    packed, scales, zeros = cuda_lib.rtn_minmax_quantize(W, 4, 128)
+    torch.cuda.synchronize()
+    rtn_codes = ortn.unpack_int4(packed.cpu().numpy())
+    assert np.array_equal(out["codes"].cpu().numpy(), rtn_codes)
+    assert torch.equal(out["scales"], scales) and torch.equal(out["zeros"], zeros)
+    codes, s_ref, _ = ortn.rtn_minmax(W.float().cpu().numpy().astype(np.float64), 4, 128)
+    assert np.array_equal(rtn_codes, codes)
+
+
+def test_correlated_inputs(cuda_lib):
+    """Strongly correlated channels (not one of the named workloads): compensation is large, so
+    one legitimate near-tie flip upstream can move later codes by more than one level. Here the
+    GPU must agree with the oracle on >= 99 % of codes and on the loss within 1 %, and each of
+    its decisions must be exact given its own earlier ones (self-consistency in fp64)."""
+    X = workloads.correlated_activations(4096, 256, rank=4, seed=3, device="cuda")
+    W = workloads.make_weights(workloads.WORKLOADS["mlp_up_7b"].replace(d_out=192, d_in=256),
+                               device="cuda")
+    out, ref, Wn, Href = run_case(cuda_lib, W, X, 3, 64, 128, True)
+    agree, l_gpu, l_ref = check_outputs(out, ref, Wn, Href, 64, max_diff=None)
+    perm = out["perm"].cpu().numpy().astype(np.int64)
+    codes = out["codes"].cpu().numpy()[:, perm].astype(np.float64)
+    sc = out["scales"].float().cpu().numpy().astype(np.float64)
+    zr = out["zeros"].float().cpu().numpy().astype(np.float64)
+    Whp = sc[:, np.arange(256) // 64] * (codes - zr[:, np.arange(256) // 64])
+    Hd, _ = ofac.damp(Href[np.ix_(perm, perm)], 0.01)
+    bad, near, sbad = self_consistency(Wn[:, perm], Whp, codes, sc, zr, Hd, 64, 3)
+    log_parity(self_consistency_bad=bad, near_ties=near, scale_bad=sbad, loss_gpu=l_gpu,
+               loss_ref=l_ref)
+    assert bad == 0 and sbad == 0, (bad, near, sbad)
+    # compensation did real work here: GPTQ beats RTN clearly
+    codes, s, z = ortn.rtn_minmax(Wn, 3, 64)
+    assert l_ref < 0.8 * oloss.recon_loss(Wn, ortn.rtn_dequant(codes, s, z, 64), Href)
+
+
+@pytest.mark.parametrize("act_order", [False, True])
+def test_inverse_factor_matches_oracle(cuda_lib, act_order):
+    wl = workloads.WORKLOADS["mlp_up_7b"].replace(d_in=1024, n_tokens=8192, seed=4)
+    X = workloads.make_activations(wl, device="cuda")
+    H = gpu_hessian(cuda_lib, X)
+    U, perm = cuda_lib.inverse_factor(H, 0.01, act_order)
+    Ug = U.cpu().numpy().astype(np.float64)
+    Href = ohess.hessian(X.cpu().numpy())
+    perm_ref, Uref = ogptq.prepare_u(Href, 0.01, act_order)
+    assert np.array_equal(perm.cpu().numpy(), perm_ref)
+    assert np.array_equal(Ug, np.triu(Ug))
+    err = np.max(np.abs(Ug - Uref)) / np.max(np.abs(Uref))
+    assert err <= 1e-3, err
+    Hd, _ = ofac.damp(Href[np.ix_(perm_ref, perm_ref)], 0.01)
+    resid = np.max(np.abs(Ug.T @ Ug @ Hd - np.eye(1024)))
+    assert resid <= 1e-3, resid
+
+
+@pytest.mark.slow
+def test_full_size_mlp_up_7b(cuda_lib):
+    """The timed workload: W 11008x4096 fp16, X 262144x4096, INT4 g128 B128, all rows."""
+    wl = workloads.WORKLOADS["mlp_up_7b"]
+    W = workloads.make_weights(wl, device="cuda")
+    X = workloads.make_activations(wl, device="cuda")
+    out, ref, Wn, Href = run_case(cuda_lib, W, X, wl.bits, wl.group_size, wl.block_size,
+                                  wl.act_order)
+    check_outputs(out, ref, Wn, Href, wl.group_size)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("bits", [4, 3])
+def test_mlp_down_7b_shape_act_order(cuda_lib, bits):
+    """d_in = 11008 with act_order, INT4 and INT3 (32768 calibration tokens)."""
+    wl = workloads.WORKLOADS["mlp_down_7b"].replace(n_tokens=32768, bits=bits)
+    W = workloads.make_weights(wl, device="cuda")
+    X = workloads.make_activations(wl, device="cuda")
+    H = gpu_hessian(cuda_lib, X)
+    out = cuda_lib.quantize_layer(W, H, bits=bits, group_size=128, act_order=True,
+                                  compute_loss=True)
+    torch.cuda.synchronize()
+    Wn = W.float().cpu().numpy().astype(np.float64)
+    Href = ohess.hessian(X.cpu().numpy())
+    ref = ogptq.gptq_blocked_ref(Wn, Href, bits, 128, act_order=True)
+    perm_gpu = out["perm"].cpu().numpy()
+    moved = np.flatnonzero(perm_gpu != ref["perm"])
+    # near-equal diagonal entries may legitimately swap within fp32 error of H; compare the
+    # columns whose processing position agrees, and require the rest to be a handful
+    assert moved.size <= 8, moved.size
+    keep = np.ones(Wn.shape[1], dtype=bool)
+    keep[perm_gpu[moved]] = False
+    keep[ref["perm"][moved]] = False
+    compare_codes(out["codes"].cpu().numpy()[:, keep], ref["codes"][:, keep])
+    l_ref = oloss.recon_loss(Wn, ref["What"], Href)
+    assert abs(out["loss"] - l_ref) <= 0.01 * l_ref, (out["loss"], l_ref)
