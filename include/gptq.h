@@ -96,10 +96,11 @@ gptq_status gptq_hessian_destroy(gptq_hessian* h);
 
 /* Handle-free form: H (device fp32 [d_in x d_in], caller-owned, 16-byte aligned, row stride
  * d_in) += 2 * X^T X on its upper triangle (tiles that straddle the diagonal also update some
- * entries below it). `unit_tokens` sets how many tokens one tensor-core accumulation covers
- * before it is added into H (0 = library default; otherwise a multiple of 64); it trades
- * accumulation precision against reduction traffic. status_dev: device int, or NULL; set
- * to GPTQ_ERR_TIMEOUT if a bounded wait gave up. */
+ * entries below it). The tensor cores accumulate at most 256 tokens at a time; those partial
+ * sums are added in fp32 with round-to-nearest, and each work unit adds its sum into H with
+ * atomic fp32 adds (so the low bits of H depend on the order units finish). `unit_tokens`
+ * sets the tokens per work unit (0 = chosen to balance the SMs; otherwise a multiple of 64).
+ * status_dev: device int, or NULL; set to GPTQ_ERR_TIMEOUT if a bounded wait gave up. */
 gptq_status gptq_hessian_accumulate_into(float* H, int d_in, const void* X, int64_t n_tokens,
                                          int unit_tokens, int* status_dev, void* stream);
 
