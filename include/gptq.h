@@ -147,6 +147,32 @@ gptq_status gptq_quantize_layer(const void* W, int w_dtype, int d_out, int d_in,
                                 int32_t* g_idx, int32_t* perm, float* loss,
                                 void* workspace, size_t workspace_bytes, void* stream);
 
+/* No-allocation form of gptq_quantize_layer, with the same arguments except the workspace.
+ * The pages have no counterpart; this is an integration aid. It is for callers that may not
+ * allocate device memory when they quantize: runtimes that reserved almost all of the GPU for
+ * their own pools at start-up, and deployments that forbid device allocation after
+ * initialisation. Such callers cannot supply a workspace either. The scratch is a fixed
+ * 32 MiB device array inside the library, reserved on every GPU that loads the library and
+ * held until the process exits.
+ *   - Layers whose gptq_quantize_layer_workspace(d_out, d_in, block_size) exceeds 32 MiB are
+ *     rejected with GPTQ_ERR_WORKSPACE before anything is launched. For example, d_in = 1024
+ *     fits up to d_out = 4096 and d_in = 512 up to d_out = 16384; d_in = 4096 does not fit.
+ *   - No cudaMalloc, cudaFree or other allocating call is made.
+ *   - The first call on each device looks up the array's device address (cudaGetSymbolAddress
+ *     with that device current). Make that first call before any stream capture on the device.
+ *   - All calls share the one array, and it keeps the previous call's contents. The status
+ *     block at its head is cleared by every call, and everything else is written before it is
+ *     read. Calls that overlap on the GPU (concurrent streams, or several host threads) race on
+ *     the array and must be serialised by the caller.
+ * Synchronises `stream` once at its end, like gptq_quantize_layer. Errors: as
+ * gptq_quantize_layer, plus WORKSPACE for layers that do not fit. */
+gptq_status gptq_quantize_layer_noalloc(const void* W, int w_dtype, int d_out, int d_in,
+                                        const float* H, int bits, int group_size, int block_size,
+                                        float percdamp, int act_order,
+                                        uint8_t* codes, uint16_t* scales, uint16_t* zeros,
+                                        int32_t* g_idx, int32_t* perm, float* loss,
+                                        void* stream);
+
 /* Stage 2 on its own: the processing order and U (upper triangular, zero below the diagonal,
  * U^T U = (P H P + lambda*I)^-1 in the processing order P) that gptq_quantize_layer uses.
  *   H        device fp32 [d_in x d_in], upper triangle read.  d_in: >= 8, multiple of 8.

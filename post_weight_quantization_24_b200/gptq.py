@@ -63,6 +63,8 @@ _SIGNATURES = {
     "gptq_inverse_factor_workspace": ([_I], _SZ),
     "gptq_inverse_factor": ([_P, _I, _F, _I, _P, _P, _P, _SZ, _P], _I),
     "rtn_minmax_quantize": ([_P, _I, _I, _I, _I, _I, _P, _P, _P, _P], _I),
+    "gptq_quantize_layer_noalloc": ([_P, _I, _I, _I, _P, _I, _I, _I, _F, _I, _P, _P, _P, _P, _P,
+                                     ctypes.POINTER(_F), _P], _I),
     "gptq_profile_enable": ([_I], None),
     "gptq_profile_read": ([ctypes.POINTER(_F), _I], _I),
     "gptq_launch_count": ([], ctypes.c_ulonglong),
@@ -229,6 +231,40 @@ def quantize_layer(W: torch.Tensor, H: torch.Tensor, bits: int = 4, group_size: 
         ctypes.byref(loss) if compute_loss else None, workspace.data_ptr(),
         workspace.numel(), _stream())
     _check(st, "gptq_quantize_layer")
+    res = dict(out)
+    res["loss"] = float(loss.value) if compute_loss else None
+    return res
+
+
+def quantize_layer_noalloc(W: torch.Tensor, H: torch.Tensor, bits: int = 4,
+                           group_size: int = 128, block_size: int = 128,
+                           percdamp: float = 0.01, act_order: bool = False,
+                           compute_loss: bool = False, out: dict | None = None) -> dict:
+    """quantize_layer without a workspace: the library uses its fixed 32 MiB device scratch.
+
+    For callers that may not allocate device memory while quantizing. Only ``out`` (the
+    caller's output tensors) is allocated here when it is not given. Layers whose workspace
+    would exceed 32 MiB raise GPTQError(GPTQ_ERR_WORKSPACE). Calls share the scratch, so they
+    must not overlap on the GPU.
+    """
+    _require_cuda(W, "W")
+    _require_cuda(H, "H")
+    d_out, d_in = W.shape
+    dev = W.device
+    if out is None:
+        ng = d_in // group_size if group_size > 0 and d_in % group_size == 0 else 1
+        out = dict(codes=torch.empty(d_out, d_in, dtype=torch.uint8, device=dev),
+                   scales=torch.empty(d_out, ng, dtype=torch.float16, device=dev),
+                   zeros=torch.empty(d_out, ng, dtype=torch.float16, device=dev),
+                   g_idx=torch.empty(d_in, dtype=torch.int32, device=dev),
+                   perm=torch.empty(d_in, dtype=torch.int32, device=dev))
+    loss = ctypes.c_float(float("nan"))
+    st = lib().gptq_quantize_layer_noalloc(
+        W.data_ptr(), _dtype_code(W), d_out, d_in, H.data_ptr(), bits, group_size, block_size,
+        float(percdamp), int(bool(act_order)), out["codes"].data_ptr(), out["scales"].data_ptr(),
+        out["zeros"].data_ptr(), out["g_idx"].data_ptr(), _ptr(out.get("perm")),
+        ctypes.byref(loss) if compute_loss else None, _stream())
+    _check(st, "gptq_quantize_layer_noalloc")
     res = dict(out)
     res["loss"] = float(loss.value) if compute_loss else None
     return res
