@@ -303,7 +303,7 @@ def run_ours(args):
     col_flops = 2.0 * d_out * d * wl.block_size / 2.0
     lazy_flops = 2.0 * d_out * sum(wl.block_size * max(0, d - j0 - wl.block_size)
                                    for j0 in range(0, d, wl.block_size))
-    loss_flops = 2.0 * 2.0 * d_out * d * d
+    loss_flops = 2.0 * d_out * d * d      # one trace GEMM (numerator from the e^2 sums)
     rtn_bytes = d_out * d * (2 + (0.5 if wl.bits == 4 else 1.0)) + d_out * (d // wl.group_size) * 4
 
     def tf(fl, ms):
@@ -511,6 +511,36 @@ def run_reference(args):
     print(json.dumps(res), flush=True)
 
 
+def run_ncu_case(name: str):
+    """Small invocations for ncu captures (inputs larger than L2, a few GB at most): the
+    profile summaries under profiles/ name these commands."""
+    from post_weight_quantization_24_b200 import gptq
+    torch.cuda.set_device(0)
+    wl = workloads.WORKLOADS["mlp_up_7b"]
+    if name == "hessian":                        # X 16384 x 4096 fp16 = 134 MB; 3 launches
+        X = workloads.make_activations(wl.replace(n_tokens=16384), device="cuda")
+        h = gptq.Hessian(wl.d_in)
+        for _ in range(3):
+            h.accumulate(X)
+    elif name == "gptq":                         # the timed layer's quantizer, 2 calls
+        X = workloads.make_activations(wl.replace(n_tokens=8192), device="cuda")
+        W = workloads.make_weights(wl, device="cuda")
+        h = gptq.Hessian(wl.d_in)
+        h.accumulate(X)
+        ws = torch.empty(gptq.quantize_layer_workspace(wl.d_out, wl.d_in), dtype=torch.uint8,
+                         device="cuda")
+        for _ in range(2):
+            gptq.quantize_layer(W, h.raw(), compute_loss=True, workspace=ws)
+    elif name == "rtn":                          # W 11008 x 4096 fp16; 3 launches
+        W = workloads.make_weights(wl, device="cuda")
+        for _ in range(3):
+            gptq.rtn_minmax_quantize(W, 4, 128)
+    else:
+        raise SystemExit(f"unknown ncu case {name}")
+    torch.cuda.synchronize()
+    print("ncu case done:", name)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -520,7 +550,12 @@ def main(argv=None):
     ap.add_argument("--workload", default="mlp_up_7b", choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ncu-case", choices=("hessian", "gptq", "rtn"),
+                    help="run one small case for an ncu capture and exit (no JSON line)")
     args = ap.parse_args(argv)
+    if args.ncu_case:
+        run_ncu_case(args.ncu_case)
+        return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":

@@ -331,7 +331,7 @@ gptq_status gptq_quantize_layer(const void* W, int w_dtype, int d_out, int d_in,
         const int bw = std::min(block_size, d_in - j0);
         tm.begin(3);
         GPTQ_TRY(gptq_block_launch(ws.Wk, d_out, d_in, j0, bw, ws.X, group_size, bits, codes_p,
-                                   scales, zeros, ws.Err, 128, status, s));
+                                   scales, zeros, ws.Err, 128, &ws.st->err_sq, status, s));
         tm.end();
         tm.begin(4);
         GPTQ_TRY(lazy_update_launch(ws.Wk, d_out, d_in, j0, bw, ws.X, ws.Err, 128, status, s));
@@ -354,7 +354,7 @@ gptq_status gptq_quantize_layer(const void* W, int w_dtype, int d_out, int d_in,
     GPTQ_CUDA_TRY(cudaStreamSynchronize(s));
     profile_collect();
     if (host.status) return static_cast<gptq_status>(host.status);
-    if (loss) *loss = static_cast<float>(host.loss_num / host.loss_den);
+    if (loss) *loss = static_cast<float>((host.err_sq - host.lam * host.delta_sq) / host.loss_den);
     return GPTQ_OK;
 }
 

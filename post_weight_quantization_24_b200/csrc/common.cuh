@@ -208,15 +208,25 @@ __device__ __forceinline__ void tmem_ld_wait() {
 // Shared-memory matrix descriptor for tcgen05.mma (sm_100 layout: start>>4 in [0,14),
 // leading-byte-offset>>4 in [16,30), stride-byte-offset>>4 in [32,46), version 1 at bit 46,
 // layout type in [61,64): 2 = 128-byte swizzle).
-__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr, uint32_t lbo_bytes,
-                                                    uint32_t sbo_bytes) {
+__device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo_bytes,
+                                              uint32_t sbo_bytes, uint32_t layout_type) {
     uint64_t d = 0;
     d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
     d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
     d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
     d |= 1ull << 46;
-    d |= 2ull << 61;
+    d |= static_cast<uint64_t>(layout_type & 7u) << 61;
     return d;
+}
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr, uint32_t lbo_bytes,
+                                                    uint32_t sbo_bytes) {
+    return umma_desc(saddr, lbo_bytes, sbo_bytes, 2u);
+}
+// 128-byte swizzle with 32-byte atoms (layout type 1): the only shared-memory layout the MMA
+// accepts for MN-major 32-bit (tf32) operands; swizzle atoms are 4 rows of 128 B.
+__device__ __forceinline__ uint64_t umma_desc_sw128_32b(uint32_t saddr, uint32_t lbo_bytes,
+                                                        uint32_t sbo_bytes) {
+    return umma_desc(saddr, lbo_bytes, sbo_bytes, 1u);
 }
 
 // Instruction descriptor, kind::f16: fp16 A and B, fp32 D, both operands MN-major.

@@ -14,7 +14,7 @@
 #include <algorithm>
 
 #include "internal.cuh"
-#include "sgemm.cuh"
+#include "tcgemm.cuh"
 
 namespace gq {
 
@@ -180,61 +180,192 @@ gptq_status gather_w_launch(const void* W, int w_dtype, int d_out, int d_in, con
 // ---------------------------------------------------------------------------------------
 // blocked Cholesky
 // ---------------------------------------------------------------------------------------
-// One CTA factors the nbc x nbc diagonal block A[k0:, k0:] in shared memory (right-looking,
-// one barrier per pivot: the trailing update uses the unscaled column divided by the pivot,
-// and the columns are scaled by 1/sqrt(pivot) at the end), writes L11 back, and computes
-// Dinv = L11^-1 by forward elimination on the identity (again one barrier per row).
-__global__ void __launch_bounds__(1024) potrf_diag_kernel(float* __restrict__ A, int d, int k0,
-                                                          int nbc, float* __restrict__ Dinv,
-                                                          int nb, int* status) {
+// ---- diagonal block: one CTA factors the 128 x 128 block A[k0:, k0:] and inverts its factor.
+// The block is split into four 32-column sub-panels. For each one, a single warp factors the
+// 32 x 32 diagonal sub-block in registers (lane i holds row i; pivots and columns travel by
+// shuffles, so the 32 sequential pivot steps need no block barrier) and inverts it the same
+// way; then all warps solve the sub-panel below it against that inverse and apply the rank-32
+// update to the trailing part of the block. Finally the inverse of the whole 128 x 128 factor
+// is assembled from the four sub-block inverses by block forward substitution. Rows and
+// columns beyond the matrix edge (last block) are padded with the identity.
+namespace pd {
+constexpr int NB = 128, LD = NB + 1, SUB = 32, THREADS = 512;
+constexpr int SMEM = (2 * NB * LD + 4 * SUB * (SUB + 1)) * 4;
+}  // namespace pd
+
+// v: row `lane` of a 32 x 32 SPD block (lower part used). On return v holds row `lane` of its
+// Cholesky factor L (zeros above the diagonal) and x holds row `lane` of L^-1.
+__device__ __forceinline__ void warp_chol_inv32(float (&v)[32], float (&x)[32], int lane,
+                                                bool& bad) {
+    const unsigned full = 0xffffffffu;
+#pragma unroll
+    for (int c = 0; c < 32; ++c) {
+        const float piv = __shfl_sync(full, v[c], c);
+        if (!(piv > 0.0f) || !isfinite(piv)) bad = true;
+        const float rs = 1.0f / sqrtf(piv);
+        const float lic = (lane >= c) ? v[c] * rs : 0.0f;
+        v[c] = lic;
+#pragma unroll
+        for (int j = c + 1; j < 32; ++j) {
+            const float ljc = __shfl_sync(full, lic, j);
+            v[j] = fmaf(-lic, ljc, v[j]);
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+        if (j > lane) v[j] = 0.0f;
+        x[j] = (j == lane) ? 1.0f : 0.0f;
+    }
+    // forward substitution on the identity: row k is final once rows < k have been applied
+#pragma unroll
+    for (int k = 0; k < 32; ++k) {
+        const float rkk = 1.0f / __shfl_sync(full, v[k], k);   // 1 / L[k][k]
+        if (lane == k) {
+#pragma unroll
+            for (int j = 0; j <= k; ++j) x[j] *= rkk;
+        }
+        const float lik = v[k];
+#pragma unroll
+        for (int j = 0; j <= k; ++j) {
+            const float xkj = __shfl_sync(full, x[j], k);
+            if (lane > k) x[j] = fmaf(-lik, xkj, x[j]);
+        }
+    }
+}
+
+__global__ void __launch_bounds__(pd::THREADS) potrf_diag_kernel(float* __restrict__ A, int d,
+                                                                int k0, int nbc,
+                                                                float* __restrict__ Dinv,
+                                                                int* status) {
     if (status_bad(status)) return;
     extern __shared__ float sm[];
-    const int LD = nb + 1;
-    float* S = sm;
-    float* X = sm + nb * LD;
-    float* dsq = X + nb * LD;
-    const int tid = threadIdx.x, tx = tid & 31, ty = tid >> 5;
+    float* S = sm;                          // [NB][LD]: the block, then its factor L
+    float* Dv = S + pd::NB * pd::LD;        // [NB][LD]: L^-1
+    float* Xs = Dv + pd::NB * pd::LD;       // [4][SUB][SUB+1]: sub-block inverses
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    constexpr int NW = pd::THREADS / 32;
 
-    for (int i = ty; i < nbc; i += 32)
-        for (int j = tx; j <= i; j += 32)
-            S[i * LD + j] = A[static_cast<int64_t>(k0 + i) * d + k0 + j];
+    for (int i = warp; i < pd::NB; i += NW)
+        for (int j = lane; j < pd::NB; j += 32) {
+            float v = (i == j) ? 1.0f : 0.0f;
+            if (i < nbc && j < nbc && j <= i) v = A[static_cast<int64_t>(k0 + i) * d + k0 + j];
+            S[i * pd::LD + j] = v;
+        }
     __syncthreads();
 
-    for (int c = 0; c < nbc; ++c) {
-        const float piv = S[c * LD + c];
-        if (tid == 0 && !(piv > 0.0f && isfinite(piv))) set_status(status, GPTQ_ERR_NOT_PD);
-        const float rinv = 1.0f / piv;
-        for (int i = c + 1 + ty; i < nbc; i += 32) {
-            const float lic = S[i * LD + c] * rinv;
-            for (int j = c + 1 + tx; j <= i; j += 32) S[i * LD + j] -= lic * S[j * LD + c];
+    bool bad = false;
+    for (int sp = 0; sp < 4; ++sp) {
+        const int c0 = pd::SUB * sp;
+        float* X = Xs + sp * pd::SUB * (pd::SUB + 1);
+        if (warp == 0) {
+            float v[32], x[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = (j <= lane) ? S[(c0 + lane) * pd::LD + c0 + j] : 0.0f;
+            warp_chol_inv32(v, x, lane, bad);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                if (j <= lane) S[(c0 + lane) * pd::LD + c0 + j] = v[j];
+                X[lane * (pd::SUB + 1) + j] = (j <= lane) ? x[j] : 0.0f;
+            }
+        }
+        __syncthreads();
+        // sub-panel below: L[r][c0+j] = sum_{k<=j} A[r][c0+k] * X[j][k]  (at most 96 x 32
+        // outputs, so at most 6 per thread; computed before any is written back)
+        const int r0 = c0 + pd::SUB, nr = pd::NB - r0;
+        float out[6];
+#pragma unroll
+        for (int t = 0; t < 6; ++t) {
+            const int idx = tid + t * pd::THREADS;
+            out[t] = 0.0f;
+            if (idx < nr * 32) {
+                const int r = r0 + (idx >> 5), j = idx & 31;
+                float acc = 0.0f;
+                for (int k = 0; k <= j; ++k)
+                    acc = fmaf(S[r * pd::LD + c0 + k], X[j * (pd::SUB + 1) + k], acc);
+                out[t] = acc;
+            }
+        }
+        __syncthreads();
+#pragma unroll
+        for (int t = 0; t < 6; ++t) {
+            const int idx = tid + t * pd::THREADS;
+            if (idx < nr * 32) S[(r0 + (idx >> 5)) * pd::LD + c0 + (idx & 31)] = out[t];
+        }
+        __syncthreads();
+        // trailing update: S[r][c] -= sum_k L[r][c0+k] L[c][c0+k] for r0 <= c <= r
+        for (int r = r0 + warp; r < pd::NB; r += NW) {
+            for (int c = r0 + lane; c <= r; c += 32) {
+                float acc = 0.0f;
+#pragma unroll 8
+                for (int k = 0; k < pd::SUB; ++k)
+                    acc = fmaf(S[r * pd::LD + c0 + k], S[c * pd::LD + c0 + k], acc);
+                S[r * pd::LD + c] -= acc;
+            }
         }
         __syncthreads();
     }
-    for (int c = tid; c < nbc; c += blockDim.x) dsq[c] = sqrtf(S[c * LD + c]);
-    __syncthreads();
-    for (int i = ty; i < nbc; i += 32)
-        for (int j = tx; j <= i; j += 32) {
-            const float l = S[i * LD + j] / dsq[j];
-            S[i * LD + j] = l;
-            A[static_cast<int64_t>(k0 + i) * d + k0 + j] = l;
-        }
-    for (int i = ty; i < nb; i += 32)
-        for (int j = tx; j < nb; j += 32) X[i * LD + j] = (i == j) ? 1.0f : 0.0f;
-    __syncthreads();
+    if (warp == 0 && lane == 0 && bad) set_status(status, GPTQ_ERR_NOT_PD);
 
-    for (int k = 0; k < nbc; ++k) {
-        const float lkk_inv = 1.0f / S[k * LD + k];
-        for (int i = k + 1 + ty; i < nbc; i += 32) {
-            const float f = S[i * LD + k] * lkk_inv;
-            for (int j = tx; j <= k; j += 32) X[i * LD + j] -= f * X[k * LD + j];
+    // inverse of the whole factor: diagonal 32-blocks are the sub-block inverses;
+    // Dv[I][J] = -X_I * sum_{K=J}^{I-1} L[I][K] Dv[K][J] for J < I
+    for (int i = warp; i < pd::NB; i += NW)
+        for (int j = lane; j < pd::NB; j += 32) {
+            const int I = i >> 5, J = j >> 5;
+            Dv[i * pd::LD + j] =
+                (I == J) ? Xs[I * pd::SUB * (pd::SUB + 1) + (i & 31) * (pd::SUB + 1) + (j & 31)]
+                         : 0.0f;
+        }
+    __syncthreads();
+    for (int I = 1; I < 4; ++I) {
+        // T = sum_K L[I][K] Dv[K][J] for all J < I: 32 rows x 32*I columns (<= 6 per thread)
+        float out[6];
+        const int ncol = 32 * I, total = 32 * ncol;
+#pragma unroll
+        for (int t = 0; t < 6; ++t) {
+            const int idx = tid + t * pd::THREADS;
+            out[t] = 0.0f;
+            if (idx < total) {
+                const int a = idx / ncol, col = idx % ncol, J = col >> 5;
+                float acc = 0.0f;
+                for (int k = 32 * J; k < 32 * I; ++k)
+                    acc = fmaf(S[(32 * I + a) * pd::LD + k], Dv[k * pd::LD + col], acc);
+                out[t] = acc;
+            }
+        }
+        __syncthreads();
+#pragma unroll
+        for (int t = 0; t < 6; ++t) {
+            const int idx = tid + t * pd::THREADS;
+            if (idx < total) Dv[(32 * I + idx / ncol) * pd::LD + idx % ncol] = out[t];
+        }
+        __syncthreads();
+        // Dv[I][J] = -X_I * T
+        const float* XI = Xs + I * pd::SUB * (pd::SUB + 1);
+#pragma unroll
+        for (int t = 0; t < 6; ++t) {
+            const int idx = tid + t * pd::THREADS;
+            out[t] = 0.0f;
+            if (idx < total) {
+                const int a = idx / ncol, col = idx % ncol;
+                float acc = 0.0f;
+                for (int k = 0; k <= a; ++k)
+                    acc = fmaf(XI[a * (pd::SUB + 1) + k], Dv[(32 * I + k) * pd::LD + col], acc);
+                out[t] = -acc;
+            }
+        }
+        __syncthreads();
+#pragma unroll
+        for (int t = 0; t < 6; ++t) {
+            const int idx = tid + t * pd::THREADS;
+            if (idx < total) Dv[(32 * I + idx / ncol) * pd::LD + idx % ncol] = out[t];
         }
         __syncthreads();
     }
-    for (int i = ty; i < nb; i += 32)
-        for (int j = tx; j < nb; j += 32) {
-            float v = 0.0f;
-            if (i < nbc && j <= i) v = X[i * LD + j] / S[i * LD + i];
-            Dinv[i * nb + j] = v;
+    for (int i = warp; i < pd::NB; i += NW)
+        for (int j = lane; j < pd::NB; j += 32) {
+            const bool in = i < nbc && j < nbc && j <= i;
+            Dinv[i * pd::NB + j] = in ? Dv[i * pd::LD + j] : 0.0f;
+            if (in) A[static_cast<int64_t>(k0 + i) * d + k0 + j] = S[i * pd::LD + j];
         }
 }
 
@@ -261,7 +392,8 @@ static int g_potrf_smem = 0;
 
 gptq_status cholesky_launch(float* A, int d, float* Dinv, float* P, int* status, cudaStream_t s) {
     const int nb = kCholBlock;
-    const int smem = (2 * nb * (nb + 1) + nb) * 4;
+    static_assert(kCholBlock == pd::NB, "diagonal-block kernel is written for 128-wide panels");
+    const int smem = pd::SMEM;
     if (g_potrf_smem != smem) {
         GPTQ_CUDA_TRY(cudaFuncSetAttribute(potrf_diag_kernel,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
@@ -271,23 +403,22 @@ gptq_status cholesky_launch(float* A, int d, float* Dinv, float* P, int* status,
     for (int m = 0; m < nbl; ++m) {
         const int k0 = m * nb, nbc = std::min(nb, d - k0);
         float* Dm = Dinv + static_cast<int64_t>(m) * nb * nb;
-        potrf_diag_kernel<<<1, 1024, smem, s>>>(A, d, k0, nbc, Dm, nb, status);
+        potrf_diag_kernel<<<1, pd::THREADS, smem, s>>>(A, d, k0, nbc, Dm, status);
         GPTQ_LAUNCHED();
         const int rem = d - k0 - nbc;
         if (rem <= 0) continue;
         float* A21 = A + static_cast<int64_t>(k0 + nbc) * d + k0;
-        SgemmArgs t{};  // P = A21 * Dinv_m^T
+        TcGemmArgs t{};  // P = A21 * Dinv_m^T
         t.M = rem; t.N = nbc; t.K = nbc; t.alpha = 1.f; t.beta = 0.f;
-        t.A = A21; t.lda = d; t.B = Dm; t.ldb = nb; t.C = P; t.ldc = nb;
-        t.abort_flag = status;
-        GPTQ_TRY(sgemm_launch(t, true, EPI_STORE, s));
+        t.A = A21; t.lda = d; t.B = Dm; t.ldb = nb; t.C = P; t.ldc = nb; t.status = status;
+        GPTQ_TRY(tcgemm_launch(t, true, TC_EPI_STORE, true, true, s));
         GPTQ_TRY(copy2d(P, nb, A21, d, rem, nbc, s));
-        SgemmArgs u{};  // A22 -= P P^T (lower tiles)
+        TcGemmArgs u{};  // A22 -= P P^T (lower tiles)
         u.M = rem; u.N = rem; u.K = nbc; u.alpha = -1.f; u.beta = 1.f;
         u.A = P; u.lda = nb; u.B = P; u.ldb = nb;
         u.C = A + static_cast<int64_t>(k0 + nbc) * d + (k0 + nbc); u.ldc = d;
-        u.lower_only = 1; u.abort_flag = status;
-        GPTQ_TRY(sgemm_launch(u, true, EPI_STORE, s));
+        u.lower_only = 1; u.status = status;
+        GPTQ_TRY(tcgemm_launch(u, true, TC_EPI_STORE, true, true, s));
     }
     return GPTQ_OK;
 }
@@ -321,20 +452,20 @@ gptq_status trtri_reverse_launch(const float* A, int d, const float* Dinv, float
     for (int m = 0; m < nbl; ++m) {
         const int k0 = m * nb, nbc = std::min(nb, d - k0), ncol = k0 + nbc;
         const float* Dm = Dinv + static_cast<int64_t>(m) * nb * nb;
-        SgemmArgs t{};  // P = Dinv_m * X[k0:k0+nbc, 0:ncol]
+        TcGemmArgs t{};  // P = Dinv_m * X[k0:k0+nbc, 0:ncol]
         t.M = nbc; t.N = ncol; t.K = nbc; t.alpha = 1.f; t.beta = 0.f;
         t.A = Dm; t.lda = nb; t.B = X + static_cast<int64_t>(k0) * d; t.ldb = d;
-        t.C = P; t.ldc = d; t.abort_flag = status;
-        GPTQ_TRY(sgemm_launch(t, false, EPI_STORE, s));
+        t.C = P; t.ldc = d; t.status = status;
+        GPTQ_TRY(tcgemm_launch(t, false, TC_EPI_STORE, true, true, s));
         GPTQ_TRY(copy2d(P, d, X + static_cast<int64_t>(k0) * d, d, nbc, ncol, s));
         const int rem = d - ncol;
         if (rem <= 0) continue;
-        SgemmArgs u{};  // X[ncol:, 0:ncol] -= L[ncol:, k0:ncol] * X[k0:ncol, 0:ncol]
+        TcGemmArgs u{};  // X[ncol:, 0:ncol] -= L[ncol:, k0:ncol] * X[k0:ncol, 0:ncol]
         u.M = rem; u.N = ncol; u.K = nbc; u.alpha = -1.f; u.beta = 1.f;
         u.A = A + static_cast<int64_t>(ncol) * d + k0; u.lda = d;
         u.B = X + static_cast<int64_t>(k0) * d; u.ldb = d;
-        u.C = X + static_cast<int64_t>(ncol) * d; u.ldc = d; u.abort_flag = status;
-        GPTQ_TRY(sgemm_launch(u, false, EPI_STORE, s));
+        u.C = X + static_cast<int64_t>(ncol) * d; u.ldc = d; u.status = status;
+        GPTQ_TRY(tcgemm_launch(u, false, TC_EPI_STORE, true, true, s));
     }
     const int64_t half = static_cast<int64_t>(d) * d / 2;
     const int blocks = static_cast<int>(std::min<int64_t>((half + 255) / 256, num_sms() * 16));

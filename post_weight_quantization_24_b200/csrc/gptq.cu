@@ -15,6 +15,7 @@
 #include "internal.cuh"
 #include "quant.cuh"
 #include "sgemm.cuh"
+#include "tcgemm.cuh"
 
 namespace gq {
 
@@ -36,7 +37,8 @@ constexpr int SMEM = (MAXB * MAXB + MAXB) * 4;
 __global__ void __launch_bounds__(gb::THREADS) gptq_block_kernel(
     float* __restrict__ Wk, int d_out, int d_in, int j0, int bw, const float* __restrict__ U,
     int g, int bits, uint8_t* __restrict__ codes_p, uint16_t* __restrict__ scales,
-    uint16_t* __restrict__ zeros, float* __restrict__ Err, int err_ld, const int* status) {
+    uint16_t* __restrict__ zeros, float* __restrict__ Err, int err_ld, double* err_sq,
+    const int* status) {
     if (status_bad(status)) return;
     extern __shared__ float smem[];
     float* Us = smem;                      // [MAXB][MAXB]
@@ -65,6 +67,7 @@ __global__ void __launch_bounds__(gb::THREADS) gptq_block_kernel(
     const unsigned full = 0xffffffffu;
     const int warps_total = gridDim.x * gb::WARPS;
     const int n_pairs = (d_out + 1) / 2;
+    double esq = 0.0;   // this lane's sum of squared errors (its own columns)
     for (int pair = blockIdx.x * gb::WARPS + warp_id(); pair < n_pairs; pair += warps_total) {
         const int r = pair * 2 + half;
         const bool row_ok = r < d_out;
@@ -141,16 +144,24 @@ __global__ void __launch_bounds__(gb::THREADS) gptq_block_kernel(
             float* er = Err + static_cast<int64_t>(r) * err_ld + c0;
             *reinterpret_cast<float4*>(er) = make_float4(e[0], e[1], e[2], e[3]);
             *reinterpret_cast<float4*>(er + 4) = make_float4(e[4], e[5], e[6], e[7]);
+            float part = 0.0f;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) part = fmaf(e[k], e[k], part);
+            esq += static_cast<double>(part);
         }
     }
+    // the OBS increments e^2 add up to tr(D H_d D^T) for the whole layer
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) esq += __shfl_xor_sync(full, esq, off);
+    if (lane == 0 && esq != 0.0) atomicAdd(err_sq, esq);
 }
 
 static bool g_block_attr_set = false;
 
 gptq_status gptq_block_launch(float* Wk, int d_out, int d_in, int j0, int bw, const float* U,
                               int group_size, int bits, uint8_t* codes_p, uint16_t* scales,
-                              uint16_t* zeros, float* Err, int err_ld, const int* status,
-                              cudaStream_t s) {
+                              uint16_t* zeros, float* Err, int err_ld, double* err_sq,
+                              const int* status, cudaStream_t s) {
     if (!g_block_attr_set) {
         GPTQ_CUDA_TRY(cudaFuncSetAttribute(gptq_block_kernel,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, gb::SMEM));
@@ -161,22 +172,22 @@ gptq_status gptq_block_launch(float* Wk, int d_out, int d_in, int j0, int bw, co
     const int grid = std::max(1, std::min(need, num_sms() * 3));
     gptq_block_kernel<<<grid, gb::THREADS, gb::SMEM, s>>>(Wk, d_out, d_in, j0, bw, U, group_size,
                                                           bits, codes_p, scales, zeros, Err,
-                                                          err_ld, status);
+                                                          err_ld, err_sq, status);
     GPTQ_LAUNCHED();
     return GPTQ_OK;
 }
 
-// W[:, j1:] -= Err_block * U[j0:j1, j1:]
+// W[:, j1:] -= Err_block * U[j0:j1, j1:]  (3xTF32 on the tensor cores)
 gptq_status lazy_update_launch(float* Wk, int d_out, int d_in, int j0, int bw, const float* U,
                                const float* Err, int err_ld, const int* status, cudaStream_t s) {
     const int j1 = j0 + bw;
     if (j1 >= d_in) return GPTQ_OK;
-    SgemmArgs a{};
+    TcGemmArgs a{};
     a.M = d_out; a.N = d_in - j1; a.K = bw; a.alpha = -1.f; a.beta = 1.f;
     a.A = Err; a.lda = err_ld;
     a.B = U + static_cast<int64_t>(j0) * d_in + j1; a.ldb = d_in;
-    a.C = Wk + j1; a.ldc = d_in; a.abort_flag = status;
-    return sgemm_launch(a, false, EPI_STORE, s);
+    a.C = Wk + j1; a.ldc = d_in; a.status = status;
+    return tcgemm_launch(a, false, TC_EPI_STORE, true, true, s);
 }
 
 // codes[r][c] = codes_p[r][invperm[c]]; g_idx[c] = invperm[c] / g; perm_out = perm
@@ -211,14 +222,15 @@ gptq_status assemble_launch(const uint8_t* codes_p, int d_out, int d_in, const i
     return GPTQ_OK;
 }
 
-// Dp[r][p] = W[r][perm[p]] - What[r][p] (processing order), What from codes, scales, zeros
+// sum over the layer of (W[r][perm[p]] - What[r][p])^2, What from codes, scales and zeros
 template <typename T>
-__global__ void delta_kernel(const T* __restrict__ W, int d_out, int d_in,
-                             const int* __restrict__ perm, const uint8_t* __restrict__ codes_p,
-                             const uint16_t* __restrict__ scales,
-                             const uint16_t* __restrict__ zeros, int g, float* __restrict__ Dp) {
+__global__ void __launch_bounds__(256) delta_sq_kernel(
+    const T* __restrict__ W, int d_out, int d_in, const int* __restrict__ perm,
+    const uint8_t* __restrict__ codes_p, const uint16_t* __restrict__ scales,
+    const uint16_t* __restrict__ zeros, int g, double* out) {
     const int64_t n = static_cast<int64_t>(d_out) * d_in;
     const int ng = d_in / g;
+    double acc = 0.0;
     for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < n;
          e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         const int64_t r = e / d_in;
@@ -227,35 +239,50 @@ __global__ void delta_kernel(const T* __restrict__ W, int d_out, int d_in,
         const float s = __half2float(__ushort_as_half(scales[gi]));
         const float z = __half2float(__ushort_as_half(zeros[gi]));
         const float wh = s * (static_cast<float>(codes_p[e]) - z);
-        Dp[e] = static_cast<float>(W[r * d_in + perm[p]]) - wh;
+        const float dlt = static_cast<float>(W[r * d_in + perm[p]]) - wh;
+        acc += static_cast<double>(dlt) * dlt;
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    __shared__ double red[8];
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        double t = 0.0;
+        for (int w = 0; w < 8; ++w) t += red[w];
+        atomicAdd(out, t);
     }
 }
 
-// tr(D H D^T) and tr(W H W^T) in the processing order (a common permutation of rows and
-// columns leaves both traces unchanged), each as a GEMM whose epilogue dots with its A operand.
+// Reconstruction loss tr(D H D^T) / tr(W H W^T) with the undamped H.
+// Numerator: the column loop already summed the OBS increments e^2, whose total is
+// tr(D H_d D^T) with H_d = H + lambda*I, so tr(D H D^T) = sum e^2 - lambda*||D||^2 (one pass
+// over the outputs). Denominator: tr(W H W^T) as a GEMM (W_p * H_p) whose epilogue dots with
+// W_p, in the processing order (a common permutation leaves the trace unchanged).
 gptq_status loss_launch(const void* W, int w_dtype, int d_out, int d_in, const float* H,
                         const int* perm, const uint8_t* codes_p, const uint16_t* scales,
                         const uint16_t* zeros, int group_size, float* Wk, float* Hp,
                         DevState* st, cudaStream_t s) {
-    GPTQ_TRY(gather_h_launch(H, d_in, perm, st, 0, Hp, &st->status, s));
     const int64_t n = static_cast<int64_t>(d_out) * d_in;
-    const int blocks = static_cast<int>(std::min<int64_t>((n + 255) / 256, num_sms() * 32));
+    const int blocks = static_cast<int>(std::min<int64_t>((n + 255) / 256, num_sms() * 8));
     if (w_dtype == GPTQ_DTYPE_F16)
-        delta_kernel<__half><<<blocks, 256, 0, s>>>(static_cast<const __half*>(W), d_out, d_in,
-                                                    perm, codes_p, scales, zeros, group_size, Wk);
+        delta_sq_kernel<__half><<<blocks, 256, 0, s>>>(static_cast<const __half*>(W), d_out,
+                                                       d_in, perm, codes_p, scales, zeros,
+                                                       group_size, &st->delta_sq);
     else
-        delta_kernel<float><<<blocks, 256, 0, s>>>(static_cast<const float*>(W), d_out, d_in,
-                                                   perm, codes_p, scales, zeros, group_size, Wk);
+        delta_sq_kernel<float><<<blocks, 256, 0, s>>>(static_cast<const float*>(W), d_out, d_in,
+                                                      perm, codes_p, scales, zeros, group_size,
+                                                      &st->delta_sq);
     GPTQ_LAUNCHED();
-    SgemmArgs a{};
+    GPTQ_TRY(gather_h_launch(H, d_in, perm, st, 0, Hp, &st->status, s));
+    GPTQ_TRY(gather_w_launch(W, w_dtype, d_out, d_in, perm, Wk, &st->status, s));
+    // Hp is symmetric, so it serves as the K-major [N x K] operand directly; fp16 weights are
+    // exact in tf32 and need no split
+    TcGemmArgs a{};
     a.M = d_out; a.N = d_in; a.K = d_in; a.alpha = 1.f; a.beta = 0.f;
     a.A = Wk; a.lda = d_in; a.B = Hp; a.ldb = d_in; a.D = Wk; a.ldd = d_in;
-    a.dot = &st->loss_num; a.abort_flag = &st->status;
-    GPTQ_TRY(sgemm_launch(a, false, EPI_DOT, s));
-    GPTQ_TRY(gather_w_launch(W, w_dtype, d_out, d_in, perm, Wk, &st->status, s));
-    a.dot = &st->loss_den;
-    GPTQ_TRY(sgemm_launch(a, false, EPI_DOT, s));
-    return GPTQ_OK;
+    a.dot = &st->loss_den; a.status = &st->status;
+    return tcgemm_launch(a, true, TC_EPI_DOT, w_dtype != GPTQ_DTYPE_F16, true, s);
 }
 
 }  // namespace gq

@@ -11,7 +11,8 @@ struct DevState {
     int pad;
     double lam;        // damping term percdamp * mean(diag H)
     double diag_sum;
-    double loss_num;   // tr(D H D^T)
+    double err_sq;     // sum of e^2 over all columns = tr(D H_d D^T) (OBS increments)
+    double delta_sq;   // ||W - What||_F^2
     double loss_den;   // tr(W H W^T)
 };
 
@@ -48,8 +49,8 @@ gptq_status trtri_reverse_launch(const float* A, int d, const float* Dinv, float
 // gptq.cu
 gptq_status gptq_block_launch(float* Wk, int d_out, int d_in, int j0, int bw, const float* U,
                               int group_size, int bits, uint8_t* codes_p, uint16_t* scales,
-                              uint16_t* zeros, float* Err, int err_ld, const int* status,
-                              cudaStream_t s);
+                              uint16_t* zeros, float* Err, int err_ld, double* err_sq,
+                              const int* status, cudaStream_t s);
 gptq_status lazy_update_launch(float* Wk, int d_out, int d_in, int j0, int bw, const float* U,
                                const float* Err, int err_ld, const int* status, cudaStream_t s);
 gptq_status assemble_launch(const uint8_t* codes_p, int d_out, int d_in, const int* perm,

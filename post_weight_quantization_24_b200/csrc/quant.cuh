@@ -66,8 +66,15 @@ __device__ __forceinline__ float round_quotient(float w, float scale, float inv_
 }
 
 __device__ __forceinline__ int quant_code(float w, const QParams& p, int maxq) {
-    float q = round_quotient(w, p.scale, p.inv_scale) + p.zero;
-    q = fminf(fmaxf(q, 0.0f), static_cast<float>(maxq));
+    // Fast path: t = w * (1/scale) is within |t| * 2.4e-7 of the exact quotient (two fp32
+    // roundings), so when its distance to the nearest half-integer exceeds that bound, rintf(t)
+    // is already the exact rounding. Otherwise (rare) decide exactly with round_quotient.
+    const float t = w * p.inv_scale;
+    float k = rintf(t);
+    if (fabsf(t - k) > 0.5f - fabsf(t) * 3.0e-7f - 1.0e-30f) {
+        k = round_quotient(w, p.scale, p.inv_scale);
+    }
+    const float q = fminf(fmaxf(k + p.zero, 0.0f), static_cast<float>(maxq));
     return static_cast<int>(q);
 }
 

@@ -17,7 +17,7 @@ struct Load8;
 
 template <>
 struct Load8<__half> {
-    static __device__ __forceinline__ void run(const __half* p, float (&v)[8]) {
+    static __device__ __forceinline__ void run(const __half* p, float* v) {
         const uint4 u = __ldcs(reinterpret_cast<const uint4*>(p));
         const __half2* h = reinterpret_cast<const __half2*>(&u);
 #pragma unroll
@@ -31,7 +31,7 @@ struct Load8<__half> {
 
 template <>
 struct Load8<float> {
-    static __device__ __forceinline__ void run(const float* p, float (&v)[8]) {
+    static __device__ __forceinline__ void run(const float* p, float* v) {
         const float4 a = __ldcs(reinterpret_cast<const float4*>(p));
         const float4 b = __ldcs(reinterpret_cast<const float4*>(p) + 1);
         v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
@@ -39,8 +39,9 @@ struct Load8<float> {
     }
 };
 
-// TPG = threads per group (group_size / 8), a power of two in [1, 32].
-template <typename T, int TPG>
+// E = weights per thread (8 or 16); TPG = threads per group (group_size / E), a power of two
+// in [1, 32]. All loads of an iteration are issued before any arithmetic.
+template <typename T, int E, int TPG>
 __global__ void __launch_bounds__(256) rtn_kernel(const T* __restrict__ W, int64_t n_chunks,
                                                   int bits, uint8_t* __restrict__ out,
                                                   uint16_t* __restrict__ scales,
@@ -53,16 +54,17 @@ __global__ void __launch_bounds__(256) rtn_kernel(const T* __restrict__ W, int64
          base < n_chunks; base += stride) {
         const int64_t t = base + (threadIdx.x & 31);
         const bool ok = t < n_chunks;
-        float v[8];
+        float v[E];
         if (ok) {
-            Load8<T>::run(W + t * 8, v);
+#pragma unroll
+            for (int h = 0; h < E / 8; ++h) Load8<T>::run(W + t * E + 8 * h, v + 8 * h);
         } else {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) v[i] = 0.0f;
+            for (int i = 0; i < E; ++i) v[i] = 0.0f;
         }
         float mn = v[0], mx = v[0];
 #pragma unroll
-        for (int i = 1; i < 8; ++i) {
+        for (int i = 1; i < E; ++i) {
             mn = fminf(mn, v[i]);
             mx = fmaxf(mx, v[i]);
         }
@@ -73,19 +75,25 @@ __global__ void __launch_bounds__(256) rtn_kernel(const T* __restrict__ W, int64
         }
         if (!ok) continue;
         const QParams p = group_params(mn, mx, maxq);
-        int q[8];
+        int q[E];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) q[i] = quant_code(v[i], p, maxq);
+        for (int i = 0; i < E; ++i) q[i] = quant_code(v[i], p, maxq);
         if (bits == 4) {
-            uint32_t packed = 0;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) packed |= static_cast<uint32_t>(q[i]) << (4 * i);
-            __stcs(reinterpret_cast<unsigned int*>(out) + t, packed);
+            for (int h = 0; h < E / 8; ++h) {
+                uint32_t packed = 0;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) packed |= static_cast<uint32_t>(q[8 * h + i]) << (4 * i);
+                __stcs(reinterpret_cast<unsigned int*>(out) + t * (E / 8) + h, packed);
+            }
         } else {
-            uint2 b;
-            b.x = q[0] | (q[1] << 8) | (q[2] << 16) | (q[3] << 24);
-            b.y = q[4] | (q[5] << 8) | (q[6] << 16) | (q[7] << 24);
-            __stcs(reinterpret_cast<uint2*>(out) + t, b);
+#pragma unroll
+            for (int h = 0; h < E / 8; ++h) {
+                uint2 b;
+                b.x = q[8 * h] | (q[8 * h + 1] << 8) | (q[8 * h + 2] << 16) | (q[8 * h + 3] << 24);
+                b.y = q[8 * h + 4] | (q[8 * h + 5] << 8) | (q[8 * h + 6] << 16) | (q[8 * h + 7] << 24);
+                __stcs(reinterpret_cast<uint2*>(out) + t * (E / 8) + h, b);
+            }
         }
         if ((t & (TPG - 1)) == 0) {
             const int64_t gi = t / TPG;
@@ -135,19 +143,24 @@ static gptq_status launch_rtn(const T* W, int64_t n, int group_size, int bits, u
                               uint16_t* scales, uint16_t* zeros, cudaStream_t s) {
     const int sms = num_sms();
     if (group_size % 8 == 0 && group_size <= 256 && (group_size & (group_size - 1)) == 0) {
-        const int64_t n_chunks = n / 8;
+        // 16 weights per thread when the group allows it, else 8
+        const int E = (group_size % 16 == 0) ? 16 : 8;
+        const int64_t n_chunks = n / E;
         int64_t blocks = (n_chunks + 255) / 256;
-        const int64_t cap = static_cast<int64_t>(sms) * 16;
+        const int64_t cap = static_cast<int64_t>(sms) * 8;
         if (blocks > cap) blocks = cap;
         if (blocks < 1) blocks = 1;
         const dim3 grid(static_cast<unsigned>(blocks)), block(256);
-        switch (group_size / 8) {
-            case 1: rtn_kernel<T, 1><<<grid, block, 0, s>>>(W, n_chunks, bits, out, scales, zeros); break;
-            case 2: rtn_kernel<T, 2><<<grid, block, 0, s>>>(W, n_chunks, bits, out, scales, zeros); break;
-            case 4: rtn_kernel<T, 4><<<grid, block, 0, s>>>(W, n_chunks, bits, out, scales, zeros); break;
-            case 8: rtn_kernel<T, 8><<<grid, block, 0, s>>>(W, n_chunks, bits, out, scales, zeros); break;
-            case 16: rtn_kernel<T, 16><<<grid, block, 0, s>>>(W, n_chunks, bits, out, scales, zeros); break;
-            default: rtn_kernel<T, 32><<<grid, block, 0, s>>>(W, n_chunks, bits, out, scales, zeros); break;
+        if (E == 16) {
+            switch (group_size / 16) {
+                case 1: rtn_kernel<T, 16, 1><<<grid, block, 0, s>>>(W, n_chunks, bits, out, scales, zeros); break;
+                case 2: rtn_kernel<T, 16, 2><<<grid, block, 0, s>>>(W, n_chunks, bits, out, scales, zeros); break;
+                case 4: rtn_kernel<T, 16, 4><<<grid, block, 0, s>>>(W, n_chunks, bits, out, scales, zeros); break;
+                case 8: rtn_kernel<T, 16, 8><<<grid, block, 0, s>>>(W, n_chunks, bits, out, scales, zeros); break;
+                default: rtn_kernel<T, 16, 16><<<grid, block, 0, s>>>(W, n_chunks, bits, out, scales, zeros); break;
+            }
+        } else {
+            rtn_kernel<T, 8, 1><<<grid, block, 0, s>>>(W, n_chunks, bits, out, scales, zeros);
         }
     } else {
         const int64_t n_groups = n / group_size;

@@ -1,0 +1,434 @@
+// fp32-accurate GEMM on the 5th-generation tensor cores (tcgen05.mma kind::tf32).
+//
+// tf32 keeps 10 explicit mantissa bits. An fp32 operand x is written as hi + lo with
+// hi = tf32(x) and lo = tf32(x - hi); the product a*b is taken as hi_a*hi_b + hi_a*lo_b +
+// lo_a*hi_b, dropping lo_a*lo_b (about 2^-22 relative). Each partial product is exact in the
+// tensor core and accumulates in fp32 in TMEM, so the result carries fp32-level error, at
+// three tf32 MMAs per step instead of one. An operand that is already exact in tf32 (for
+// example fp16 weights) is not split, and its pass is skipped.
+//
+// Kernel (persistent, one CTA per SM; output tiles of 128 x 128, k-blocks of 32):
+//   warp 0      TMA producer: A tile 128 x 32 (K-major, 128-byte swizzle); B tile either
+//               K-major 128 x 32, or MN-major as four 32 x 32 boxes (128-byte swizzle with
+//               32-byte atoms, the layout the MMA needs for MN-major tf32); 3-stage ring.
+//   warps 2-9   converters: split the fp32 tiles in shared memory into hi (in place) and lo,
+//               then make the writes visible to the tensor core (proxy fence).
+//   warp 1      TMEM allocator and MMA issuer: per k-block 4 k-steps x (1..3) MMAs
+//               M128 N128 K8 into one of two 128-column TMEM accumulators.
+//   warps 10-13 epilogue: tcgen05.ld, then C = alpha*acc + beta*C, or a dot with D.
+// Every mbarrier wait is bounded; on timeout the kernel records GPTQ_ERR_TIMEOUT, drains its
+// copies and MMAs, frees TMEM and returns.
+#include <algorithm>
+
+#include "tcgemm.cuh"
+
+namespace gq {
+
+namespace tg {
+constexpr int BM = 128, BN = 128, BK = 32, STAGES = 3;
+constexpr int TILE_A = BM * BK * 4;                  // 16 KB
+constexpr int TILE_B = BN * BK * 4;                  // 16 KB
+constexpr int OFF_A_LO = TILE_A;
+constexpr int OFF_B = 2 * TILE_A;
+constexpr int OFF_B_LO = 2 * TILE_A + TILE_B;
+constexpr int STAGE = 2 * TILE_A + 2 * TILE_B;       // 64 KB
+constexpr int CONV_WARPS = 8;
+constexpr int EPI_WARP0 = 2 + CONV_WARPS;            // warps 10..13
+constexpr int THREADS = (EPI_WARP0 + 4) * 32;        // 448
+constexpr int BAR_BYTES = 256;
+constexpr int SMEM = 1024 + STAGES * STAGE + BAR_BYTES;
+constexpr uint32_t TMEM_COLS = 256;
+constexpr int BAND = 16;                             // m-tiles per raster band (L2 reuse)
+}  // namespace tg
+
+// kind::tf32 instruction descriptor: A, B tf32 (format 2), D f32, A K-major, B K- or MN-major
+__host__ __device__ constexpr uint32_t umma_idesc_tf32(int M, int N, bool b_mn) {
+    return (1u << 4) | (2u << 7) | (2u << 10) | (0u << 15) | ((b_mn ? 1u : 0u) << 16) |
+           (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_tf32(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                          uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ float tf32_rna(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return __uint_as_float(r);
+}
+
+struct TcParams {
+    TcGemmArgs a;
+    int n_mt, n_nt, n_kb;
+    long long n_tiles;
+};
+
+__device__ __forceinline__ bool tc_tile(const TcParams& p, long long t, int& m0, int& n0) {
+    // bands of BAND m-tiles; inside a band the m-tile varies fastest
+    const long long per_band = static_cast<long long>(tg::BAND) * p.n_nt;
+    const int band = static_cast<int>(t / per_band);
+    const int rem = static_cast<int>(t % per_band);
+    const int band_m = min(tg::BAND, p.n_mt - band * tg::BAND);
+    const int mt = band * tg::BAND + rem % band_m;
+    const int nt = rem / band_m;
+    m0 = mt * tg::BM;
+    n0 = nt * tg::BN;
+    if (nt >= p.n_nt) return false;
+    if (p.a.lower_only && m0 + tg::BM - 1 < n0) return false;
+    return true;
+}
+
+template <bool B_K, int EPI, bool SPLIT_A, bool SPLIT_B>
+__global__ void __launch_bounds__(tg::THREADS, 1)
+    tcgemm_kernel(const __grid_constant__ CUtensorMap amap,
+                  const __grid_constant__ CUtensorMap bmap, const TcParams p) {
+    if (status_bad(p.a.status)) return;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + tg::STAGES * tg::STAGE);
+    uint64_t* full = bars;                          // [STAGES] TMA landed
+    uint64_t* conv = bars + tg::STAGES;             // [STAGES] split done
+    uint64_t* empty = bars + 2 * tg::STAGES;        // [STAGES] MMAs done reading
+    uint64_t* acc_full = bars + 3 * tg::STAGES;     // [2]
+    uint64_t* acc_empty = acc_full + 2;             // [2]
+    uint64_t* drained = acc_empty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drained + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    int* status = const_cast<int*>(p.a.status);
+
+    const int warp = warp_id(), lane = lane_id();
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < tg::STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&conv[s], tg::CONV_WARPS);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_empty[b], 4);
+        }
+        mbar_init(drained, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&amap);
+        tma_prefetch_desc(&bmap);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, tg::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ---------------- TMA producer ----------------
+        if (lane == 0) {
+            int it = 0;
+            for (long long t = blockIdx.x; t < p.n_tiles && !*abort_flag; t += gridDim.x) {
+                int m0, n0;
+                if (!tc_tile(p, t, m0, n0)) continue;
+                for (int kb = 0; kb < p.n_kb; ++kb, ++it) {
+                    const int st = it % tg::STAGES;
+                    if (!mbar_wait(&empty[st], ((it / tg::STAGES) & 1) ^ 1)) {
+                        set_status(status, GPTQ_ERR_TIMEOUT);
+                        *abort_flag = 1;
+                        break;
+                    }
+                    uint8_t* sa = smem + st * tg::STAGE;
+                    const int k0 = kb * tg::BK;
+                    mbar_arrive_expect_tx(&full[st], tg::TILE_A + tg::TILE_B);
+                    tma_load_2d(sa, &amap, &full[st], k0, m0);
+                    if (B_K) {
+                        tma_load_2d(sa + tg::OFF_B, &bmap, &full[st], k0, n0);
+                    } else {
+#pragma unroll
+                        for (int c = 0; c < 4; ++c)
+                            tma_load_2d(sa + tg::OFF_B + c * 4096, &bmap, &full[st], n0 + 32 * c, k0);
+                    }
+                }
+            }
+            const int n_tail = it < tg::STAGES ? it : tg::STAGES;
+            for (int k = it - n_tail; k < it; ++k) {
+                if (!mbar_wait(&full[k % tg::STAGES], (k / tg::STAGES) & 1)) {
+                    set_status(status, GPTQ_ERR_TIMEOUT);
+                    *abort_flag = 1;
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            constexpr uint32_t IDESC = umma_idesc_tf32(tg::BM, tg::BN, !B_K);
+            int it = 0, lt = 0;
+            bool ok = true;
+            for (long long t = blockIdx.x; ok && t < p.n_tiles && !*abort_flag; t += gridDim.x) {
+                int m0, n0;
+                if (!tc_tile(p, t, m0, n0)) continue;
+                const int b = lt & 1;
+                if (!mbar_wait(&acc_empty[b], ((lt >> 1) & 1) ^ 1)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * tg::BN);
+                for (int kb = 0; kb < p.n_kb; ++kb, ++it) {
+                    const int st = it % tg::STAGES;
+                    if (!mbar_wait(&conv[st], (it / tg::STAGES) & 1)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t s0 = smem_u32(smem + st * tg::STAGE);
+#pragma unroll
+                    for (int kk = 0; kk < tg::BK / 8; ++kk) {
+                        // A: K-major rows of 128 B; a k-step of 8 tf32 is 32 B along the row
+                        const uint64_t a_hi = umma_desc_sw128(s0 + kk * 32, 16, 1024);
+                        const uint64_t a_lo = umma_desc_sw128(s0 + tg::OFF_A_LO + kk * 32, 16, 1024);
+                        uint64_t b_hi, b_lo;
+                        if (B_K) {
+                            b_hi = umma_desc_sw128(s0 + tg::OFF_B + kk * 32, 16, 1024);
+                            b_lo = umma_desc_sw128(s0 + tg::OFF_B_LO + kk * 32, 16, 1024);
+                        } else {
+                            // MN-major tf32: 128-byte swizzle with 32-byte atoms; 32-column
+                            // chunks 4 KB apart, 4-row swizzle atoms 512 B apart, a k-step is
+                            // 8 rows (1 KB)
+                            b_hi = umma_desc_sw128_32b(s0 + tg::OFF_B + kk * 1024, 4096, 512);
+                            b_lo = umma_desc_sw128_32b(s0 + tg::OFF_B_LO + kk * 1024, 4096, 512);
+                        }
+                        umma_tf32(d_tmem, a_hi, b_hi, IDESC, (kb > 0 || kk > 0) ? 1u : 0u);
+                        if (SPLIT_B) umma_tf32(d_tmem, a_hi, b_lo, IDESC, 1u);
+                        if (SPLIT_A) umma_tf32(d_tmem, a_lo, b_hi, IDESC, 1u);
+                    }
+                    umma_commit(&empty[st]);
+                }
+                if (!ok) break;
+                umma_commit(&acc_full[b]);
+                ++lt;
+            }
+            if (!ok) {
+                set_status(status, GPTQ_ERR_TIMEOUT);
+                *abort_flag = 1;
+            }
+            umma_commit(drained);
+            if (!mbar_wait(drained, 0)) set_status(status, GPTQ_ERR_TIMEOUT);
+        }
+        __syncwarp();
+    } else if (warp < tg::EPI_WARP0) {
+        // ---------------- converters: fp32 -> tf32 hi (in place) + lo ----------------
+        const int ct = (warp - 2) * 32 + lane;   // 0..255
+        int it = 0;
+        bool stop = false;
+        for (long long t = blockIdx.x; t < p.n_tiles && !stop; t += gridDim.x) {
+            int m0, n0;
+            if (!tc_tile(p, t, m0, n0)) continue;
+            for (int kb = 0; kb < p.n_kb; ++kb, ++it) {
+                const int st = it % tg::STAGES;
+                int ok = 1;
+                if (lane == 0) ok = mbar_wait(&full[st], (it / tg::STAGES) & 1) ? 1 : 0;
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok || __shfl_sync(0xffffffffu, *abort_flag, 0)) {
+                    if (lane == 0 && !ok) {
+                        set_status(status, GPTQ_ERR_TIMEOUT);
+                        *abort_flag = 1;
+                    }
+                    stop = true;
+                    break;
+                }
+                uint8_t* sa = smem + st * tg::STAGE;
+                if (SPLIT_A) {
+                    float4* hi = reinterpret_cast<float4*>(sa);
+                    float4* lo = reinterpret_cast<float4*>(sa + tg::OFF_A_LO);
+#pragma unroll
+                    for (int j = 0; j < tg::TILE_A / 16 / 256; ++j) {
+                        const int i = ct + 256 * j;
+                        const float4 x = hi[i];
+                        float4 h, l;
+                        h.x = tf32_rna(x.x); l.x = tf32_rna(x.x - h.x);
+                        h.y = tf32_rna(x.y); l.y = tf32_rna(x.y - h.y);
+                        h.z = tf32_rna(x.z); l.z = tf32_rna(x.z - h.z);
+                        h.w = tf32_rna(x.w); l.w = tf32_rna(x.w - h.w);
+                        hi[i] = h;
+                        lo[i] = l;
+                    }
+                }
+                if (SPLIT_B) {
+                    float4* hi = reinterpret_cast<float4*>(sa + tg::OFF_B);
+                    float4* lo = reinterpret_cast<float4*>(sa + tg::OFF_B_LO);
+#pragma unroll
+                    for (int j = 0; j < tg::TILE_B / 16 / 256; ++j) {
+                        const int i = ct + 256 * j;
+                        const float4 x = hi[i];
+                        float4 h, l;
+                        h.x = tf32_rna(x.x); l.x = tf32_rna(x.x - h.x);
+                        h.y = tf32_rna(x.y); l.y = tf32_rna(x.y - h.y);
+                        h.z = tf32_rna(x.z); l.z = tf32_rna(x.z - h.z);
+                        h.w = tf32_rna(x.w); l.w = tf32_rna(x.w - h.w);
+                        hi[i] = h;
+                        lo[i] = l;
+                    }
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&conv[st]);
+            }
+        }
+        __syncwarp();
+    } else {
+        // ---------------- epilogue ----------------
+        const int q = warp & 3;
+        const uint32_t t_lane = static_cast<uint32_t>(32 * q) << 16;
+        double dot = 0.0;
+        int lt = 0;
+        bool stop = false;
+        for (long long t = blockIdx.x; t < p.n_tiles && !stop; t += gridDim.x) {
+            int m0, n0;
+            if (!tc_tile(p, t, m0, n0)) continue;
+            const int b = lt & 1;
+            int ok = 1;
+            if (lane == 0) ok = mbar_wait(&acc_full[b], (lt >> 1) & 1) ? 1 : 0;
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok || __shfl_sync(0xffffffffu, *abort_flag, 0)) {
+                if (lane == 0 && !ok) {
+                    set_status(status, GPTQ_ERR_TIMEOUT);
+                    *abort_flag = 1;
+                }
+                stop = true;
+                break;
+            }
+            tc_fence_after();
+            const int row = m0 + 32 * q + lane;
+#pragma unroll 1
+            for (int c = 0; c < tg::BN / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld_32x32b_x32(tmem_base + t_lane + static_cast<uint32_t>(b * tg::BN + 32 * c), r);
+                tmem_ld_wait();
+                const int col0 = n0 + 32 * c;
+                if (row < p.a.M && col0 < p.a.N) {
+                    if (EPI == TC_EPI_STORE) {
+                        float* cp = p.a.C + static_cast<int64_t>(row) * p.a.ldc + col0;
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) {
+                            if (col0 + 4 * k < p.a.N) {
+                                float4 v = make_float4(p.a.alpha * __uint_as_float(r[4 * k]),
+                                                       p.a.alpha * __uint_as_float(r[4 * k + 1]),
+                                                       p.a.alpha * __uint_as_float(r[4 * k + 2]),
+                                                       p.a.alpha * __uint_as_float(r[4 * k + 3]));
+                                if (p.a.beta != 0.0f) {
+                                    const float4 o = *reinterpret_cast<const float4*>(cp + 4 * k);
+                                    v.x = fmaf(p.a.beta, o.x, v.x);
+                                    v.y = fmaf(p.a.beta, o.y, v.y);
+                                    v.z = fmaf(p.a.beta, o.z, v.z);
+                                    v.w = fmaf(p.a.beta, o.w, v.w);
+                                }
+                                *reinterpret_cast<float4*>(cp + 4 * k) = v;
+                            }
+                        }
+                    } else {
+                        const float* dp = p.a.D + static_cast<int64_t>(row) * p.a.ldd + col0;
+                        float part = 0.0f;
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) {
+                            if (col0 + 4 * k < p.a.N) {
+                                const float4 dv = *reinterpret_cast<const float4*>(dp + 4 * k);
+                                part = fmaf(__uint_as_float(r[4 * k]), dv.x, part);
+                                part = fmaf(__uint_as_float(r[4 * k + 1]), dv.y, part);
+                                part = fmaf(__uint_as_float(r[4 * k + 2]), dv.z, part);
+                                part = fmaf(__uint_as_float(r[4 * k + 3]), dv.w, part);
+                            }
+                        }
+                        dot += static_cast<double>(part);
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[b]);
+            ++lt;
+        }
+        if (EPI == TC_EPI_DOT) {
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
+            if (lane == 0 && dot != 0.0) atomicAdd(p.a.dot, static_cast<double>(p.a.alpha) * dot);
+        }
+        __syncwarp();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem_base, tg::TMEM_COLS);
+}
+
+template <bool B_K, int EPI, bool SA, bool SB>
+static gptq_status launch_variant(const CUtensorMap& am, const CUtensorMap& bm, const TcParams& p,
+                                  int grid, cudaStream_t s) {
+    static bool attr = false;
+    if (!attr) {
+        GPTQ_CUDA_TRY(cudaFuncSetAttribute(tcgemm_kernel<B_K, EPI, SA, SB>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, tg::SMEM));
+        attr = true;
+    }
+    tcgemm_kernel<B_K, EPI, SA, SB><<<grid, tg::THREADS, tg::SMEM, s>>>(am, bm, p);
+    GPTQ_LAUNCHED();
+    return GPTQ_OK;
+}
+
+template <bool B_K, int EPI>
+static gptq_status launch_split(const CUtensorMap& am, const CUtensorMap& bm, const TcParams& p,
+                                int grid, bool sa, bool sb, cudaStream_t s) {
+    if (sa && sb) return launch_variant<B_K, EPI, true, true>(am, bm, p, grid, s);
+    if (sa) return launch_variant<B_K, EPI, true, false>(am, bm, p, grid, s);
+    if (sb) return launch_variant<B_K, EPI, false, true>(am, bm, p, grid, s);
+    return launch_variant<B_K, EPI, false, false>(am, bm, p, grid, s);
+}
+
+gptq_status tcgemm_launch(const TcGemmArgs& a, bool b_kmajor, int epi, bool split_a, bool split_b,
+                          cudaStream_t s) {
+    if (a.M <= 0 || a.N <= 0 || a.K <= 0) return GPTQ_OK;
+    if (a.lda % 4 || a.ldb % 4 || a.N % 4 || (epi == TC_EPI_STORE && a.ldc % 4) ||
+        (epi == TC_EPI_DOT && a.ldd % 4))
+        return GPTQ_ERR_ARG;
+    if ((reinterpret_cast<uintptr_t>(a.A) & 15) || (reinterpret_cast<uintptr_t>(a.B) & 15))
+        return GPTQ_ERR_ARG;
+    CUtensorMap am, bm;
+    GPTQ_TRY(encode_tensor_map_2d(&am, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, const_cast<float*>(a.A),
+                                  a.K, a.M, static_cast<uint64_t>(a.lda) * 4, 32, 128,
+                                  CU_TENSOR_MAP_SWIZZLE_128B));
+    if (b_kmajor) {
+        GPTQ_TRY(encode_tensor_map_2d(&bm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, const_cast<float*>(a.B),
+                                      a.K, a.N, static_cast<uint64_t>(a.ldb) * 4, 32, 128,
+                                      CU_TENSOR_MAP_SWIZZLE_128B));
+    } else {
+        GPTQ_TRY(encode_tensor_map_2d(&bm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, const_cast<float*>(a.B),
+                                      a.N, a.K, static_cast<uint64_t>(a.ldb) * 4, 32, 32,
+                                      CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B));
+    }
+    TcParams p;
+    p.a = a;
+    p.n_mt = (a.M + tg::BM - 1) / tg::BM;
+    p.n_nt = (a.N + tg::BN - 1) / tg::BN;
+    p.n_kb = (a.K + tg::BK - 1) / tg::BK;
+    const int n_bands = (p.n_mt + tg::BAND - 1) / tg::BAND;
+    p.n_tiles = static_cast<long long>(n_bands) * tg::BAND * p.n_nt;
+    long long useful = static_cast<long long>(p.n_mt) * p.n_nt;
+    if (a.lower_only) useful = useful / 2 + p.n_mt;
+    const int grid = static_cast<int>(std::max<long long>(1, std::min<long long>(useful, num_sms())));
+    if (b_kmajor) {
+        return epi == TC_EPI_STORE ? launch_split<true, TC_EPI_STORE>(am, bm, p, grid, split_a, split_b, s)
+                                   : launch_split<true, TC_EPI_DOT>(am, bm, p, grid, split_a, split_b, s);
+    }
+    return epi == TC_EPI_STORE ? launch_split<false, TC_EPI_STORE>(am, bm, p, grid, split_a, split_b, s)
+                               : launch_split<false, TC_EPI_DOT>(am, bm, p, grid, split_a, split_b, s);
+}
+
+}  // namespace gq
