@@ -15,7 +15,9 @@
 //               then make the writes visible to the tensor core (proxy fence).
 //   warp 1      TMEM allocator and MMA issuer: per k-block 4 k-steps x (1..3) MMAs
 //               M128 N128 K8 into one of two 128-column TMEM accumulators.
-//   warps 10-13 epilogue: tcgen05.ld, then C = alpha*acc + beta*C, or a dot with D.
+//   warps 10-13 epilogue: tcgen05.ld, scale by alpha, stage 32 x 32 pieces in swizzled shared
+//               memory and let TMA write them: a tensor reduce-add (C += alpha*A*B, the add
+//               happens in L2) when beta = 1, a tensor store when beta = 0; or a dot with D.
 // Every mbarrier wait is bounded; on timeout the kernel records GPTQ_ERR_TIMEOUT, drains its
 // copies and MMAs, frees TMEM and returns.
 #include <algorithm>
@@ -35,8 +37,10 @@ constexpr int STAGE = 2 * TILE_A + 2 * TILE_B;       // 64 KB
 constexpr int CONV_WARPS = 8;
 constexpr int EPI_WARP0 = 2 + CONV_WARPS;            // warps 10..13
 constexpr int THREADS = (EPI_WARP0 + 4) * 32;        // 448
+constexpr int EPI_BUF = 32 * 32 * 4;                // 4 KB: 32 rows x 32 fp32
+constexpr int EPI_BYTES = 4 * 2 * EPI_BUF;           // 4 warps, double-buffered
 constexpr int BAR_BYTES = 256;
-constexpr int SMEM = 1024 + STAGES * STAGE + BAR_BYTES;
+constexpr int SMEM = 1024 + STAGES * STAGE + EPI_BYTES + BAR_BYTES;
 constexpr uint32_t TMEM_COLS = 256;
 constexpr int BAND = 16;                             // m-tiles per raster band (L2 reuse)
 }  // namespace tg
@@ -65,6 +69,7 @@ __device__ __forceinline__ float tf32_rna(float x) {
 
 struct TcParams {
     TcGemmArgs a;
+    int beta_one;
     int n_mt, n_nt, n_kb;
     long long n_tiles;
 };
@@ -87,12 +92,14 @@ __device__ __forceinline__ bool tc_tile(const TcParams& p, long long t, int& m0,
 template <bool B_K, int EPI, bool SPLIT_A, bool SPLIT_B>
 __global__ void __launch_bounds__(tg::THREADS, 1)
     tcgemm_kernel(const __grid_constant__ CUtensorMap amap,
-                  const __grid_constant__ CUtensorMap bmap, const TcParams p) {
+                  const __grid_constant__ CUtensorMap bmap,
+                  const __grid_constant__ CUtensorMap cmap, const TcParams p) {
     if (status_bad(p.a.status)) return;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + tg::STAGES * tg::STAGE);
+    float* epi_smem = reinterpret_cast<float*>(smem + tg::STAGES * tg::STAGE);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + tg::STAGES * tg::STAGE + tg::EPI_BYTES);
     uint64_t* full = bars;                          // [STAGES] TMA landed
     uint64_t* conv = bars + tg::STAGES;             // [STAGES] split done
     uint64_t* empty = bars + 2 * tg::STAGES;        // [STAGES] MMAs done reading
@@ -119,6 +126,7 @@ __global__ void __launch_bounds__(tg::THREADS, 1)
         fence_mbar_init();
         tma_prefetch_desc(&amap);
         tma_prefetch_desc(&bmap);
+        if (EPI == TC_EPI_STORE) tma_prefetch_desc(&cmap);
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, tg::TMEM_COLS);
@@ -287,8 +295,9 @@ __global__ void __launch_bounds__(tg::THREADS, 1)
         // ---------------- epilogue ----------------
         const int q = warp & 3;
         const uint32_t t_lane = static_cast<uint32_t>(32 * q) << 16;
+        float* stage_buf = epi_smem + (warp - tg::EPI_WARP0) * 2 * (tg::EPI_BUF / 4);
         double dot = 0.0;
-        int lt = 0;
+        int lt = 0, nbulk = 0;
         bool stop = false;
         for (long long t = blockIdx.x; t < p.n_tiles && !stop; t += gridDim.x) {
             int m0, n0;
@@ -306,48 +315,49 @@ __global__ void __launch_bounds__(tg::THREADS, 1)
                 break;
             }
             tc_fence_after();
-            const int row = m0 + 32 * q + lane;
+            const int row0 = m0 + 32 * q;
+            const int row = row0 + lane;
 #pragma unroll 1
             for (int c = 0; c < tg::BN / 32; ++c) {
                 uint32_t r[32];
                 tmem_ld_32x32b_x32(tmem_base + t_lane + static_cast<uint32_t>(b * tg::BN + 32 * c), r);
                 tmem_ld_wait();
                 const int col0 = n0 + 32 * c;
-                if (row < p.a.M && col0 < p.a.N) {
-                    if (EPI == TC_EPI_STORE) {
-                        float* cp = p.a.C + static_cast<int64_t>(row) * p.a.ldc + col0;
+                if (row0 >= p.a.M || col0 >= p.a.N) continue;       // warp-uniform
+                if (EPI == TC_EPI_STORE) {
+                    // stage this warp's 32 x 32 piece with the 128-byte swizzle of the C map
+                    float* buf = stage_buf + (nbulk & 1) * (tg::EPI_BUF / 4);
+                    if (lane == 0) bulk_wait_read<1>();
+                    __syncwarp();
+                    float4* rowp = reinterpret_cast<float4*>(buf + lane * 32);
 #pragma unroll
-                        for (int k = 0; k < 8; ++k) {
-                            if (col0 + 4 * k < p.a.N) {
-                                float4 v = make_float4(p.a.alpha * __uint_as_float(r[4 * k]),
-                                                       p.a.alpha * __uint_as_float(r[4 * k + 1]),
-                                                       p.a.alpha * __uint_as_float(r[4 * k + 2]),
-                                                       p.a.alpha * __uint_as_float(r[4 * k + 3]));
-                                if (p.a.beta != 0.0f) {
-                                    const float4 o = *reinterpret_cast<const float4*>(cp + 4 * k);
-                                    v.x = fmaf(p.a.beta, o.x, v.x);
-                                    v.y = fmaf(p.a.beta, o.y, v.y);
-                                    v.z = fmaf(p.a.beta, o.z, v.z);
-                                    v.w = fmaf(p.a.beta, o.w, v.w);
-                                }
-                                *reinterpret_cast<float4*>(cp + 4 * k) = v;
-                            }
-                        }
-                    } else {
-                        const float* dp = p.a.D + static_cast<int64_t>(row) * p.a.ldd + col0;
-                        float part = 0.0f;
-#pragma unroll
-                        for (int k = 0; k < 8; ++k) {
-                            if (col0 + 4 * k < p.a.N) {
-                                const float4 dv = *reinterpret_cast<const float4*>(dp + 4 * k);
-                                part = fmaf(__uint_as_float(r[4 * k]), dv.x, part);
-                                part = fmaf(__uint_as_float(r[4 * k + 1]), dv.y, part);
-                                part = fmaf(__uint_as_float(r[4 * k + 2]), dv.z, part);
-                                part = fmaf(__uint_as_float(r[4 * k + 3]), dv.w, part);
-                            }
-                        }
-                        dot += static_cast<double>(part);
+                    for (int j = 0; j < 8; ++j) {
+                        rowp[j ^ (lane & 7)] = make_float4(
+                            p.a.alpha * __uint_as_float(r[4 * j]), p.a.alpha * __uint_as_float(r[4 * j + 1]),
+                            p.a.alpha * __uint_as_float(r[4 * j + 2]), p.a.alpha * __uint_as_float(r[4 * j + 3]));
                     }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        if (p.beta_one) tma_reduce_add_2d(&cmap, buf, col0, row0);
+                        else tma_store_2d(&cmap, buf, col0, row0);
+                        bulk_commit();
+                    }
+                    ++nbulk;
+                } else if (row < p.a.M) {
+                    const float* dp = p.a.D + static_cast<int64_t>(row) * p.a.ldd + col0;
+                    float part = 0.0f;
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        if (col0 + 4 * k < p.a.N) {
+                            const float4 dv = *reinterpret_cast<const float4*>(dp + 4 * k);
+                            part = fmaf(__uint_as_float(r[4 * k]), dv.x, part);
+                            part = fmaf(__uint_as_float(r[4 * k + 1]), dv.y, part);
+                            part = fmaf(__uint_as_float(r[4 * k + 2]), dv.z, part);
+                            part = fmaf(__uint_as_float(r[4 * k + 3]), dv.w, part);
+                        }
+                    }
+                    dot += static_cast<double>(part);
                 }
             }
             tc_fence_before();
@@ -355,7 +365,9 @@ __global__ void __launch_bounds__(tg::THREADS, 1)
             if (lane == 0) mbar_arrive(&acc_empty[b]);
             ++lt;
         }
-        if (EPI == TC_EPI_DOT) {
+        if (EPI == TC_EPI_STORE) {
+            if (lane == 0) bulk_wait_all();
+        } else {
 #pragma unroll
             for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
             if (lane == 0 && dot != 0.0) atomicAdd(p.a.dot, static_cast<double>(p.a.alpha) * dot);
@@ -370,26 +382,28 @@ __global__ void __launch_bounds__(tg::THREADS, 1)
 }
 
 template <bool B_K, int EPI, bool SA, bool SB>
-static gptq_status launch_variant(const CUtensorMap& am, const CUtensorMap& bm, const TcParams& p,
-                                  int grid, cudaStream_t s) {
+static gptq_status launch_variant(const CUtensorMap& am, const CUtensorMap& bm,
+                                  const CUtensorMap& cm, const TcParams& p, int grid,
+                                  cudaStream_t s) {
     static bool attr = false;
     if (!attr) {
         GPTQ_CUDA_TRY(cudaFuncSetAttribute(tcgemm_kernel<B_K, EPI, SA, SB>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, tg::SMEM));
         attr = true;
     }
-    tcgemm_kernel<B_K, EPI, SA, SB><<<grid, tg::THREADS, tg::SMEM, s>>>(am, bm, p);
+    tcgemm_kernel<B_K, EPI, SA, SB><<<grid, tg::THREADS, tg::SMEM, s>>>(am, bm, cm, p);
     GPTQ_LAUNCHED();
     return GPTQ_OK;
 }
 
 template <bool B_K, int EPI>
-static gptq_status launch_split(const CUtensorMap& am, const CUtensorMap& bm, const TcParams& p,
-                                int grid, bool sa, bool sb, cudaStream_t s) {
-    if (sa && sb) return launch_variant<B_K, EPI, true, true>(am, bm, p, grid, s);
-    if (sa) return launch_variant<B_K, EPI, true, false>(am, bm, p, grid, s);
-    if (sb) return launch_variant<B_K, EPI, false, true>(am, bm, p, grid, s);
-    return launch_variant<B_K, EPI, false, false>(am, bm, p, grid, s);
+static gptq_status launch_split(const CUtensorMap& am, const CUtensorMap& bm,
+                                const CUtensorMap& cm, const TcParams& p, int grid, bool sa,
+                                bool sb, cudaStream_t s) {
+    if (sa && sb) return launch_variant<B_K, EPI, true, true>(am, bm, cm, p, grid, s);
+    if (sa) return launch_variant<B_K, EPI, true, false>(am, bm, cm, p, grid, s);
+    if (sb) return launch_variant<B_K, EPI, false, true>(am, bm, cm, p, grid, s);
+    return launch_variant<B_K, EPI, false, false>(am, bm, cm, p, grid, s);
 }
 
 gptq_status tcgemm_launch(const TcGemmArgs& a, bool b_kmajor, int epi, bool split_a, bool split_b,
@@ -400,7 +414,18 @@ gptq_status tcgemm_launch(const TcGemmArgs& a, bool b_kmajor, int epi, bool spli
         return GPTQ_ERR_ARG;
     if ((reinterpret_cast<uintptr_t>(a.A) & 15) || (reinterpret_cast<uintptr_t>(a.B) & 15))
         return GPTQ_ERR_ARG;
-    CUtensorMap am, bm;
+    // the stored result goes out through TMA: beta must be 0 (store) or 1 (reduce-add)
+    if (epi == TC_EPI_STORE &&
+        ((a.beta != 0.0f && a.beta != 1.0f) || (reinterpret_cast<uintptr_t>(a.C) & 15)))
+        return GPTQ_ERR_ARG;
+    CUtensorMap am, bm, cm;
+    if (epi == TC_EPI_STORE) {
+        GPTQ_TRY(encode_tensor_map_2d(&cm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.C, a.N, a.M,
+                                      static_cast<uint64_t>(a.ldc) * 4, 32, 32,
+                                      CU_TENSOR_MAP_SWIZZLE_128B));
+    } else {
+        cm = am;   // unused by the dot epilogue
+    }
     GPTQ_TRY(encode_tensor_map_2d(&am, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, const_cast<float*>(a.A),
                                   a.K, a.M, static_cast<uint64_t>(a.lda) * 4, 32, 128,
                                   CU_TENSOR_MAP_SWIZZLE_128B));
@@ -415,6 +440,7 @@ gptq_status tcgemm_launch(const TcGemmArgs& a, bool b_kmajor, int epi, bool spli
     }
     TcParams p;
     p.a = a;
+    p.beta_one = (a.beta == 1.0f) ? 1 : 0;
     p.n_mt = (a.M + tg::BM - 1) / tg::BM;
     p.n_nt = (a.N + tg::BN - 1) / tg::BN;
     p.n_kb = (a.K + tg::BK - 1) / tg::BK;
@@ -424,11 +450,13 @@ gptq_status tcgemm_launch(const TcGemmArgs& a, bool b_kmajor, int epi, bool spli
     if (a.lower_only) useful = useful / 2 + p.n_mt;
     const int grid = static_cast<int>(std::max<long long>(1, std::min<long long>(useful, num_sms())));
     if (b_kmajor) {
-        return epi == TC_EPI_STORE ? launch_split<true, TC_EPI_STORE>(am, bm, p, grid, split_a, split_b, s)
-                                   : launch_split<true, TC_EPI_DOT>(am, bm, p, grid, split_a, split_b, s);
+        return epi == TC_EPI_STORE
+                   ? launch_split<true, TC_EPI_STORE>(am, bm, cm, p, grid, split_a, split_b, s)
+                   : launch_split<true, TC_EPI_DOT>(am, bm, cm, p, grid, split_a, split_b, s);
     }
-    return epi == TC_EPI_STORE ? launch_split<false, TC_EPI_STORE>(am, bm, p, grid, split_a, split_b, s)
-                               : launch_split<false, TC_EPI_DOT>(am, bm, p, grid, split_a, split_b, s);
+    return epi == TC_EPI_STORE
+               ? launch_split<false, TC_EPI_STORE>(am, bm, cm, p, grid, split_a, split_b, s)
+               : launch_split<false, TC_EPI_DOT>(am, bm, cm, p, grid, split_a, split_b, s);
 }
 
 }  // namespace gq
