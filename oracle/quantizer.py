@@ -10,11 +10,16 @@ Sources
 Readings taken where the pages are silent:
   * Codes use the unsigned range [0, maxq], maxq = 2**bits - 1 (the INT8 example's signed range
     differs only by an offset of 2**(bits-1)).
-  * The range is the literal min and max of the group.
+  * The range is the group's min and max widened to contain 0. §2.1's formula sends the real
+    value 0 to the code zero_point, so zero_point is itself a code in [0, maxq] and, with
+    §4.2's fp16 storage, exact; a group entirely above (below) 0 gets the range [0, max]
+    ([min, 0]). For groups that contain 0 (the worked example's [-2.5, 3.7]) this is the
+    literal min and max.
   * scale = (xmax - xmin)/maxq rounded UP to fp16, so that the stored scale is what the codes
     are computed with and |w - ŵ| <= scale/2 holds exactly for every entry.
-  * zero = rint(-xmin/scale), round half to even; an integer, stored as an fp16 value.
-  * A group with xmax == xmin gets scale 1.
+  * zero = rint(-xmin/scale), round half to even; an integer in [0, maxq] (+0, never -0),
+    stored as an fp16 value.
+  * An all-zero group (xmax == xmin == 0 after widening) gets scale 1.
   * q = clamp(rint(w/scale) + zero, 0, maxq), round half to even; ŵ = scale·(q - zero).
 """
 
@@ -37,15 +42,16 @@ def fp16_round_up(x):
 def group_params(xmin, xmax, maxq):
     """(scale, zero) for groups with the given minima and maxima (fp64 arrays).
 
-    scale is fp16-representable (held in fp64), zero is integer-valued (held in fp64).
+    The range [xmin, xmax] is first widened to contain 0. scale is fp16-representable (held
+    in fp64), zero is an integer in [0, maxq] (held in fp64).
     """
-    xmin = np.asarray(xmin, dtype=np.float64)
-    xmax = np.asarray(xmax, dtype=np.float64)
+    xmin = np.minimum(np.asarray(xmin, dtype=np.float64), 0.0)
+    xmax = np.maximum(np.asarray(xmax, dtype=np.float64), 0.0)
     span = xmax - xmin
     with np.errstate(divide="ignore", invalid="ignore"):
         scale = fp16_round_up(span / maxq)
         scale = np.where(span == 0.0, 1.0, scale)
-        zero = np.rint(-xmin / scale)
+        zero = np.rint(-xmin / scale) + 0.0
     return scale, zero
 
 

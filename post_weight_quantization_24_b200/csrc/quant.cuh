@@ -3,8 +3,10 @@
 // 0539edu.com/news/6111416 §2.1: q = round(x/scale) + zero_point, scale = (max-min)/(qmax-qmin).
 // §4.2: one fp16 scale and one fp16 zero point per group.
 //
-// Group scalars are computed in fp64:  scale = smallest fp16 >= (xmax - xmin)/maxq (1 when the
-// group is constant), zero = rint(-xmin/scale) (half to even). Per-element codes
+// The group's range [xmin, xmax] is widened to contain 0 (the formula maps real 0 to the code
+// zero_point, so the zero point is a code in [0, maxq] and exact in fp16). Group scalars are
+// computed in fp64:  scale = smallest fp16 >= (xmax - xmin)/maxq (1 for an all-zero group),
+// zero = rint(-xmin/scale) (half to even, +0 rather than -0). Per-element codes
 // q = clamp(rint(w/scale) + zero, 0, maxq) are decided EXACTLY in fp32: an approximate
 // quotient gives a candidate k, and the sign of w - (k +- 1/2)*scale, computed with a single
 // fused multiply-add (one rounding of the exact value, so its sign is exact), moves k by one
@@ -38,14 +40,22 @@ struct QParams {
 };
 
 __device__ __forceinline__ QParams group_params(float xmin, float xmax, int maxq) {
-    const double span = static_cast<double>(xmax) - static_cast<double>(xmin);
+    const double lo = fmin(static_cast<double>(xmin), 0.0);
+    const double hi = fmax(static_cast<double>(xmax), 0.0);
+    const double span = hi - lo;
     const double s = (span == 0.0) ? 1.0 : fp16_ceil(span / static_cast<double>(maxq));
-    const double z = rint(-static_cast<double>(xmin) / s);
+    const double z = rint(-lo / s) + 0.0;
     QParams p;
     p.scale = static_cast<float>(s);
     p.zero = static_cast<float>(z);
     p.inv_scale = static_cast<float>(1.0 / s);
     return p;
+}
+
+// The same, kept out of line: for loops that reach it rarely (once per group) and would
+// otherwise carry one inlined copy of the fp64 sequence per unrolled iteration.
+static __device__ __noinline__ QParams group_params_call(float xmin, float xmax, int maxq) {
+    return group_params(xmin, xmax, maxq);
 }
 
 // rint(w / scale) with the exact tie-to-even decision described above.

@@ -111,7 +111,7 @@ def recurrence_consistency(Wn, H, out, g, bits, percdamp, rows, tie_tol=0.05):
         gi = q // g
         if q % g == 0:
             grp = w[:, q:q + g]
-            span = grp.max(1) - grp.min(1)
+            span = np.maximum(grp.max(1), 0.0) - np.minimum(grp.min(1), 0.0)
             s_ex = (span / maxq).astype(np.float16).astype(np.float64)
             lo = np.nextafter(s_ex.astype(np.float16), np.float16(-np.inf)).astype(np.float64)
             hi = np.nextafter(np.nextafter(s_ex.astype(np.float16), np.float16(np.inf)),
@@ -213,7 +213,8 @@ def check_outputs(out, ref, Wn, Href, g, perm_must_match=True, max_diff=1):
 
 @pytest.mark.parametrize("bits,g,B,act_order", [
     (4, 128, 128, False), (4, 128, 128, True), (3, 128, 128, True), (4, 64, 128, False),
-    (4, 32, 64, True), (2, 128, 128, False), (8, 128, 128, True), (4, 8, 16, False)])
+    (4, 32, 64, True), (2, 128, 128, False), (8, 128, 128, True), (4, 8, 16, False),
+    (3, 2, 16, False)])
 def test_linear_512(cuda_lib, bits, g, B, act_order):
     wl = workloads.WORKLOADS["linear_512"]
     W = workloads.make_weights(wl, device="cuda")
@@ -224,7 +225,7 @@ def test_linear_512(cuda_lib, bits, g, B, act_order):
 
 @pytest.mark.parametrize("d_out,d_in,n,g,B,act_order", [
     (77, 384, 1500, 64, 128, True), (31, 200, 800, 8, 64, False), (64, 264, 900, 8, 128, True),
-    (5, 136, 300, 8, 64, False), (129, 1024, 3000, 128, 128, True)])
+    (5, 136, 300, 8, 64, False), (129, 1024, 3000, 128, 128, True), (37, 120, 600, 6, 24, True)])
 def test_ragged_shapes(cuda_lib, d_out, d_in, n, g, B, act_order):
     wl = workloads.WORKLOADS["mlp_up_7b"].replace(d_out=d_out, d_in=d_in, n_tokens=n, seed=d_in)
     W = workloads.make_weights(wl, device="cuda")

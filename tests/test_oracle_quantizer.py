@@ -76,8 +76,17 @@ def test_quantizer_error_bound_and_nearest_level(bits):
         levels = quantizer.dequantize(np.arange(maxq + 1), s, z)
         best = np.min(np.abs(w[:, None] - levels[None, :]), axis=1)
         assert np.all(np.abs(w - wh) <= best)
-        # the group minimum maps to code 0 exactly
-        assert q[np.argmin(w)] == 0
+        # the zero point is a code and real 0 sits exactly on it
+        assert z == np.rint(z) and 0 <= z <= maxq and not np.signbit(z)
+        assert quantizer.dequantize(np.array([z]), s, z)[0] == 0.0
+        # the widened range's lower end maps to code 0 (rint(-x) = -rint(x) under half-even;
+        # the upper end may land one code short because z is rounded)
+        lo = min(w.min(), 0.0)
+        assert quantizer.quantize(np.array([lo]), s, z, maxq)[0] == 0
+        if w.min() >= 0:
+            assert z == 0 and q[np.argmin(w)] == np.clip(np.rint(w.min() / s), 0, maxq)
+        else:
+            assert q[np.argmin(w)] == 0
 
 
 def test_quantizer_ties_round_half_even():
@@ -88,10 +97,23 @@ def test_quantizer_ties_round_half_even():
 
 
 def test_degenerate_group_scale_one():
+    s, z = quantizer.group_params(0.0, 0.0, 15)
+    assert s == 1.0 and z == 0.0 and not np.signbit(z)
+    assert quantizer.quantize(np.array([0.0]), s, z, 15)[0] == 0
+
+
+def test_one_signed_groups_widen_to_zero():
+    # a constant positive group: range [0, 0.3], the value lands on the top code
     s, z = quantizer.group_params(0.3, 0.3, 15)
-    assert s == 1.0 and z == 0.0
-    q = quantizer.quantize(np.array([0.3]), s, z, 15)
-    assert abs(0.3 - quantizer.dequantize(q, s, z)[0]) <= 0.5
+    assert z == 0.0 and s == quantizer.fp16_round_up(0.3 / 15)
+    assert quantizer.quantize(np.array([0.3]), s, z, 15)[0] == 15
+    # a negative group [-0.7, -0.2]: range [-0.7, 0], zero point at the top code
+    s, z = quantizer.group_params(-0.7, -0.2, 7)
+    assert s == quantizer.fp16_round_up(0.7 / 7) and z == 7.0
+    assert list(quantizer.quantize(np.array([-0.7, 0.0]), s, z, 7)) == [0, 7]
+    # a tiny span far from 0 no longer gives a zero point beyond fp16's exact integers
+    s, z = quantizer.group_params(1.0, 1.0 + 2.0 ** -20, 7)
+    assert z == 0.0 and np.float16(z) == z
 
 
 def test_rtn_matches_per_group_brute_force():
@@ -101,7 +123,7 @@ def test_rtn_matches_per_group_brute_force():
     for r in range(16):
         for gi in range(4):
             w = W[r, gi * 16:(gi + 1) * 16]
-            span = w.max() - w.min()
+            span = max(w.max(), 0.0) - min(w.min(), 0.0)
             s = quantizer.fp16_round_up(span / 15)
             assert scales[r, gi] == s
             levels = s * (np.arange(16) - zeros[r, gi])
