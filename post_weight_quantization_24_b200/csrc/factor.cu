@@ -187,10 +187,15 @@ gptq_status gather_w_launch(const void* W, int w_dtype, int d_out, int d_in, con
 // way; then all warps solve the sub-panel below it against that inverse and apply the rank-32
 // update to the trailing part of the block. Finally the inverse of the whole 128 x 128 factor
 // is assembled from the four sub-block inverses by block forward substitution. Rows and
-// columns beyond the matrix edge (last block) are padded with the identity.
+// columns beyond the matrix edge (last block) are padded with the identity. The solve, update
+// and assembly loops work on 4-column strips so one shared-memory load feeds four FMAs; the
+// operands they stream across columns are kept transposed for that.
 namespace pd {
-constexpr int NB = 128, LD = NB + 1, SUB = 32, THREADS = 512;
-constexpr int SMEM = (2 * NB * LD + 4 * SUB * (SUB + 1)) * 4;
+constexpr int NB = 128, SUB = 32, THREADS = 512;
+constexpr int LD = NB + 1;        // S: scalar row access
+constexpr int LDV = NB + 4;       // Dv, LT: float4 row access
+constexpr int LDX = SUB + 4;      // XT: float4 row access
+constexpr int SMEM = (NB * LD + NB * LDV + SUB * LDV + 4 * SUB * LDX) * 4;
 }  // namespace pd
 
 // v: row `lane` of a 32 x 32 SPD block (lower part used). On return v holds row `lane` of its
@@ -198,12 +203,15 @@ constexpr int SMEM = (2 * NB * LD + 4 * SUB * (SUB + 1)) * 4;
 __device__ __forceinline__ void warp_chol_inv32(float (&v)[32], float (&x)[32], int lane,
                                                 bool& bad) {
     const unsigned full = 0xffffffffu;
+    float rdiag = 1.0f;   // 1 / L[lane][lane]
 #pragma unroll
     for (int c = 0; c < 32; ++c) {
         const float piv = __shfl_sync(full, v[c], c);
         if (!(piv > 0.0f) || !isfinite(piv)) bad = true;
-        const float rs = 1.0f / sqrtf(piv);
-        const float lic = (lane >= c) ? v[c] * rs : 0.0f;
+        float r = rsqrtf(piv);
+        r = r * fmaf(-0.5f * piv, r * r, 1.5f);   // one Newton step: r = 1/sqrt(piv)
+        if (lane == c) rdiag = r;
+        const float lic = (lane >= c) ? v[c] * r : 0.0f;
         v[c] = lic;
 #pragma unroll
         for (int j = c + 1; j < 32; ++j) {
@@ -216,21 +224,20 @@ __device__ __forceinline__ void warp_chol_inv32(float (&v)[32], float (&x)[32], 
         if (j > lane) v[j] = 0.0f;
         x[j] = (j == lane) ? 1.0f : 0.0f;
     }
-    // forward substitution on the identity: row k is final once rows < k have been applied
+    // forward substitution on the identity with the row scaling deferred: when row k is
+    // broadcast it is scaled by 1/L[k][k] on the fly; each lane scales its own row at the end
 #pragma unroll
     for (int k = 0; k < 32; ++k) {
-        const float rkk = 1.0f / __shfl_sync(full, v[k], k);   // 1 / L[k][k]
-        if (lane == k) {
-#pragma unroll
-            for (int j = 0; j <= k; ++j) x[j] *= rkk;
-        }
-        const float lik = v[k];
+        const float rkk = __shfl_sync(full, rdiag, k);
+        const float nlik = (lane > k) ? -v[k] : 0.0f;
 #pragma unroll
         for (int j = 0; j <= k; ++j) {
-            const float xkj = __shfl_sync(full, x[j], k);
-            if (lane > k) x[j] = fmaf(-lik, xkj, x[j]);
+            const float xkj = __shfl_sync(full, x[j], k) * rkk;
+            x[j] = fmaf(nlik, xkj, x[j]);
         }
     }
+#pragma unroll
+    for (int j = 0; j < 32; ++j) x[j] *= rdiag;
 }
 
 __global__ void __launch_bounds__(pd::THREADS) potrf_diag_kernel(float* __restrict__ A, int d,
@@ -238,25 +245,34 @@ __global__ void __launch_bounds__(pd::THREADS) potrf_diag_kernel(float* __restri
                                                                 float* __restrict__ Dinv,
                                                                 int* status) {
     if (status_bad(status)) return;
-    extern __shared__ float sm[];
+    extern __shared__ __align__(16) float sm[];
     float* S = sm;                          // [NB][LD]: the block, then its factor L
-    float* Dv = S + pd::NB * pd::LD;        // [NB][LD]: L^-1
-    float* Xs = Dv + pd::NB * pd::LD;       // [4][SUB][SUB+1]: sub-block inverses
+    float* Dv = S + pd::NB * pd::LD;        // [NB][LDV]: L^-1
+    float* LT = Dv + pd::NB * pd::LDV;      // [SUB][LDV]: current sub-panel of L, transposed
+    float* XT = LT + pd::SUB * pd::LDV;     // [4][SUB][LDX]: sub-block inverses, transposed
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     constexpr int NW = pd::THREADS / 32;
 
-    for (int i = warp; i < pd::NB; i += NW)
-        for (int j = lane; j < pd::NB; j += 32) {
-            float v = (i == j) ? 1.0f : 0.0f;
-            if (i < nbc && j < nbc && j <= i) v = A[static_cast<int64_t>(k0 + i) * d + k0 + j];
-            S[i * pd::LD + j] = v;
+    // load: 32 independent loads per thread, then the stores (identity padding past the edge)
+    {
+        float vals[32];
+#pragma unroll
+        for (int t = 0; t < 32; ++t) {
+            const int e = tid + t * pd::THREADS, i = e >> 7, j = e & 127;
+            vals[t] = (i < nbc && j <= i) ? A[static_cast<int64_t>(k0 + i) * d + k0 + j] : 0.0f;
         }
+#pragma unroll
+        for (int t = 0; t < 32; ++t) {
+            const int e = tid + t * pd::THREADS, i = e >> 7, j = e & 127;
+            S[i * pd::LD + j] = (i >= nbc && i == j) ? 1.0f : vals[t];
+        }
+    }
     __syncthreads();
 
     bool bad = false;
     for (int sp = 0; sp < 4; ++sp) {
         const int c0 = pd::SUB * sp;
-        float* X = Xs + sp * pd::SUB * (pd::SUB + 1);
+        float* X = XT + sp * pd::SUB * pd::LDX;      // X^T: X[j][k] stored at [k][j]
         if (warp == 0) {
             float v[32], x[32];
 #pragma unroll
@@ -265,41 +281,67 @@ __global__ void __launch_bounds__(pd::THREADS) potrf_diag_kernel(float* __restri
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
                 if (j <= lane) S[(c0 + lane) * pd::LD + c0 + j] = v[j];
-                X[lane * (pd::SUB + 1) + j] = (j <= lane) ? x[j] : 0.0f;
+                X[j * pd::LDX + lane] = x[j];        // row lane of X -> column lane of X^T
+                LT[j * pd::LDV + c0 + lane] = v[j];  // L[c0+lane][c0+j] -> LT[j][c0+lane]
             }
         }
         __syncthreads();
-        // sub-panel below: L[r][c0+j] = sum_{k<=j} A[r][c0+k] * X[j][k]  (at most 96 x 32
-        // outputs, so at most 6 per thread; computed before any is written back)
+        // sub-panel below: L[r][c0+j] = sum_{k<=j} A[r][c0+k] * X[j][k], computed for 4
+        // consecutive j per thread (rows r0..127: at most 96 x 8 strips, 2 per thread)
         const int r0 = c0 + pd::SUB, nr = pd::NB - r0;
-        float out[6];
+        float4 out[2];
 #pragma unroll
-        for (int t = 0; t < 6; ++t) {
+        for (int t = 0; t < 2; ++t) {
             const int idx = tid + t * pd::THREADS;
-            out[t] = 0.0f;
-            if (idx < nr * 32) {
-                const int r = r0 + (idx >> 5), j = idx & 31;
-                float acc = 0.0f;
-                for (int k = 0; k <= j; ++k)
-                    acc = fmaf(S[r * pd::LD + c0 + k], X[j * (pd::SUB + 1) + k], acc);
+            out[t] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (idx < nr * 8) {
+                const int r = r0 + (idx >> 3), j4 = (idx & 7) * 4;
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                for (int k = 0; k < j4 + 4; ++k) {
+                    const float a = S[r * pd::LD + c0 + k];
+                    const float4 xv = *reinterpret_cast<const float4*>(&X[k * pd::LDX + j4]);
+                    acc.x = fmaf(a, xv.x, acc.x);
+                    acc.y = fmaf(a, xv.y, acc.y);
+                    acc.z = fmaf(a, xv.z, acc.z);
+                    acc.w = fmaf(a, xv.w, acc.w);
+                }
                 out[t] = acc;
             }
         }
         __syncthreads();
 #pragma unroll
-        for (int t = 0; t < 6; ++t) {
+        for (int t = 0; t < 2; ++t) {
             const int idx = tid + t * pd::THREADS;
-            if (idx < nr * 32) S[(r0 + (idx >> 5)) * pd::LD + c0 + (idx & 31)] = out[t];
+            if (idx < nr * 8) {
+                const int r = r0 + (idx >> 3), j4 = (idx & 7) * 4;
+                float* dst = &S[r * pd::LD + c0 + j4];
+                dst[0] = out[t].x; dst[1] = out[t].y; dst[2] = out[t].z; dst[3] = out[t].w;
+                LT[(j4 + 0) * pd::LDV + r] = out[t].x;
+                LT[(j4 + 1) * pd::LDV + r] = out[t].y;
+                LT[(j4 + 2) * pd::LDV + r] = out[t].z;
+                LT[(j4 + 3) * pd::LDV + r] = out[t].w;
+            }
         }
         __syncthreads();
-        // trailing update: S[r][c] -= sum_k L[r][c0+k] L[c][c0+k] for r0 <= c <= r
+        // trailing update: S[r][c..c+3] -= sum_k L[r][c0+k] L[c..c+3][c0+k] for r0 <= c <= r
         for (int r = r0 + warp; r < pd::NB; r += NW) {
-            for (int c = r0 + lane; c <= r; c += 32) {
-                float acc = 0.0f;
+            for (int cq = r0 / 4 + lane; cq * 4 <= r; cq += 32) {
+                const int c = cq * 4;
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 8
-                for (int k = 0; k < pd::SUB; ++k)
-                    acc = fmaf(S[r * pd::LD + c0 + k], S[c * pd::LD + c0 + k], acc);
-                S[r * pd::LD + c] -= acc;
+                for (int k = 0; k < pd::SUB; ++k) {
+                    const float a = S[r * pd::LD + c0 + k];
+                    const float4 lv = *reinterpret_cast<const float4*>(&LT[k * pd::LDV + c]);
+                    acc.x = fmaf(a, lv.x, acc.x);
+                    acc.y = fmaf(a, lv.y, acc.y);
+                    acc.z = fmaf(a, lv.z, acc.z);
+                    acc.w = fmaf(a, lv.w, acc.w);
+                }
+                float* dst = &S[r * pd::LD + c];
+                dst[0] -= acc.x;
+                if (c + 1 <= r) dst[1] -= acc.y;
+                if (c + 2 <= r) dst[2] -= acc.z;
+                if (c + 3 <= r) dst[3] -= acc.w;
             }
         }
         __syncthreads();
@@ -308,65 +350,77 @@ __global__ void __launch_bounds__(pd::THREADS) potrf_diag_kernel(float* __restri
 
     // inverse of the whole factor: diagonal 32-blocks are the sub-block inverses;
     // Dv[I][J] = -X_I * sum_{K=J}^{I-1} L[I][K] Dv[K][J] for J < I
-    for (int i = warp; i < pd::NB; i += NW)
-        for (int j = lane; j < pd::NB; j += 32) {
-            const int I = i >> 5, J = j >> 5;
-            Dv[i * pd::LD + j] =
-                (I == J) ? Xs[I * pd::SUB * (pd::SUB + 1) + (i & 31) * (pd::SUB + 1) + (j & 31)]
-                         : 0.0f;
-        }
+    for (int e = tid; e < pd::NB * pd::NB; e += pd::THREADS) {
+        const int i = e >> 7, j = e & 127, I = i >> 5, J = j >> 5;
+        Dv[i * pd::LDV + j] =
+            (I == J) ? XT[I * pd::SUB * pd::LDX + (j & 31) * pd::LDX + (i & 31)] : 0.0f;
+    }
     __syncthreads();
     for (int I = 1; I < 4; ++I) {
-        // T = sum_K L[I][K] Dv[K][J] for all J < I: 32 rows x 32*I columns (<= 6 per thread)
-        float out[6];
-        const int ncol = 32 * I, total = 32 * ncol;
+        // T = sum_K L[I][K] Dv[K][J] for all J < I: 32 rows x 8*I four-column strips
+        const int nq = 8 * I, total = 32 * nq;
+        float4 out[2];
 #pragma unroll
-        for (int t = 0; t < 6; ++t) {
+        for (int t = 0; t < 2; ++t) {
             const int idx = tid + t * pd::THREADS;
-            out[t] = 0.0f;
+            out[t] = make_float4(0.f, 0.f, 0.f, 0.f);
             if (idx < total) {
-                const int a = idx / ncol, col = idx % ncol, J = col >> 5;
-                float acc = 0.0f;
-                for (int k = 32 * J; k < 32 * I; ++k)
-                    acc = fmaf(S[(32 * I + a) * pd::LD + k], Dv[k * pd::LD + col], acc);
+                const int a = idx / nq, col = (idx % nq) * 4, J = col >> 5;
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                for (int k = 32 * J; k < 32 * I; ++k) {
+                    const float l = S[(32 * I + a) * pd::LD + k];
+                    const float4 dv = *reinterpret_cast<const float4*>(&Dv[k * pd::LDV + col]);
+                    acc.x = fmaf(l, dv.x, acc.x);
+                    acc.y = fmaf(l, dv.y, acc.y);
+                    acc.z = fmaf(l, dv.z, acc.z);
+                    acc.w = fmaf(l, dv.w, acc.w);
+                }
                 out[t] = acc;
             }
         }
         __syncthreads();
 #pragma unroll
-        for (int t = 0; t < 6; ++t) {
+        for (int t = 0; t < 2; ++t) {
             const int idx = tid + t * pd::THREADS;
-            if (idx < total) Dv[(32 * I + idx / ncol) * pd::LD + idx % ncol] = out[t];
+            if (idx < total)
+                *reinterpret_cast<float4*>(&Dv[(32 * I + idx / nq) * pd::LDV + (idx % nq) * 4]) = out[t];
         }
         __syncthreads();
-        // Dv[I][J] = -X_I * T
-        const float* XI = Xs + I * pd::SUB * (pd::SUB + 1);
+        // Dv[I][J] = -X_I * T  (X_I lower: X_I[a][k] = XT_I[k][a])
+        const float* XI = XT + I * pd::SUB * pd::LDX;
 #pragma unroll
-        for (int t = 0; t < 6; ++t) {
+        for (int t = 0; t < 2; ++t) {
             const int idx = tid + t * pd::THREADS;
-            out[t] = 0.0f;
+            out[t] = make_float4(0.f, 0.f, 0.f, 0.f);
             if (idx < total) {
-                const int a = idx / ncol, col = idx % ncol;
-                float acc = 0.0f;
-                for (int k = 0; k <= a; ++k)
-                    acc = fmaf(XI[a * (pd::SUB + 1) + k], Dv[(32 * I + k) * pd::LD + col], acc);
-                out[t] = -acc;
+                const int a = idx / nq, col = (idx % nq) * 4;
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                for (int k = 0; k <= a; ++k) {
+                    const float xa = XI[k * pd::LDX + a];
+                    const float4 tv = *reinterpret_cast<const float4*>(&Dv[(32 * I + k) * pd::LDV + col]);
+                    acc.x = fmaf(xa, tv.x, acc.x);
+                    acc.y = fmaf(xa, tv.y, acc.y);
+                    acc.z = fmaf(xa, tv.z, acc.z);
+                    acc.w = fmaf(xa, tv.w, acc.w);
+                }
+                out[t] = make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
             }
         }
         __syncthreads();
 #pragma unroll
-        for (int t = 0; t < 6; ++t) {
+        for (int t = 0; t < 2; ++t) {
             const int idx = tid + t * pd::THREADS;
-            if (idx < total) Dv[(32 * I + idx / ncol) * pd::LD + idx % ncol] = out[t];
+            if (idx < total)
+                *reinterpret_cast<float4*>(&Dv[(32 * I + idx / nq) * pd::LDV + (idx % nq) * 4]) = out[t];
         }
         __syncthreads();
     }
-    for (int i = warp; i < pd::NB; i += NW)
-        for (int j = lane; j < pd::NB; j += 32) {
-            const bool in = i < nbc && j < nbc && j <= i;
-            Dinv[i * pd::NB + j] = in ? Dv[i * pd::LD + j] : 0.0f;
-            if (in) A[static_cast<int64_t>(k0 + i) * d + k0 + j] = S[i * pd::LD + j];
-        }
+    for (int e = tid; e < pd::NB * pd::NB; e += pd::THREADS) {
+        const int i = e >> 7, j = e & 127;
+        const bool in = i < nbc && j < nbc && j <= i;
+        Dinv[i * pd::NB + j] = in ? Dv[i * pd::LDV + j] : 0.0f;
+        if (in) A[static_cast<int64_t>(k0 + i) * d + k0 + j] = S[i * pd::LD + j];
+    }
 }
 
 __global__ void copy2d_kernel(const float* __restrict__ src, int lds, float* __restrict__ dst,
