@@ -156,12 +156,227 @@ __global__ void __launch_bounds__(gb::THREADS) gptq_block_kernel(
     if (lane == 0 && esq != 0.0) atomicAdd(err_sq, esq);
 }
 
+// ---------------------------------------------------------------------------------------
+// Row-resident column loop (group sizes that are a multiple of 4).
+//
+// One thread owns one row of the block and keeps its (up to 128) block weights in registers,
+// so quantizing a column is done once per row, with no cross-lane traffic; U sits in shared
+// memory and every lane reads the same U entries (broadcast loads). The column loop runs in
+// chunks of 4 columns: at the start of the chunk that begins at block column i0, register
+// w[c] holds block column i0 + c. Step k of the chunk quantizes w[k] and applies
+// w[c] -= err * U[i0+k][i0+c] to the columns c > k; the last step writes each result four
+// registers lower, so the window moves by 4 columns per chunk without copies and every
+// register index stays a compile-time constant. A chunk's entries of U start at column i0, a
+// multiple of 4, so they are read as aligned float4. The register window shrinks in phases
+// of 16 columns (W = 128, 112, ..., 16): a chunk in phase p only touches w[0..W).
+// Group starts fall on chunk starts (group_size % 4 == 0, blocks start on group starts).
+// ---------------------------------------------------------------------------------------
+namespace gr {
+constexpr int MAXB = 128;                    // widest block handled in one launch
+constexpr int LD = MAXB + 16;                // shared row stride of U (floats), zero padded
+constexpr int PH = 16;                       // block columns per window phase
+constexpr int NPH = MAXB / PH;
+constexpr int WARPS = 2;
+constexpr int THREADS = WARPS * 32;          // one row per thread
+constexpr int SMEM = MAXB * LD * 4 + WARPS * MAXB * 4 + NPH * 8;
+}  // namespace gr
+
+struct RowCtx {
+    const float* Us;      // [MAXB][LD]: Us[i][c] = U[j0+i][j0+c] for i, c < bw, else 0 (c >= bw)
+    const float* dinv;    // this warp's copy of 1 / U[j0+i][j0+i]
+    int bw, g, maxq, j0, d_in, n_groups_row, err_ld;
+    bool row_ok;
+    int64_t r;
+    uint8_t* codes_p;
+    uint16_t* scales;
+    uint16_t* zeros;
+    float* Err;
+    QParams P;
+    int next_gs;          // block column of the next group start
+    double esq;           // this row's sum of squared OBS errors
+};
+
+template <int W>
+__device__ __forceinline__ void rows_phase(float (&w)[gr::MAXB], int p0, RowCtx& x) {
+    const int i_end = min(p0 + gr::PH, x.bw);
+#pragma unroll 1
+    for (int i0 = p0; i0 < i_end; i0 += 4) {
+        if (i0 == x.next_gs) {
+            // group [i0, i0+g): min/max of its current weights, w[0..g)
+            x.next_gs += x.g;
+            float mn = w[0], mx = w[0];
+#pragma unroll
+            for (int c4 = 0; c4 < W; c4 += 4) {
+                if (c4 >= x.g) break;
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    mn = fminf(mn, w[c4 + t]);
+                    mx = fmaxf(mx, w[c4 + t]);
+                }
+            }
+            x.P = group_params(mn, mx, x.maxq);
+            if (x.row_ok) {
+                const int64_t gi = x.r * x.n_groups_row + (x.j0 + i0) / x.g;
+                x.scales[gi] = half_bits(x.P.scale);
+                x.zeros[gi] = half_bits(x.P.zero);
+            }
+        }
+        const float4 dv = *reinterpret_cast<const float4*>(x.dinv + i0);
+        const float dk[4] = {dv.x, dv.y, dv.z, dv.w};
+        float e[4];
+        uint32_t qword = 0u;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float wi = w[k];
+            const int qi = quant_code(wi, x.P, x.maxq);
+            const float err = (wi - dequant(qi, x.P)) * dk[k];
+            e[k] = err;
+            qword |= static_cast<uint32_t>(qi) << (8 * k);
+            const float* urow = x.Us + (i0 + k) * gr::LD + i0;
+            if (k < 3) {
+#pragma unroll
+                for (int c4 = 0; c4 < W; c4 += 4) {
+                    const float4 u = *reinterpret_cast<const float4*>(urow + c4);
+                    const float uu[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                    for (int t = 0; t < 4; ++t)
+                        if (c4 + t > k) w[c4 + t] = fmaf(-err, uu[t], w[c4 + t]);
+                }
+            } else {
+#pragma unroll
+                for (int c4 = 4; c4 < W; c4 += 4) {
+                    const float4 u = *reinterpret_cast<const float4*>(urow + c4);
+                    const float uu[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) w[c4 - 4 + t] = fmaf(-err, uu[t], w[c4 + t]);
+                }
+#pragma unroll
+                for (int t = 0; t < 4; ++t) w[W - 4 + t] = 0.0f;
+            }
+        }
+        if (x.row_ok) {
+            *reinterpret_cast<float4*>(x.Err + x.r * x.err_ld + i0) =
+                make_float4(e[0], e[1], e[2], e[3]);
+            *reinterpret_cast<uint32_t*>(x.codes_p + x.r * x.d_in + x.j0 + i0) = qword;
+        }
+        float part = e[0] * e[0];
+        part = fmaf(e[1], e[1], part);
+        part = fmaf(e[2], e[2], part);
+        part = fmaf(e[3], e[3], part);
+        x.esq += static_cast<double>(part);
+    }
+}
+
+// Waits for phase P's rows of U, derives their 1/U_ii, runs the phase, then the next one.
+// Returns false if a wait ran out of its cycle limit.
+template <int P>
+__device__ __forceinline__ bool rows_phases(float (&w)[gr::MAXB], RowCtx& x, uint64_t* bars,
+                                            float* dinv, int lane) {
+    if constexpr (P < gr::NPH) {
+        const int p0 = P * gr::PH;
+        if (p0 >= x.bw) return true;
+        const bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[P], 0));
+        if (!ok) return false;
+        if (lane < gr::PH) {
+            const int i = p0 + lane;
+            dinv[i] = i < x.bw ? 1.0f / x.Us[i * gr::LD + i] : 0.0f;
+        }
+        __syncwarp();
+        rows_phase<gr::MAXB - P * gr::PH>(w, p0, x);
+        return rows_phases<P + 1>(w, x, bars, dinv, lane);
+    }
+    return true;
+}
+
+__global__ void __launch_bounds__(gr::THREADS, 3) gptq_rows_kernel(
+    const float* __restrict__ Wk, int d_out, int d_in, int j0, int bw, const float* __restrict__ U,
+    int g, int bits, uint8_t* __restrict__ codes_p, uint16_t* __restrict__ scales,
+    uint16_t* __restrict__ zeros, float* __restrict__ Err, int err_ld, double* err_sq,
+    int* status) {
+    if (status_bad(status)) return;
+    extern __shared__ __align__(128) unsigned char rows_smem[];
+    float* Us = reinterpret_cast<float*>(rows_smem);
+    float* dinv_all = Us + gr::MAXB * gr::LD;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(dinv_all + gr::WARPS * gr::MAXB);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+    // zero the pad columns [bw, LD) of the rows in use; the bulk copies fill [0, bw)
+    const int pad = gr::LD - bw;
+    for (int e = tid; e < bw * pad; e += gr::THREADS) Us[(e / pad) * gr::LD + bw + e % pad] = 0.f;
+    if (tid == 0) {
+        for (int p = 0; p < gr::NPH; ++p) mbar_init(&bars[p], 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (warp == 0) {
+        // rows [16p, 16p+16) of U's diagonal block arrive on barrier p
+        if (lane < gr::NPH) {
+            const int rows = min(max(bw - lane * gr::PH, 0), gr::PH);
+            if (rows > 0) mbar_arrive_expect_tx(&bars[lane], static_cast<uint32_t>(rows * bw * 4));
+        }
+        __syncwarp();
+        for (int i = lane; i < bw; i += 32)
+            bulk_load_1d(Us + i * gr::LD, U + static_cast<int64_t>(j0 + i) * d_in + j0,
+                         static_cast<uint32_t>(bw * 4), &bars[i / gr::PH]);
+    }
+
+    RowCtx x;
+    x.Us = Us;
+    x.dinv = dinv_all + warp * gr::MAXB;
+    x.bw = bw; x.g = g; x.maxq = (1 << bits) - 1; x.j0 = j0; x.d_in = d_in;
+    x.n_groups_row = d_in / g; x.err_ld = err_ld;
+    x.r = static_cast<int64_t>(blockIdx.x) * gr::THREADS + tid;
+    x.row_ok = x.r < d_out;
+    x.codes_p = codes_p; x.scales = scales; x.zeros = zeros; x.Err = Err;
+    x.P.scale = 1.f; x.P.zero = 0.f; x.P.inv_scale = 1.f;
+    x.next_gs = 0;   // j0 is a multiple of g
+    x.esq = 0.0;
+
+    float w[gr::MAXB];
+    const float* wrow = Wk + x.r * d_in + j0;
+#pragma unroll
+    for (int c4 = 0; c4 < gr::MAXB; c4 += 4) {
+        float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (x.row_ok && c4 < bw) a = *reinterpret_cast<const float4*>(wrow + c4);
+        w[c4] = a.x; w[c4 + 1] = a.y; w[c4 + 2] = a.z; w[c4 + 3] = a.w;
+    }
+
+    if (!rows_phases<0>(w, x, bars, dinv_all + warp * gr::MAXB, lane)) {
+        set_status(status, GPTQ_ERR_TIMEOUT);
+        // let the copies still in flight land before the block exits (bounded again)
+        if (warp == 0 && lane < gr::NPH && lane * gr::PH < bw) mbar_wait(&bars[lane], 0);
+        __syncwarp();
+        return;
+    }
+    // the OBS increments e^2 add up to tr(D H_d D^T) for the whole layer
+    double esq = x.esq;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) esq += __shfl_xor_sync(0xffffffffu, esq, off);
+    if (lane == 0 && esq != 0.0) atomicAdd(err_sq, esq);
+}
+
+static bool g_rows_attr_set = false;
+
 static bool g_block_attr_set = false;
 
 gptq_status gptq_block_launch(float* Wk, int d_out, int d_in, int j0, int bw, const float* U,
                               int group_size, int bits, uint8_t* codes_p, uint16_t* scales,
                               uint16_t* zeros, float* Err, int err_ld, double* err_sq,
-                              const int* status, cudaStream_t s) {
+                              int* status, cudaStream_t s) {
+    if (group_size % 4 == 0) {
+        if (!g_rows_attr_set) {
+            GPTQ_CUDA_TRY(cudaFuncSetAttribute(gptq_rows_kernel,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               gr::SMEM));
+            g_rows_attr_set = true;
+        }
+        const int grid = (d_out + gr::THREADS - 1) / gr::THREADS;
+        gptq_rows_kernel<<<grid, gr::THREADS, gr::SMEM, s>>>(Wk, d_out, d_in, j0, bw, U,
+                                                            group_size, bits, codes_p, scales,
+                                                            zeros, Err, err_ld, err_sq, status);
+        GPTQ_LAUNCHED();
+        return GPTQ_OK;
+    }
     if (!g_block_attr_set) {
         GPTQ_CUDA_TRY(cudaFuncSetAttribute(gptq_block_kernel,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, gb::SMEM));

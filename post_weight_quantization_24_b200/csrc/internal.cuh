@@ -50,7 +50,7 @@ gptq_status trtri_reverse_launch(const float* A, int d, const float* Dinv, float
 gptq_status gptq_block_launch(float* Wk, int d_out, int d_in, int j0, int bw, const float* U,
                               int group_size, int bits, uint8_t* codes_p, uint16_t* scales,
                               uint16_t* zeros, float* Err, int err_ld, double* err_sq,
-                              const int* status, cudaStream_t s);
+                              int* status, cudaStream_t s);
 gptq_status lazy_update_launch(float* Wk, int d_out, int d_in, int j0, int bw, const float* U,
                                const float* Err, int err_ld, const int* status, cudaStream_t s);
 gptq_status assemble_launch(const uint8_t* codes_p, int d_out, int d_in, const int* perm,
