@@ -41,6 +41,7 @@ PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
                   "sm_max_mhz": 1965.0}
 N_SM, FP32_LANES_PER_SM = 148, 128
+TF32_PER_BF16 = round(1.1 / 2.25, 4)   # nominal dense tf32 : bf16 tensor rates on B200
 
 
 def load_peaks():
@@ -294,58 +295,64 @@ def run_ours(args):
     # ---- per-stage roofline ----
     clock_mhz = (clocks or {}).get("sm_mhz") or peaks.get("clocks_under_load", {}).get("sm_mhz_median", 1312.0)
     fp32_peak_tf = N_SM * FP32_LANES_PER_SM * 2 * clock_mhz * 1e6 / 1e12
-    fp32_peak_max_tf = N_SM * FP32_LANES_PER_SM * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
-    hess_flops = float(n) * d * (d + 1)                          # symmetric 2·XᵀX
+    tc_peak = peaks["bf16_tflops"]                       # fp16 MMA runs at the bf16 rate
+    tf32_peak = tc_peak * TF32_PER_BF16                  # nominal dense tf32 : bf16 ratio
+    hess_flops = float(n) * d * (d + 1)                  # symmetric 2·XᵀX
     hess_tf = hess_flops / (hess_ms / 1e3) / 1e12
-    tc_peak = peaks["bf16_tflops"]                               # fp16 MMA rate = bf16 rate
     chol_flops = d ** 3 / 3.0
     trtri_flops = d ** 3 / 3.0
-    col_flops = 2.0 * d_out * d * wl.block_size / 2.0
+    col_flops = float(d_out) * d * wl.block_size         # d_out·d·B/2 FMAs
     lazy_flops = 2.0 * d_out * sum(wl.block_size * max(0, d - j0 - wl.block_size)
                                    for j0 in range(0, d, wl.block_size))
-    loss_flops = 2.0 * d_out * d * d      # one trace GEMM (numerator from the e^2 sums)
+    w_f16 = wl.w_dtype == "f16"
+    loss_flops = float(d_out) * d * (d + 1) if w_f16 else 2.0 * d_out * d * d
     rtn_bytes = d_out * d * (2 + (0.5 if wl.bits == 4 else 1.0)) + d_out * (d // wl.group_size) * 4
 
-    def tf(fl, ms):
-        return fl / (ms / 1e3) / 1e12 if ms > 0 else None
+    def stage(ms, bound, flops=None, peak=None, note=None):
+        out = {"ms": ms, "bound": bound}
+        if flops is not None and ms > 0:
+            out["tflops"] = flops / (ms / 1e3) / 1e12
+            out["peak_tflops"] = peak
+            out["frac"] = out["tflops"] / peak
+        if note:
+            out["peak_note"] = note
+        return out
 
+    tf32x3 = f"tf32 = {TF32_PER_BF16} x measured bf16, / 3 MMA passes (3xTF32)"
     stages = {
-        "hessian": {"ms": hess_ms, "bound": "tensor", "tflops": hess_tf,
-                    "frac": hess_tf / tc_peak, "calib_tokens_per_s": n / (hess_ms / 1e3)},
+        "hessian": dict(stage(hess_ms, "tensor", hess_flops, tc_peak, "measured bf16 dense burst"),
+                        calib_tokens_per_s=n / (hess_ms / 1e3)),
         "prepare": {"ms": lib_ms["prepare"]},
-        "cholesky": {"ms": lib_ms["cholesky"], "bound": "alu",
-                     "tflops": tf(chol_flops, lib_ms["cholesky"])},
-        "trtri": {"ms": lib_ms["trtri"], "bound": "alu", "tflops": tf(trtri_flops, lib_ms["trtri"])},
-        "column_loop": {"ms": lib_ms["column_loop"], "bound": "alu",
-                        "tflops": tf(col_flops, lib_ms["column_loop"])},
-        "lazy_update": {"ms": lib_ms["lazy_update"], "bound": "alu",
-                        "tflops": tf(lazy_flops, lib_ms["lazy_update"])},
+        "cholesky": stage(lib_ms["cholesky"], "tensor", chol_flops, tf32_peak / 3, tf32x3),
+        "trtri": stage(lib_ms["trtri"], "tensor", trtri_flops, tf32_peak / 3, tf32x3),
+        "column_loop": stage(lib_ms["column_loop"], "alu", col_flops, fp32_peak_tf,
+                             f"FFMA 148 SM x 128 lanes x 2 at the sampled {clock_mhz:.0f} MHz"),
+        "lazy_update": stage(lib_ms["lazy_update"], "tensor", lazy_flops, tf32_peak / 3, tf32x3),
         "assemble": {"ms": lib_ms["assemble"]},
-        "loss": {"ms": lib_ms["loss"], "bound": "alu", "tflops": tf(loss_flops, lib_ms["loss"])},
+        "loss": stage(lib_ms["loss"], "tensor", loss_flops,
+                      tc_peak if w_f16 else tf32_peak / 3,
+                      "Gram matrix WᵀW on the fp16 path; measured bf16 dense burst" if w_f16
+                      else tf32x3),
         "rtn": {"ms": rtn_ms, "bound": "hbm", "gbs": rtn_bytes / (rtn_ms / 1e3) / 1e9,
                 "frac": rtn_bytes / (rtn_ms / 1e3) / 1e9 / peaks["hbm_gbs"]},
     }
-    for k in ("cholesky", "trtri", "column_loop", "lazy_update", "loss"):
-        if stages[k].get("tflops") is not None:
-            stages[k]["frac"] = stages[k]["tflops"] / fp32_peak_tf
 
-    # dominant kernel by time share
-    dom = max(("hessian", "lazy_update", "loss", "cholesky", "trtri", "column_loop"),
+    # the dominant kernel (largest stage) carries the roofline object
+    traffic, _ = ncu_traffic("hessian_tc_kernel_mlp_up_7b.md", "hessian.cu")
+    roof = {"kernel": "hessian_tc_kernel", "bound": "tensor", "achieved": hess_tf,
+            "peak": tc_peak, "unit": "TFLOP/s", "frac": hess_tf / tc_peak,
+            "traffic": traffic,
+            "peak_note": "measured bf16 dense burst (fp16 MMA runs at the bf16 rate); of measured"
+            if peaks["source"] == "measured" else "fallback"}
+    dom = max((k for k in stages if "frac" in stages[k] or k == "hessian"),
               key=lambda k: stages[k]["ms"])
-    if dom == "hessian":
-        traffic, _ = ncu_traffic("hessian_tc_kernel_mlp_up_7b.md", "hessian.cu")
-        roof = {"kernel": "hessian_tc_kernel", "bound": "tensor", "achieved": hess_tf,
-                "peak": tc_peak, "unit": "TFLOP/s", "frac": hess_tf / tc_peak,
-                "traffic": traffic,
-                "peak_note": "measured bf16 dense burst (fp16 MMA runs at the bf16 rate); of measured"
-                if peaks["source"] == "measured" else "fallback"}
-    else:
-        traffic, _ = ncu_traffic("sgemm_kernel_mlp_up_7b.md", "sgemm.cuh")
-        roof = {"kernel": dom, "bound": "alu", "achieved": stages[dom]["tflops"],
-                "peak": fp32_peak_tf, "unit": "TFLOP/s",
-                "frac": stages[dom]["tflops"] / fp32_peak_tf, "traffic": traffic,
-                "peak_note": f"FFMA peak 148 SM x 128 lanes x 2 flop at the sampled "
-                             f"{clock_mhz:.0f} MHz ({fp32_peak_max_tf:.1f} TF at max clock)"}
+    if dom != "hessian":
+        roof = {"kernel": dom, "bound": stages[dom]["bound"],
+                "achieved": stages[dom].get("tflops", stages[dom].get("gbs")),
+                "peak": stages[dom].get("peak_tflops", peaks["hbm_gbs"]),
+                "unit": "TFLOP/s" if "tflops" in stages[dom] else "GB/s",
+                "frac": stages[dom]["frac"], "traffic": None,
+                "peak_note": stages[dom].get("peak_note", "")}
 
     # ---- end to end through the public API with host buffers ----
     e2e = None
@@ -362,8 +369,9 @@ def run_ours(args):
                                f"B{wl.block_size} percdamp {wl.percdamp} act_order {wl.act_order}",
                    "per_rank": "one independent layer per GPU (seed = rank)",
                    "l2": "X (2.1 GB) larger than L2, plus a 512 MB L2 flush between steps",
-                   "arithmetic": "Hessian fp16 x fp16 -> fp32 on tcgen05; factorisation, column "
-                                 "loop, lazy update, loss in fp32 FFMA; group scalars fp64"},
+                   "arithmetic": "Hessian and loss Gram matrix fp16 x fp16 -> fp32 on tcgen05; "
+                                 "factorisation and lazy update fp32 as 3xTF32 on tcgen05; "
+                                 "column loop fp32 FFMA; group scalars fp64"},
         "calib_tokens_per_s": world * n / (hess_ms / 1e3),
         "layer_loss": step.loss,
         "stages": stages,

@@ -474,6 +474,41 @@ __global__ void __launch_bounds__(256) delta_sq_kernel(
 // tr(D H_d D^T) with H_d = H + lambda*I, so tr(D H D^T) = sum e^2 - lambda*||D||^2 (one pass
 // over the outputs). Denominator: tr(W H W^T) as a GEMM (W_p * H_p) whose epilogue dots with
 // W_p, in the processing order (a common permutation leaves the trace unchanged).
+// sum_{i,j} H[i][j] * G[i][j] / 2 from the upper triangles of two symmetric matrices
+// (G = 2 W^T W, as the Hessian kernel writes it), accumulated in fp64
+__global__ void __launch_bounds__(256) upper_dot_kernel(const float* __restrict__ H,
+                                                        const float* __restrict__ G, int d,
+                                                        double* out) {
+    double acc = 0.0;
+    for (int i = blockIdx.x; i < d; i += gridDim.x) {
+        const float* h = H + static_cast<int64_t>(i) * d;
+        const float* g = G + static_cast<int64_t>(i) * d;
+        for (int c = (i & ~3) + 4 * static_cast<int>(threadIdx.x); c < d; c += 4 * 256) {
+            const float4 a = *reinterpret_cast<const float4*>(h + c);
+            const float4 b = *reinterpret_cast<const float4*>(g + c);
+            const float pa[4] = {a.x * b.x, a.y * b.y, a.z * b.z, a.w * b.w};
+            float v = 0.0f;
+#pragma unroll
+            for (int t = 0; t < 4; ++t) v += (c + t > i) ? 2.0f * pa[t] : (c + t == i ? pa[t] : 0.0f);
+            acc += static_cast<double>(v);
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    __shared__ double red[8];
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        double t = 0.0;
+        for (int w = 0; w < 8; ++w) t += red[w];
+        atomicAdd(out, 0.5 * t);
+    }
+}
+
+// The denominator tr(W H W^T) equals <H, W^T W>. For fp16 W, G = 2 W^T W comes from the
+// Hessian kernel (W's rows play the tokens; exact fp16 products, fp32 accumulation) into the
+// d_in^2 scratch G, followed by one pass over the two upper triangles. fp32 W (not exact in
+// fp16) takes the tf32x3 GEMM route: tr(W H W^T) with W and H in the processing order.
 gptq_status loss_launch(const void* W, int w_dtype, int d_out, int d_in, const float* H,
                         const int* perm, const uint8_t* codes_p, const uint16_t* scales,
                         const uint16_t* zeros, int group_size, float* Wk, float* Hp,
@@ -489,15 +524,23 @@ gptq_status loss_launch(const void* W, int w_dtype, int d_out, int d_in, const f
                                                       perm, codes_p, scales, zeros, group_size,
                                                       &st->delta_sq);
     GPTQ_LAUNCHED();
+    if (w_dtype == GPTQ_DTYPE_F16) {
+        float* G = Hp;
+        GPTQ_CUDA_TRY(cudaMemsetAsync(G, 0, static_cast<size_t>(d_in) * d_in * sizeof(float), s));
+        GPTQ_TRY(hessian_launch(G, d_in, W, d_out, 0, &st->status, s));
+        const int gb = std::max(1, std::min(d_in, num_sms() * 8));
+        upper_dot_kernel<<<gb, 256, 0, s>>>(H, G, d_in, &st->loss_den);
+        GPTQ_LAUNCHED();
+        return GPTQ_OK;
+    }
     GPTQ_TRY(gather_h_launch(H, d_in, perm, st, 0, Hp, &st->status, s));
     GPTQ_TRY(gather_w_launch(W, w_dtype, d_out, d_in, perm, Wk, &st->status, s));
-    // Hp is symmetric, so it serves as the K-major [N x K] operand directly; fp16 weights are
-    // exact in tf32 and need no split
+    // Hp is symmetric, so it serves as the K-major [N x K] operand directly
     TcGemmArgs a{};
     a.M = d_out; a.N = d_in; a.K = d_in; a.alpha = 1.f; a.beta = 0.f;
     a.A = Wk; a.lda = d_in; a.B = Hp; a.ldb = d_in; a.D = Wk; a.ldd = d_in;
     a.dot = &st->loss_den; a.status = &st->status;
-    return tcgemm_launch(a, true, TC_EPI_DOT, w_dtype != GPTQ_DTYPE_F16, true, s);
+    return tcgemm_launch(a, true, TC_EPI_DOT, true, true, s);
 }
 
 }  // namespace gq
