@@ -181,246 +181,138 @@ gptq_status gather_w_launch(const void* W, int w_dtype, int d_out, int d_in, con
 // blocked Cholesky
 // ---------------------------------------------------------------------------------------
 // ---- diagonal block: one CTA factors the 128 x 128 block A[k0:, k0:] and inverts its factor.
-// The block is split into four 32-column sub-panels. For each one, a single warp factors the
-// 32 x 32 diagonal sub-block in registers (lane i holds row i; pivots and columns travel by
-// shuffles, so the 32 sequential pivot steps need no block barrier) and inverts it the same
-// way; then all warps solve the sub-panel below it against that inverse and apply the rank-32
-// update to the trailing part of the block. Finally the inverse of the whole 128 x 128 factor
-// is assembled from the four sub-block inverses by block forward substitution. Rows and
-// columns beyond the matrix edge (last block) are padded with the identity. The solve, update
-// and assembly loops work on 4-column strips so one shared-memory load feeds four FMAs; the
-// operands they stream across columns are kept transposed for that.
+// Pass 1 (factor) is right-looking elimination with one thread per row. At step c every
+// thread publishes its current column-c entry a_ic; by symmetry the pivot row's entries a_cm
+// are the published a_mc, so the column is all a step needs. Thread i then applies
+// a_im -= (a_ic / a_cc) a_mc to its row and records L[i][c] = a_ic / sqrt(a_cc).
+// Pass 2 (inverse) gives thread i column i of L^-1 by forward substitution against the
+// recorded columns of L: x_m -= L[m][c] * x_c / L[c][c], with x_c / L[c][c] = (L^-1)[c][i].
+// In both passes a thread's values sit in a register window that moves down one position
+// per step (position p holds matrix index c + p), so the running step is always position 0
+// and every register index is a compile-time constant; the window narrows in phases of 16
+// steps. One barrier per step in pass 1 (the published column is double-buffered); none in
+// pass 2. Rows and columns beyond the matrix edge are padded with the identity.
 namespace pd {
-constexpr int NB = 128, SUB = 32, THREADS = 512;
-constexpr int LD = NB + 1;        // S: scalar row access
-constexpr int LDV = NB + 4;       // Dv, LT: float4 row access
-constexpr int LDX = SUB + 4;      // XT: float4 row access
-constexpr int SMEM = (NB * LD + NB * LDV + SUB * LDV + 4 * SUB * LDX) * 4;
+constexpr int NB = 128, THREADS = NB, PH = 16;
+constexpr int LS = NB + 4;          // Lsh row stride: Lsh[c][m - c + 3] = L[m][c], m >= c
+constexpr int CB = NB + 8;          // published column: cb[i - c + 3] = a_ic of step c
+constexpr int SMEM = (NB * LS + 2 * CB + NB) * 4;   // + rs[c] = 1 / L[c][c]
 }  // namespace pd
 
-// v: row `lane` of a 32 x 32 SPD block (lower part used). On return v holds row `lane` of its
-// Cholesky factor L (zeros above the diagonal) and x holds row `lane` of L^-1.
-__device__ __forceinline__ void warp_chol_inv32(float (&v)[32], float (&x)[32], int lane,
-                                                bool& bad) {
-    const unsigned full = 0xffffffffu;
-    float rdiag = 1.0f;   // 1 / L[lane][lane]
+template <int W>
+__device__ __forceinline__ void potrf_factor_phase(float (&w)[pd::NB], int q, int i, float* Lsh,
+                                                   float* cb, float* rs, bool& bad) {
+#pragma unroll 1
+    for (int c = q * pd::PH; c < (q + 1) * pd::PH; ++c) {
+        float* buf = cb + (c & 1) * pd::CB;
+        if (i >= c) buf[i - c + 3] = w[0];
+        __syncthreads();
+        if ((i | 31) >= c) {                 // this warp still has a row at or below the pivot
+            const float p = buf[3];
+            const float rp = __frcp_rn(p);
+            const float sp = sqrtf(p);
+            const float rsp = __frcp_rn(sp);
+            const float w0 = w[0];
+            if (i == c) {
+                if (!(p > 0.0f) || !isfinite(p)) bad = true;
+                Lsh[c * pd::LS + 3] = sp;
+                rs[c] = rsp;
+            } else if (i > c) {
+                Lsh[c * pd::LS + i - c + 3] = w0 * rsp;
+            }
+            const float t = w0 * rp;
+            const float* col = buf + 4;      // col[k] = a_{c+1+k, c}
 #pragma unroll
-    for (int c = 0; c < 32; ++c) {
-        const float piv = __shfl_sync(full, v[c], c);
-        if (!(piv > 0.0f) || !isfinite(piv)) bad = true;
-        float r = rsqrtf(piv);
-        r = r * fmaf(-0.5f * piv, r * r, 1.5f);   // one Newton step: r = 1/sqrt(piv)
-        if (lane == c) rdiag = r;
-        const float lic = (lane >= c) ? v[c] * r : 0.0f;
-        v[c] = lic;
+            for (int k4 = 0; k4 < W; k4 += 4) {
+                const float4 v = *reinterpret_cast<const float4*>(col + k4);
+                const float vv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-        for (int j = c + 1; j < 32; ++j) {
-            const float ljc = __shfl_sync(full, lic, j);
-            v[j] = fmaf(-lic, ljc, v[j]);
+                for (int u = 0; u < 4; ++u)
+                    if (k4 + u + 1 < W) w[k4 + u] = fmaf(-t, vv[u], w[k4 + u + 1]);
+            }
+            w[W - 1] = 0.0f;
         }
     }
-#pragma unroll
-    for (int j = 0; j < 32; ++j) {
-        if (j > lane) v[j] = 0.0f;
-        x[j] = (j == lane) ? 1.0f : 0.0f;
-    }
-    // forward substitution on the identity with the row scaling deferred: when row k is
-    // broadcast it is scaled by 1/L[k][k] on the fly; each lane scales its own row at the end
-#pragma unroll
-    for (int k = 0; k < 32; ++k) {
-        const float rkk = __shfl_sync(full, rdiag, k);
-        const float nlik = (lane > k) ? -v[k] : 0.0f;
-#pragma unroll
-        for (int j = 0; j <= k; ++j) {
-            const float xkj = __shfl_sync(full, x[j], k) * rkk;
-            x[j] = fmaf(nlik, xkj, x[j]);
-        }
-    }
-#pragma unroll
-    for (int j = 0; j < 32; ++j) x[j] *= rdiag;
 }
 
-__global__ void __launch_bounds__(pd::THREADS) potrf_diag_kernel(float* __restrict__ A, int d,
-                                                                int k0, int nbc,
-                                                                float* __restrict__ Dinv,
-                                                                int* status) {
+template <int W>
+__device__ __forceinline__ void potrf_inverse_phase(float (&w)[pd::NB], int q, int i, int nbc,
+                                                    const float* Lsh, const float* rs,
+                                                    float* __restrict__ Dinv) {
+#pragma unroll 1
+    for (int c = q * pd::PH; c < (q + 1) * pd::PH; ++c) {
+        const float t2 = w[0] * rs[c];       // (L^-1)[c][i]
+        Dinv[c * pd::NB + i] = (c < nbc && i < nbc) ? t2 : 0.0f;
+        const float* col = Lsh + c * pd::LS + 4;   // col[k] = L[c+1+k][c]
+#pragma unroll
+        for (int k4 = 0; k4 < W; k4 += 4) {
+            const float4 v = *reinterpret_cast<const float4*>(col + k4);
+            const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (k4 + u + 1 < W) w[k4 + u] = fmaf(-t2, vv[u], w[k4 + u + 1]);
+        }
+        w[W - 1] = 0.0f;
+    }
+}
+
+__global__ void __launch_bounds__(pd::THREADS, 1) potrf_diag_kernel(float* __restrict__ A, int d,
+                                                                   int k0, int nbc,
+                                                                   float* __restrict__ Dinv,
+                                                                   int* status) {
     if (status_bad(status)) return;
     extern __shared__ __align__(16) float sm[];
-    float* S = sm;                          // [NB][LD]: the block, then its factor L
-    float* Dv = S + pd::NB * pd::LD;        // [NB][LDV]: L^-1
-    float* LT = Dv + pd::NB * pd::LDV;      // [SUB][LDV]: current sub-panel of L, transposed
-    float* XT = LT + pd::SUB * pd::LDV;     // [4][SUB][LDX]: sub-block inverses, transposed
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    constexpr int NW = pd::THREADS / 32;
+    float* Lsh = sm;                          // [NB][LS]
+    float* cb = Lsh + pd::NB * pd::LS;        // [2][CB]
+    float* rs = cb + 2 * pd::CB;              // [NB]
+    const int i = threadIdx.x, warp = i >> 5;
 
-    // load: 32 independent loads per thread, then the stores (identity padding past the edge)
-    {
-        float vals[32];
+    for (int e = i; e < (pd::NB * pd::LS + 2 * pd::CB) / 4; e += pd::THREADS)
+        reinterpret_cast<float4*>(sm)[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+
+    // row i of the block's lower triangle (zeros above the diagonal; identity past the edge)
+    float w[pd::NB];
+    const float* arow = A + static_cast<int64_t>(k0 + i) * d + k0;
 #pragma unroll
-        for (int t = 0; t < 32; ++t) {
-            const int e = tid + t * pd::THREADS, i = e >> 7, j = e & 127;
-            vals[t] = (i < nbc && j <= i) ? A[static_cast<int64_t>(k0 + i) * d + k0 + j] : 0.0f;
-        }
+    for (int p4 = 0; p4 < pd::NB; p4 += 4) {
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (i < nbc && p4 <= i && p4 < nbc) v = *reinterpret_cast<const float4*>(arow + p4);
+        const float vv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-        for (int t = 0; t < 32; ++t) {
-            const int e = tid + t * pd::THREADS, i = e >> 7, j = e & 127;
-            S[i * pd::LD + j] = (i >= nbc && i == j) ? 1.0f : vals[t];
-        }
+        for (int u = 0; u < 4; ++u)
+            w[p4 + u] = (i < nbc) ? (p4 + u <= i ? vv[u] : 0.0f) : (p4 + u == i ? 1.0f : 0.0f);
     }
     __syncthreads();
 
     bool bad = false;
-    for (int sp = 0; sp < 4; ++sp) {
-        const int c0 = pd::SUB * sp;
-        float* X = XT + sp * pd::SUB * pd::LDX;      // X^T: X[j][k] stored at [k][j]
-        if (warp == 0) {
-            float v[32], x[32];
-#pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = (j <= lane) ? S[(c0 + lane) * pd::LD + c0 + j] : 0.0f;
-            warp_chol_inv32(v, x, lane, bad);
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                if (j <= lane) S[(c0 + lane) * pd::LD + c0 + j] = v[j];
-                X[j * pd::LDX + lane] = x[j];        // row lane of X -> column lane of X^T
-                LT[j * pd::LDV + c0 + lane] = v[j];  // L[c0+lane][c0+j] -> LT[j][c0+lane]
-            }
-        }
-        __syncthreads();
-        // sub-panel below: L[r][c0+j] = sum_{k<=j} A[r][c0+k] * X[j][k], computed for 4
-        // consecutive j per thread (rows r0..127: at most 96 x 8 strips, 2 per thread)
-        const int r0 = c0 + pd::SUB, nr = pd::NB - r0;
-        float4 out[2];
-#pragma unroll
-        for (int t = 0; t < 2; ++t) {
-            const int idx = tid + t * pd::THREADS;
-            out[t] = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (idx < nr * 8) {
-                const int r = r0 + (idx >> 3), j4 = (idx & 7) * 4;
-                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-                for (int k = 0; k < j4 + 4; ++k) {
-                    const float a = S[r * pd::LD + c0 + k];
-                    const float4 xv = *reinterpret_cast<const float4*>(&X[k * pd::LDX + j4]);
-                    acc.x = fmaf(a, xv.x, acc.x);
-                    acc.y = fmaf(a, xv.y, acc.y);
-                    acc.z = fmaf(a, xv.z, acc.z);
-                    acc.w = fmaf(a, xv.w, acc.w);
-                }
-                out[t] = acc;
-            }
-        }
-        __syncthreads();
-#pragma unroll
-        for (int t = 0; t < 2; ++t) {
-            const int idx = tid + t * pd::THREADS;
-            if (idx < nr * 8) {
-                const int r = r0 + (idx >> 3), j4 = (idx & 7) * 4;
-                float* dst = &S[r * pd::LD + c0 + j4];
-                dst[0] = out[t].x; dst[1] = out[t].y; dst[2] = out[t].z; dst[3] = out[t].w;
-                LT[(j4 + 0) * pd::LDV + r] = out[t].x;
-                LT[(j4 + 1) * pd::LDV + r] = out[t].y;
-                LT[(j4 + 2) * pd::LDV + r] = out[t].z;
-                LT[(j4 + 3) * pd::LDV + r] = out[t].w;
-            }
-        }
-        __syncthreads();
-        // trailing update: S[r][c..c+3] -= sum_k L[r][c0+k] L[c..c+3][c0+k] for r0 <= c <= r
-        for (int r = r0 + warp; r < pd::NB; r += NW) {
-            for (int cq = r0 / 4 + lane; cq * 4 <= r; cq += 32) {
-                const int c = cq * 4;
-                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 8
-                for (int k = 0; k < pd::SUB; ++k) {
-                    const float a = S[r * pd::LD + c0 + k];
-                    const float4 lv = *reinterpret_cast<const float4*>(&LT[k * pd::LDV + c]);
-                    acc.x = fmaf(a, lv.x, acc.x);
-                    acc.y = fmaf(a, lv.y, acc.y);
-                    acc.z = fmaf(a, lv.z, acc.z);
-                    acc.w = fmaf(a, lv.w, acc.w);
-                }
-                float* dst = &S[r * pd::LD + c];
-                dst[0] -= acc.x;
-                if (c + 1 <= r) dst[1] -= acc.y;
-                if (c + 2 <= r) dst[2] -= acc.z;
-                if (c + 3 <= r) dst[3] -= acc.w;
-            }
-        }
-        __syncthreads();
-    }
-    if (warp == 0 && lane == 0 && bad) set_status(status, GPTQ_ERR_NOT_PD);
+    potrf_factor_phase<128>(w, 0, i, Lsh, cb, rs, bad);
+    potrf_factor_phase<112>(w, 1, i, Lsh, cb, rs, bad);
+    potrf_factor_phase<96>(w, 2, i, Lsh, cb, rs, bad);
+    potrf_factor_phase<80>(w, 3, i, Lsh, cb, rs, bad);
+    potrf_factor_phase<64>(w, 4, i, Lsh, cb, rs, bad);
+    potrf_factor_phase<48>(w, 5, i, Lsh, cb, rs, bad);
+    potrf_factor_phase<32>(w, 6, i, Lsh, cb, rs, bad);
+    potrf_factor_phase<16>(w, 7, i, Lsh, cb, rs, bad);
+    if (__syncthreads_or(bad) && i == 0) set_status(status, GPTQ_ERR_NOT_PD);
 
-    // inverse of the whole factor: diagonal 32-blocks are the sub-block inverses;
-    // Dv[I][J] = -X_I * sum_{K=J}^{I-1} L[I][K] Dv[K][J] for J < I
-    for (int e = tid; e < pd::NB * pd::NB; e += pd::THREADS) {
-        const int i = e >> 7, j = e & 127, I = i >> 5, J = j >> 5;
-        Dv[i * pd::LDV + j] =
-            (I == J) ? XT[I * pd::SUB * pd::LDX + (j & 31) * pd::LDX + (i & 31)] : 0.0f;
-    }
-    __syncthreads();
-    for (int I = 1; I < 4; ++I) {
-        // T = sum_K L[I][K] Dv[K][J] for all J < I: 32 rows x 8*I four-column strips
-        const int nq = 8 * I, total = 32 * nq;
-        float4 out[2];
+    // L back into A: thread i writes column i (row segments stay coalesced across threads)
+    for (int m = i; m < nbc; ++m)
+        if (i < nbc) A[static_cast<int64_t>(k0 + m) * d + k0 + i] = Lsh[i * pd::LS + m - i + 3];
+
+    // pass 2: column i of L^-1. Warp w's columns are zero above row 32w, so it starts at step
+    // 32w with x_i = 1 at window position i - 32w, and writes zeros for the earlier steps.
+    for (int c = 0; c < 32 * warp; ++c) Dinv[c * pd::NB + i] = 0.0f;
 #pragma unroll
-        for (int t = 0; t < 2; ++t) {
-            const int idx = tid + t * pd::THREADS;
-            out[t] = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (idx < total) {
-                const int a = idx / nq, col = (idx % nq) * 4, J = col >> 5;
-                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-                for (int k = 32 * J; k < 32 * I; ++k) {
-                    const float l = S[(32 * I + a) * pd::LD + k];
-                    const float4 dv = *reinterpret_cast<const float4*>(&Dv[k * pd::LDV + col]);
-                    acc.x = fmaf(l, dv.x, acc.x);
-                    acc.y = fmaf(l, dv.y, acc.y);
-                    acc.z = fmaf(l, dv.z, acc.z);
-                    acc.w = fmaf(l, dv.w, acc.w);
-                }
-                out[t] = acc;
-            }
-        }
-        __syncthreads();
-#pragma unroll
-        for (int t = 0; t < 2; ++t) {
-            const int idx = tid + t * pd::THREADS;
-            if (idx < total)
-                *reinterpret_cast<float4*>(&Dv[(32 * I + idx / nq) * pd::LDV + (idx % nq) * 4]) = out[t];
-        }
-        __syncthreads();
-        // Dv[I][J] = -X_I * T  (X_I lower: X_I[a][k] = XT_I[k][a])
-        const float* XI = XT + I * pd::SUB * pd::LDX;
-#pragma unroll
-        for (int t = 0; t < 2; ++t) {
-            const int idx = tid + t * pd::THREADS;
-            out[t] = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (idx < total) {
-                const int a = idx / nq, col = (idx % nq) * 4;
-                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-                for (int k = 0; k <= a; ++k) {
-                    const float xa = XI[k * pd::LDX + a];
-                    const float4 tv = *reinterpret_cast<const float4*>(&Dv[(32 * I + k) * pd::LDV + col]);
-                    acc.x = fmaf(xa, tv.x, acc.x);
-                    acc.y = fmaf(xa, tv.y, acc.y);
-                    acc.z = fmaf(xa, tv.z, acc.z);
-                    acc.w = fmaf(xa, tv.w, acc.w);
-                }
-                out[t] = make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
-            }
-        }
-        __syncthreads();
-#pragma unroll
-        for (int t = 0; t < 2; ++t) {
-            const int idx = tid + t * pd::THREADS;
-            if (idx < total)
-                *reinterpret_cast<float4*>(&Dv[(32 * I + idx / nq) * pd::LDV + (idx % nq) * 4]) = out[t];
-        }
-        __syncthreads();
-    }
-    for (int e = tid; e < pd::NB * pd::NB; e += pd::THREADS) {
-        const int i = e >> 7, j = e & 127;
-        const bool in = i < nbc && j < nbc && j <= i;
-        Dinv[i * pd::NB + j] = in ? Dv[i * pd::LDV + j] : 0.0f;
-        if (in) A[static_cast<int64_t>(k0 + i) * d + k0 + j] = S[i * pd::LD + j];
-    }
+    for (int p = 0; p < pd::NB; ++p) w[p] = (p == i - 32 * warp) ? 1.0f : 0.0f;
+    const int q0 = 2 * warp;
+    if (q0 <= 0) potrf_inverse_phase<128>(w, 0, i, nbc, Lsh, rs, Dinv);
+    if (q0 <= 1) potrf_inverse_phase<112>(w, 1, i, nbc, Lsh, rs, Dinv);
+    if (q0 <= 2) potrf_inverse_phase<96>(w, 2, i, nbc, Lsh, rs, Dinv);
+    if (q0 <= 3) potrf_inverse_phase<80>(w, 3, i, nbc, Lsh, rs, Dinv);
+    if (q0 <= 4) potrf_inverse_phase<64>(w, 4, i, nbc, Lsh, rs, Dinv);
+    if (q0 <= 5) potrf_inverse_phase<48>(w, 5, i, nbc, Lsh, rs, Dinv);
+    if (q0 <= 6) potrf_inverse_phase<32>(w, 6, i, nbc, Lsh, rs, Dinv);
+    potrf_inverse_phase<16>(w, 7, i, nbc, Lsh, rs, Dinv);
 }
 
 __global__ void copy2d_kernel(const float* __restrict__ src, int lds, float* __restrict__ dst,
