@@ -120,6 +120,8 @@ gptq_status act_order_launch(const float* H, int d, int act_order, int* perm, in
 __global__ void gather_h_kernel(const float* __restrict__ H, int d, const int* __restrict__ perm,
                                 const DevState* __restrict__ st, int reversed,
                                 float* __restrict__ A, int* status) {
+    // the Cholesky reads only the lower triangle of the reversed matrix: skip tiles above it
+    if (reversed && blockIdx.y < blockIdx.x) return;
     const int j = blockIdx.x * 32 + threadIdx.x;
     if (j >= d) return;
     const int b = reversed ? perm[d - 1 - j] : perm[j];
@@ -128,6 +130,7 @@ __global__ void gather_h_kernel(const float* __restrict__ H, int d, const int* _
     for (int k = threadIdx.y; k < 32; k += blockDim.y) {
         const int i = blockIdx.y * 32 + k;
         if (i >= d) break;
+        if (reversed && i < j) continue;
         const int a = reversed ? perm[d - 1 - i] : perm[i];
         const int lo = min(a, b), hi = max(a, b);
         float v = H[static_cast<int64_t>(lo) * d + hi];
@@ -150,23 +153,22 @@ template <typename T>
 __global__ void gather_w_kernel(const T* __restrict__ W, int d_out, int d_in,
                                 const int* __restrict__ perm, float* __restrict__ Wk,
                                 int* status) {
-    const int64_t n = static_cast<int64_t>(d_out) * d_in;
     int bad = 0;
-    for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < n;
-         e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        const int64_t r = e / d_in;
-        const int p = static_cast<int>(e - r * d_in);
-        const float v = static_cast<float>(W[r * d_in + perm[p]]);
-        if (!isfinite(v)) bad = 1;
-        Wk[e] = v;
+    for (int r = blockIdx.x; r < d_out; r += gridDim.x) {
+        const T* wr = W + static_cast<int64_t>(r) * d_in;
+        float* out = Wk + static_cast<int64_t>(r) * d_in;
+        for (int p = threadIdx.x; p < d_in; p += blockDim.x) {
+            const float v = static_cast<float>(wr[perm[p]]);
+            if (!isfinite(v)) bad = 1;
+            out[p] = v;
+        }
     }
     if (bad) set_status(status, GPTQ_ERR_NONFINITE);
 }
 
 gptq_status gather_w_launch(const void* W, int w_dtype, int d_out, int d_in, const int* perm,
                             float* Wk, int* status, cudaStream_t s) {
-    const int64_t n = static_cast<int64_t>(d_out) * d_in;
-    const int blocks = static_cast<int>(std::min<int64_t>((n + 255) / 256, num_sms() * 32));
+    const int blocks = std::min(d_out, num_sms() * 16);
     if (w_dtype == GPTQ_DTYPE_F16)
         gather_w_kernel<__half><<<blocks, 256, 0, s>>>(static_cast<const __half*>(W), d_out, d_in,
                                                        perm, Wk, status);

@@ -14,176 +14,54 @@
 
 #include "internal.cuh"
 #include "quant.cuh"
-#include "sgemm.cuh"
 #include "tcgemm.cuh"
 
 namespace gq {
 
-namespace gb {
-constexpr int MAXB = 128;            // widest block handled in one launch
-constexpr int LANES_PER_ROW = 16;    // 8 columns per lane, two rows per warp
-constexpr int WARPS = 8;
-constexpr int THREADS = WARPS * 32;
-constexpr int SMEM = (MAXB * MAXB + MAXB) * 4;
-}  // namespace gb
-
-// In-block column loop. The block's U[j0:j0+bw, j0:j0+bw] (zero below the diagonal) and the
-// reciprocals of its diagonal sit in shared memory. Each half-warp owns one row and holds its
-// bw (<= 128) block weights in registers, 8 per lane. Column i is owned by lane i/8: it is
-// broadcast with a shuffle, every lane of the row computes the same code and error, and each
-// lane applies the rank-1 update to its 8 columns with one row of U (entries left of column
-// i are zero, so no masking is needed). Group scale/zero come from a half-warp min/max
-// reduction over the group's current weights at the group's first column.
-__global__ void __launch_bounds__(gb::THREADS) gptq_block_kernel(
-    float* __restrict__ Wk, int d_out, int d_in, int j0, int bw, const float* __restrict__ U,
-    int g, int bits, uint8_t* __restrict__ codes_p, uint16_t* __restrict__ scales,
-    uint16_t* __restrict__ zeros, float* __restrict__ Err, int err_ld, double* err_sq,
-    const int* status) {
-    if (status_bad(status)) return;
-    extern __shared__ float smem[];
-    float* Us = smem;                      // [MAXB][MAXB]
-    float* dinv = smem + gb::MAXB * gb::MAXB;
-    const int maxq = (1 << bits) - 1;
-    const int n_groups_row = d_in / g;
-
-    for (int e = threadIdx.x; e < gb::MAXB * gb::MAXB / 4; e += blockDim.x) {
-        const int i = e / (gb::MAXB / 4), c4 = (e % (gb::MAXB / 4)) * 4;
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (i < bw && c4 < bw) {
-            v = *reinterpret_cast<const float4*>(U + static_cast<int64_t>(j0 + i) * d_in + j0 + c4);
-            if (c4 + 0 < i) v.x = 0.f;
-            if (c4 + 1 < i) v.y = 0.f;
-            if (c4 + 2 < i) v.z = 0.f;
-            if (c4 + 3 < i) v.w = 0.f;
-        }
-        *reinterpret_cast<float4*>(Us + i * gb::MAXB + c4) = v;
-    }
-    for (int i = threadIdx.x; i < gb::MAXB; i += blockDim.x)
-        dinv[i] = i < bw ? 1.0f / U[static_cast<int64_t>(j0 + i) * d_in + j0 + i] : 0.0f;
-    __syncthreads();
-
-    const int lane = lane_id(), half = lane >> 4, hl = lane & 15;
-    const int c0 = hl * 8;                           // this lane's first block column
-    const unsigned full = 0xffffffffu;
-    const int warps_total = gridDim.x * gb::WARPS;
-    const int n_pairs = (d_out + 1) / 2;
-    double esq = 0.0;   // this lane's sum of squared errors (its own columns)
-    for (int pair = blockIdx.x * gb::WARPS + warp_id(); pair < n_pairs; pair += warps_total) {
-        const int r = pair * 2 + half;
-        const bool row_ok = r < d_out;
-        float w[8];
-        float* wrow = Wk + static_cast<int64_t>(r) * d_in + j0;
-        if (row_ok && c0 < bw) {
-            const float4 a = *reinterpret_cast<const float4*>(wrow + c0);
-            const float4 b = *reinterpret_cast<const float4*>(wrow + c0 + 4);
-            w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
-            w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
-        } else {
-#pragma unroll
-            for (int k = 0; k < 8; ++k) w[k] = 0.f;
-        }
-        float e[8];
-        uint32_t qlo = 0, qhi = 0;
-        QParams P;
-        P.scale = 1.f; P.zero = 0.f; P.inv_scale = 1.f;
-#pragma unroll 1
-        for (int i0 = 0; i0 < bw; i0 += 8) {
-            const int owner = (half << 4) | (i0 >> 3);
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const int i = i0 + c;
-                if (i >= bw) break;
-                if ((j0 + i) % g == 0) {
-                    // group [i, i+g) of the block: min/max of its current weights in this row
-                    float mn = INFINITY, mx = -INFINITY;
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        const int col = c0 + k;
-                        if (col >= i && col < i + g && col < bw) {
-                            mn = fminf(mn, w[k]);
-                            mx = fmaxf(mx, w[k]);
-                        }
-                    }
-#pragma unroll
-                    for (int off = 8; off > 0; off >>= 1) {
-                        mn = fminf(mn, __shfl_xor_sync(full, mn, off));
-                        mx = fmaxf(mx, __shfl_xor_sync(full, mx, off));
-                    }
-                    P = group_params(mn, mx, maxq);
-                    if (hl == 0 && row_ok) {
-                        const int64_t gi = static_cast<int64_t>(r) * n_groups_row + (j0 + i) / g;
-                        scales[gi] = half_bits(P.scale);
-                        zeros[gi] = half_bits(P.zero);
-                    }
-                }
-                const float wi = __shfl_sync(full, w[c], owner);
-                const int qi = quant_code(wi, P, maxq);
-                const float err = (wi - dequant(qi, P)) * dinv[i];
-                if (hl == (i0 >> 3)) {
-                    e[c] = err;
-                    if (c < 4) qlo |= static_cast<uint32_t>(qi) << (8 * c);
-                    else qhi |= static_cast<uint32_t>(qi) << (8 * (c - 4));
-                }
-                const float4 u0 = *reinterpret_cast<const float4*>(Us + i * gb::MAXB + c0);
-                const float4 u1 = *reinterpret_cast<const float4*>(Us + i * gb::MAXB + c0 + 4);
-                w[0] = fmaf(-err, u0.x, w[0]);
-                w[1] = fmaf(-err, u0.y, w[1]);
-                w[2] = fmaf(-err, u0.z, w[2]);
-                w[3] = fmaf(-err, u0.w, w[3]);
-                w[4] = fmaf(-err, u1.x, w[4]);
-                w[5] = fmaf(-err, u1.y, w[5]);
-                w[6] = fmaf(-err, u1.z, w[6]);
-                w[7] = fmaf(-err, u1.w, w[7]);
-            }
-        }
-        if (row_ok && c0 < bw) {
-            uint2 qv;
-            qv.x = qlo;
-            qv.y = qhi;
-            *reinterpret_cast<uint2*>(codes_p + static_cast<int64_t>(r) * d_in + j0 + c0) = qv;
-            float* er = Err + static_cast<int64_t>(r) * err_ld + c0;
-            *reinterpret_cast<float4*>(er) = make_float4(e[0], e[1], e[2], e[3]);
-            *reinterpret_cast<float4*>(er + 4) = make_float4(e[4], e[5], e[6], e[7]);
-            float part = 0.0f;
-#pragma unroll
-            for (int k = 0; k < 8; ++k) part = fmaf(e[k], e[k], part);
-            esq += static_cast<double>(part);
-        }
-    }
-    // the OBS increments e^2 add up to tr(D H_d D^T) for the whole layer
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) esq += __shfl_xor_sync(full, esq, off);
-    if (lane == 0 && esq != 0.0) atomicAdd(err_sq, esq);
-}
-
 // ---------------------------------------------------------------------------------------
-// Row-resident column loop (group sizes that are a multiple of 4).
+// Column loop, one row per thread.
 //
 // One thread owns one row of the block and keeps its (up to 128) block weights in registers,
-// so quantizing a column is done once per row, with no cross-lane traffic; U sits in shared
-// memory and every lane reads the same U entries (broadcast loads). The column loop runs in
-// chunks of 4 columns: at the start of the chunk that begins at block column i0, register
-// w[c] holds block column i0 + c. Step k of the chunk quantizes w[k] and applies
-// w[c] -= err * U[i0+k][i0+c] to the columns c > k; the last step writes each result four
-// registers lower, so the window moves by 4 columns per chunk without copies and every
-// register index stays a compile-time constant. A chunk's entries of U start at column i0, a
-// multiple of 4, so they are read as aligned float4. The register window shrinks in phases
-// of 16 columns (W = 128, 112, ..., 16): a chunk in phase p only touches w[0..W).
-// Group starts fall on chunk starts (group_size % 4 == 0, blocks start on group starts).
+// so each column is quantized once per row, with no cross-lane traffic. Register w[k] holds
+// block column i + k while column i is processed: the step quantizes w[0] and applies
+// w[c] -= err * U[i][i+c] to the later columns, writing each result one register lower, so
+// the window moves by one column per step without copies and every register index stays a
+// compile-time constant. The loop body is a single step (a few KB of code, so it stays in
+// the instruction cache); the window narrows in phases of 16 columns (W = 128, 112, ..., 16).
+// The step reads row i of U starting at column i+1, so the block's U comes as an image whose
+// row i is U[i][i+1 ...] (16-byte aligned, zero past the block), brought into shared memory
+// by bulk copies, 16 rows per mbarrier, together with the reciprocals of U's diagonal.
+// Errors and codes are kept for four columns and stored together.
 // ---------------------------------------------------------------------------------------
 namespace gr {
 constexpr int MAXB = 128;                    // widest block handled in one launch
-constexpr int LD = MAXB + 16;                // shared row stride of U (floats), zero padded
 constexpr int PH = 16;                       // block columns per window phase
 constexpr int NPH = MAXB / PH;
 constexpr int WARPS = 2;
 constexpr int THREADS = WARPS * 32;          // one row per thread
-constexpr int SMEM = MAXB * LD * 4 + WARPS * MAXB * 4 + NPH * 8;
+constexpr int SMEM = MAXB * MAXB * 4 + MAXB * 4 + NPH * 8;
 }  // namespace gr
 
+// img[R][k] = U[R][R+1+k] while R+1+k stays inside R's block (else 0); rdiag[R] = 1/U[R][R]
+__global__ void column_images_kernel(const float* __restrict__ U, int d, int bs,
+                                     float* __restrict__ img, float* __restrict__ rdiag) {
+    const int R = blockIdx.x, k = threadIdx.x;
+    const int j0 = (R / bs) * bs, bw = min(bs, d - j0), i = R - j0;
+    const float* urow = U + static_cast<int64_t>(R) * d;
+    img[static_cast<int64_t>(R) * gr::MAXB + k] = (i + 1 + k < bw) ? urow[R + 1 + k] : 0.0f;
+    if (k == 0) rdiag[R] = 1.0f / urow[R];
+}
+
+gptq_status column_images_launch(const float* U, int d, int block_size, float* img, float* rdiag,
+                                 cudaStream_t s) {
+    column_images_kernel<<<d, gr::MAXB, 0, s>>>(U, d, block_size, img, rdiag);
+    GPTQ_LAUNCHED();
+    return GPTQ_OK;
+}
+
 struct RowCtx {
-    const float* Us;      // [MAXB][LD]: Us[i][c] = U[j0+i][j0+c] for i, c < bw, else 0 (c >= bw)
-    const float* dinv;    // this warp's copy of 1 / U[j0+i][j0+i]
+    const float* Us;      // [MAXB][MAXB]: Us[i][k] = U[j0+i][j0+i+1+k] inside the block, else 0
+    const float* rd;      // [MAXB]: 1 / U[j0+i][j0+i]
     int bw, g, maxq, j0, d_in, n_groups_row, err_ld;
     bool row_ok;
     int64_t r;
@@ -193,6 +71,8 @@ struct RowCtx {
     float* Err;
     QParams P;
     int next_gs;          // block column of the next group start
+    float e0, e1, e2, e3; // errors of the last four columns (e0 newest)
+    uint32_t qword;       // their codes, oldest in the low byte
     double esq;           // this row's sum of squared OBS errors
 };
 
@@ -200,9 +80,9 @@ template <int W>
 __device__ __forceinline__ void rows_phase(float (&w)[gr::MAXB], int p0, RowCtx& x) {
     const int i_end = min(p0 + gr::PH, x.bw);
 #pragma unroll 1
-    for (int i0 = p0; i0 < i_end; i0 += 4) {
-        if (i0 == x.next_gs) {
-            // group [i0, i0+g): min/max of its current weights, w[0..g)
+    for (int i = p0; i < i_end; ++i) {
+        if (i == x.next_gs) {
+            // group [i, i+g): min/max of its current weights, w[0..g)
             x.next_gs += x.g;
             float mn = w[0], mx = w[0];
 #pragma unroll
@@ -210,119 +90,96 @@ __device__ __forceinline__ void rows_phase(float (&w)[gr::MAXB], int p0, RowCtx&
                 if (c4 >= x.g) break;
 #pragma unroll
                 for (int t = 0; t < 4; ++t) {
-                    mn = fminf(mn, w[c4 + t]);
-                    mx = fmaxf(mx, w[c4 + t]);
+                    if (c4 + t < x.g) {
+                        mn = fminf(mn, w[c4 + t]);
+                        mx = fmaxf(mx, w[c4 + t]);
+                    }
                 }
             }
             x.P = group_params(mn, mx, x.maxq);
             if (x.row_ok) {
-                const int64_t gi = x.r * x.n_groups_row + (x.j0 + i0) / x.g;
+                const int64_t gi = x.r * x.n_groups_row + (x.j0 + i) / x.g;
                 x.scales[gi] = half_bits(x.P.scale);
                 x.zeros[gi] = half_bits(x.P.zero);
             }
         }
-        const float4 dv = *reinterpret_cast<const float4*>(x.dinv + i0);
-        const float dk[4] = {dv.x, dv.y, dv.z, dv.w};
-        float e[4];
-        uint32_t qword = 0u;
+        const float wi = w[0];
+        const int qi = quant_code(wi, x.P, x.maxq);
+        const float err = (wi - dequant(qi, x.P)) * x.rd[i];
+        x.e3 = x.e2; x.e2 = x.e1; x.e1 = x.e0; x.e0 = err;
+        x.qword = (x.qword >> 8) | (static_cast<uint32_t>(qi) << 24);
+        const float* urow = x.Us + i * gr::MAXB;   // urow[k] = U[i][i+1+k]
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const float wi = w[k];
-            const int qi = quant_code(wi, x.P, x.maxq);
-            const float err = (wi - dequant(qi, x.P)) * dk[k];
-            e[k] = err;
-            qword |= static_cast<uint32_t>(qi) << (8 * k);
-            const float* urow = x.Us + (i0 + k) * gr::LD + i0;
-            if (k < 3) {
+        for (int k4 = 0; k4 < W; k4 += 4) {
+            const float4 u = *reinterpret_cast<const float4*>(urow + k4);
+            const float uu[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-                for (int c4 = 0; c4 < W; c4 += 4) {
-                    const float4 u = *reinterpret_cast<const float4*>(urow + c4);
-                    const float uu[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-                    for (int t = 0; t < 4; ++t)
-                        if (c4 + t > k) w[c4 + t] = fmaf(-err, uu[t], w[c4 + t]);
-                }
-            } else {
-#pragma unroll
-                for (int c4 = 4; c4 < W; c4 += 4) {
-                    const float4 u = *reinterpret_cast<const float4*>(urow + c4);
-                    const float uu[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-                    for (int t = 0; t < 4; ++t) w[c4 - 4 + t] = fmaf(-err, uu[t], w[c4 + t]);
-                }
-#pragma unroll
-                for (int t = 0; t < 4; ++t) w[W - 4 + t] = 0.0f;
+            for (int t = 0; t < 4; ++t)
+                if (k4 + t + 1 < W) w[k4 + t] = fmaf(-err, uu[t], w[k4 + t + 1]);
+        }
+        w[W - 1] = 0.0f;
+        if ((i & 3) == 3) {
+            if (x.row_ok) {
+                *reinterpret_cast<float4*>(x.Err + x.r * x.err_ld + i - 3) =
+                    make_float4(x.e3, x.e2, x.e1, x.e0);
+                *reinterpret_cast<uint32_t*>(x.codes_p + x.r * x.d_in + x.j0 + i - 3) = x.qword;
             }
+            float part = x.e0 * x.e0;
+            part = fmaf(x.e1, x.e1, part);
+            part = fmaf(x.e2, x.e2, part);
+            part = fmaf(x.e3, x.e3, part);
+            x.esq += static_cast<double>(part);
         }
-        if (x.row_ok) {
-            *reinterpret_cast<float4*>(x.Err + x.r * x.err_ld + i0) =
-                make_float4(e[0], e[1], e[2], e[3]);
-            *reinterpret_cast<uint32_t*>(x.codes_p + x.r * x.d_in + x.j0 + i0) = qword;
-        }
-        float part = e[0] * e[0];
-        part = fmaf(e[1], e[1], part);
-        part = fmaf(e[2], e[2], part);
-        part = fmaf(e[3], e[3], part);
-        x.esq += static_cast<double>(part);
     }
 }
 
-// Waits for phase P's rows of U, derives their 1/U_ii, runs the phase, then the next one.
-// Returns false if a wait ran out of its cycle limit.
+// Waits for phase P's rows of the image, runs the phase, then the next one. Returns false if
+// a wait ran out of its cycle limit.
 template <int P>
-__device__ __forceinline__ bool rows_phases(float (&w)[gr::MAXB], RowCtx& x, uint64_t* bars,
-                                            float* dinv, int lane) {
+__device__ __forceinline__ bool rows_phases(float (&w)[gr::MAXB], RowCtx& x, uint64_t* bars) {
     if constexpr (P < gr::NPH) {
         const int p0 = P * gr::PH;
         if (p0 >= x.bw) return true;
         const bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[P], 0));
         if (!ok) return false;
-        if (lane < gr::PH) {
-            const int i = p0 + lane;
-            dinv[i] = i < x.bw ? 1.0f / x.Us[i * gr::LD + i] : 0.0f;
-        }
-        __syncwarp();
         rows_phase<gr::MAXB - P * gr::PH>(w, p0, x);
-        return rows_phases<P + 1>(w, x, bars, dinv, lane);
+        return rows_phases<P + 1>(w, x, bars);
     }
     return true;
 }
 
 __global__ void __launch_bounds__(gr::THREADS, 3) gptq_rows_kernel(
-    const float* __restrict__ Wk, int d_out, int d_in, int j0, int bw, const float* __restrict__ U,
-    int g, int bits, uint8_t* __restrict__ codes_p, uint16_t* __restrict__ scales,
-    uint16_t* __restrict__ zeros, float* __restrict__ Err, int err_ld, double* err_sq,
-    int* status) {
+    const float* __restrict__ Wk, int d_out, int d_in, int j0, int bw,
+    const float* __restrict__ img, const float* __restrict__ rdiag, int g, int bits,
+    uint8_t* __restrict__ codes_p, uint16_t* __restrict__ scales, uint16_t* __restrict__ zeros,
+    float* __restrict__ Err, int err_ld, double* err_sq, int* status) {
     if (status_bad(status)) return;
     extern __shared__ __align__(128) unsigned char rows_smem[];
     float* Us = reinterpret_cast<float*>(rows_smem);
-    float* dinv_all = Us + gr::MAXB * gr::LD;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(dinv_all + gr::WARPS * gr::MAXB);
+    float* rd = Us + gr::MAXB * gr::MAXB;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(rd + gr::MAXB);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
-    // zero the pad columns [bw, LD) of the rows in use; the bulk copies fill [0, bw)
-    const int pad = gr::LD - bw;
-    for (int e = tid; e < bw * pad; e += gr::THREADS) Us[(e / pad) * gr::LD + bw + e % pad] = 0.f;
     if (tid == 0) {
         for (int p = 0; p < gr::NPH; ++p) mbar_init(&bars[p], 1);
         fence_mbar_init();
     }
     __syncthreads();
-    if (warp == 0) {
-        // rows [16p, 16p+16) of U's diagonal block arrive on barrier p
-        if (lane < gr::NPH) {
-            const int rows = min(max(bw - lane * gr::PH, 0), gr::PH);
-            if (rows > 0) mbar_arrive_expect_tx(&bars[lane], static_cast<uint32_t>(rows * bw * 4));
+    if (warp == 0 && lane < gr::NPH) {
+        // image rows [16p, 16p+16) of the block arrive on barrier p (+ the diagonal on 0)
+        const int p = lane, rows = min(max(bw - p * gr::PH, 0), gr::PH);
+        if (rows > 0) {
+            const uint32_t bytes = static_cast<uint32_t>(rows * gr::MAXB * 4);
+            mbar_arrive_expect_tx(&bars[p], bytes + (p == 0 ? static_cast<uint32_t>(bw * 4) : 0u));
+            bulk_load_1d(Us + p * gr::PH * gr::MAXB,
+                         img + static_cast<int64_t>(j0 + p * gr::PH) * gr::MAXB, bytes, &bars[p]);
+            if (p == 0) bulk_load_1d(rd, rdiag + j0, static_cast<uint32_t>(bw * 4), &bars[0]);
         }
-        __syncwarp();
-        for (int i = lane; i < bw; i += 32)
-            bulk_load_1d(Us + i * gr::LD, U + static_cast<int64_t>(j0 + i) * d_in + j0,
-                         static_cast<uint32_t>(bw * 4), &bars[i / gr::PH]);
     }
 
     RowCtx x;
     x.Us = Us;
-    x.dinv = dinv_all + warp * gr::MAXB;
+    x.rd = rd;
     x.bw = bw; x.g = g; x.maxq = (1 << bits) - 1; x.j0 = j0; x.d_in = d_in;
     x.n_groups_row = d_in / g; x.err_ld = err_ld;
     x.r = static_cast<int64_t>(blockIdx.x) * gr::THREADS + tid;
@@ -330,6 +187,8 @@ __global__ void __launch_bounds__(gr::THREADS, 3) gptq_rows_kernel(
     x.codes_p = codes_p; x.scales = scales; x.zeros = zeros; x.Err = Err;
     x.P.scale = 1.f; x.P.zero = 0.f; x.P.inv_scale = 1.f;
     x.next_gs = 0;   // j0 is a multiple of g
+    x.e0 = x.e1 = x.e2 = x.e3 = 0.f;
+    x.qword = 0u;
     x.esq = 0.0;
 
     float w[gr::MAXB];
@@ -341,7 +200,7 @@ __global__ void __launch_bounds__(gr::THREADS, 3) gptq_rows_kernel(
         w[c4] = a.x; w[c4 + 1] = a.y; w[c4 + 2] = a.z; w[c4 + 3] = a.w;
     }
 
-    if (!rows_phases<0>(w, x, bars, dinv_all + warp * gr::MAXB, lane)) {
+    if (!rows_phases<0>(w, x, bars)) {
         set_status(status, GPTQ_ERR_TIMEOUT);
         // let the copies still in flight land before the block exits (bounded again)
         if (warp == 0 && lane < gr::NPH && lane * gr::PH < bw) mbar_wait(&bars[lane], 0);
@@ -357,51 +216,34 @@ __global__ void __launch_bounds__(gr::THREADS, 3) gptq_rows_kernel(
 
 static bool g_rows_attr_set = false;
 
-static bool g_block_attr_set = false;
-
-gptq_status gptq_block_launch(float* Wk, int d_out, int d_in, int j0, int bw, const float* U,
-                              int group_size, int bits, uint8_t* codes_p, uint16_t* scales,
-                              uint16_t* zeros, float* Err, int err_ld, double* err_sq,
-                              int* status, cudaStream_t s) {
-    if (group_size % 4 == 0) {
-        if (!g_rows_attr_set) {
-            GPTQ_CUDA_TRY(cudaFuncSetAttribute(gptq_rows_kernel,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               gr::SMEM));
-            g_rows_attr_set = true;
-        }
-        const int grid = (d_out + gr::THREADS - 1) / gr::THREADS;
-        gptq_rows_kernel<<<grid, gr::THREADS, gr::SMEM, s>>>(Wk, d_out, d_in, j0, bw, U,
-                                                            group_size, bits, codes_p, scales,
-                                                            zeros, Err, err_ld, err_sq, status);
-        GPTQ_LAUNCHED();
-        return GPTQ_OK;
+gptq_status gptq_block_launch(float* Wk, int d_out, int d_in, int j0, int bw, const float* img,
+                              const float* rdiag, int group_size, int bits, uint8_t* codes_p,
+                              uint16_t* scales, uint16_t* zeros, float* Err, int err_ld,
+                              double* err_sq, int* status, cudaStream_t s) {
+    if (!g_rows_attr_set) {
+        GPTQ_CUDA_TRY(cudaFuncSetAttribute(gptq_rows_kernel,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           gr::SMEM));
+        g_rows_attr_set = true;
     }
-    if (!g_block_attr_set) {
-        GPTQ_CUDA_TRY(cudaFuncSetAttribute(gptq_block_kernel,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize, gb::SMEM));
-        g_block_attr_set = true;
-    }
-    const int n_pairs = (d_out + 1) / 2;
-    const int need = (n_pairs + gb::WARPS - 1) / gb::WARPS;
-    const int grid = std::max(1, std::min(need, num_sms() * 3));
-    gptq_block_kernel<<<grid, gb::THREADS, gb::SMEM, s>>>(Wk, d_out, d_in, j0, bw, U, group_size,
-                                                          bits, codes_p, scales, zeros, Err,
-                                                          err_ld, err_sq, status);
+    const int grid = (d_out + gr::THREADS - 1) / gr::THREADS;
+    gptq_rows_kernel<<<grid, gr::THREADS, gr::SMEM, s>>>(Wk, d_out, d_in, j0, bw, img, rdiag,
+                                                        group_size, bits, codes_p, scales, zeros,
+                                                        Err, err_ld, err_sq, status);
     GPTQ_LAUNCHED();
     return GPTQ_OK;
 }
 
-// W[:, j1:] -= Err_block * U[j0:j1, j1:]  (3xTF32 on the tensor cores)
-gptq_status lazy_update_launch(float* Wk, int d_out, int d_in, int j0, int bw, const float* U,
-                               const float* Err, int err_ld, const int* status, cudaStream_t s) {
-    const int j1 = j0 + bw;
-    if (j1 >= d_in) return GPTQ_OK;
+// W[:, c0:c1] -= Err[:, 0:k1-k0] * U[k0:k1, c0:c1]  (3xTF32 on the tensor cores)
+gptq_status lazy_update_launch(float* Wk, int d_out, int d_in, int k0, int k1, int c0, int c1,
+                               const float* U, const float* Err, int err_ld, const int* status,
+                               cudaStream_t s) {
+    if (c1 <= c0 || k1 <= k0) return GPTQ_OK;
     TcGemmArgs a{};
-    a.M = d_out; a.N = d_in - j1; a.K = bw; a.alpha = -1.f; a.beta = 1.f;
+    a.M = d_out; a.N = c1 - c0; a.K = k1 - k0; a.alpha = -1.f; a.beta = 1.f;
     a.A = Err; a.lda = err_ld;
-    a.B = U + static_cast<int64_t>(j0) * d_in + j1; a.ldb = d_in;
-    a.C = Wk + j1; a.ldc = d_in; a.status = status;
+    a.B = U + static_cast<int64_t>(k0) * d_in + c0; a.ldb = d_in;
+    a.C = Wk + c0; a.ldc = d_in; a.status = status;
     return tcgemm_launch(a, false, TC_EPI_STORE, true, true, s);
 }
 
@@ -410,27 +252,24 @@ __global__ void assemble_kernel(const uint8_t* __restrict__ codes_p, int d_out, 
                                 const int* __restrict__ perm, const int* __restrict__ invperm,
                                 int g, int act_order, uint8_t* __restrict__ codes,
                                 int32_t* __restrict__ g_idx, int32_t* __restrict__ perm_out) {
-    const int64_t n = static_cast<int64_t>(d_out) * d_in;
-    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-    const int64_t t0 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-    for (int64_t c = t0; c < d_in; c += stride) {
+    const int t0 = blockIdx.x * blockDim.x + threadIdx.x, stride = gridDim.x * blockDim.x;
+    for (int c = t0; c < d_in; c += stride) {
         g_idx[c] = invperm[c] / g;
         if (perm_out) perm_out[c] = perm[c];
     }
     if (!act_order) return;
-    for (int64_t e = t0; e < n; e += stride) {
-        const int64_t r = e / d_in;
-        const int c = static_cast<int>(e - r * d_in);
-        codes[e] = codes_p[r * d_in + invperm[c]];
+    for (int r = blockIdx.x; r < d_out; r += gridDim.x) {
+        const uint8_t* src = codes_p + static_cast<int64_t>(r) * d_in;
+        uint8_t* dst = codes + static_cast<int64_t>(r) * d_in;
+        for (int c = threadIdx.x; c < d_in; c += blockDim.x) dst[c] = src[invperm[c]];
     }
 }
 
 gptq_status assemble_launch(const uint8_t* codes_p, int d_out, int d_in, const int* perm,
                             const int* invperm, int group_size, int act_order, uint8_t* codes,
                             int32_t* g_idx, int32_t* perm_out, cudaStream_t s) {
-    const int64_t n = act_order ? static_cast<int64_t>(d_out) * d_in : d_in;
-    const int blocks = static_cast<int>(std::min<int64_t>((n + 255) / 256, num_sms() * 16));
-    assemble_kernel<<<std::max(blocks, 1), 256, 0, s>>>(codes_p, d_out, d_in, perm, invperm,
+    const int blocks = std::max(1, std::min(std::max(d_out, (d_in + 255) / 256), num_sms() * 16));
+    assemble_kernel<<<blocks, 256, 0, s>>>(codes_p, d_out, d_in, perm, invperm,
                                                        group_size, act_order, codes, g_idx,
                                                        perm_out);
     GPTQ_LAUNCHED();
@@ -443,19 +282,25 @@ __global__ void __launch_bounds__(256) delta_sq_kernel(
     const T* __restrict__ W, int d_out, int d_in, const int* __restrict__ perm,
     const uint8_t* __restrict__ codes_p, const uint16_t* __restrict__ scales,
     const uint16_t* __restrict__ zeros, int g, double* out) {
-    const int64_t n = static_cast<int64_t>(d_out) * d_in;
     const int ng = d_in / g;
+    const float inv_g = 1.0f / static_cast<float>(g);
     double acc = 0.0;
-    for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < n;
-         e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        const int64_t r = e / d_in;
-        const int p = static_cast<int>(e - r * d_in);
-        const int64_t gi = r * ng + p / g;
-        const float s = __half2float(__ushort_as_half(scales[gi]));
-        const float z = __half2float(__ushort_as_half(zeros[gi]));
-        const float wh = s * (static_cast<float>(codes_p[e]) - z);
-        const float dlt = static_cast<float>(W[r * d_in + perm[p]]) - wh;
-        acc += static_cast<double>(dlt) * dlt;
+    for (int r = blockIdx.x; r < d_out; r += gridDim.x) {
+        const int64_t row = static_cast<int64_t>(r) * d_in;
+        float part = 0.0f;
+        for (int p = threadIdx.x; p < d_in; p += blockDim.x) {
+            // p / g from a float quotient, corrected by one either way (p < 2^17)
+            int q = __float2int_rz(static_cast<float>(p) * inv_g);
+            if (q * g > p) --q;
+            else if ((q + 1) * g <= p) ++q;
+            const int64_t gi = static_cast<int64_t>(r) * ng + q;
+            const float s = __half2float(__ushort_as_half(scales[gi]));
+            const float z = __half2float(__ushort_as_half(zeros[gi]));
+            const float wh = s * (static_cast<float>(codes_p[row + p]) - z);
+            const float dlt = static_cast<float>(W[row + perm[p]]) - wh;
+            part = fmaf(dlt, dlt, part);
+        }
+        acc += static_cast<double>(part);
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
@@ -513,8 +358,7 @@ gptq_status loss_launch(const void* W, int w_dtype, int d_out, int d_in, const f
                         const int* perm, const uint8_t* codes_p, const uint16_t* scales,
                         const uint16_t* zeros, int group_size, float* Wk, float* Hp,
                         DevState* st, cudaStream_t s) {
-    const int64_t n = static_cast<int64_t>(d_out) * d_in;
-    const int blocks = static_cast<int>(std::min<int64_t>((n + 255) / 256, num_sms() * 8));
+    const int blocks = std::min(d_out, num_sms() * 8);
     if (w_dtype == GPTQ_DTYPE_F16)
         delta_sq_kernel<__half><<<blocks, 256, 0, s>>>(static_cast<const __half*>(W), d_out,
                                                        d_in, perm, codes_p, scales, zeros,

@@ -17,6 +17,7 @@ struct DevState {
 };
 
 constexpr int kCholBlock = 128;   // panel width of the blocked Cholesky / triangular inverse
+constexpr int kSuperCols = 512;   // columns whose errors are collected before the far update
 
 // rtn.cu
 gptq_status rtn_launch(const void* W, int w_dtype, int d_out, int d_in, int bits,
@@ -47,12 +48,19 @@ gptq_status trtri_reverse_launch(const float* A, int d, const float* Dinv, float
                                  int* status, cudaStream_t s);
 
 // gptq.cu
-gptq_status gptq_block_launch(float* Wk, int d_out, int d_in, int j0, int bw, const float* U,
-                              int group_size, int bits, uint8_t* codes_p, uint16_t* scales,
-                              uint16_t* zeros, float* Err, int err_ld, double* err_sq,
-                              int* status, cudaStream_t s);
-gptq_status lazy_update_launch(float* Wk, int d_out, int d_in, int j0, int bw, const float* U,
-                               const float* Err, int err_ld, const int* status, cudaStream_t s);
+// Per-row images of U's diagonal blocks for the column loop: img [d x 128],
+// img[R][k] = U[R][R+1+k] inside R's block of block_size columns (else 0); rdiag[R] = 1/U[R][R].
+gptq_status column_images_launch(const float* U, int d, int block_size, float* img, float* rdiag,
+                                 cudaStream_t s);
+// The column loop of the block [j0, j0+bw), with img/rdiag as column_images_launch writes them
+gptq_status gptq_block_launch(float* Wk, int d_out, int d_in, int j0, int bw, const float* img,
+                              const float* rdiag, int group_size, int bits, uint8_t* codes_p,
+                              uint16_t* scales, uint16_t* zeros, float* Err, int err_ld,
+                              double* err_sq, int* status, cudaStream_t s);
+// W[:, c0:c1] -= Err[:, 0:k1-k0] * U[k0:k1, c0:c1]
+gptq_status lazy_update_launch(float* Wk, int d_out, int d_in, int k0, int k1, int c0, int c1,
+                               const float* U, const float* Err, int err_ld, const int* status,
+                               cudaStream_t s);
 gptq_status assemble_launch(const uint8_t* codes_p, int d_out, int d_in, const int* perm,
                             const int* invperm, int group_size, int act_order, uint8_t* codes,
                             int32_t* g_idx, int32_t* perm_out, cudaStream_t s);
