@@ -6,6 +6,7 @@
 #include <vector>
 
 #include "internal.cuh"
+#include "tcgemm.cuh"
 
 namespace gq {
 
@@ -133,7 +134,8 @@ struct Workspace {
     float* A;        // d^2: damped, permuted, reversed H -> Cholesky factor; later undamped Hp
     float* X;        // d^2: L^-1, then U
     float* Wk;       // d_out x d_in working weights (processing order)
-    float* Err;      // d_out x kSuperCols errors of the current super-block
+    float* Err;      // d_out x kSuperCols errors of the current super-block (tf32 hi part)
+    float* ErrLo;    // d_out x kSuperCols (tf32 lo part)
     uint8_t* codes_p;// d_out x d_in codes in processing order
     float* P;        // d x 128 panel scratch
     float* Dinv;     // ceil(d/128) x 128 x 128 inverses of the Cholesky diagonal blocks
@@ -157,6 +159,7 @@ static Workspace layout(void* base, int d_out, int d_in) {
     w.X = reinterpret_cast<float*>(take(d * d * 4));
     w.Wk = reinterpret_cast<float*>(take(static_cast<size_t>(d_out) * d * 4));
     w.Err = reinterpret_cast<float*>(take(static_cast<size_t>(d_out) * kSuperCols * 4));
+    w.ErrLo = reinterpret_cast<float*>(take(static_cast<size_t>(d_out) * kSuperCols * 4));
     w.codes_p = take(static_cast<size_t>(d_out) * d);
     w.P = reinterpret_cast<float*>(take(d * kCholBlock * 4));
     w.Dinv = reinterpret_cast<float*>(take(nbl * kCholBlock * kCholBlock * 4));
@@ -332,6 +335,10 @@ gptq_status gptq_quantize_layer(const void* W, int w_dtype, int d_out, int d_in,
     tm.begin(3);
     GPTQ_TRY(column_images_launch(ws.X, d_in, block_size, ws.P, ws.Dinv, s));
     tm.end();
+    // U as tf32 hi (in place) and lo (into the factor's buffer, free now) for the lazy updates
+    tm.begin(4);
+    GPTQ_TRY(tcgemm_split_launch(ws.X, ws.X, ws.A, d_in, d_in, d_in, true, s));
+    tm.end();
     // Lazy batch updates on two levels: the errors of a super-block of whole blocks (about
     // kSuperCols columns) are kept; after each block only the rest of its super-block is
     // updated, and the columns beyond the super-block get one update per super-block. Every
@@ -341,20 +348,21 @@ gptq_status gptq_quantize_layer(const void* W, int w_dtype, int d_out, int d_in,
         const int s1 = std::min(s0 + super, d_in);
         for (int j0 = s0; j0 < s1; j0 += block_size) {
             const int bw = std::min(block_size, s1 - j0), j1 = j0 + bw;
-            float* err_blk = ws.Err + (j0 - s0);
+            float* err_hi = ws.Err + (j0 - s0);
+            float* err_lo = ws.ErrLo + (j0 - s0);
             tm.begin(3);
             GPTQ_TRY(gptq_block_launch(ws.Wk, d_out, d_in, j0, bw, ws.P, ws.Dinv, group_size,
-                                       bits, codes_p, scales, zeros, err_blk, kSuperCols,
+                                       bits, codes_p, scales, zeros, err_hi, err_lo, kSuperCols,
                                        &ws.st->err_sq, status, s));
             tm.end();
             tm.begin(4);
-            GPTQ_TRY(lazy_update_launch(ws.Wk, d_out, d_in, j0, j1, j1, s1, ws.X, err_blk,
-                                        kSuperCols, status, s));
+            GPTQ_TRY(lazy_update_launch(ws.Wk, d_out, d_in, j0, j1, j1, s1, ws.X, ws.A, err_hi,
+                                        err_lo, kSuperCols, status, s));
             tm.end();
         }
         tm.begin(4);
-        GPTQ_TRY(lazy_update_launch(ws.Wk, d_out, d_in, s0, s1, s1, d_in, ws.X, ws.Err,
-                                    kSuperCols, status, s));
+        GPTQ_TRY(lazy_update_launch(ws.Wk, d_out, d_in, s0, s1, s1, d_in, ws.X, ws.A, ws.Err,
+                                    ws.ErrLo, kSuperCols, status, s));
         tm.end();
     }
     // ---- stage 5: outputs in the original column order ----

@@ -68,7 +68,8 @@ struct RowCtx {
     uint8_t* codes_p;
     uint16_t* scales;
     uint16_t* zeros;
-    float* Err;
+    float* Err;           // tf32 hi and lo parts of the errors (the lazy update's operand)
+    float* ErrLo;
     QParams P;
     int next_gs;          // block column of the next group start
     float e0, e1, e2, e3; // errors of the last four columns (e0 newest)
@@ -120,8 +121,17 @@ __device__ __forceinline__ void rows_phase(float (&w)[gr::MAXB], int p0, RowCtx&
         w[W - 1] = 0.0f;
         if ((i & 3) == 3) {
             if (x.row_ok) {
+                const float ev[4] = {x.e3, x.e2, x.e1, x.e0};
+                float hv[4], lv[4];
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    hv[t] = tf32_rna(ev[t]);
+                    lv[t] = tf32_rna(ev[t] - hv[t]);
+                }
                 *reinterpret_cast<float4*>(x.Err + x.r * x.err_ld + i - 3) =
-                    make_float4(x.e3, x.e2, x.e1, x.e0);
+                    make_float4(hv[0], hv[1], hv[2], hv[3]);
+                *reinterpret_cast<float4*>(x.ErrLo + x.r * x.err_ld + i - 3) =
+                    make_float4(lv[0], lv[1], lv[2], lv[3]);
                 *reinterpret_cast<uint32_t*>(x.codes_p + x.r * x.d_in + x.j0 + i - 3) = x.qword;
             }
             float part = x.e0 * x.e0;
@@ -152,7 +162,7 @@ __global__ void __launch_bounds__(gr::THREADS, 3) gptq_rows_kernel(
     const float* __restrict__ Wk, int d_out, int d_in, int j0, int bw,
     const float* __restrict__ img, const float* __restrict__ rdiag, int g, int bits,
     uint8_t* __restrict__ codes_p, uint16_t* __restrict__ scales, uint16_t* __restrict__ zeros,
-    float* __restrict__ Err, int err_ld, double* err_sq, int* status) {
+    float* __restrict__ Err, float* __restrict__ ErrLo, int err_ld, double* err_sq, int* status) {
     if (status_bad(status)) return;
     extern __shared__ __align__(128) unsigned char rows_smem[];
     float* Us = reinterpret_cast<float*>(rows_smem);
@@ -184,7 +194,7 @@ __global__ void __launch_bounds__(gr::THREADS, 3) gptq_rows_kernel(
     x.n_groups_row = d_in / g; x.err_ld = err_ld;
     x.r = static_cast<int64_t>(blockIdx.x) * gr::THREADS + tid;
     x.row_ok = x.r < d_out;
-    x.codes_p = codes_p; x.scales = scales; x.zeros = zeros; x.Err = Err;
+    x.codes_p = codes_p; x.scales = scales; x.zeros = zeros; x.Err = Err; x.ErrLo = ErrLo;
     x.P.scale = 1.f; x.P.zero = 0.f; x.P.inv_scale = 1.f;
     x.next_gs = 0;   // j0 is a multiple of g
     x.e0 = x.e1 = x.e2 = x.e3 = 0.f;
@@ -218,8 +228,8 @@ static bool g_rows_attr_set = false;
 
 gptq_status gptq_block_launch(float* Wk, int d_out, int d_in, int j0, int bw, const float* img,
                               const float* rdiag, int group_size, int bits, uint8_t* codes_p,
-                              uint16_t* scales, uint16_t* zeros, float* Err, int err_ld,
-                              double* err_sq, int* status, cudaStream_t s) {
+                              uint16_t* scales, uint16_t* zeros, float* Err, float* ErrLo,
+                              int err_ld, double* err_sq, int* status, cudaStream_t s) {
     if (!g_rows_attr_set) {
         GPTQ_CUDA_TRY(cudaFuncSetAttribute(gptq_rows_kernel,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -229,22 +239,25 @@ gptq_status gptq_block_launch(float* Wk, int d_out, int d_in, int j0, int bw, co
     const int grid = (d_out + gr::THREADS - 1) / gr::THREADS;
     gptq_rows_kernel<<<grid, gr::THREADS, gr::SMEM, s>>>(Wk, d_out, d_in, j0, bw, img, rdiag,
                                                         group_size, bits, codes_p, scales, zeros,
-                                                        Err, err_ld, err_sq, status);
+                                                        Err, ErrLo, err_ld, err_sq, status);
     GPTQ_LAUNCHED();
     return GPTQ_OK;
 }
 
-// W[:, c0:c1] -= Err[:, 0:k1-k0] * U[k0:k1, c0:c1]  (3xTF32 on the tensor cores)
+// W[:, c0:c1] -= Err[:, 0:k1-k0] * U[k0:k1, c0:c1]  (3xTF32 on the tensor cores, with both
+// operands split into tf32 hi/lo once: U after the factorisation, Err by the column loop)
 gptq_status lazy_update_launch(float* Wk, int d_out, int d_in, int k0, int k1, int c0, int c1,
-                               const float* U, const float* Err, int err_ld, const int* status,
+                               const float* U_hi, const float* U_lo, const float* Err_hi,
+                               const float* Err_lo, int err_ld, const int* status,
                                cudaStream_t s) {
     if (c1 <= c0 || k1 <= k0) return GPTQ_OK;
+    const int64_t boff = static_cast<int64_t>(k0) * d_in + c0;
     TcGemmArgs a{};
     a.M = d_out; a.N = c1 - c0; a.K = k1 - k0; a.alpha = -1.f; a.beta = 1.f;
-    a.A = Err; a.lda = err_ld;
-    a.B = U + static_cast<int64_t>(k0) * d_in + c0; a.ldb = d_in;
+    a.A = Err_hi; a.A_lo = Err_lo; a.lda = err_ld;
+    a.B = U_hi + boff; a.B_lo = U_lo + boff; a.ldb = d_in;
     a.C = Wk + c0; a.ldc = d_in; a.status = status;
-    return tcgemm_launch(a, false, TC_EPI_STORE, true, true, s);
+    return tcgemm_presplit_launch(a, s);
 }
 
 // codes[r][c] = codes_p[r][invperm[c]]; g_idx[c] = invperm[c] / g; perm_out = perm

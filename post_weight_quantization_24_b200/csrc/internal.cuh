@@ -55,11 +55,12 @@ gptq_status column_images_launch(const float* U, int d, int block_size, float* i
 // The column loop of the block [j0, j0+bw), with img/rdiag as column_images_launch writes them
 gptq_status gptq_block_launch(float* Wk, int d_out, int d_in, int j0, int bw, const float* img,
                               const float* rdiag, int group_size, int bits, uint8_t* codes_p,
-                              uint16_t* scales, uint16_t* zeros, float* Err, int err_ld,
-                              double* err_sq, int* status, cudaStream_t s);
-// W[:, c0:c1] -= Err[:, 0:k1-k0] * U[k0:k1, c0:c1]
+                              uint16_t* scales, uint16_t* zeros, float* Err, float* ErrLo,
+                              int err_ld, double* err_sq, int* status, cudaStream_t s);
+// W[:, c0:c1] -= Err[:, 0:k1-k0] * U[k0:k1, c0:c1], both operands given as tf32 hi/lo parts
 gptq_status lazy_update_launch(float* Wk, int d_out, int d_in, int k0, int k1, int c0, int c1,
-                               const float* U, const float* Err, int err_ld, const int* status,
+                               const float* U_hi, const float* U_lo, const float* Err_hi,
+                               const float* Err_lo, int err_ld, const int* status,
                                cudaStream_t s);
 gptq_status assemble_launch(const uint8_t* codes_p, int d_out, int d_in, const int* perm,
                             const int* invperm, int group_size, int act_order, uint8_t* codes,

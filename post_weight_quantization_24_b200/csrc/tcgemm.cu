@@ -61,12 +61,6 @@ __device__ __forceinline__ void umma_tf32(uint32_t d_tmem, uint64_t adesc, uint6
         : "memory");
 }
 
-__device__ __forceinline__ float tf32_rna(float x) {
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return __uint_as_float(r);
-}
-
 struct TcParams {
     TcGemmArgs a;
     int beta_one;
@@ -89,11 +83,14 @@ __device__ __forceinline__ bool tc_tile(const TcParams& p, long long t, int& m0,
     return true;
 }
 
-template <bool B_K, int EPI, bool SPLIT_A, bool SPLIT_B>
+template <bool B_K, int EPI, bool SPLIT_A, bool SPLIT_B, bool PRE>
 __global__ void __launch_bounds__(tg::THREADS, 1)
     tcgemm_kernel(const __grid_constant__ CUtensorMap amap,
                   const __grid_constant__ CUtensorMap bmap,
-                  const __grid_constant__ CUtensorMap cmap, const TcParams p) {
+                  const __grid_constant__ CUtensorMap cmap,
+                  const __grid_constant__ CUtensorMap alomap,
+                  const __grid_constant__ CUtensorMap blomap, const TcParams p) {
+    static_assert(!PRE || (SPLIT_A && SPLIT_B), "pre-split operands come in hi/lo pairs");
     if (status_bad(p.a.status)) return;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -127,6 +124,10 @@ __global__ void __launch_bounds__(tg::THREADS, 1)
         tma_prefetch_desc(&amap);
         tma_prefetch_desc(&bmap);
         if (EPI == TC_EPI_STORE) tma_prefetch_desc(&cmap);
+        if (PRE) {
+            tma_prefetch_desc(&alomap);
+            tma_prefetch_desc(&blomap);
+        }
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, tg::TMEM_COLS);
@@ -153,14 +154,20 @@ __global__ void __launch_bounds__(tg::THREADS, 1)
                     }
                     uint8_t* sa = smem + st * tg::STAGE;
                     const int k0 = kb * tg::BK;
-                    mbar_arrive_expect_tx(&full[st], tg::TILE_A + tg::TILE_B);
+                    mbar_arrive_expect_tx(&full[st], (PRE ? 2 : 1) * (tg::TILE_A + tg::TILE_B));
                     tma_load_2d(sa, &amap, &full[st], k0, m0);
+                    if (PRE) tma_load_2d(sa + tg::OFF_A_LO, &alomap, &full[st], k0, m0);
                     if (B_K) {
                         tma_load_2d(sa + tg::OFF_B, &bmap, &full[st], k0, n0);
+                        if (PRE) tma_load_2d(sa + tg::OFF_B_LO, &blomap, &full[st], k0, n0);
                     } else {
 #pragma unroll
-                        for (int c = 0; c < 4; ++c)
+                        for (int c = 0; c < 4; ++c) {
                             tma_load_2d(sa + tg::OFF_B + c * 4096, &bmap, &full[st], n0 + 32 * c, k0);
+                            if (PRE)
+                                tma_load_2d(sa + tg::OFF_B_LO + c * 4096, &blomap, &full[st],
+                                            n0 + 32 * c, k0);
+                        }
                     }
                 }
             }
@@ -191,7 +198,7 @@ __global__ void __launch_bounds__(tg::THREADS, 1)
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * tg::BN);
                 for (int kb = 0; kb < p.n_kb; ++kb, ++it) {
                     const int st = it % tg::STAGES;
-                    if (!mbar_wait(&conv[st], (it / tg::STAGES) & 1)) {
+                    if (!mbar_wait(PRE ? &full[st] : &conv[st], (it / tg::STAGES) & 1)) {
                         ok = false;
                         break;
                     }
@@ -233,64 +240,66 @@ __global__ void __launch_bounds__(tg::THREADS, 1)
         __syncwarp();
     } else if (warp < tg::EPI_WARP0) {
         // ---------------- converters: fp32 -> tf32 hi (in place) + lo ----------------
-        const int ct = (warp - 2) * 32 + lane;   // 0..255
-        int it = 0;
-        bool stop = false;
-        for (long long t = blockIdx.x; t < p.n_tiles && !stop; t += gridDim.x) {
-            int m0, n0;
-            if (!tc_tile(p, t, m0, n0)) continue;
-            for (int kb = 0; kb < p.n_kb; ++kb, ++it) {
-                const int st = it % tg::STAGES;
-                int ok = 1;
-                if (lane == 0) ok = mbar_wait(&full[st], (it / tg::STAGES) & 1) ? 1 : 0;
-                ok = __shfl_sync(0xffffffffu, ok, 0);
-                if (!ok || __shfl_sync(0xffffffffu, *abort_flag, 0)) {
-                    if (lane == 0 && !ok) {
-                        set_status(status, GPTQ_ERR_TIMEOUT);
-                        *abort_flag = 1;
+        if constexpr (!PRE) {   // (pre-split operands arrive ready for the MMA)
+            const int ct = (warp - 2) * 32 + lane;   // 0..255
+            int it = 0;
+            bool stop = false;
+            for (long long t = blockIdx.x; t < p.n_tiles && !stop; t += gridDim.x) {
+                int m0, n0;
+                if (!tc_tile(p, t, m0, n0)) continue;
+                for (int kb = 0; kb < p.n_kb; ++kb, ++it) {
+                    const int st = it % tg::STAGES;
+                    int ok = 1;
+                    if (lane == 0) ok = mbar_wait(&full[st], (it / tg::STAGES) & 1) ? 1 : 0;
+                    ok = __shfl_sync(0xffffffffu, ok, 0);
+                    if (!ok || __shfl_sync(0xffffffffu, *abort_flag, 0)) {
+                        if (lane == 0 && !ok) {
+                            set_status(status, GPTQ_ERR_TIMEOUT);
+                            *abort_flag = 1;
+                        }
+                        stop = true;
+                        break;
                     }
-                    stop = true;
-                    break;
-                }
-                uint8_t* sa = smem + st * tg::STAGE;
-                if (SPLIT_A) {
-                    float4* hi = reinterpret_cast<float4*>(sa);
-                    float4* lo = reinterpret_cast<float4*>(sa + tg::OFF_A_LO);
-#pragma unroll
-                    for (int j = 0; j < tg::TILE_A / 16 / 256; ++j) {
-                        const int i = ct + 256 * j;
-                        const float4 x = hi[i];
-                        float4 h, l;
-                        h.x = tf32_rna(x.x); l.x = tf32_rna(x.x - h.x);
-                        h.y = tf32_rna(x.y); l.y = tf32_rna(x.y - h.y);
-                        h.z = tf32_rna(x.z); l.z = tf32_rna(x.z - h.z);
-                        h.w = tf32_rna(x.w); l.w = tf32_rna(x.w - h.w);
-                        hi[i] = h;
-                        lo[i] = l;
+                    uint8_t* sa = smem + st * tg::STAGE;
+                    if (SPLIT_A) {
+                        float4* hi = reinterpret_cast<float4*>(sa);
+                        float4* lo = reinterpret_cast<float4*>(sa + tg::OFF_A_LO);
+    #pragma unroll
+                        for (int j = 0; j < tg::TILE_A / 16 / 256; ++j) {
+                            const int i = ct + 256 * j;
+                            const float4 x = hi[i];
+                            float4 h, l;
+                            h.x = tf32_rna(x.x); l.x = tf32_rna(x.x - h.x);
+                            h.y = tf32_rna(x.y); l.y = tf32_rna(x.y - h.y);
+                            h.z = tf32_rna(x.z); l.z = tf32_rna(x.z - h.z);
+                            h.w = tf32_rna(x.w); l.w = tf32_rna(x.w - h.w);
+                            hi[i] = h;
+                            lo[i] = l;
+                        }
                     }
-                }
-                if (SPLIT_B) {
-                    float4* hi = reinterpret_cast<float4*>(sa + tg::OFF_B);
-                    float4* lo = reinterpret_cast<float4*>(sa + tg::OFF_B_LO);
-#pragma unroll
-                    for (int j = 0; j < tg::TILE_B / 16 / 256; ++j) {
-                        const int i = ct + 256 * j;
-                        const float4 x = hi[i];
-                        float4 h, l;
-                        h.x = tf32_rna(x.x); l.x = tf32_rna(x.x - h.x);
-                        h.y = tf32_rna(x.y); l.y = tf32_rna(x.y - h.y);
-                        h.z = tf32_rna(x.z); l.z = tf32_rna(x.z - h.z);
-                        h.w = tf32_rna(x.w); l.w = tf32_rna(x.w - h.w);
-                        hi[i] = h;
-                        lo[i] = l;
+                    if (SPLIT_B) {
+                        float4* hi = reinterpret_cast<float4*>(sa + tg::OFF_B);
+                        float4* lo = reinterpret_cast<float4*>(sa + tg::OFF_B_LO);
+    #pragma unroll
+                        for (int j = 0; j < tg::TILE_B / 16 / 256; ++j) {
+                            const int i = ct + 256 * j;
+                            const float4 x = hi[i];
+                            float4 h, l;
+                            h.x = tf32_rna(x.x); l.x = tf32_rna(x.x - h.x);
+                            h.y = tf32_rna(x.y); l.y = tf32_rna(x.y - h.y);
+                            h.z = tf32_rna(x.z); l.z = tf32_rna(x.z - h.z);
+                            h.w = tf32_rna(x.w); l.w = tf32_rna(x.w - h.w);
+                            hi[i] = h;
+                            lo[i] = l;
+                        }
                     }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&conv[st]);
                 }
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&conv[st]);
             }
+            __syncwarp();
         }
-        __syncwarp();
     } else {
         // ---------------- epilogue ----------------
         const int q = warp & 3;
@@ -381,17 +390,19 @@ __global__ void __launch_bounds__(tg::THREADS, 1)
     if (warp == 1) tmem_dealloc(tmem_base, tg::TMEM_COLS);
 }
 
-template <bool B_K, int EPI, bool SA, bool SB>
+template <bool B_K, int EPI, bool SA, bool SB, bool PRE>
 static gptq_status launch_variant(const CUtensorMap& am, const CUtensorMap& bm,
-                                  const CUtensorMap& cm, const TcParams& p, int grid,
+                                  const CUtensorMap& cm, const CUtensorMap& alom,
+                                  const CUtensorMap& blom, const TcParams& p, int grid,
                                   cudaStream_t s) {
     static bool attr = false;
     if (!attr) {
-        GPTQ_CUDA_TRY(cudaFuncSetAttribute(tcgemm_kernel<B_K, EPI, SA, SB>,
+        GPTQ_CUDA_TRY(cudaFuncSetAttribute(tcgemm_kernel<B_K, EPI, SA, SB, PRE>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, tg::SMEM));
         attr = true;
     }
-    tcgemm_kernel<B_K, EPI, SA, SB><<<grid, tg::THREADS, tg::SMEM, s>>>(am, bm, cm, p);
+    tcgemm_kernel<B_K, EPI, SA, SB, PRE><<<grid, tg::THREADS, tg::SMEM, s>>>(am, bm, cm, alom,
+                                                                             blom, p);
     GPTQ_LAUNCHED();
     return GPTQ_OK;
 }
@@ -400,15 +411,13 @@ template <bool B_K, int EPI>
 static gptq_status launch_split(const CUtensorMap& am, const CUtensorMap& bm,
                                 const CUtensorMap& cm, const TcParams& p, int grid, bool sa,
                                 bool sb, cudaStream_t s) {
-    if (sa && sb) return launch_variant<B_K, EPI, true, true>(am, bm, cm, p, grid, s);
-    if (sa) return launch_variant<B_K, EPI, true, false>(am, bm, cm, p, grid, s);
-    if (sb) return launch_variant<B_K, EPI, false, true>(am, bm, cm, p, grid, s);
-    return launch_variant<B_K, EPI, false, false>(am, bm, cm, p, grid, s);
+    if (sa && sb) return launch_variant<B_K, EPI, true, true, false>(am, bm, cm, am, bm, p, grid, s);
+    if (sa) return launch_variant<B_K, EPI, true, false, false>(am, bm, cm, am, bm, p, grid, s);
+    if (sb) return launch_variant<B_K, EPI, false, true, false>(am, bm, cm, am, bm, p, grid, s);
+    return launch_variant<B_K, EPI, false, false, false>(am, bm, cm, am, bm, p, grid, s);
 }
 
-gptq_status tcgemm_launch(const TcGemmArgs& a, bool b_kmajor, int epi, bool split_a, bool split_b,
-                          cudaStream_t s) {
-    if (a.M <= 0 || a.N <= 0 || a.K <= 0) return GPTQ_OK;
+static gptq_status check_args(const TcGemmArgs& a, int epi) {
     if (a.lda % 4 || a.ldb % 4 || a.N % 4 || (epi == TC_EPI_STORE && a.ldc % 4) ||
         (epi == TC_EPI_DOT && a.ldd % 4))
         return GPTQ_ERR_ARG;
@@ -418,26 +427,32 @@ gptq_status tcgemm_launch(const TcGemmArgs& a, bool b_kmajor, int epi, bool spli
     if (epi == TC_EPI_STORE &&
         ((a.beta != 0.0f && a.beta != 1.0f) || (reinterpret_cast<uintptr_t>(a.C) & 15)))
         return GPTQ_ERR_ARG;
-    CUtensorMap am, bm, cm;
-    if (epi == TC_EPI_STORE) {
-        GPTQ_TRY(encode_tensor_map_2d(&cm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.C, a.N, a.M,
-                                      static_cast<uint64_t>(a.ldc) * 4, 32, 32,
-                                      CU_TENSOR_MAP_SWIZZLE_128B));
-    } else {
-        cm = am;   // unused by the dot epilogue
-    }
-    GPTQ_TRY(encode_tensor_map_2d(&am, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, const_cast<float*>(a.A),
-                                  a.K, a.M, static_cast<uint64_t>(a.lda) * 4, 32, 128,
-                                  CU_TENSOR_MAP_SWIZZLE_128B));
-    if (b_kmajor) {
-        GPTQ_TRY(encode_tensor_map_2d(&bm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, const_cast<float*>(a.B),
-                                      a.K, a.N, static_cast<uint64_t>(a.ldb) * 4, 32, 128,
-                                      CU_TENSOR_MAP_SWIZZLE_128B));
-    } else {
-        GPTQ_TRY(encode_tensor_map_2d(&bm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, const_cast<float*>(a.B),
-                                      a.N, a.K, static_cast<uint64_t>(a.ldb) * 4, 32, 32,
-                                      CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B));
-    }
+    return GPTQ_OK;
+}
+
+static gptq_status encode_a(CUtensorMap* m, const float* A, const TcGemmArgs& a) {
+    return encode_tensor_map_2d(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, const_cast<float*>(A), a.K,
+                                a.M, static_cast<uint64_t>(a.lda) * 4, 32, 128,
+                                CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+static gptq_status encode_b(CUtensorMap* m, const float* B, const TcGemmArgs& a, bool b_kmajor) {
+    if (b_kmajor)
+        return encode_tensor_map_2d(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, const_cast<float*>(B),
+                                    a.K, a.N, static_cast<uint64_t>(a.ldb) * 4, 32, 128,
+                                    CU_TENSOR_MAP_SWIZZLE_128B);
+    return encode_tensor_map_2d(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, const_cast<float*>(B), a.N,
+                                a.K, static_cast<uint64_t>(a.ldb) * 4, 32, 32,
+                                CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B);
+}
+
+static gptq_status encode_c(CUtensorMap* m, const TcGemmArgs& a) {
+    return encode_tensor_map_2d(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.C, a.N, a.M,
+                                static_cast<uint64_t>(a.ldc) * 4, 32, 32,
+                                CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+static TcParams make_params(const TcGemmArgs& a, int& grid) {
     TcParams p;
     p.a = a;
     p.beta_one = (a.beta == 1.0f) ? 1 : 0;
@@ -448,7 +463,21 @@ gptq_status tcgemm_launch(const TcGemmArgs& a, bool b_kmajor, int epi, bool spli
     p.n_tiles = static_cast<long long>(n_bands) * tg::BAND * p.n_nt;
     long long useful = static_cast<long long>(p.n_mt) * p.n_nt;
     if (a.lower_only) useful = useful / 2 + p.n_mt;
-    const int grid = static_cast<int>(std::max<long long>(1, std::min<long long>(useful, num_sms())));
+    grid = static_cast<int>(std::max<long long>(1, std::min<long long>(useful, num_sms())));
+    return p;
+}
+
+gptq_status tcgemm_launch(const TcGemmArgs& a, bool b_kmajor, int epi, bool split_a, bool split_b,
+                          cudaStream_t s) {
+    if (a.M <= 0 || a.N <= 0 || a.K <= 0) return GPTQ_OK;
+    GPTQ_TRY(check_args(a, epi));
+    CUtensorMap am, bm, cm;
+    GPTQ_TRY(encode_a(&am, a.A, a));
+    GPTQ_TRY(encode_b(&bm, a.B, a, b_kmajor));
+    if (epi == TC_EPI_STORE) GPTQ_TRY(encode_c(&cm, a));
+    else cm = am;   // unused by the dot epilogue
+    int grid;
+    const TcParams p = make_params(a, grid);
     if (b_kmajor) {
         return epi == TC_EPI_STORE
                    ? launch_split<true, TC_EPI_STORE>(am, bm, cm, p, grid, split_a, split_b, s)
@@ -457,6 +486,51 @@ gptq_status tcgemm_launch(const TcGemmArgs& a, bool b_kmajor, int epi, bool spli
     return epi == TC_EPI_STORE
                ? launch_split<false, TC_EPI_STORE>(am, bm, cm, p, grid, split_a, split_b, s)
                : launch_split<false, TC_EPI_DOT>(am, bm, cm, p, grid, split_a, split_b, s);
+}
+
+gptq_status tcgemm_presplit_launch(const TcGemmArgs& a, cudaStream_t s) {
+    if (a.M <= 0 || a.N <= 0 || a.K <= 0) return GPTQ_OK;
+    GPTQ_TRY(check_args(a, TC_EPI_STORE));
+    if (!a.A_lo || !a.B_lo || (reinterpret_cast<uintptr_t>(a.A_lo) & 15) ||
+        (reinterpret_cast<uintptr_t>(a.B_lo) & 15))
+        return GPTQ_ERR_ARG;
+    CUtensorMap am, bm, cm, alom, blom;
+    GPTQ_TRY(encode_a(&am, a.A, a));
+    GPTQ_TRY(encode_a(&alom, a.A_lo, a));
+    GPTQ_TRY(encode_b(&bm, a.B, a, false));
+    GPTQ_TRY(encode_b(&blom, a.B_lo, a, false));
+    GPTQ_TRY(encode_c(&cm, a));
+    int grid;
+    const TcParams p = make_params(a, grid);
+    return launch_variant<false, TC_EPI_STORE, true, true, true>(am, bm, cm, alom, blom, p, grid, s);
+}
+
+__global__ void tf32_split_kernel(const float* src, float* hi, float* __restrict__ lo, int rows,
+                                  int cols, int ld, int upper) {
+    for (int r = blockIdx.x; r < rows; r += gridDim.x) {
+        const int64_t row = static_cast<int64_t>(r) * ld;
+        for (int c = (upper ? (r & ~3) : 0) + 4 * static_cast<int>(threadIdx.x); c < cols;
+             c += 4 * blockDim.x) {
+            const float4 x = *reinterpret_cast<const float4*>(src + row + c);
+            float4 h, l;
+            h.x = tf32_rna(x.x); l.x = tf32_rna(x.x - h.x);
+            h.y = tf32_rna(x.y); l.y = tf32_rna(x.y - h.y);
+            h.z = tf32_rna(x.z); l.z = tf32_rna(x.z - h.z);
+            h.w = tf32_rna(x.w); l.w = tf32_rna(x.w - h.w);
+            *reinterpret_cast<float4*>(hi + row + c) = h;
+            *reinterpret_cast<float4*>(lo + row + c) = l;
+        }
+    }
+}
+
+gptq_status tcgemm_split_launch(const float* src, float* hi, float* lo, int rows, int cols, int ld,
+                                bool upper, cudaStream_t s) {
+    if (rows <= 0 || cols <= 0) return GPTQ_OK;
+    if (cols % 4 || ld % 4) return GPTQ_ERR_ARG;
+    const int blocks = std::min(rows, num_sms() * 8);
+    tf32_split_kernel<<<blocks, 256, 0, s>>>(src, hi, lo, rows, cols, ld, upper ? 1 : 0);
+    GPTQ_LAUNCHED();
+    return GPTQ_OK;
 }
 
 }  // namespace gq

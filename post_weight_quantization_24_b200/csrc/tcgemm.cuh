@@ -9,6 +9,13 @@ namespace gq {
 
 enum { TC_EPI_STORE = 0, TC_EPI_DOT = 1 };
 
+// x rounded to tf32 (10 explicit mantissa bits), nearest with ties away from zero
+__device__ __forceinline__ float tf32_rna(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return __uint_as_float(r);
+}
+
 struct TcGemmArgs {
     int M, N, K;
     float alpha, beta;
@@ -23,6 +30,10 @@ struct TcGemmArgs {
     double* dot;
     int lower_only;   // skip output tiles entirely above the diagonal
     const int* status;  // optional: skip all work when *status != 0; receives TIMEOUT
+    // Pre-split operands (tcgemm_presplit_launch): A and B hold the tf32 hi parts, A_lo and
+    // B_lo the lo parts, with the layouts and strides of A and B.
+    const float* A_lo;
+    const float* B_lo;
 };
 
 // split_a / split_b: represent that operand as hi + lo tf32 parts (an operand that is already
@@ -30,5 +41,15 @@ struct TcGemmArgs {
 // ldd multiples of 4; A, B 16-byte aligned; N a multiple of 4.
 gptq_status tcgemm_launch(const TcGemmArgs& a, bool b_kmajor, int epi, bool split_a, bool split_b,
                           cudaStream_t s);
+
+// C = alpha*A*B + beta*C (store epilogue) with both operands already split into tf32 hi and lo
+// (hi = tf32_rna(x), lo = tf32_rna(x - hi), as tcgemm_split_launch writes them); B MN-major.
+// Operands reused by many tiles are split once instead of in every tile.
+gptq_status tcgemm_presplit_launch(const TcGemmArgs& a, cudaStream_t s);
+
+// hi[i][j] = tf32_rna(x), lo[i][j] = tf32_rna(x - hi) for x = src[i][j], j0(i) <= j < cols,
+// j0(i) = upper ? i & ~3 : 0 (rows of stride ld; hi may alias src)
+gptq_status tcgemm_split_launch(const float* src, float* hi, float* lo, int rows, int cols, int ld,
+                                bool upper, cudaStream_t s);
 
 }  // namespace gq
