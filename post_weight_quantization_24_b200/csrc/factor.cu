@@ -184,57 +184,75 @@ gptq_status gather_w_launch(const void* W, int w_dtype, int d_out, int d_in, con
 // ---------------------------------------------------------------------------------------
 // ---- diagonal block: one CTA factors the 128 x 128 block A[k0:, k0:] and inverts its factor.
 // Pass 1 (factor) is right-looking elimination with one thread per row. At step c every
-// thread publishes its current column-c entry a_ic; by symmetry the pivot row's entries a_cm
-// are the published a_mc, so the column is all a step needs. Thread i then applies
+// thread has published its current column-c entry a_ic; by symmetry the pivot row's entries
+// a_cm are the published a_mc, so the column is all a step needs. Thread i then applies
 // a_im -= (a_ic / a_cc) a_mc to its row and records L[i][c] = a_ic / sqrt(a_cc).
 // Pass 2 (inverse) gives thread i column i of L^-1 by forward substitution against the
 // recorded columns of L: x_m -= L[m][c] * x_c / L[c][c], with x_c / L[c][c] = (L^-1)[c][i].
 // In both passes a thread's values sit in a register window that moves down one position
 // per step (position p holds matrix index c + p), so the running step is always position 0
 // and every register index is a compile-time constant; the window narrows in phases of 16
-// steps. One barrier per step in pass 1 (the published column is double-buffered); none in
-// pass 2. Rows and columns beyond the matrix edge are padded with the identity.
+// steps. In pass 1 a thread computes its next column entry first, publishes it and arrives
+// on the next step's mbarrier before it sweeps the rest of its row, so the exchange of one
+// step overlaps the arithmetic of the previous one (three column buffers, one mbarrier
+// each). Pass 2 needs no synchronisation. Rows and columns beyond the matrix edge are padded
+// with the identity.
 namespace pd {
-constexpr int NB = 128, THREADS = NB, PH = 16;
+constexpr int NB = 128, THREADS = NB, PH = 16, NBUF = 3;
 constexpr int LS = NB + 4;          // Lsh row stride: Lsh[c][m - c + 3] = L[m][c], m >= c
 constexpr int CB = NB + 8;          // published column: cb[i - c + 3] = a_ic of step c
-constexpr int SMEM = (NB * LS + 2 * CB + NB) * 4;   // + rs[c] = 1 / L[c][c]
+constexpr int SMEM = (NB * LS + NBUF * CB + NB) * 4 + NBUF * 8;   // + rs[c], mbarriers
 }  // namespace pd
 
+__device__ __forceinline__ float rcp_approx(float x) {
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
+__device__ __forceinline__ float rsqrt_approx(float x) {
+    float r;
+    asm("rsqrt.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
 template <int W>
-__device__ __forceinline__ void potrf_factor_phase(float (&w)[pd::NB], int q, int i, float* Lsh,
-                                                   float* cb, float* rs, bool& bad) {
+__device__ __forceinline__ bool potrf_factor_phase(float (&w)[pd::NB], int q, int i, float* Lsh,
+                                                   float* cb, uint64_t* mb, float* rs, bool& bad) {
 #pragma unroll 1
     for (int c = q * pd::PH; c < (q + 1) * pd::PH; ++c) {
-        float* buf = cb + (c & 1) * pd::CB;
-        if (i >= c) buf[i - c + 3] = w[0];
-        __syncthreads();
+        const int b = c % pd::NBUF, nb = (c + 1) % pd::NBUF;
+        if (!mbar_wait(&mb[b], (c / pd::NBUF) & 1)) return false;
+        const float* buf = cb + b * pd::CB;
+        const float* col = buf + 4;          // col[k] = a_{c+1+k, c}
         if ((i | 31) >= c) {                 // this warp still has a row at or below the pivot
             const float p = buf[3];
-            const float rp = __frcp_rn(p);
-            const float sp = sqrtf(p);
-            const float rsp = __frcp_rn(sp);
-            const float w0 = w[0];
+            const float t = w[0] * rcp_approx(p);
+            // the next step's column entry first: publish it, then sweep the rest of the row
+            const float nw0 = fmaf(-t, col[0], w[1]);
+            if (i > c) cb[nb * pd::CB + i - c + 2] = nw0;
+            mbar_arrive(&mb[nb]);
+            const float rsp = rsqrt_approx(p);
+            if (i >= c) Lsh[c * pd::LS + i - c + 3] = (i == c) ? p * rsp : w[0] * rsp;
             if (i == c) {
-                if (!(p > 0.0f) || !isfinite(p)) bad = true;
-                Lsh[c * pd::LS + 3] = sp;
                 rs[c] = rsp;
-            } else if (i > c) {
-                Lsh[c * pd::LS + i - c + 3] = w0 * rsp;
+                if (!(p > 0.0f) || !isfinite(p)) bad = true;
             }
-            const float t = w0 * rp;
-            const float* col = buf + 4;      // col[k] = a_{c+1+k, c}
+            w[0] = nw0;
 #pragma unroll
             for (int k4 = 0; k4 < W; k4 += 4) {
                 const float4 v = *reinterpret_cast<const float4*>(col + k4);
                 const float vv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
                 for (int u = 0; u < 4; ++u)
-                    if (k4 + u + 1 < W) w[k4 + u] = fmaf(-t, vv[u], w[k4 + u + 1]);
+                    if (k4 + u >= 1 && k4 + u + 1 < W) w[k4 + u] = fmaf(-t, vv[u], w[k4 + u + 1]);
             }
             w[W - 1] = 0.0f;
+        } else {
+            mbar_arrive(&mb[nb]);
         }
     }
+    return true;
 }
 
 template <int W>
@@ -265,12 +283,17 @@ __global__ void __launch_bounds__(pd::THREADS, 1) potrf_diag_kernel(float* __res
     if (status_bad(status)) return;
     extern __shared__ __align__(16) float sm[];
     float* Lsh = sm;                          // [NB][LS]
-    float* cb = Lsh + pd::NB * pd::LS;        // [2][CB]
-    float* rs = cb + 2 * pd::CB;              // [NB]
+    float* cb = Lsh + pd::NB * pd::LS;        // [NBUF][CB]
+    float* rs = cb + pd::NBUF * pd::CB;       // [NB]
+    uint64_t* mb = reinterpret_cast<uint64_t*>(rs + pd::NB);   // [NBUF], 128 arrivals each
     const int i = threadIdx.x, warp = i >> 5;
 
-    for (int e = i; e < (pd::NB * pd::LS + 2 * pd::CB) / 4; e += pd::THREADS)
+    for (int e = i; e < (pd::NB * pd::LS + pd::NBUF * pd::CB) / 4; e += pd::THREADS)
         reinterpret_cast<float4*>(sm)[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (i == 0) {
+        for (int b = 0; b < pd::NBUF; ++b) mbar_init(&mb[b], pd::THREADS);
+        fence_mbar_init();
+    }
 
     // row i of the block's lower triangle (zeros above the diagonal; identity past the edge)
     float w[pd::NB];
@@ -285,17 +308,22 @@ __global__ void __launch_bounds__(pd::THREADS, 1) potrf_diag_kernel(float* __res
             w[p4 + u] = (i < nbc) ? (p4 + u <= i ? vv[u] : 0.0f) : (p4 + u == i ? 1.0f : 0.0f);
     }
     __syncthreads();
+    // step 0's column: every thread publishes a_i0
+    cb[i + 3] = w[0];
+    mbar_arrive(&mb[0]);
 
     bool bad = false;
-    potrf_factor_phase<128>(w, 0, i, Lsh, cb, rs, bad);
-    potrf_factor_phase<112>(w, 1, i, Lsh, cb, rs, bad);
-    potrf_factor_phase<96>(w, 2, i, Lsh, cb, rs, bad);
-    potrf_factor_phase<80>(w, 3, i, Lsh, cb, rs, bad);
-    potrf_factor_phase<64>(w, 4, i, Lsh, cb, rs, bad);
-    potrf_factor_phase<48>(w, 5, i, Lsh, cb, rs, bad);
-    potrf_factor_phase<32>(w, 6, i, Lsh, cb, rs, bad);
-    potrf_factor_phase<16>(w, 7, i, Lsh, cb, rs, bad);
+    bool ok = potrf_factor_phase<128>(w, 0, i, Lsh, cb, mb, rs, bad);
+    ok = ok && potrf_factor_phase<112>(w, 1, i, Lsh, cb, mb, rs, bad);
+    ok = ok && potrf_factor_phase<96>(w, 2, i, Lsh, cb, mb, rs, bad);
+    ok = ok && potrf_factor_phase<80>(w, 3, i, Lsh, cb, mb, rs, bad);
+    ok = ok && potrf_factor_phase<64>(w, 4, i, Lsh, cb, mb, rs, bad);
+    ok = ok && potrf_factor_phase<48>(w, 5, i, Lsh, cb, mb, rs, bad);
+    ok = ok && potrf_factor_phase<32>(w, 6, i, Lsh, cb, mb, rs, bad);
+    ok = ok && potrf_factor_phase<16>(w, 7, i, Lsh, cb, mb, rs, bad);
+    if (!ok) set_status(status, GPTQ_ERR_TIMEOUT);
     if (__syncthreads_or(bad) && i == 0) set_status(status, GPTQ_ERR_NOT_PD);
+    if (__syncthreads_or(!ok)) return;
 
     // L back into A: thread i writes column i (row segments stay coalesced across threads)
     for (int m = i; m < nbc; ++m)
