@@ -234,6 +234,43 @@ class LayerStep:
         return {k: a.elapsed_time(b) for k, (a, b) in self.ev.items()}
 
 
+def rtn_stack_measure(gptq, device, reps: int = 3):
+    """Group min-max RTN (INT4, g128) over the weights of a 7B-shaped decoder stack: 32 layers x
+    {q, k, v, o 4096x4096; gate, up 11008x4096; down 4096x11008}, 6.48e9 fp16 weights (13 GB),
+    far larger than L2. The matrices of one input width are quantized as one row block (RTN is
+    row-independent), so each repetition is two launches; CUDA events bracket back-to-back
+    repetitions on the launching stream. Weights: N(0, 0.02) with 0.1% of input columns x20."""
+    g = torch.Generator(device=device).manual_seed(1234)
+    shapes = ((32 * (4 * 4096 + 2 * 11008), 4096), (32 * 4096, 11008))
+    bufs = []
+    for rows, cols in shapes:
+        W = torch.randn(rows, cols, generator=g, device=device, dtype=torch.float16)
+        W.mul_(0.02)
+        outl = torch.randperm(cols, generator=g, device=device)[:max(1, round(0.001 * cols))]
+        W[:, outl] *= 20
+        out = (torch.empty(rows, cols // 2, dtype=torch.uint8, device=device),
+               torch.empty(rows, cols // 128, dtype=torch.float16, device=device),
+               torch.empty(rows, cols // 128, dtype=torch.float16, device=device))
+        bufs.append((W, out))
+    n = sum(r * c for r, c in shapes)
+    for W, out in bufs:                       # warm-up
+        gptq.rtn_minmax_quantize(W, 4, 128, out=out)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        for W, out in bufs:
+            gptq.rtn_minmax_quantize(W, 4, 128, out=out)
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / reps
+    nbytes = n * 2.5 + n // 128 * 4
+    del bufs
+    torch.cuda.empty_cache()
+    return {"ms": ms, "weights": n, "bytes": nbytes, "gbs": nbytes / (ms / 1e3) / 1e9,
+            "weights_per_s": n / (ms / 1e3), "launches": 2 * reps}
+
+
 def run_ours(args):
     world, rank, local = dist_env()
     distributed = init_dist(world, local)
@@ -279,6 +316,7 @@ def run_ours(args):
     launches = gptq.launch_count() - launches0
     clocks = sampler.stop()
     barrier(distributed)
+    rtn_stack = None if args.no_rtn_stack else rtn_stack_measure(gptq, device)
 
     K = args.steps
     total_ms_max = max_over_ranks(total_ms, distributed, device)
@@ -334,8 +372,15 @@ def run_ours(args):
                       "Gram matrix WᵀW on the fp16 path; measured bf16 dense burst" if w_f16
                       else tf32x3),
         "rtn": {"ms": rtn_ms, "bound": "hbm", "gbs": rtn_bytes / (rtn_ms / 1e3) / 1e9,
-                "frac": rtn_bytes / (rtn_ms / 1e3) / 1e9 / peaks["hbm_gbs"]},
+                "frac": rtn_bytes / (rtn_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+                "note": "one call on this layer's W (90 MB, inside L2) right after a synchronising "
+                        "call: includes the host submission gap; see rtn_7b_stack"},
     }
+    if rtn_stack is not None:
+        stages["rtn_7b_stack"] = dict(rtn_stack, bound="hbm",
+                                      frac=rtn_stack["gbs"] / peaks["hbm_gbs"],
+                                      note="INT4 g128 RTN over a 7B decoder stack's 224 matrices "
+                                           "(6.48e9 fp16 weights), outside the timed step")
 
     # the dominant kernel (largest stage) carries the roofline object
     traffic, _ = ncu_traffic("hessian_tc_kernel_mlp_up_7b.md", "hessian.cu")
@@ -558,6 +603,8 @@ def main(argv=None):
     ap.add_argument("--workload", default="mlp_up_7b", choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-rtn-stack", action="store_true",
+                    help="skip the RTN measurement over a 7B decoder stack (13 GB of weights)")
     ap.add_argument("--ncu-case", choices=("hessian", "gptq", "rtn"),
                     help="run one small case for an ncu capture and exit (no JSON line)")
     args = ap.parse_args(argv)

@@ -29,8 +29,10 @@ __device__ __forceinline__ double fp16_ceil(double x) {
     const long long bits = __double_as_longlong(x);
     int e = static_cast<int>((bits >> 52) & 0x7FF) - 1023;   // floor(log2 x) for normal x
     if (e < -14) e = -14;
+    // spacing = 2^(e-10) and its exact reciprocal 2^(10-e); x * 2^(10-e) is exact in fp64
     const double spacing = __longlong_as_double(static_cast<long long>(e - 10 + 1023) << 52);
-    return ceil(x / spacing) * spacing;
+    const double inv_spacing = __longlong_as_double(static_cast<long long>(10 - e + 1023) << 52);
+    return ceil(x * inv_spacing) * spacing;
 }
 
 struct QParams {
@@ -39,16 +41,36 @@ struct QParams {
     float inv_scale;  // approximate 1/scale, only used to form the candidate code
 };
 
+// rint(-lo / s) (half to even) for -lo >= 0 and 0 < s, with -lo/s <= 2^20: a candidate from an
+// approximate quotient, then the exact fp64 residual -lo - k*s (k*s is exact: k has at most 21
+// bits and s 11) moves it to the nearest integer and settles exact halves to even. It equals
+// rint of the correctly rounded fp64 quotient, which cannot land on a half-integer the exact
+// quotient is not on (-lo has 24 significant bits, so a nonzero distance to one is far larger
+// than an fp64 rounding).
+__device__ __forceinline__ double rint_quotient(double nlo, double s) {
+    float r;   // approximate 1/s: the candidate only has to be within one of the answer
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(static_cast<float>(s)));
+    double k = rint(nlo * static_cast<double>(r));
+    const double e = fma(-k, s, nlo);        // exact
+    if (2.0 * e > s) k += 1.0;
+    else if (2.0 * e < -s) k -= 1.0;
+    const double e2 = fma(-k, s, nlo);       // exact; |e2| <= s/2
+    if ((2.0 * e2 == s || 2.0 * e2 == -s) && (static_cast<long long>(k) & 1))
+        k += (e2 > 0.0 ? 1.0 : -1.0);        // a tie: take the even neighbour
+    return k;
+}
+
 __device__ __forceinline__ QParams group_params(float xmin, float xmax, int maxq) {
     const double lo = fmin(static_cast<double>(xmin), 0.0);
     const double hi = fmax(static_cast<double>(xmax), 0.0);
     const double span = hi - lo;
     const double s = (span == 0.0) ? 1.0 : fp16_ceil(span / static_cast<double>(maxq));
-    const double z = rint(-lo / s) + 0.0;
+    // -lo/s <= span/s <= maxq; an infinite s (span/maxq above the fp16 range) gives zero 0
+    const double z = (isinf(s) ? 0.0 : rint_quotient(-lo, s)) + 0.0;
     QParams p;
     p.scale = static_cast<float>(s);
     p.zero = static_cast<float>(z);
-    p.inv_scale = static_cast<float>(1.0 / s);
+    p.inv_scale = __frcp_rn(p.scale);   // fp32 1/scale, within one rounding of the exact value
     return p;
 }
 
@@ -86,6 +108,19 @@ __device__ __forceinline__ int quant_code(float w, const QParams& p, int maxq) {
     }
     const float q = fminf(fmaxf(k + p.zero, 0.0f), static_cast<float>(maxq));
     return static_cast<int>(q);
+}
+
+// The same code as quant_code, kept as an integer-valued float (for packing without F2I).
+__device__ __forceinline__ float quant_codef(float w, const QParams& p, float maxqf) {
+    const float t = w * p.inv_scale;
+    float k = rintf(t);
+    if (fabsf(t - k) > 0.5f - fabsf(t) * 3.0e-7f - 1.0e-30f) k = round_quotient(w, p.scale, p.inv_scale);
+    return fminf(fmaxf(k + p.zero, 0.0f), maxqf);
+}
+
+// Integer bits of an integer-valued float in [0, 2^22): add 2^23 and read the mantissa.
+__device__ __forceinline__ uint32_t small_int_bits(float v) {
+    return __float_as_uint(v + 8388608.0f) - 0x4B000000u;
 }
 
 __device__ __forceinline__ float dequant(int q, const QParams& p) {

@@ -7,6 +7,9 @@
 // shuffles, compute the group's scalars in fp64, and write 8 codes (4 bytes packed INT4, or
 // 8 bytes) plus, from the group's first thread, the fp16 scale and zero. Bytes per weight:
 // 2 (fp16 in) + 0.5 (INT4 out) + 4/group_size (scale + zero).
+#include <algorithm>
+#include <type_traits>
+
 #include "common.cuh"
 #include "quant.cuh"
 
@@ -103,6 +106,222 @@ __global__ void __launch_bounds__(256) rtn_kernel(const T* __restrict__ W, int64
     }
 }
 
+// fp16 weights, power-of-two groups of 32..256: 32 weights per thread (four 16-byte loads),
+// TPG = group_size / 32 threads per group. Codes stay integer-valued floats until they are
+// packed with byte permutes, so no float-to-int conversions are issued.
+// One chunk of 32 fp16 weights on the exact path (quant_codef), packed and stored like the
+// fast path does. Kept out of line: the fast path reaches it rarely.
+__device__ __noinline__ void rtn_chunk_exact(const __half* w, QParams p, int bits,
+                                             uint8_t* __restrict__ out, int64_t t) {
+    constexpr int E = 32;
+    const float maxqf = static_cast<float>((1 << bits) - 1);
+    if (bits == 4) {
+        for (int b = 0; b < E / 2; ++b) {
+            const float lo = quant_codef(__half2float(w[2 * b]), p, maxqf);
+            const float hi = quant_codef(__half2float(w[2 * b + 1]), p, maxqf);
+            out[(E / 2) * t + b] = static_cast<uint8_t>(small_int_bits(fmaf(hi, 16.0f, lo)));
+        }
+    } else {
+        for (int i = 0; i < E; ++i)
+            out[E * t + i] = static_cast<uint8_t>(small_int_bits(quant_codef(__half2float(w[i]), p, maxqf)));
+    }
+}
+
+namespace rp {
+constexpr int WARPS = 8, THREADS = WARPS * 32;
+constexpr int E = 32;                          // weights per lane
+constexpr int STAGES = 4;                      // per-warp ring of 2 KB stages
+constexpr int STAGE_BYTES = 32 * E * 2;        // one warp-iteration: 32 lanes x 32 fp16
+constexpr int SMEM = WARPS * STAGES * STAGE_BYTES;   // 64 KB
+}  // namespace rp
+
+// The group scalars of group_params (same values, bit for bit) without branches, for the
+// streaming kernel: s = smallest fp16 >= span/maxq (the one fp64 division is the same IEEE
+// operation), z = rint(-lo/s) corrected with the exact residual (ties to even), and an
+// approximate 1/s (relative error <= 2^-23; the codes only use it for a candidate that the
+// caller checks).
+__device__ __forceinline__ QParams group_params_stream(float xmin, float xmax, int maxq) {
+    const double lo = fmin(static_cast<double>(xmin), 0.0);
+    const double hi = fmax(static_cast<double>(xmax), 0.0);
+    const double span = hi - lo;
+    const double q = span / static_cast<double>(maxq);
+    // fp16_ceil(q) for q > 0: spacing 2^(e-10), e = max(floor(log2 q), -14)
+    const long long qb = __double_as_longlong(q);
+    const int e = max(static_cast<int>((qb >> 52) & 0x7FF) - 1023, -14);
+    const double spacing = __longlong_as_double(static_cast<long long>(e - 10 + 1023) << 52);
+    const double inv_spacing = __longlong_as_double(static_cast<long long>(10 - e + 1023) << 52);
+    double sc = ceil(q * inv_spacing) * spacing;
+    sc = (q > 65504.0) ? __longlong_as_double(0x7FF0000000000000LL) : sc;
+    sc = (span == 0.0) ? 1.0 : sc;
+    // z = rint(-lo / sc): candidate, then one exact correction and the tie rule
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(static_cast<float>(sc)));
+    const double nlo = -lo;
+    double k = rint(nlo * static_cast<double>(r));
+    const double e1 = fma(-k, sc, nlo);
+    k += (2.0 * e1 > sc) ? 1.0 : ((2.0 * e1 < -sc) ? -1.0 : 0.0);
+    const double e2 = fma(-k, sc, nlo);
+    const bool tie = (2.0 * e2 == sc || 2.0 * e2 == -sc) && (static_cast<long long>(k) & 1);
+    k += tie ? (e2 > 0.0 ? 1.0 : -1.0) : 0.0;
+    k = isinf(sc) ? 0.0 : k;
+    QParams p;
+    p.scale = static_cast<float>(sc);
+    p.zero = static_cast<float>(k + 0.0);
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(p.inv_scale) : "f"(p.scale));
+    return p;
+}
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// fp16 weights, power-of-two groups of 32..256: a lane quantizes 32 consecutive weights
+// (TPG = group_size / 32 lanes per group). Each warp streams its 2 KB per iteration through a
+// 4-stage shared-memory ring with per-lane async copies (coalesced: lane L copies bytes
+// 16L + 512h), keeping three iterations in flight while it computes one, which is what keeps
+// enough bytes outstanding to run at HBM speed. Codes come out of the rounding as float bit
+// patterns and are packed with byte permutes. Chunk indices are 32-bit (the launcher checks).
+template <int TPG, bool INT4>
+__global__ void __launch_bounds__(rp::THREADS, 3) rtn_f16_kernel(const __half* __restrict__ W,
+                                                                int n_chunks, int bits,
+                                                                uint8_t* __restrict__ out,
+                                                                uint16_t* __restrict__ scales,
+                                                                uint16_t* __restrict__ zeros) {
+    extern __shared__ __align__(16) uint8_t rtn_smem[];
+    const int lane = lane_id(), warp = warp_id();
+    uint8_t* ring = rtn_smem + warp * rp::STAGES * rp::STAGE_BYTES;
+    const int maxq = (1 << bits) - 1;
+    const int n_wit = (n_chunks + 31) / 32;                        // warp-iterations in total
+    const int wstride = gridDim.x * rp::WARPS;
+    const int w0 = blockIdx.x * rp::WARPS + warp;
+    const uint8_t* wbytes = reinterpret_cast<const uint8_t*>(W);
+    auto issue = [&](int wi, int st) {
+        if (wi < n_wit) {
+            const uint8_t* src = wbytes + static_cast<int64_t>(wi) * rp::STAGE_BYTES + 16 * lane;
+            uint8_t* dst = ring + st * rp::STAGE_BYTES + 16 * lane;
+            const int valid = min(32, n_chunks - wi * 32) * (2 * rp::E) - 16 * lane;   // bytes
+#pragma unroll
+            for (int h = 0; h < 4; ++h)
+                if (512 * h < valid) cp_async16(dst + 512 * h, src + 512 * h);
+        }
+        cp_async_commit();
+    };
+#pragma unroll
+    for (int k = 0; k < rp::STAGES - 1; ++k) issue(w0 + k * wstride, k);
+    int st = 0;
+    for (int wi = w0; wi < n_wit; wi += wstride) {
+        __syncwarp();     // every lane is done reading the stage the next copy overwrites
+        issue(wi + (rp::STAGES - 1) * wstride, (st + rp::STAGES - 1) & (rp::STAGES - 1));
+        cp_async_wait<rp::STAGES - 1>();
+        __syncwarp();     // this iteration's 2 KB, copied by all lanes, is in shared memory
+        const int t = wi * 32 + lane;
+        const uint4* mine = reinterpret_cast<const uint4*>(ring + st * rp::STAGE_BYTES + 64 * lane);
+        st = (st + 1) & (rp::STAGES - 1);
+        uint4 raw[4];
+#pragma unroll
+        for (int h = 0; h < 4; ++h) raw[h] = mine[h];   // (lanes past the end hold stale data, unused)
+        // group min/max on the fp16 pairs (exact: the fp16 -> fp32 conversion is monotone)
+        const __half2* hp = reinterpret_cast<const __half2*>(raw);
+        __half2 mn2 = __hmin2(hp[0], hp[1]), mx2 = __hmax2(hp[0], hp[1]);
+#pragma unroll
+        for (int i = 2; i < 16; ++i) {
+            mn2 = __hmin2(mn2, hp[i]);
+            mx2 = __hmax2(mx2, hp[i]);
+        }
+        float mn = fminf(__low2float(mn2), __high2float(mn2));
+        float mx = fmaxf(__low2float(mx2), __high2float(mx2));
+#pragma unroll
+        for (int off = TPG / 2; off > 0; off >>= 1) {
+            mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        }
+        if (t >= n_chunks) continue;
+        const QParams p = group_params_stream(mn, mx, maxq);
+        // u = w/scale + zero in one fma; every w lies inside the group's range, so u is in
+        // [-0.5, maxq + 0.5] up to 4.5e-5 (1/scale within 2^-23, one rounding in the fma).
+        // Adding 1.5 * 2^23 rounds u to the nearest integer (half to even) and leaves it in
+        // the low mantissa bits. The rounding is exact unless u is within 4.5e-5 of a
+        // half-integer; if any of the 32 is, the chunk is redone on the exact path. Otherwise
+        // every code is in [0, maxq], so no clamp is needed.
+        constexpr float kMagic = 12582912.0f;                  // 1.5 * 2^23
+        float kf[32];
+        uint32_t mb[32];
+        float dev = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const float2 f = __half22float2(hp[i]);
+            const float u0 = fmaf(f.x, p.inv_scale, p.zero), u1 = fmaf(f.y, p.inv_scale, p.zero);
+            const float m0 = u0 + kMagic, m1 = u1 + kMagic;
+            kf[2 * i] = m0 - kMagic;
+            kf[2 * i + 1] = m1 - kMagic;
+            mb[2 * i] = __float_as_uint(m0);
+            mb[2 * i + 1] = __float_as_uint(m1);
+            dev = fmaxf(dev, fmaxf(fabsf(u0 - kf[2 * i]), fabsf(u1 - kf[2 * i + 1])));
+        }
+        if (dev > 0.5f - 6.0e-5f) {
+            // rare: a code within 4.5e-5 of a rounding boundary; redo the chunk on the exact path
+            rtn_chunk_exact(reinterpret_cast<const __half*>(mine), p, bits, out, t);
+        } else if (INT4) {
+            // byte b holds codes 2b (low nibble) and 2b+1: q0 + 16 q1 (exact), magic-added, has
+            // it in its low byte
+            uint32_t by[16];
+#pragma unroll
+            for (int b = 0; b < 16; ++b)
+                by[b] = __float_as_uint(fmaf(kf[2 * b + 1], 16.0f, kf[2 * b]) + kMagic);
+            uint32_t word[4];
+#pragma unroll
+            for (int w4 = 0; w4 < 4; ++w4)
+                word[w4] = __byte_perm(__byte_perm(by[4 * w4], by[4 * w4 + 1], 0x0040),
+                                       __byte_perm(by[4 * w4 + 2], by[4 * w4 + 3], 0x0040), 0x5410);
+            __stcs(reinterpret_cast<uint4*>(out) + t, make_uint4(word[0], word[1], word[2], word[3]));
+        } else {
+            // one code per byte: the low byte of the magic-added pattern is the code
+            uint32_t word[8];
+#pragma unroll
+            for (int w4 = 0; w4 < 8; ++w4)
+                word[w4] = __byte_perm(__byte_perm(mb[4 * w4], mb[4 * w4 + 1], 0x0040),
+                                       __byte_perm(mb[4 * w4 + 2], mb[4 * w4 + 3], 0x0040), 0x5410);
+            __stcs(reinterpret_cast<uint4*>(out) + 2 * t, make_uint4(word[0], word[1], word[2], word[3]));
+            __stcs(reinterpret_cast<uint4*>(out) + 2 * t + 1, make_uint4(word[4], word[5], word[6], word[7]));
+        }
+        if ((t & (TPG - 1)) == 0) {
+            scales[t / TPG] = half_bits(p.scale);
+            zeros[t / TPG] = half_bits(p.zero);
+        }
+    }
+}
+
+template <int TPG, bool INT4>
+static gptq_status launch_rtn_f16(const __half* W, int64_t n, int bits, uint8_t* out,
+                                  uint16_t* scales, uint16_t* zeros, cudaStream_t s) {
+    static bool attr = false;
+    if (!attr) {
+        GPTQ_CUDA_TRY(cudaFuncSetAttribute(rtn_f16_kernel<TPG, INT4>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, rp::SMEM));
+        attr = true;
+    }
+    // three resident blocks per SM; warps stride over warp-iterations of 1024 weights
+    const int n_chunks = static_cast<int>(n / rp::E);
+    const int64_t n_wit = (n_chunks + 31) / 32;
+    const int64_t want = (n_wit + rp::WARPS - 1) / rp::WARPS;
+    const unsigned grid = static_cast<unsigned>(
+        std::max<int64_t>(1, std::min<int64_t>(want, 3 * static_cast<int64_t>(num_sms()))));
+    rtn_f16_kernel<TPG, INT4><<<grid, rp::THREADS, rp::SMEM, s>>>(W, n_chunks, bits, out, scales, zeros);
+    GPTQ_LAUNCHED();
+    return GPTQ_OK;
+}
+
+template <int TPG>
+static gptq_status launch_rtn_f16_bits(const __half* W, int64_t n, int bits, uint8_t* out,
+                                       uint16_t* scales, uint16_t* zeros, cudaStream_t s) {
+    return bits == 4 ? launch_rtn_f16<TPG, true>(W, n, bits, out, scales, zeros, s)
+                     : launch_rtn_f16<TPG, false>(W, n, bits, out, scales, zeros, s);
+}
+
 // Any group size: one thread per group.
 template <typename T>
 __global__ void rtn_generic_kernel(const T* __restrict__ W, int64_t n_groups, int group_size,
@@ -142,7 +361,16 @@ template <typename T>
 static gptq_status launch_rtn(const T* W, int64_t n, int group_size, int bits, uint8_t* out,
                               uint16_t* scales, uint16_t* zeros, cudaStream_t s) {
     const int sms = num_sms();
-    if (group_size % 8 == 0 && group_size <= 256 && (group_size & (group_size - 1)) == 0) {
+    const bool pow2 = (group_size & (group_size - 1)) == 0;
+    if (std::is_same<T, __half>::value && pow2 && group_size >= 32 && group_size <= 256 &&
+        n / rp::E < (int64_t(1) << 31) - 64) {
+        const __half* Wh = reinterpret_cast<const __half*>(W);
+        if (group_size == 32) GPTQ_TRY(launch_rtn_f16_bits<1>(Wh, n, bits, out, scales, zeros, s));
+        else if (group_size == 64) GPTQ_TRY(launch_rtn_f16_bits<2>(Wh, n, bits, out, scales, zeros, s));
+        else if (group_size == 128) GPTQ_TRY(launch_rtn_f16_bits<4>(Wh, n, bits, out, scales, zeros, s));
+        else GPTQ_TRY(launch_rtn_f16_bits<8>(Wh, n, bits, out, scales, zeros, s));
+        return GPTQ_OK;
+    } else if (group_size % 8 == 0 && group_size <= 256 && pow2) {
         // 16 weights per thread when the group allows it, else 8
         const int E = (group_size % 16 == 0) ? 16 : 8;
         const int64_t n_chunks = n / E;
