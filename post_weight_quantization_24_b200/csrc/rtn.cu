@@ -241,37 +241,36 @@ __global__ void __launch_bounds__(rp::THREADS, 3) rtn_f16_kernel(const __half* _
         }
         if (t >= n_chunks) continue;
         const QParams p = group_params_stream(mn, mx, maxq);
-        // u = w/scale + zero in one fma; every w lies inside the group's range, so u is in
-        // [-0.5, maxq + 0.5] up to 4.5e-5 (1/scale within 2^-23, one rounding in the fma).
-        // Adding 1.5 * 2^23 rounds u to the nearest integer (half to even) and leaves it in
-        // the low mantissa bits. The rounding is exact unless u is within 4.5e-5 of a
-        // half-integer; if any of the 32 is, the chunk is redone on the exact path. Otherwise
-        // every code is in [0, maxq], so no clamp is needed.
+        // m = fma(w, 1/scale, zero + 1.5 * 2^23): the product is exact inside the fma and the
+        // single rounding (ulp 1 at 1.5 * 2^23) rounds w/scale + zero to the nearest integer,
+        // half to even, leaving it in the low mantissa bits. Every w lies inside the group's
+        // range, so the rounded value is within 3.1e-5 of the exact w/scale + zero (1/scale is
+        // within 2^-23). A second fma gives the residual r = w/scale + zero - code; if every |r|
+        // stays 6e-5 clear of 1/2, every code is the exact rounding and lies in [0, maxq] (no
+        // clamp); otherwise the chunk is redone on the exact path.
         constexpr float kMagic = 12582912.0f;                  // 1.5 * 2^23
-        float kf[32];
-        uint32_t mb[32];
+        const float C = p.zero + kMagic;                         // exact: zero is an integer
+        float m[32];
         float dev = 0.0f;
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
             const float2 f = __half22float2(hp[i]);
-            const float u0 = fmaf(f.x, p.inv_scale, p.zero), u1 = fmaf(f.y, p.inv_scale, p.zero);
-            const float m0 = u0 + kMagic, m1 = u1 + kMagic;
-            kf[2 * i] = m0 - kMagic;
-            kf[2 * i + 1] = m1 - kMagic;
-            mb[2 * i] = __float_as_uint(m0);
-            mb[2 * i + 1] = __float_as_uint(m1);
-            dev = fmaxf(dev, fmaxf(fabsf(u0 - kf[2 * i]), fabsf(u1 - kf[2 * i + 1])));
+            m[2 * i] = fmaf(f.x, p.inv_scale, C);
+            m[2 * i + 1] = fmaf(f.y, p.inv_scale, C);
+            const float r0 = fmaf(f.x, p.inv_scale, C - m[2 * i]);      // C - m is exact
+            const float r1 = fmaf(f.y, p.inv_scale, C - m[2 * i + 1]);
+            dev = fmaxf(dev, fmaxf(fabsf(r0), fabsf(r1)));
         }
         if (dev > 0.5f - 6.0e-5f) {
-            // rare: a code within 4.5e-5 of a rounding boundary; redo the chunk on the exact path
+            // rare: a code within 6e-5 of a rounding boundary; redo the chunk on the exact path
             rtn_chunk_exact(reinterpret_cast<const __half*>(mine), p, bits, out, t);
         } else if (INT4) {
-            // byte b holds codes 2b (low nibble) and 2b+1: q0 + 16 q1 (exact), magic-added, has
-            // it in its low byte
+            // byte b holds codes 2b (low nibble) and 2b+1: (M + q0) + 16 q1 has q0 + 16 q1 in its
+            // low byte (exact: all values are integers below 2^24)
             uint32_t by[16];
 #pragma unroll
             for (int b = 0; b < 16; ++b)
-                by[b] = __float_as_uint(fmaf(kf[2 * b + 1], 16.0f, kf[2 * b]) + kMagic);
+                by[b] = __float_as_uint(fmaf(m[2 * b + 1] - kMagic, 16.0f, m[2 * b]));
             uint32_t word[4];
 #pragma unroll
             for (int w4 = 0; w4 < 4; ++w4)
@@ -283,8 +282,8 @@ __global__ void __launch_bounds__(rp::THREADS, 3) rtn_f16_kernel(const __half* _
             uint32_t word[8];
 #pragma unroll
             for (int w4 = 0; w4 < 8; ++w4)
-                word[w4] = __byte_perm(__byte_perm(mb[4 * w4], mb[4 * w4 + 1], 0x0040),
-                                       __byte_perm(mb[4 * w4 + 2], mb[4 * w4 + 3], 0x0040), 0x5410);
+                word[w4] = __byte_perm(__byte_perm(__float_as_uint(m[4 * w4]), __float_as_uint(m[4 * w4 + 1]), 0x0040),
+                                       __byte_perm(__float_as_uint(m[4 * w4 + 2]), __float_as_uint(m[4 * w4 + 3]), 0x0040), 0x5410);
             __stcs(reinterpret_cast<uint4*>(out) + 2 * t, make_uint4(word[0], word[1], word[2], word[3]));
             __stcs(reinterpret_cast<uint4*>(out) + 2 * t + 1, make_uint4(word[4], word[5], word[6], word[7]));
         }
