@@ -395,8 +395,8 @@ def run_ours(args):
                                            "(6.48e9 fp16 weights), outside the timed step")
 
     # the dominant kernel (largest stage) carries the roofline object
-    traffic, _ = ncu_traffic("hessian_tc_kernel_mlp_up_7b.md", "hessian.cu")
-    roof = {"kernel": "hessian_tc_kernel", "bound": "tensor", "achieved": hess_tf,
+    traffic, _ = ncu_traffic("hessian_pair_kernel_mlp_up_7b.md", "hessian.cu")
+    roof = {"kernel": "hessian_pair_kernel", "bound": "tensor", "achieved": hess_tf,
             "peak": tc_peak, "unit": "TFLOP/s", "frac": hess_tf / tc_peak,
             "traffic": traffic,
             "peak_note": "measured bf16 dense burst (fp16 MMA runs at the bf16 rate); of measured"
