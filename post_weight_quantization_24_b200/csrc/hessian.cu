@@ -64,7 +64,7 @@ constexpr int BM = 128;                             // rows per CTA
 constexpr int BNC = 128;                            // B columns loaded per CTA
 constexpr int BN = 256;                             // accumulator columns
 constexpr int BK = 64, STAGES = 6;
-constexpr int CHUNK_KB = 4;                         // k-blocks per tensor-core partial sum
+constexpr int CHUNK_KB = 8;                         // k-blocks per tensor-core partial sum
 constexpr int BOX_BYTES = 64 * BK * 2;              // 64 channels x 64 tokens fp16 = 8 KB
 constexpr int A_BYTES = BM * BK * 2;                // 16 KB
 constexpr int B_BYTES = BNC * BK * 2;               // 16 KB
@@ -273,7 +273,12 @@ __global__ void __launch_bounds__(hp2::THREADS, 1)
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&acc_empty[b]), 0));
+                if (lane == 0) {
+                    // the leader's barrier: a local arrive for the leader's warps, a cluster-scope
+                    // remote one for the peer's
+                    if (leader) mbar_arrive(&acc_empty[b]);
+                    else mbar_arrive_cluster(mapa_shared(smem_u32(&acc_empty[b]), 0));
+                }
             }
             if (stop) break;
             // unit complete: H[row][cols] += 2 * acc for this CTA's rows of the pair tile
