@@ -137,7 +137,7 @@ struct Workspace {
     float* Err;      // d_out x kSuperCols errors of the current super-block (tf32 hi part)
     float* ErrLo;    // d_out x kSuperCols (tf32 lo part)
     uint8_t* codes_p;// d_out x d_in codes in processing order
-    float* P;        // d x 128 panel scratch
+    float* P;        // d x 128: the column loop's images of U's diagonal blocks
     float* Dinv;     // ceil(d/128) x 128 x 128 inverses of the Cholesky diagonal blocks
     int* perm;
     int* invperm;
@@ -321,24 +321,20 @@ gptq_status gptq_quantize_layer(const void* W, int w_dtype, int d_out, int d_in,
     GPTQ_TRY(gather_h_launch(H, d_in, ws.perm, ws.st, 1, ws.A, status, s));
     GPTQ_TRY(gather_w_launch(W, w_dtype, d_out, d_in, ws.perm, ws.Wk, status, s));
     tm.end();
-    // ---- stage 1-2: U with U^T U = H_d^-1 ----
+    // ---- stage 1: U with U^T U = H_d^-1 (factor and inverse overlap on two streams) ----
     tm.begin(1);
-    GPTQ_TRY(cholesky_launch(ws.A, d_in, ws.Dinv, ws.P, status, s));
+    GPTQ_TRY(factor_inverse_launch(ws.A, d_in, ws.Dinv, ws.X, status, s));
     tm.end();
-    tm.begin(2);
-    GPTQ_TRY(trtri_reverse_launch(ws.A, d_in, ws.Dinv, ws.X, ws.P, status, s));
-    tm.end();
-    // ---- stage 3-4: column loop and lazy batch updates ----
+    // ---- stage 2: the forms of U that the column loop and the lazy updates read ----
     uint8_t* codes_p = act_order ? ws.codes_p : codes;
-    // the panel scratch and the block inverses are free after the triangular inverse: they
-    // take the column loop's images of U's diagonal blocks and 1/U_ii
-    tm.begin(3);
+    // the block inverses are free after the triangular inverse: they take 1/U_ii, and P the
+    // column loop's images of U's diagonal blocks
+    tm.begin(2);
     GPTQ_TRY(column_images_launch(ws.X, d_in, block_size, ws.P, ws.Dinv, s));
-    tm.end();
     // U as tf32 hi (in place) and lo (into the factor's buffer, free now) for the lazy updates
-    tm.begin(4);
     GPTQ_TRY(tcgemm_split_launch(ws.X, ws.X, ws.A, d_in, d_in, d_in, true, s));
     tm.end();
+    // ---- stage 3-4: column loop and lazy batch updates ----
     // Lazy batch updates on two levels: the errors of a super-block of whole blocks (about
     // kSuperCols columns) are kept; after each block only the rest of its super-block is
     // updated, and the columns beyond the super-block get one update per super-block. Every
@@ -409,8 +405,7 @@ gptq_status gptq_inverse_factor(const float* H, int d_in, float percdamp, int ac
     GPTQ_TRY(diag_stats_launch(H, d_in, static_cast<double>(percdamp), ws.st, s));
     GPTQ_TRY(act_order_launch(H, d_in, act_order, ws.perm, ws.invperm, s));
     GPTQ_TRY(gather_h_launch(H, d_in, ws.perm, ws.st, 1, ws.A, status, s));
-    GPTQ_TRY(cholesky_launch(ws.A, d_in, ws.Dinv, ws.P, status, s));
-    GPTQ_TRY(trtri_reverse_launch(ws.A, d_in, ws.Dinv, ws.X, ws.P, status, s));
+    GPTQ_TRY(factor_inverse_launch(ws.A, d_in, ws.Dinv, ws.X, status, s));
     GPTQ_CUDA_TRY(cudaMemcpyAsync(U, ws.X, static_cast<size_t>(d_in) * d_in * 4,
                                   cudaMemcpyDeviceToDevice, s));
     if (perm)

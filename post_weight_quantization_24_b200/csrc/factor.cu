@@ -12,6 +12,7 @@
 // U^T U = H_d^-1 (the unique upper Cholesky factor of the inverse). The permutation and the
 // reversal are folded into one gather of H.
 #include <algorithm>
+#include <mutex>
 
 #include "internal.cuh"
 #include "tcgemm.cuh"
@@ -345,59 +346,7 @@ __global__ void __launch_bounds__(pd::THREADS, 1) potrf_diag_kernel(float* __res
     potrf_inverse_phase<16>(w, 7, i, nbc, Lsh, rs, Dinv);
 }
 
-__global__ void copy2d_kernel(const float* __restrict__ src, int lds, float* __restrict__ dst,
-                              int ldd, int rows, int cols4) {
-    const int c = blockIdx.x * blockDim.x + threadIdx.x;
-    const int r = blockIdx.y;
-    if (r < rows && c < cols4)
-        reinterpret_cast<float4*>(dst + static_cast<int64_t>(r) * ldd)[c] =
-            reinterpret_cast<const float4*>(src + static_cast<int64_t>(r) * lds)[c];
-}
-
-static gptq_status copy2d(const float* src, int lds, float* dst, int ldd, int rows, int cols,
-                          cudaStream_t s) {
-    if (rows <= 0 || cols <= 0) return GPTQ_OK;
-    const int cols4 = cols / 4;
-    const dim3 grid((cols4 + 127) / 128, rows);
-    copy2d_kernel<<<grid, 128, 0, s>>>(src, lds, dst, ldd, rows, cols4);
-    GPTQ_LAUNCHED();
-    return GPTQ_OK;
-}
-
 static int g_potrf_smem = 0;
-
-gptq_status cholesky_launch(float* A, int d, float* Dinv, float* P, int* status, cudaStream_t s) {
-    const int nb = kCholBlock;
-    static_assert(kCholBlock == pd::NB, "diagonal-block kernel is written for 128-wide panels");
-    const int smem = pd::SMEM;
-    if (g_potrf_smem != smem) {
-        GPTQ_CUDA_TRY(cudaFuncSetAttribute(potrf_diag_kernel,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
-        g_potrf_smem = smem;
-    }
-    const int nbl = (d + nb - 1) / nb;
-    for (int m = 0; m < nbl; ++m) {
-        const int k0 = m * nb, nbc = std::min(nb, d - k0);
-        float* Dm = Dinv + static_cast<int64_t>(m) * nb * nb;
-        potrf_diag_kernel<<<1, pd::THREADS, smem, s>>>(A, d, k0, nbc, Dm, status);
-        GPTQ_LAUNCHED();
-        const int rem = d - k0 - nbc;
-        if (rem <= 0) continue;
-        float* A21 = A + static_cast<int64_t>(k0 + nbc) * d + k0;
-        TcGemmArgs t{};  // P = A21 * Dinv_m^T
-        t.M = rem; t.N = nbc; t.K = nbc; t.alpha = 1.f; t.beta = 0.f;
-        t.A = A21; t.lda = d; t.B = Dm; t.ldb = nb; t.C = P; t.ldc = nb; t.status = status;
-        GPTQ_TRY(tcgemm_launch(t, true, TC_EPI_STORE, true, true, s));
-        GPTQ_TRY(copy2d(P, nb, A21, d, rem, nbc, s));
-        TcGemmArgs u{};  // A22 -= P P^T (lower tiles)
-        u.M = rem; u.N = rem; u.K = nbc; u.alpha = -1.f; u.beta = 1.f;
-        u.A = P; u.lda = nb; u.B = P; u.ldb = nb;
-        u.C = A + static_cast<int64_t>(k0 + nbc) * d + (k0 + nbc); u.ldc = d;
-        u.lower_only = 1; u.status = status;
-        GPTQ_TRY(tcgemm_launch(u, true, TC_EPI_STORE, true, true, s));
-    }
-    return GPTQ_OK;
-}
 
 // ---------------------------------------------------------------------------------------
 // triangular inverse and reversal
@@ -418,35 +367,141 @@ __global__ void reverse_inplace_kernel(float* X, int64_t half) {
     }
 }
 
-gptq_status trtri_reverse_launch(const float* A, int d, const float* Dinv, float* X, float* P,
-                                 int* status, cudaStream_t s) {
-    const int nb = kCholBlock;
-    GPTQ_CUDA_TRY(cudaMemsetAsync(X, 0, static_cast<size_t>(d) * d * 4, s));
-    set_identity_kernel<<<(d + 255) / 256, 256, 0, s>>>(X, d);
-    GPTQ_LAUNCHED();
-    const int nbl = (d + nb - 1) / nb;
-    for (int m = 0; m < nbl; ++m) {
-        const int k0 = m * nb, nbc = std::min(nb, d - k0), ncol = k0 + nbc;
-        const float* Dm = Dinv + static_cast<int64_t>(m) * nb * nb;
-        TcGemmArgs t{};  // P = Dinv_m * X[k0:k0+nbc, 0:ncol]
-        t.M = nbc; t.N = ncol; t.K = nbc; t.alpha = 1.f; t.beta = 0.f;
-        t.A = Dm; t.lda = nb; t.B = X + static_cast<int64_t>(k0) * d; t.ldb = d;
-        t.C = P; t.ldc = d; t.status = status;
-        GPTQ_TRY(tcgemm_launch(t, false, TC_EPI_STORE, true, true, s));
-        GPTQ_TRY(copy2d(P, d, X + static_cast<int64_t>(k0) * d, d, nbc, ncol, s));
-        const int rem = d - ncol;
-        if (rem <= 0) continue;
-        TcGemmArgs u{};  // X[ncol:, 0:ncol] -= L[ncol:, k0:ncol] * X[k0:ncol, 0:ncol]
-        u.M = rem; u.N = ncol; u.K = nbc; u.alpha = -1.f; u.beta = 1.f;
-        u.A = A + static_cast<int64_t>(ncol) * d + k0; u.lda = d;
-        u.B = X + static_cast<int64_t>(k0) * d; u.ldb = d;
-        u.C = X + static_cast<int64_t>(ncol) * d; u.ldc = d; u.status = status;
-        GPTQ_TRY(tcgemm_launch(u, false, TC_EPI_STORE, true, true, s));
+// ---------------------------------------------------------------------------------------
+// factor and inverse on two streams
+// ---------------------------------------------------------------------------------------
+// Per device: a second stream and the events that order the two streams. The enqueue of one
+// factorisation holds the mutex, so the events are never recorded by two sequences at once.
+namespace {
+struct SideStreams {
+    cudaStream_t side = nullptr;
+    cudaEvent_t fork = nullptr, trsm = nullptr, rest = nullptr, join = nullptr;
+};
+constexpr int kMaxDevices = 64;
+SideStreams g_side[kMaxDevices];
+std::mutex g_side_mu;
+
+gptq_status side_streams(SideStreams** out) {
+    int dev = 0;
+    GPTQ_CUDA_TRY(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= kMaxDevices) return GPTQ_ERR_UNSUPPORTED;
+    SideStreams& ss = g_side[dev];
+    if (!ss.side) {
+        GPTQ_CUDA_TRY(cudaStreamCreateWithFlags(&ss.side, cudaStreamNonBlocking));
+        for (cudaEvent_t* e : {&ss.fork, &ss.trsm, &ss.rest, &ss.join})
+            GPTQ_CUDA_TRY(cudaEventCreateWithFlags(e, cudaEventDisableTiming));
     }
-    const int64_t half = static_cast<int64_t>(d) * d / 2;
-    const int blocks = static_cast<int>(std::min<int64_t>((half + 255) / 256, num_sms() * 16));
-    reverse_inplace_kernel<<<blocks, 256, 0, s>>>(X, half);
-    GPTQ_LAUNCHED();
+    *out = &ss;
+    return GPTQ_OK;
+}
+}  // namespace
+
+// Blocked right-looking Cholesky of A with one step of lookahead, and the blocked triangular
+// inverse X = L^-1, then U = reverse(X).
+//
+// Main stream, panel m (columns k0 .. e-1, e = k0 + nbc; rem = d - e rows below):
+//   diag(m)   L11 and its inverse Dinv_m (one CTA)
+//   trsm(m)   L21 = A21 Dinv_m^T, in place (each output tile is the input tile it reads)
+//   next(m)   the trailing update of panel m+1's columns only: A[e:, e:e+128] -= L21 L21^T
+// Side stream, after trsm(m):
+//   rest(m)   the rest of the trailing update: A[e+128:, e+128:] -= L21' L21'^T (lower tiles)
+//   inv(m)    X[k0:e, 0:e] = Dinv_m X[k0:e, 0:e] (in place), X[e:, 0:e] -= L21 X[k0:e, 0:e]
+// next(m) waits for rest(m-1), the only other writer of its columns; diag(m+1) and trsm(m+1)
+// need only next(m), so rest(m) and inv(m) overlap them. The side stream's GEMMs leave as many
+// SMs free as the main stream's kernels of the next panel have CTAs (one, or one per 128 rows
+// below it; at most half the GPU), so the chain of diagonal blocks does not wait for an SM.
+gptq_status factor_inverse_launch(float* A, int d, float* Dinv, float* X, int* status,
+                                  cudaStream_t s) {
+    const int nb = kCholBlock;
+    static_assert(kCholBlock == pd::NB, "diagonal-block kernel is written for 128-wide panels");
+    const int smem = pd::SMEM;
+    if (g_potrf_smem != smem) {
+        GPTQ_CUDA_TRY(cudaFuncSetAttribute(potrf_diag_kernel,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+        g_potrf_smem = smem;
+    }
+    std::lock_guard<std::mutex> lock(g_side_mu);
+    SideStreams* ss = nullptr;
+    GPTQ_TRY(side_streams(&ss));
+    cudaStream_t t2 = ss->side;
+    const int sms = num_sms();
+
+    GPTQ_CUDA_TRY(cudaEventRecord(ss->fork, s));
+    GPTQ_CUDA_TRY(cudaStreamWaitEvent(t2, ss->fork, 0));
+    // Everything below is enqueued on both streams; on an error the side stream is joined
+    // back before returning, so a capture of `s` stays well formed.
+    auto body = [&]() -> gptq_status {
+        GPTQ_CUDA_TRY(cudaMemsetAsync(X, 0, static_cast<size_t>(d) * d * 4, t2));
+        set_identity_kernel<<<(d + 255) / 256, 256, 0, t2>>>(X, d);
+        GPTQ_LAUNCHED();
+        const int nbl = (d + nb - 1) / nb;
+        for (int m = 0; m < nbl; ++m) {
+            const int k0 = m * nb, nbc = std::min(nb, d - k0), e = k0 + nbc, rem = d - e;
+            float* Dm = Dinv + static_cast<int64_t>(m) * nb * nb;
+            float* A21 = A + static_cast<int64_t>(e) * d + k0;
+            // SMs kept free for the main stream while this panel's side work runs: diag(m+1)
+            // takes one, trsm(m+1) and next(m+1) one per 128 rows below panel m+1
+            const int reserve = std::min(sms / 2, std::max(1, (rem + nb - 1) / nb));
+            const int side_ctas = std::max(1, sms - reserve);
+            potrf_diag_kernel<<<1, pd::THREADS, smem, s>>>(A, d, k0, nbc, Dm, status);
+            GPTQ_LAUNCHED();
+            if (rem > 0) {
+                TcGemmArgs t{};  // A21 = A21 * Dinv_m^T
+                t.M = rem; t.N = nbc; t.K = nbc; t.alpha = 1.f; t.beta = 0.f;
+                t.A = A21; t.lda = d; t.B = Dm; t.ldb = nb; t.C = A21; t.ldc = d;
+                t.status = status;
+                GPTQ_TRY(tcgemm_launch(t, true, TC_EPI_STORE, true, true, s));
+                GPTQ_CUDA_TRY(cudaEventRecord(ss->trsm, s));
+                // next(m) after rest(m-1): the event's last record is still rest(m-1)'s
+                if (m > 0) GPTQ_CUDA_TRY(cudaStreamWaitEvent(s, ss->rest, 0));
+                TcGemmArgs u{};  // A[e:, e:e+128] -= A21 A21[0:128]^T
+                u.M = rem; u.N = std::min(nb, rem); u.K = nbc; u.alpha = -1.f; u.beta = 1.f;
+                u.A = A21; u.lda = d; u.B = A21; u.ldb = d;
+                u.C = A + static_cast<int64_t>(e) * d + e; u.ldc = d;
+                u.lower_only = 1; u.status = status;
+                GPTQ_TRY(tcgemm_launch(u, true, TC_EPI_STORE, true, true, s));
+                GPTQ_CUDA_TRY(cudaStreamWaitEvent(t2, ss->trsm, 0));
+                if (rem > nb) {
+                    const float* A21r = A21 + static_cast<int64_t>(nb) * d;
+                    TcGemmArgs r{};  // A[e+128:, e+128:] -= A21' A21'^T (lower tiles)
+                    r.M = rem - nb; r.N = rem - nb; r.K = nbc; r.alpha = -1.f; r.beta = 1.f;
+                    r.A = A21r; r.lda = d; r.B = A21r; r.ldb = d;
+                    r.C = A + static_cast<int64_t>(e + nb) * d + (e + nb); r.ldc = d;
+                    r.lower_only = 1; r.status = status; r.max_ctas = side_ctas;
+                    GPTQ_TRY(tcgemm_launch(r, true, TC_EPI_STORE, true, true, t2));
+                }
+                GPTQ_CUDA_TRY(cudaEventRecord(ss->rest, t2));
+            } else {
+                GPTQ_CUDA_TRY(cudaEventRecord(ss->trsm, s));
+                GPTQ_CUDA_TRY(cudaStreamWaitEvent(t2, ss->trsm, 0));
+            }
+            float* Xk = X + static_cast<int64_t>(k0) * d;
+            TcGemmArgs v{};  // X[k0:e, 0:e] = Dinv_m * X[k0:e, 0:e], in place
+            v.M = nbc; v.N = e; v.K = nbc; v.alpha = 1.f; v.beta = 0.f;
+            v.A = Dm; v.lda = nb; v.B = Xk; v.ldb = d; v.C = Xk; v.ldc = d;
+            v.status = status; v.max_ctas = side_ctas;
+            GPTQ_TRY(tcgemm_launch(v, false, TC_EPI_STORE, true, true, t2));
+            if (rem > 0) {
+                TcGemmArgs w{};  // X[e:, 0:e] -= L21 * X[k0:e, 0:e]
+                w.M = rem; w.N = e; w.K = nbc; w.alpha = -1.f; w.beta = 1.f;
+                w.A = A21; w.lda = d; w.B = Xk; w.ldb = d;
+                w.C = X + static_cast<int64_t>(e) * d; w.ldc = d;
+                w.status = status; w.max_ctas = side_ctas;
+                GPTQ_TRY(tcgemm_launch(w, false, TC_EPI_STORE, true, true, t2));
+            }
+        }
+        const int64_t half = static_cast<int64_t>(d) * d / 2;
+        const int blocks =
+            static_cast<int>(std::min<int64_t>((half + 255) / 256, num_sms() * 16));
+        reverse_inplace_kernel<<<blocks, 256, 0, t2>>>(X, half);
+        GPTQ_LAUNCHED();
+        return GPTQ_OK;
+    };
+    const gptq_status rc = body();
+    const cudaError_t e1 = cudaEventRecord(ss->join, t2);
+    const cudaError_t e2 = cudaStreamWaitEvent(s, ss->join, 0);
+    if (rc != GPTQ_OK) return rc;
+    if (e1 != cudaSuccess || e2 != cudaSuccess) return GPTQ_ERR_CUDA;
     return GPTQ_OK;
 }
 

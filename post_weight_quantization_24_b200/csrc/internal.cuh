@@ -40,12 +40,11 @@ gptq_status gather_h_launch(const float* H, int d, const int* perm, const DevSta
                             int reversed, float* A, int* status, cudaStream_t s);
 gptq_status gather_w_launch(const void* W, int w_dtype, int d_out, int d_in, const int* perm,
                             float* Wk, int* status, cudaStream_t s);
-// In-place lower Cholesky of A (lda = d); writes the inverses of the diagonal blocks to Dinv
-// (ceil(d/nb) blocks of nb x nb, row-major, zero above the diagonal). P: d*nb floats scratch.
-gptq_status cholesky_launch(float* A, int d, float* Dinv, float* P, int* status, cudaStream_t s);
-// X = L^-1 (lower) from the factor in A and Dinv; then U = reverse(X) in place in X.
-gptq_status trtri_reverse_launch(const float* A, int d, const float* Dinv, float* X, float* P,
-                                 int* status, cudaStream_t s);
+// In-place lower Cholesky factor L of A (lda = d), the inverses of its diagonal blocks in Dinv
+// (ceil(d/nb) blocks of nb x nb, row-major, zero above the diagonal), and U = reverse(L^-1) in
+// X. Uses a second stream of its own, forked from and joined back to s.
+gptq_status factor_inverse_launch(float* A, int d, float* Dinv, float* X, int* status,
+                                  cudaStream_t s);
 
 // gptq.cu
 // Per-row images of U's diagonal blocks for the column loop: img [d x 128],

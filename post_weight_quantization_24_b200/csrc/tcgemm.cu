@@ -463,7 +463,9 @@ static TcParams make_params(const TcGemmArgs& a, int& grid) {
     p.n_tiles = static_cast<long long>(n_bands) * tg::BAND * p.n_nt;
     long long useful = static_cast<long long>(p.n_mt) * p.n_nt;
     if (a.lower_only) useful = useful / 2 + p.n_mt;
-    grid = static_cast<int>(std::max<long long>(1, std::min<long long>(useful, num_sms())));
+    long long cap = num_sms();
+    if (a.max_ctas > 0) cap = std::min<long long>(cap, a.max_ctas);
+    grid = static_cast<int>(std::max<long long>(1, std::min<long long>(useful, cap)));
     return p;
 }
 

@@ -34,6 +34,7 @@ struct TcGemmArgs {
     // B_lo the lo parts, with the layouts and strides of A and B.
     const float* A_lo;
     const float* B_lo;
+    int max_ctas;     // > 0: launch at most this many CTAs (leaves SMs to concurrent work)
 };
 
 // split_a / split_b: represent that operand as hi + lo tf32 parts (an operand that is already

@@ -28,7 +28,7 @@ STATUS = {0: "GPTQ_OK", -1: "GPTQ_ERR_ARG", -2: "GPTQ_ERR_NOT_PD", -3: "GPTQ_ERR
           -4: "GPTQ_ERR_CUDA", -5: "GPTQ_ERR_OOM", -6: "GPTQ_ERR_TIMEOUT",
           -7: "GPTQ_ERR_WORKSPACE", -8: "GPTQ_ERR_UNSUPPORTED"}
 DTYPE_F16, DTYPE_F32 = 0, 1
-STAGES = ("prepare", "cholesky", "trtri", "column_loop", "lazy_update", "assemble", "loss")
+STAGES = ("prepare", "factor", "images", "column_loop", "lazy_update", "assemble", "loss")
 
 
 class GPTQError(RuntimeError):
