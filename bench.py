@@ -170,26 +170,30 @@ class ClockSampler:
 # ------------------------------------------------------------------------------------------
 # the committed ncu summary of the dominant kernel (traffic is null if the kernel changed)
 # ------------------------------------------------------------------------------------------
+def code_sha(source_file: str) -> str:
+    """sha256 of a kernel source with comments and blank lines removed: an edit of comments
+    alone leaves it unchanged, any edit of the code changes it."""
+    src = os.path.join(ROOT, "post_weight_quantization_24_b200", "csrc", source_file)
+    text = re.sub(r"/\*.*?\*/", "", open(src).read(), flags=re.S)
+    lines = [ln.split("//", 1)[0].rstrip() for ln in text.splitlines()]
+    return hashlib.sha256("\n".join(ln for ln in lines if ln).encode()).hexdigest()
+
+
 def ncu_traffic(summary_name: str, source_file: str):
+    """DRAM bytes per full-size launch from a committed ncu summary, or None when the summary is
+    missing or the kernel's code has changed since its capture."""
     path = os.path.join(ROOT, "profiles", summary_name)
     try:
         text = open(path).read()
     except OSError:
         return None, None
-    m_h = re.search(r"kernel_source_sha256:\s*([0-9a-f]{64})", text)
+    m_h = re.search(r"kernel_code_sha256:\s*([0-9a-f]{64})", text)
     m_b = re.search(r"dram_bytes_per_launch_full_size:\s*([0-9.eE+]+)", text)
     if not (m_h and m_b):
         return None, path
-    src = os.path.join(ROOT, "post_weight_quantization_24_b200", "csrc", source_file)
-    cur = hashlib.sha256(open(src, "rb").read()).hexdigest()
-    if cur != m_h.group(1):
+    if code_sha(source_file) != m_h.group(1):
         return None, path
     return float(m_b.group(1)), path
-
-
-def source_sha(source_file: str) -> str:
-    src = os.path.join(ROOT, "post_weight_quantization_24_b200", "csrc", source_file)
-    return hashlib.sha256(open(src, "rb").read()).hexdigest()
 
 
 # ------------------------------------------------------------------------------------------

@@ -15,15 +15,16 @@
 //     columns (2 boxes) into a 6-stage ring;
 //   * warp 1: TMEM allocation in both CTAs; in the leader CTA the single-thread issuer of
 //     4 x tcgen05.mma.cta_group::2 (M256 N256 K16, fp16 in, fp32 accumulate) per k-block into
-//     one of two 256-column TMEM accumulators, switching every CHUNK_KB k-blocks (256 tokens);
+//     one of two 256-column TMEM accumulators, switching every CHUNK_KB k-blocks (512 tokens);
 //   * warps 2-17 of each CTA: promotion epilogue - each warp owns 32 of its CTA's rows x 64
-//     columns in 64 fp32 registers per thread. When a 256-token chunk is complete it reads its
+//     columns in 64 fp32 registers per thread. When a 512-token chunk is complete it reads its
 //     slice from TMEM (tcgen05.ld) and adds it to the registers, then hands the accumulator
 //     back. At the end of a unit it adds 2x the registers into H with vector atomics (fp32 add
 //     in L2), so token slices of the same tile and successive calls accumulate in place.
 // Why promote: the tensor cores' fp32 accumulation truncates, so a long accumulation drifts
-// low (about -4e-5 relative over 8192 tokens, measured on B200); 256-token partial sums keep
-// that drift near 1e-6 and the register sums round to nearest.
+// low (about -4e-5 relative over 8192 tokens, measured on B200); 512-token partial sums keep
+// that drift near 2e-6 over 262144 tokens (1024-token sums: 5e-6) and the register sums round
+// to nearest.
 // Every mbarrier wait is bounded; on timeout the kernel records GPTQ_ERR_TIMEOUT, drains its
 // own copies and MMAs, frees TMEM and returns.
 #include <algorithm>
@@ -50,7 +51,7 @@ struct HessianParams {
 // instead of the 48 KB a single-CTA 128 x 256 tile needs for the same flops per SM. The
 // leader CTA (rank 0) issues M256 N256 K16 MMAs that read A by rows and B by columns from both
 // CTAs' shared memory; each CTA's TMEM receives its 128 rows x 256 columns, and each CTA's
-// warps promote and flush their own rows exactly as in the single-CTA kernel above.
+// warps promote and flush their own rows.
 // Synchronisation: both CTAs' TMA loads complete on the leader's stage barrier (the leader
 // expects both halves); the leader's MMA commits arrive, multicast, on the stage-free and
 // accumulator-full barriers of both CTAs; both CTAs' promotion warps release an accumulator on
