@@ -347,3 +347,134 @@ def test_mlp_down_7b_act_order(cuda_lib, mlp_down_inputs, bits):
         assert bad == 0 and sbad == 0, (bad, near, sbad)
         l_ref = oloss.recon_loss(Wn, ref["What"], Href)
         assert abs(out["loss"] - l_ref) <= 0.01 * l_ref, (out["loss"], l_ref)
+
+
+@pytest.mark.slow
+def test_full_size_attn_o_70b(cuda_lib):
+    """The 70B attention-output layer: W 8192x8192 fp16, X 65536x8192, INT4 g128 B128, all rows,
+    against the full fp64 oracle."""
+    wl = workloads.WORKLOADS["attn_o_70b"]
+    W = workloads.make_weights(wl, device="cuda")
+    X = workloads.make_activations(wl, device="cuda")
+    out, ref, Wn, Href = run_case(cuda_lib, W, X, wl.bits, wl.group_size, wl.block_size,
+                                  wl.act_order)
+    assert np.array_equal(out["perm"].cpu().numpy(), ref["perm"])
+    assert np.array_equal(out["g_idx"].cpu().numpy(), ref["g_idx"])
+    full_size_checks(out, ref, Wn, Href, wl.group_size, wl.bits)
+
+
+def recurrence_consistency_dev(W, H, out, g, bits, percdamp, rows, tie_tol=0.05):
+    """recurrence_consistency for layers whose d_in makes host fp64 linear algebra too slow: the
+    same replay, with the fp64 factorisation and the column steps run by torch on the device.
+    U is the upper Cholesky factor of the inverse of the damped, permuted H (here by the index
+    reversal: U = flip(chol_lower(flip(H_d))^-1), which satisfies U^T U = H_d^-1)."""
+    dev = H.device
+    maxq = 2 ** bits - 1
+    perm = out["perm"].to(dev).long()
+    d = perm.numel()
+    Hd = H.double()[perm][:, perm]
+    Hd.diagonal().add_(percdamp * torch.mean(torch.diagonal(Hd)))
+    L = torch.linalg.cholesky(torch.flip(Hd, [0, 1]))
+    del Hd
+    eye = torch.eye(d, dtype=torch.float64, device=dev)
+    U = torch.flip(torch.linalg.solve_triangular(L, eye, upper=False), [0, 1])
+    del L, eye
+    r = torch.as_tensor(rows, device=dev).long()
+    codes = out["codes"][r][:, perm].double()
+    sc = out["scales"][r].double()
+    zr = out["zeros"][r].double()
+    w = W[r].double()[:, perm].clone()
+    bad = near = sbad = 0
+    for q in range(d):
+        gi = q // g
+        if q % g == 0:
+            grp = w[:, q:q + g]
+            span = (torch.clamp(grp.max(1).values, min=0.0) - torch.clamp(grp.min(1).values, max=0.0))
+            s_ex = (span / maxq).cpu().numpy().astype(np.float16)
+            lo = np.nextafter(s_ex, np.float16(-np.inf)).astype(np.float64)
+            hi = np.nextafter(np.nextafter(s_ex, np.float16(np.inf)), np.float16(np.inf))
+            sgi = sc[:, gi].cpu().numpy()
+            sbad += int(np.sum((sgi < lo) | (sgi > hi.astype(np.float64))))
+        s, z = sc[:, gi], zr[:, gi]
+        t = w[:, q] / s
+        want = torch.clamp(torch.round(t) + z, 0, maxq)   # torch.round: half to even
+        mism = want != codes[:, q]
+        tie = torch.abs(torch.abs(t - torch.floor(t)) - 0.5) < tie_tol
+        bad += int(torch.sum(mism & ~tie))
+        near += int(torch.sum(mism & tie))
+        what = s * (codes[:, q] - z)
+        e = (w[:, q] - what) / U[q, q]
+        w[:, q + 1:] -= torch.outer(e, U[q, q + 1:])
+        w[:, q] = what
+    return bad, near, sbad
+
+
+@pytest.mark.slow
+def test_mlp_down_70b_sampled(cuda_lib, request):
+    """The 70B down projection: W 8192x28672 fp16, X 65536x28672 (3.8 GB), INT4 g128 B128. The
+    fp64 oracle is too slow for the whole layer in a test, so parity is checked on sampled
+    outputs and through properties that hold at any size:
+      * H against the oracle on its diagonal and on a sampled 96x96 block (1e-5 relative);
+      * every GPU decision on sampled rows is the rounding of its exactly compensated weight
+        (fp64 replay driven by the GPU's own decisions, on the GPU's H, which the first check
+        ties to the oracle);
+      * the loss the library reports equals tr(ΔHΔᵀ)/tr(WHWᵀ) on that H in fp64 within 1 %;
+      * RTN of the same W is bit-exact against the oracle."""
+    wl = workloads.WORKLOADS["mlp_down_70b"]
+    W = workloads.make_weights(wl, device="cuda")
+    X = workloads.make_activations(wl, device="cuda")
+    H = gpu_hessian(cuda_lib, X)
+    d = wl.d_in
+    # H: sampled block and diagonal against the oracle
+    Xc = X.cpu().numpy()
+    del X
+    rng = np.random.default_rng(0)
+    rows_h = np.sort(rng.choice(d, 96, replace=False))
+    cols_h = np.sort(rng.choice(d, 96, replace=False))
+    ref_blk = ohess.hessian_entries(Xc, rows_h, cols_h)
+    got_blk = H[torch.as_tensor(rows_h, device="cuda")][:, torch.as_tensor(cols_h, device="cuda")]
+    got_blk = got_blk.cpu().numpy().astype(np.float64)
+    ref_diag = np.empty(d)
+    for c0 in range(0, d, 1024):
+        x64 = Xc[:, c0:c0 + 1024].astype(np.float64)
+        ref_diag[c0:c0 + 1024] = 2.0 * np.einsum("ti,ti->i", x64, x64)
+    del Xc, x64
+    got_diag = torch.diagonal(H).cpu().numpy().astype(np.float64)
+
+    def rel_fro(a, b):
+        return float(np.linalg.norm(a - b) / np.linalg.norm(b))
+
+    log_parity(h_rel_fro_diag=rel_fro(got_diag, ref_diag), h_rel_fro_block=rel_fro(got_blk, ref_blk))
+    assert rel_fro(got_diag, ref_diag) <= 1e-5
+    assert rel_fro(got_blk, ref_blk) <= 1e-5
+
+    out = cuda_lib.quantize_layer(W, H, bits=wl.bits, group_size=wl.group_size,
+                                  block_size=wl.block_size, act_order=wl.act_order,
+                                  compute_loss=True)
+    torch.cuda.synchronize()
+    assert np.array_equal(out["perm"].cpu().numpy(), np.arange(d))
+    assert np.array_equal(out["g_idx"].cpu().numpy(), np.arange(d) // wl.group_size)
+    codes = out["codes"]
+    assert int(codes.max()) <= 2 ** wl.bits - 1
+    # the library's loss against tr(ΔHΔᵀ)/tr(WHWᵀ) in fp64 on the same H
+    gi = out["g_idx"].long()
+    What = out["scales"].double()[:, gi] * (codes.double() - out["zeros"].double()[:, gi])
+    W64, H64 = W.double(), H.double()
+    D = W64 - What
+    l64 = float(torch.sum((D @ H64) * D) / torch.sum((W64 @ H64) * W64))
+    del D, What, H64
+    log_parity(loss_lib=out["loss"], loss_fp64_same_h=l64)
+    assert abs(out["loss"] - l64) <= 0.01 * l64, (out["loss"], l64)
+    # replay on sampled rows
+    rows = np.sort(rng.choice(wl.d_out, 16, replace=False))
+    bad, near, sbad = recurrence_consistency_dev(W, H, out, wl.group_size, wl.bits, 0.01, rows)
+    log_parity(recurrence_bad=bad, recurrence_near=near, scale_bad=sbad)
+    assert bad == 0 and sbad == 0, (bad, near, sbad)
+    # RTN of the same weights, bit-exact
+    packed, scales, zeros = cuda_lib.rtn_minmax_quantize(W, wl.bits, wl.group_size)
+    torch.cuda.synchronize()
+    c_ref, s_ref, z_ref = ortn.rtn_minmax(W.float().cpu().numpy().astype(np.float64), wl.bits,
+                                          wl.group_size)
+    assert np.array_equal(ortn.unpack_int4(packed.cpu().numpy()), c_ref)
+    assert np.array_equal(scales.float().cpu().numpy().astype(np.float64), s_ref)
+    assert np.array_equal(zeros.float().cpu().numpy().astype(np.float64), z_ref)
