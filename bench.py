@@ -287,6 +287,57 @@ def rtn_stack_measure(gptq, device, reps: int = 3):
             "weights_per_s": n / (ms / 1e3), "launches": 2 * reps}
 
 
+def decoder_layer_measure(gptq, device, n_tokens: int = 131072, reps: int = 2):
+    """GPTQ over one 7B decoder layer: the Hessians of its four distinct inputs (attention in,
+    o_proj in, MLP in: 4096 channels; down_proj in: 11008) over 131072 tokens each, then INT4
+    g128 B128 GPTQ of its seven linears (q, k, v read one Hessian, gate and up another). Inputs,
+    weights and workspaces are resident; every quantize call synchronises once, as a user's
+    would. CUDA events bracket `reps` layers after one warm-up layer; a 32-layer stack takes
+    32 times as long."""
+    base = workloads.WORKLOADS["mlp_up_7b"]
+    inputs = {}
+    for idx, (name, d) in enumerate(workloads.DECODER_7B_INPUTS.items()):
+        wl = base.replace(name=name, d_in=d, n_tokens=n_tokens, seed=100 + idx)
+        inputs[name] = workloads.make_activations(wl, device=device)
+    linears = []
+    for idx, (name, d_out, d_in, src) in enumerate(workloads.DECODER_7B_LINEARS):
+        wl = base.replace(name=name, d_out=d_out, d_in=d_in, seed=200 + idx)
+        W = workloads.make_weights(wl, device=device)
+        ws = torch.empty(gptq.quantize_layer_workspace(d_out, d_in), dtype=torch.uint8,
+                         device=device)
+        linears.append((W, src, ws))
+    hs = {k: gptq.Hessian(X.shape[1]) for k, X in inputs.items()}
+
+    def layer():
+        for k, X in inputs.items():
+            hs[k].reset()
+            hs[k].accumulate(X)
+        raws = {k: h.raw() for k, h in hs.items()}
+        for W, src, ws in linears:
+            gptq.quantize_layer(W, raws[src], bits=4, group_size=128, block_size=128,
+                                workspace=ws)
+
+    layer()
+    torch.cuda.synchronize()
+    launches0 = gptq.launch_count()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        layer()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / reps
+    n_w = sum(d_out * d_in for _, d_out, d_in, _ in workloads.DECODER_7B_LINEARS)
+    out = {"ms": ms, "layers_per_s": 1e3 / ms, "weights": n_w, "weights_per_s": n_w / (ms / 1e3),
+           "tokens_per_input": n_tokens, "stack_32_layers_s": 32 * ms / 1e3,
+           "launches": (gptq.launch_count() - launches0) // reps,
+           "note": "one 7B decoder layer: 4 Hessians over 131072 tokens + GPTQ of 7 linears "
+                   "(INT4 g128 B128), outside the timed step"}
+    del inputs, linears, hs
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_ours(args):
     world, rank, local = dist_env()
     distributed = init_dist(world, local)
@@ -340,6 +391,12 @@ def run_ours(args):
             lib_stage_tot[k] += v
     gptq.profile_enable(False)
     rtn_stack = None if args.no_rtn_stack else rtn_stack_measure(gptq, device)
+    decoder = None
+    if not args.no_decoder_layer:
+        try:
+            decoder = decoder_layer_measure(gptq, device)
+        except Exception as exc:                      # reported in the line, never fatal
+            decoder = {"error": f"{type(exc).__name__}: {exc}"[:300]}
 
     K = args.steps
     total_ms_max = max_over_ranks(total_ms, distributed, device)
@@ -387,8 +444,9 @@ def run_ours(args):
         "factor": stage(lib_ms["factor"], "tensor", chol_flops + trtri_flops, tf32_peak / 3,
                         tf32x3 + "; Cholesky and triangular inverse, overlapped on two streams"),
         "images": {"ms": lib_ms["images"]},
-        "column_loop": stage(lib_ms["column_loop"], "alu", col_flops, fp32_peak_tf,
-                             f"FFMA 148 SM x 128 lanes x 2 at the sampled {clock_mhz:.0f} MHz"),
+        "column_loop": dict(stage(lib_ms["column_loop"], "alu", col_flops, fp32_peak_tf,
+                                  f"FFMA 148 SM x 128 lanes x 2 at the sampled {clock_mhz:.0f} MHz"),
+                            us_per_column_step=lib_ms["column_loop"] * 1e3 / d),
         "lazy_update": stage(lib_ms["lazy_update"], "tensor", lazy_flops, tf32_peak / 3, tf32x3),
         "assemble": {"ms": lib_ms["assemble"]},
         "loss": stage(lib_ms["loss"], "tensor", loss_flops,
@@ -400,6 +458,8 @@ def run_ours(args):
                 "note": "one call on this layer's W (90 MB, inside L2) right after a synchronising "
                         "call: includes the host submission gap; see rtn_7b_stack"},
     }
+    if decoder is not None:
+        stages["gptq_7b_decoder_layer"] = decoder
     if rtn_stack is not None:
         stages["rtn_7b_stack"] = dict(rtn_stack, bound="hbm",
                                       frac=rtn_stack["gbs"] / peaks["hbm_gbs"],
@@ -414,7 +474,8 @@ def run_ours(args):
             "peak_note": "measured bf16 dense burst (fp16 MMA runs at the bf16 rate); of measured"
             if peaks["source"] == "measured" else "fallback"}
     # (the 7B-stack RTN measurement runs outside the step and does not compete)
-    dom = max((k for k in stages if k != "rtn_7b_stack" and ("frac" in stages[k] or k == "hessian")),
+    dom = max((k for k in stages if k not in ("rtn_7b_stack", "gptq_7b_decoder_layer")
+               and ("frac" in stages[k] or k == "hessian")),
               key=lambda k: stages[k]["ms"])
     if dom != "hessian":
         roof = {"kernel": dom, "bound": stages[dom]["bound"],
@@ -630,6 +691,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-rtn-stack", action="store_true",
                     help="skip the RTN measurement over a 7B decoder stack (13 GB of weights)")
+    ap.add_argument("--no-decoder-layer", action="store_true",
+                    help="skip the GPTQ measurement over one 7B decoder layer (about 10 GB)")
     ap.add_argument("--ncu-case", choices=("hessian", "gptq", "rtn"),
                     help="run one small case for an ncu capture and exit (no JSON line)")
     args = ap.parse_args(argv)
