@@ -24,6 +24,12 @@
  *     them. No call allocates device memory except gptq_hessian_create.
  *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream). Work is
  *     ordered on it. Calls are not thread-safe on the same handle or workspace.
+ *   - gptq_quantize_layer and gptq_inverse_factor also run part of the factorisation on a
+ *     second stream that the library owns (one per device). It is forked from `stream` and
+ *     joined back to it by events inside the call, so the call stays ordered on `stream`.
+ *   - One process drives one GPU. The library sets its kernels' shared-memory limits once per
+ *     process, on the device current at the first call; a process that switches devices
+ *     between calls is not supported (launches on the second device fail with CUDA).
  *   - Argument errors are detected on the host before any launch and return GPTQ_ERR_ARG.
  *   - fp16 values are passed as their 16-bit patterns (uint16_t).
  *   - The library runs only on sm_100 devices; elsewhere calls return GPTQ_ERR_UNSUPPORTED.
