@@ -145,7 +145,7 @@ def adjacent_level(out, ref, g):
 def full_size_checks(out, ref, Wn, Href, g, bits, percdamp=0.01, n_rows=48, rows=None):
     """Parity for full-size layers.
 
-    Spec tolerances: >= 99 % identical codes; loss within 1 %; every mismatch one level
+    Target tolerances: >= 99 % identical codes; loss within 1 %; every mismatch one level
     (read as: the reconstructed weight lies within 1.5 oracle steps, which is exactly +-1 code
     where both sides use the same group grid).
     At full size GPTQ's greedy chain makes a few entries cascade: one legitimate near-tie flip
