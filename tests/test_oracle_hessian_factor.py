@@ -83,3 +83,31 @@ def test_upper_factor_residual_and_routes_agree(d, n):
     assert np.max(np.abs(R)) <= 1e-9
     U2 = factor.upper_chol_of_inverse_reversed(Hd)
     assert np.max(np.abs(U - U2)) <= 1e-10 * np.max(np.abs(U))
+
+
+@pytest.mark.parametrize("act_order", [False, True])
+def test_prepare_u_is_the_upper_factor_of_the_damped_ordered_inverse(act_order):
+    """The (perm, U) pair the GPU's inverse factor is compared with: perm is the processing
+    order (identity, or diag(H) descending with ties by lower index), and U is the unique upper
+    triangular factor with a positive diagonal of (P H P + lambda I)^-1, lambda = 0.01 mean(diag H)."""
+    from oracle import gptq as og
+    rng = np.random.default_rng(11)
+    X = rng.standard_normal((300, 24)) * np.exp(rng.standard_normal(24))
+    X[:, 5] = X[:, 9]                      # a tie on the diagonal and a rank-deficient pair
+    H = 2.0 * X.T @ X
+    perm, U = og.prepare_u(H, 0.01, act_order)
+    d = H.shape[0]
+    diag = np.diag(H)
+    if act_order:
+        assert sorted(perm.tolist()) == list(range(d))
+        dp = diag[perm]
+        assert np.all(np.diff(dp) <= 0)
+        for a in range(d - 1):             # equal keys keep index order
+            if dp[a] == dp[a + 1]:
+                assert perm[a] < perm[a + 1]
+        assert list(perm).index(5) < list(perm).index(9)
+    else:
+        assert np.array_equal(perm, np.arange(d))
+    assert np.array_equal(U, np.triu(U)) and np.all(np.diag(U) > 0)
+    Hd = H[np.ix_(perm, perm)] + 0.01 * np.mean(diag) * np.eye(d)
+    assert np.max(np.abs(U.T @ U @ Hd - np.eye(d))) <= 1e-9
