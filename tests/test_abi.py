@@ -94,3 +94,28 @@ def test_workspace_sizes(L):
                   + r256(nbl * 128 * 128 * 4) + 2 * r256(d_in * 4))
         assert L.gptq_quantize_layer_workspace(d_out, d_in, 128) == expect
     assert L.gptq_quantize_layer_workspace(0, 512, 128) == 0
+
+
+def test_missing_library_fails_loudly(monkeypatch):
+    """No silent fallback: without the built library every entry point raises."""
+    from post_weight_quantization_24_b200 import gptq
+    monkeypatch.setattr(gptq, "LIB_PATH", os.path.join(ROOT, "no_such_dir", "libgptq_b200.so"))
+    monkeypatch.setattr(gptq, "_lib", None)
+    with pytest.raises(RuntimeError, match="not built"):
+        gptq.lib()
+    with pytest.raises(RuntimeError, match="not built"):
+        gptq.quantize_layer_workspace(16, 128)
+
+
+def test_host_tensors_are_refused():
+    """The binding only marshals device tensors; host tensors raise instead of running on the CPU."""
+    import torch
+    from post_weight_quantization_24_b200 import gptq
+    W = torch.zeros(4, 128, dtype=torch.float16)
+    H = torch.eye(128)
+    with pytest.raises(ValueError, match="CUDA"):
+        gptq.rtn_minmax_quantize(W, 4, 32)
+    with pytest.raises(ValueError, match="CUDA"):
+        gptq.quantize_layer(W, H, bits=4, group_size=32)
+    with pytest.raises(ValueError, match="CUDA"):
+        gptq.quantize_layer_noalloc(W, H, bits=4, group_size=32)
