@@ -102,7 +102,7 @@ gptq_status gptq_hessian_destroy(gptq_hessian* h);
 
 /* Handle-free form: H (device fp32 [d_in x d_in], caller-owned, 16-byte aligned, row stride
  * d_in) += 2 * X^T X on its upper triangle (tiles that straddle the diagonal also update some
- * entries below it). The tensor cores accumulate at most 256 tokens at a time; those partial
+ * entries below it). The tensor cores accumulate at most 512 tokens at a time; those partial
  * sums are added in fp32 with round-to-nearest, and each work unit adds its sum into H with
  * atomic fp32 adds (so the low bits of H depend on the order units finish). `unit_tokens`
  * sets the tokens per work unit (0 = chosen to balance the SMs; otherwise a multiple of 64).
@@ -158,8 +158,10 @@ gptq_status gptq_quantize_layer(const void* W, int w_dtype, int d_out, int d_in,
  * allocate device memory when they quantize: runtimes that reserved almost all of the GPU for
  * their own pools at start-up, and deployments that forbid device allocation after
  * initialisation. Such callers cannot supply a workspace either. The scratch is a fixed
- * 32 MiB device array inside the library, reserved on every GPU that loads the library and
- * held until the process exits.
+ * 32 MiB device array inside the library, held until the process exits. It takes device
+ * memory when the library's device code is loaded onto a GPU; under CUDA's lazy module loading
+ * (the default) that happens at this entry point's first call on each device, so a caller
+ * that reserves its memory pools at start-up should make one call before reserving them.
  *   - Layers whose gptq_quantize_layer_workspace(d_out, d_in, block_size) exceeds 32 MiB are
  *     rejected with GPTQ_ERR_WORKSPACE before anything is launched. For example, d_in = 1024
  *     fits up to d_out = 2615 and d_in = 512 up to d_out = 4646; d_in = 4096 does not fit.
@@ -218,6 +220,18 @@ int gptq_profile_read(float* ms_out, int max_stages);
 
 /* Total number of kernels this library has launched in the process (all entry points). */
 unsigned long long gptq_launch_count(void);
+
+/* ------------------------------------------------------------------------------------------
+ * Test hook for the bounded-wait path (no counterpart on the pages). Every device-side wait of
+ * the library gives up after a cycle limit and makes the call return GPTQ_ERR_TIMEOUT instead
+ * of hanging. With on != 0, the factorisation's diagonal-block kernel first waits on an
+ * mbarrier that nothing arrives at, with a limit of about 1 ms, so the next
+ * gptq_quantize_layer / gptq_inverse_factor on the current device returns GPTQ_ERR_TIMEOUT;
+ * the kernels after it skip their work on the status word and the CUDA context stays usable.
+ * on = 0 restores normal operation. The switch is per device (current device) and process-wide;
+ * it is for tests only. Errors: CUDA, UNSUPPORTED.
+ * ------------------------------------------------------------------------------------------ */
+gptq_status gptq_test_stall_factor(int on);
 
 #ifdef __cplusplus
 }

@@ -25,13 +25,22 @@ class NotPositiveDefinite(ArithmeticError):
     pass
 
 
-def damp(H, percdamp):
-    """Return (H + λI, λ) with λ = percdamp · mean(diag H)."""
+def damping(H, percdamp):
+    """λ = percdamp · mean(diag H); NotPositiveDefinite unless it is positive and finite."""
     H = np.asarray(H, dtype=np.float64)
     lam = float(percdamp) * float(np.mean(np.diag(H)))
     if not np.isfinite(lam) or lam <= 0.0:
         raise NotPositiveDefinite(f"damping term lambda={lam!r} is not positive")
-    return H + lam * np.eye(H.shape[0]), lam
+    return lam
+
+
+def damp(H, percdamp):
+    """Return (H + λI, λ) with λ = percdamp · mean(diag H) (λ added to each diagonal entry)."""
+    H = np.asarray(H, dtype=np.float64)
+    lam = damping(H, percdamp)
+    Hd = H.copy()
+    Hd[np.diag_indices(H.shape[0])] += lam
+    return Hd, lam
 
 
 def upper_chol_of_inverse(Hd):

@@ -35,7 +35,7 @@ Rows of W are independent given H, so both accept ``rows`` to run a subset of ro
 
 import numpy as np
 
-from .factor import damp, upper_chol_of_inverse
+from .factor import damp, damping, upper_chol_of_inverse, upper_chol_of_inverse_reversed
 from .quantizer import group_params, quantize, dequantize
 
 
@@ -45,15 +45,19 @@ def act_order_perm(H):
     return np.argsort(-diag, kind="stable")
 
 
-def _prepare(W, H, percdamp, act_order, rows):
+def _prepare(W, H, percdamp, act_order, rows, need_hd=True):
+    """Rows of W, W in the processing order, the order, and (when asked for) the damped
+    Hessian in that order; λ always (it does not depend on the order)."""
     W = np.asarray(W, dtype=np.float64)
     H = np.asarray(H, dtype=np.float64)
     if rows is not None:
         W = W[np.asarray(rows)]
     d_in = H.shape[0]
     perm = act_order_perm(H) if act_order else np.arange(d_in)
-    Hp = H[np.ix_(perm, perm)]
-    Hd, lam = damp(Hp, percdamp)
+    if need_hd:
+        Hd, lam = damp(H[np.ix_(perm, perm)], percdamp)
+    else:
+        Hd, lam = None, damping(H, percdamp)
     return W, W[:, perm].copy(), perm, Hd, lam
 
 
@@ -107,16 +111,21 @@ def gptq_obs_ref(W, H, bits, group_size, percdamp=0.01, act_order=False, rows=No
 
 
 def gptq_blocked_ref(W, H, bits, group_size, block_size=128, percdamp=0.01, act_order=False,
-                     rows=None, U=None):
+                     rows=None, U=None, trace=False):
     """Blocked reference with lazy batch updates, driven by U (UᵀU = H_d⁻¹).
 
     ``U`` may be passed in when it was already computed by ``prepare_u`` for the same
     (H, percdamp, act_order); rows of W are processed independently either way.
+
+    With ``trace`` the result also holds the values each rounding decision was taken on, in
+    the processing order: ``pre`` [d_out, d_in], the compensated weight of every column just
+    before it is quantized; ``step`` and ``zquot`` [d_out, d_in/g], each group's unrounded
+    step (max − min)/maxq and zero quotient −min/scale (see ``quantizer.group_params``).
     """
     d_in = np.asarray(H).shape[0]
     _check_args(d_in, bits, group_size, block_size)
     maxq = 2 ** bits - 1
-    _, Wp, perm, Hd, lam = _prepare(W, H, percdamp, act_order, rows)
+    _, Wp, perm, Hd, lam = _prepare(W, H, percdamp, act_order, rows, need_hd=U is None)
     if U is None:
         U = upper_chol_of_inverse(Hd)
     d_out = Wp.shape[0]
@@ -124,16 +133,25 @@ def gptq_blocked_ref(W, H, bits, group_size, block_size=128, percdamp=0.01, act_
     What = np.zeros((d_out, d_in))
     scales = np.zeros((d_out, d_in // group_size))
     zeros = np.zeros((d_out, d_in // group_size))
+    if trace:
+        pre = np.zeros((d_out, d_in))
+        steps = np.zeros((d_out, d_in // group_size))
+        zquots = np.zeros((d_out, d_in // group_size))
     for j0 in range(0, d_in, block_size):
         j1 = min(j0 + block_size, d_in)
         Err = np.zeros((d_out, j1 - j0))
         for q in range(j0, j1):
             if q % group_size == 0:
                 grp = Wp[:, q:q + group_size]
-                s, z = group_params(grp.min(axis=1), grp.max(axis=1), maxq)
+                s, z, step, zquot = group_params(grp.min(axis=1), grp.max(axis=1), maxq,
+                                                 trace=True)
                 scales[:, q // group_size], zeros[:, q // group_size] = s, z
+                if trace:
+                    steps[:, q // group_size], zquots[:, q // group_size] = step, zquot
             s, z = scales[:, q // group_size], zeros[:, q // group_size]
             w = Wp[:, q].copy()
+            if trace:
+                pre[:, q] = w
             codes[:, q] = quantize(w, s, z, maxq)
             What[:, q] = dequantize(codes[:, q], s, z)
             err = (w - What[:, q]) / U[q, q]
@@ -143,12 +161,24 @@ def gptq_blocked_ref(W, H, bits, group_size, block_size=128, percdamp=0.01, act_
         Wp[:, j1:] -= Err @ U[j0:j1, j1:]          # lazy batch update of all later columns
     out = _assemble(codes, What, scales, zeros, perm, group_size)
     out["lam"] = lam
+    if trace:
+        out.update(pre=pre, step=steps, zquot=zquots, codes_p=codes)
     return out
 
 
-def prepare_u(H, percdamp=0.01, act_order=False):
-    """(perm, U) for a Hessian: the processing order and the factor the blocked loop uses."""
+def prepare_u(H, percdamp=0.01, act_order=False, route="textbook"):
+    """(perm, U) for a Hessian: the processing order and the factor the blocked loop uses.
+
+    ``route`` picks one of the two factorisations in ``factor`` (they agree to rounding, which
+    the oracle's tests check): "textbook" (Cholesky, explicit inverse, Cholesky again) or
+    "reversed" (one Cholesky of the index-reversed matrix and one triangular solve), the
+    cheaper one for the widest layers.
+    """
     H = np.asarray(H, dtype=np.float64)
     perm = act_order_perm(H) if act_order else np.arange(H.shape[0])
     Hd, _ = damp(H[np.ix_(perm, perm)], percdamp)
+    if route == "reversed":
+        return perm, upper_chol_of_inverse_reversed(Hd)
+    if route != "textbook":
+        raise ValueError(f"unknown route {route!r}")
     return perm, upper_chol_of_inverse(Hd)

@@ -39,19 +39,28 @@ def fp16_round_up(x):
     return h.astype(np.float64)
 
 
-def group_params(xmin, xmax, maxq):
+def group_params(xmin, xmax, maxq, trace=False):
     """(scale, zero) for groups with the given minima and maxima (fp64 arrays).
 
     The range [xmin, xmax] is first widened to contain 0. scale is fp16-representable (held
     in fp64), zero is an integer in [0, maxq] (held in fp64).
+
+    With ``trace`` the two quantities before their rounding come back as well: the unrounded
+    step (xmax - xmin)/maxq (before the round-up to fp16) and the zero quotient -xmin/scale
+    (before rint). They locate the group's rounding decisions: a scale whose unrounded step
+    sits on an fp16 value, or a zero whose quotient sits on a half-integer, is a tie.
     """
     xmin = np.minimum(np.asarray(xmin, dtype=np.float64), 0.0)
     xmax = np.maximum(np.asarray(xmax, dtype=np.float64), 0.0)
     span = xmax - xmin
     with np.errstate(divide="ignore", invalid="ignore"):
-        scale = fp16_round_up(span / maxq)
+        step = span / maxq
+        scale = fp16_round_up(step)
         scale = np.where(span == 0.0, 1.0, scale)
-        zero = np.rint(-xmin / scale) + 0.0
+        zquot = -xmin / scale
+        zero = np.rint(zquot) + 0.0
+    if trace:
+        return scale, zero, step, zquot
     return scale, zero
 
 

@@ -439,6 +439,11 @@ void gptq_profile_enable(int on) {
 
 unsigned long long gptq_launch_count(void) { return g_launches.load(); }
 
+gptq_status gptq_test_stall_factor(int on) {
+    GPTQ_TRY(check_device());
+    return factor_stall_set(on);
+}
+
 int gptq_profile_read(float* ms_out, int max_stages) {
     std::lock_guard<std::mutex> lock(g_prof.mu);
     const int n = max_stages < kStages ? max_stages : kStages;

@@ -81,14 +81,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Wait for the phase with the given parity to complete; false if the cycle limit ran out.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// Wait for the phase with the given parity to complete; false once `limit` cycles have passed.
+__device__ __forceinline__ bool mbar_wait_cycles(uint64_t* bar, uint32_t parity,
+                                                 long long limit) {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (!mbar_try_wait(bar, parity)) {
-        if (clock64() - t0 > kWaitLimitCycles) return false;
+        if (clock64() - t0 > limit) return false;
     }
     return true;
+}
+
+// Wait for the phase with the given parity to complete; false if the cycle limit ran out.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+    return mbar_wait_cycles(bar, parity, kWaitLimitCycles);
 }
 
 // ---------------------------------------------------------------------------------------

@@ -202,8 +202,17 @@ namespace pd {
 constexpr int NB = 128, THREADS = NB, PH = 16, NBUF = 3;
 constexpr int LS = NB + 4;          // Lsh row stride: Lsh[c][m - c + 3] = L[m][c], m >= c
 constexpr int CB = NB + 8;          // published column: cb[i - c + 3] = a_ic of step c
-constexpr int SMEM = (NB * LS + NBUF * CB + NB) * 4 + NBUF * 8;   // + rs[c], mbarriers
+// + rs[c]; NBUF exchange mbarriers and one that nothing arrives at (the stall test below)
+constexpr int SMEM = (NB * LS + NBUF * CB + NB) * 4 + (NBUF + 1) * 8;
+constexpr long long STALL_LIMIT_CYCLES = 2000000;   // about 1 ms
 }  // namespace pd
+
+// Test switch for the bounded-wait path (set by gptq_test_stall_factor): when nonzero, every
+// thread of the diagonal-block kernel first waits on an mbarrier that nothing arrives at. The
+// wait gives up after STALL_LIMIT_CYCLES, the kernel records GPTQ_ERR_TIMEOUT and returns, and
+// the rest of the factorisation skips its work on the status word. The kernel's barriers are
+// fed by its own threads' arrivals only; no copy or MMA is in flight when it gives up.
+__device__ int g_factor_stall = 0;
 
 __device__ __forceinline__ float rcp_approx(float x) {
     float r;
@@ -293,6 +302,7 @@ __global__ void __launch_bounds__(pd::THREADS, 1) potrf_diag_kernel(float* __res
         reinterpret_cast<float4*>(sm)[e] = make_float4(0.f, 0.f, 0.f, 0.f);
     if (i == 0) {
         for (int b = 0; b < pd::NBUF; ++b) mbar_init(&mb[b], pd::THREADS);
+        mbar_init(&mb[pd::NBUF], 1);
         fence_mbar_init();
     }
 
@@ -314,7 +324,9 @@ __global__ void __launch_bounds__(pd::THREADS, 1) potrf_diag_kernel(float* __res
     mbar_arrive(&mb[0]);
 
     bool bad = false;
-    bool ok = potrf_factor_phase<128>(w, 0, i, Lsh, cb, mb, rs, bad);
+    bool ok = true;
+    if (*(volatile int*)&g_factor_stall) ok = mbar_wait_cycles(&mb[pd::NBUF], 0, pd::STALL_LIMIT_CYCLES);
+    ok = ok && potrf_factor_phase<128>(w, 0, i, Lsh, cb, mb, rs, bad);
     ok = ok && potrf_factor_phase<112>(w, 1, i, Lsh, cb, mb, rs, bad);
     ok = ok && potrf_factor_phase<96>(w, 2, i, Lsh, cb, mb, rs, bad);
     ok = ok && potrf_factor_phase<80>(w, 3, i, Lsh, cb, mb, rs, bad);
@@ -347,6 +359,12 @@ __global__ void __launch_bounds__(pd::THREADS, 1) potrf_diag_kernel(float* __res
 }
 
 static int g_potrf_smem = 0;
+
+gptq_status factor_stall_set(int on) {
+    const int v = on ? 1 : 0;
+    GPTQ_CUDA_TRY(cudaMemcpyToSymbol(g_factor_stall, &v, sizeof(int)));
+    return GPTQ_OK;
+}
 
 // ---------------------------------------------------------------------------------------
 // triangular inverse and reversal

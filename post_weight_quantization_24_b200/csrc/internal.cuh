@@ -45,6 +45,8 @@ gptq_status gather_w_launch(const void* W, int w_dtype, int d_out, int d_in, con
 // X. Uses a second stream of its own, forked from and joined back to s.
 gptq_status factor_inverse_launch(float* A, int d, float* Dinv, float* X, int* status,
                                   cudaStream_t s);
+// Test switch: the diagonal-block kernel waits on a barrier nothing arrives at (bounded).
+gptq_status factor_stall_set(int on);
 
 // gptq.cu
 // Per-row images of U's diagonal blocks for the column loop: img [d x 128],

@@ -17,8 +17,12 @@
 
 namespace gq {
 
-// Largest workspace this entry point can serve: 32 MiB, held on every GPU that loads the
-// library until the process exits.
+// Largest workspace this entry point can serve: 32 MiB. The array is part of the library's
+// device code: it takes device memory when that code is loaded onto a GPU and keeps it until
+// the process exits. With CUDA's lazy module loading (the default) the load happens at the
+// first use on each device, which for this array is the address lookup in the first call of
+// gptq_quantize_layer_noalloc there; a caller that reserves its pools at start-up should make
+// that first call before reserving them.
 constexpr size_t kStaticScratchBytes = size_t(32) << 20;
 
 static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
@@ -36,7 +40,10 @@ static gptq_status static_scratch(void** out) {
     if (!g_scratch_addr[dev]) {
         void* p = nullptr;
         const cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
-        if (e != cudaSuccess || !p) return GPTQ_ERR_CUDA;
+        if (e != cudaSuccess || !p) {
+            cudaGetLastError();   // do not leave the failure for an unrelated later check
+            return GPTQ_ERR_CUDA;
+        }
         g_scratch_addr[dev] = p;
     }
     *out = g_scratch_addr[dev];

@@ -68,6 +68,7 @@ _SIGNATURES = {
     "gptq_profile_enable": ([_I], None),
     "gptq_profile_read": ([ctypes.POINTER(_F), _I], _I),
     "gptq_launch_count": ([], ctypes.c_ulonglong),
+    "gptq_test_stall_factor": ([_I], _I),
 }
 
 
@@ -325,6 +326,11 @@ def profile_read() -> dict:
 def launch_count() -> int:
     """Kernels launched by the library so far in this process."""
     return int(lib().gptq_launch_count())
+
+
+def test_stall_factor(on: bool) -> None:
+    """Test hook: make the factorisation's bounded wait run out (see include/gptq.h)."""
+    _check(lib().gptq_test_stall_factor(int(bool(on))), "gptq_test_stall_factor")
 
 
 def status_string(status: int) -> str:

@@ -69,3 +69,31 @@ def test_bad_arguments(cuda_lib):
         with pytest.raises(cuda_lib.GPTQError) as e:
             cuda_lib.quantize_layer(_w(), H, **kw)
         assert e.value.name == "GPTQ_ERR_ARG"
+
+
+def test_bounded_wait_gives_timeout_and_the_library_recovers(cuda_lib):
+    """The factorisation's diagonal-block kernel is switched to wait on an mbarrier that nothing
+    arrives at. Its bounded wait gives up after about 1 ms: the call returns GPTQ_ERR_TIMEOUT
+    (no hang, no fault), and with the switch off again the next call succeeds and matches a
+    call made before the stall."""
+    X = workloads.make_activations(workloads.WORKLOADS["linear_512"].replace(d_in=256),
+                                   device="cuda", n_tokens=2048, d_in=256)
+    h = cuda_lib.Hessian(256)
+    h.accumulate(X)
+    H = h.get()
+    W = _w()
+    before = cuda_lib.quantize_layer(W, H, compute_loss=True)
+    codes_before = before["codes"].clone()
+    cuda_lib.test_stall_factor(True)
+    try:
+        with pytest.raises(cuda_lib.GPTQError) as e:
+            cuda_lib.inverse_factor(H)
+        assert e.value.name == "GPTQ_ERR_TIMEOUT"
+        with pytest.raises(cuda_lib.GPTQError) as e:
+            cuda_lib.quantize_layer(W, H)
+        assert e.value.name == "GPTQ_ERR_TIMEOUT"
+    finally:
+        cuda_lib.test_stall_factor(False)
+    after = cuda_lib.quantize_layer(W, H, compute_loss=True)
+    assert torch.equal(after["codes"], codes_before)
+    assert torch.equal(after["scales"], before["scales"])

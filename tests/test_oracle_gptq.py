@@ -86,6 +86,51 @@ def test_least_squares_resolve_closed_form(act_order, seed):
             assert abs(What[r, q] - quantizer.dequantize(code, s, z)) == 0.0
 
 
+@pytest.mark.parametrize("act_order", [False, True])
+def test_trace_values_are_the_least_squares_resolve(act_order):
+    """The traced pre-rounding weight of every column equals the closed-form LS re-solve given
+    the earlier quantized columns, and the traced group quantities are the ones the scale and
+    zero are rounded from: fp16 round-up of the step, rint of the zero quotient, the group's
+    widened range."""
+    d, g, bits = 24, 8, 3
+    maxq = 2 ** bits - 1
+    X, H = _hessian(80, d, 31, correlated=True)
+    W = _weights(5, d, 7)
+    out = gptq.gptq_blocked_ref(W, H, bits, g, block_size=16, act_order=act_order, trace=True)
+    perm = out["perm"]
+    Hd, _ = factor.damp(H[np.ix_(perm, perm)], 0.01)
+    W0 = W[:, perm]
+    What = out["What"][:, perm]
+    for r in range(W.shape[0]):
+        for q in range(d):
+            Q, R = np.arange(q), np.arange(q, d)
+            wR = W0[r, R] - np.linalg.solve(Hd[np.ix_(R, R)], Hd[np.ix_(R, Q)] @ (What[r, Q] - W0[r, Q]))
+            assert abs(out["pre"][r, q] - wR[0]) <= 1e-9 * np.max(np.abs(W))
+            if q % g == 0:
+                lo, hi = min(wR[:g].min(), 0.0), max(wR[:g].max(), 0.0)
+                assert out["step"][r, q // g] == pytest.approx((hi - lo) / maxq, rel=1e-9)
+                assert out["zquot"][r, q // g] == pytest.approx(-lo / out["scales"][r, q // g],
+                                                                rel=1e-9, abs=1e-12)
+    assert np.array_equal(out["scales"], quantizer.fp16_round_up(out["step"]))
+    assert np.array_equal(out["zeros"], np.rint(out["zquot"]))
+    assert np.array_equal(out["codes_p"], out["codes"][:, perm])
+
+
+def test_factorisation_routes_drive_the_same_gptq():
+    """prepare_u's two routes give U within rounding of each other, and the GPTQ outputs they
+    drive are identical on a layer with no near ties."""
+    X, H = _hessian(500, 96, 41)
+    W = _weights(40, 96, 8)
+    _, U1 = gptq.prepare_u(H, 0.01, True, route="textbook")
+    _, U2 = gptq.prepare_u(H, 0.01, True, route="reversed")
+    assert np.max(np.abs(U1 - U2)) <= 1e-10 * np.max(np.abs(U1))
+    a = gptq.gptq_blocked_ref(W, H, 4, 32, act_order=True, U=U1)
+    b = gptq.gptq_blocked_ref(W, H, 4, 32, act_order=True, U=U2)
+    assert np.array_equal(a["codes"], b["codes"]) and np.array_equal(a["scales"], b["scales"])
+    with pytest.raises(ValueError):
+        gptq.prepare_u(H, route="other")
+
+
 def test_single_column_update_closed_form():
     d = 9
     X, H = _hessian(50, d, 21, correlated=True)
