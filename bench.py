@@ -287,55 +287,212 @@ def rtn_stack_measure(gptq, device, reps: int = 3):
             "weights_per_s": n / (ms / 1e3), "launches": 2 * reps}
 
 
-def decoder_layer_measure(gptq, device, n_tokens: int = 131072, reps: int = 2):
-    """GPTQ over one 7B decoder layer: the Hessians of its four distinct inputs (attention in,
-    o_proj in, MLP in: 4096 channels; down_proj in: 11008) over 131072 tokens each, then INT4
-    g128 B128 GPTQ of its seven linears (q, k, v read one Hessian, gate and up another). Inputs,
-    weights and workspaces are resident; every quantize call synchronises once, as a user's
-    would. CUDA events bracket `reps` layers after one warm-up layer; a 32-layer stack takes
-    32 times as long."""
-    base = workloads.WORKLOADS["mlp_up_7b"]
-    inputs = {}
-    for idx, (name, d) in enumerate(workloads.DECODER_7B_INPUTS.items()):
-        wl = base.replace(name=name, d_in=d, n_tokens=n_tokens, seed=100 + idx)
-        inputs[name] = workloads.make_activations(wl, device=device)
-    linears = []
-    for idx, (name, d_out, d_in, src) in enumerate(workloads.DECODER_7B_LINEARS):
-        wl = base.replace(name=name, d_out=d_out, d_in=d_in, seed=200 + idx)
-        W = workloads.make_weights(wl, device=device)
-        ws = torch.empty(gptq.quantize_layer_workspace(d_out, d_in), dtype=torch.uint8,
-                         device=device)
-        linears.append((W, src, ws))
-    hs = {k: gptq.Hessian(X.shape[1]) for k, X in inputs.items()}
+def gptq_flops(d_out: int, d: int, B: int, w_f16: bool = True) -> dict:
+    """Algorithmic flops of one quantize_layer call, per stage (symmetric Hessian work is
+    counted once; the loss denominator is the Gram matrix on the fp16 path)."""
+    return {"factor": 2.0 * d ** 3 / 3.0,
+            "column_loop": float(d_out) * d * B,
+            "lazy_update": 2.0 * d_out * sum(B * max(0, d - j0 - B) for j0 in range(0, d, B)),
+            "loss": float(d_out) * d * (d + 1) if w_f16 else 2.0 * d_out * d * d}
 
-    def layer():
-        for k, X in inputs.items():
-            hs[k].reset()
-            hs[k].accumulate(X)
-        raws = {k: h.raw() for k, h in hs.items()}
-        for W, src, ws in linears:
-            gptq.quantize_layer(W, raws[src], bits=4, group_size=128, block_size=128,
-                                workspace=ws)
 
-    layer()
+def peaks_for(peaks, clock_mhz):
+    tc = peaks["bf16_tflops"]                            # fp16 MMA runs at the bf16 rate
+    return {"tensor": tc, "tf32x3": tc * TF32_PER_BF16 / 3.0,
+            "ffma": N_SM * FP32_LANES_PER_SM * 2 * clock_mhz * 1e6 / 1e12}
+
+
+def stage_entry(ms, bound, flops=None, peak=None, note=None):
+    out = {"ms": ms, "bound": bound}
+    if flops is not None and ms > 0:
+        out["tflops"] = flops / (ms / 1e3) / 1e12
+        out["peak_tflops"] = peak
+        out["frac"] = out["tflops"] / peak
+    if note:
+        out["peak_note"] = note
+    return out
+
+
+TF32X3_NOTE = f"tf32 = {TF32_PER_BF16} x measured bf16, / 3 MMA passes (3xTF32)"
+
+
+def gptq_stage_table(hess_flops, hess_ms, lib_ms, fl, pk, clock_mhz, w_f16=True, n_tokens=None,
+                     d=None):
+    """Per-stage times and roofline fractions of one layer (or a sum of layers)."""
+    st = {
+        "hessian": stage_entry(hess_ms, "tensor", hess_flops, pk["tensor"],
+                               "measured bf16 dense burst"),
+        "prepare": {"ms": lib_ms["prepare"]},
+        "factor": stage_entry(lib_ms["factor"], "tensor", fl["factor"], pk["tf32x3"],
+                              TF32X3_NOTE + "; Cholesky and triangular inverse, two streams"),
+        "images": {"ms": lib_ms["images"]},
+        "column_loop": stage_entry(lib_ms["column_loop"], "alu", fl["column_loop"], pk["ffma"],
+                                   f"FFMA 148 SM x 128 lanes x 2 at the sampled {clock_mhz:.0f} MHz"),
+        "lazy_update": stage_entry(lib_ms["lazy_update"], "tensor", fl["lazy_update"],
+                                   pk["tf32x3"], TF32X3_NOTE),
+        "assemble": {"ms": lib_ms["assemble"]},
+        "loss": stage_entry(lib_ms["loss"], "tensor", fl["loss"],
+                            pk["tensor"] if w_f16 else pk["tf32x3"],
+                            "Gram matrix on the fp16 path; measured bf16 dense burst" if w_f16
+                            else TF32X3_NOTE),
+    }
+    if n_tokens is not None and hess_ms > 0:
+        st["hessian"]["calib_tokens_per_s"] = n_tokens / (hess_ms / 1e3)
+    if d is not None and lib_ms["column_loop"] > 0:
+        st["column_loop"]["us_per_column_step"] = lib_ms["column_loop"] * 1e3 / d
+    return st
+
+
+def measure_config(gptq, wl, device, flush, steps, warmup, peaks, clock_mhz):
+    """One timed line for a layer workload: the same step as the headline (Hessian, GPTQ with
+    loss, RTN of the same W), with its per-stage roofline fractions."""
+    step = LayerStep(gptq, wl, device)
+    gptq.profile_enable(False)
+    for _ in range(warmup):
+        step.run()
     torch.cuda.synchronize()
-    launches0 = gptq.launch_count()
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record()
-    for _ in range(reps):
-        layer()
-    b.record()
-    torch.cuda.synchronize()
-    ms = a.elapsed_time(b) / reps
-    n_w = sum(d_out * d_in for _, d_out, d_in, _ in workloads.DECODER_7B_LINEARS)
-    out = {"ms": ms, "layers_per_s": 1e3 / ms, "weights": n_w, "weights_per_s": n_w / (ms / 1e3),
-           "tokens_per_input": n_tokens, "stack_32_layers_s": 32 * ms / 1e3,
-           "launches": (gptq.launch_count() - launches0) // reps,
-           "note": "one 7B decoder layer: 4 Hessians over 131072 tokens + GPTQ of 7 linears "
-                   "(INT4 g128 B128), outside the timed step"}
-    del inputs, linears, hs
+    tot, stage_tot = 0.0, {k: 0.0 for k in ("hessian", "gptq", "rtn")}
+    for _ in range(steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        step.run(timed=True)
+        b.record()
+        torch.cuda.synchronize()
+        tot += a.elapsed_time(b)
+        for k, v in step.stage_ms().items():
+            stage_tot[k] += v
+    lib_tot = {k: 0.0 for k in gptq.STAGES}
+    gptq.profile_enable(True)
+    for _ in range(steps):
+        flush.zero_()
+        step.run()
+        torch.cuda.synchronize()
+        for k, v in gptq.profile_read().items():
+            lib_tot[k] += v
+    gptq.profile_enable(False)
+    ms = tot / steps
+    d, n, d_out = wl.d_in, wl.n_tokens, wl.d_out
+    pk = peaks_for(peaks, clock_mhz)
+    fl = gptq_flops(d_out, d, wl.block_size, wl.w_dtype == "f16")
+    hess_ms = stage_tot["hessian"] / steps
+    st = gptq_stage_table(float(n) * d * (d + 1), hess_ms, {k: v / steps for k, v in lib_tot.items()},
+                          fl, pk, clock_mhz, wl.w_dtype == "f16", n, d)
+    rtn_ms = stage_tot["rtn"] / steps
+    rtn_bytes = d_out * d * ((2 if wl.w_dtype == "f16" else 4) + (0.5 if wl.bits == 4 else 1.0)) \
+        + d_out * (d // wl.group_size) * 4
+    st["rtn"] = {"ms": rtn_ms, "bound": "hbm", "gbs": rtn_bytes / (rtn_ms / 1e3) / 1e9,
+                 "frac": rtn_bytes / (rtn_ms / 1e3) / 1e9 / peaks["hbm_gbs"]}
+    out = {"workload": f"{wl.name}: W {d_out}x{d} {wl.w_dtype}, X {n}x{d} fp16, INT{wl.bits} "
+                       f"g{wl.group_size} B{wl.block_size} act_order {wl.act_order}",
+           "steps": steps, "warmup": warmup, "ms_per_step": ms,
+           "weights_per_s": d_out * d / (ms / 1e3), "layers_per_s": 1e3 / ms,
+           "calib_tokens_per_s": n / (hess_ms / 1e3), "loss": step.loss,
+           "gptq_ms": stage_tot["gptq"] / steps, "stages": st}
+    del step
     torch.cuda.empty_cache()
     return out
+
+
+CONFIG_LINES = (("linear_512", {}), ("mlp_down_7b_int4", {"base": "mlp_down_7b", "bits": 4}),
+                ("mlp_down_7b_int3", {"base": "mlp_down_7b", "bits": 3}),
+                ("attn_o_70b", {}), ("mlp_down_70b", {}))
+
+
+def configs_measure(gptq, device, flush, peaks, clock_mhz, steps=3, warmup=3):
+    res = {}
+    for name, kw in CONFIG_LINES:
+        wl = workloads.WORKLOADS[kw.get("base", name)]
+        if "bits" in kw:
+            wl = wl.replace(bits=kw["bits"], name=name)
+        try:
+            res[name] = measure_config(gptq, wl, device, flush, steps, warmup, peaks, clock_mhz)
+        except Exception as exc:                      # reported in the line, never fatal
+            res[name] = {"error": f"{type(exc).__name__}: {exc}"[:300]}
+            torch.cuda.empty_cache()
+    return res
+
+
+def stack_measure(gptq, device, peaks, clock_mhz, n_layers=32, n_tokens=131072,
+                  variants=((128, False), (128, True), (64, False), (64, True))):
+    """GPTQ over a full 7B-shaped decoder stack, end to end: for each of `n_layers` layers,
+    fresh synthetic inputs (four distinct inputs of `n_tokens` tokens, the 7B activation recipe)
+    and fresh fp16 weights are generated, the four Hessians are accumulated, and the layer's
+    linears are quantized (INT4, B128, loss on), q;k;v and gate;up each in one call on their
+    row-stacked weights (rows are independent given the shared Hessian, so this is the same
+    result as separate calls with one factorisation instead of three or two). Every quantize
+    call synchronises once, as a user's would. Device time (CUDA events around the Hessians and
+    the quantize calls of each layer, input synthesis excluded) and host wall time (synthesis
+    included) are reported per variant, with per-stage times and roofline fractions summed over
+    the stack."""
+    hs = {k: gptq.Hessian(d) for k, d in workloads.DECODER_7B_INPUTS.items()}
+    shapes = []
+    for name, parts, d_in, src in workloads.DECODER_7B_FUSED:
+        rows = sum(d_out for n_, d_out, _, _ in workloads.DECODER_7B_LINEARS if n_ in parts)
+        shapes.append((name, rows, d_in, src))
+    ws = torch.empty(max(gptq.quantize_layer_workspace(r, d) for _, r, d, _ in shapes),
+                     dtype=torch.uint8, device=device)
+    pk = peaks_for(peaks, clock_mhz)
+    n_w = sum(r * d for _, r, d, _ in shapes)
+    res = {}
+    gptq.profile_enable(True)
+    try:
+        for g, ao in variants:
+            outs = {name: dict(codes=torch.empty(r, d, dtype=torch.uint8, device=device),
+                               scales=torch.empty(r, d // g, dtype=torch.float16, device=device),
+                               zeros=torch.empty(r, d // g, dtype=torch.float16, device=device),
+                               g_idx=torch.empty(d, dtype=torch.int32, device=device),
+                               perm=torch.empty(d, dtype=torch.int32, device=device))
+                    for name, r, d, _ in shapes}
+            lib_ms = {k: 0.0 for k in gptq.STAGES}
+            hess_ms = dev_ms = 0.0
+            losses = {name: [] for name, _, _, _ in shapes}
+            launches0 = gptq.launch_count()
+            torch.cuda.synchronize()
+            wall0 = time.perf_counter()
+            for layer in range(n_layers):
+                inputs, fused = workloads.make_decoder_layer(layer, n_tokens, device=device)
+                a, b, c = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+                a.record()
+                for k, X in inputs.items():
+                    hs[k].reset()
+                    hs[k].accumulate(X)
+                b.record()
+                for name, W, src in fused:
+                    r = gptq.quantize_layer(W, hs[src].raw(), bits=4, group_size=g,
+                                            block_size=128, act_order=ao, compute_loss=True,
+                                            workspace=ws, out=outs[name])
+                    losses[name].append(r["loss"])
+                    for k, v in gptq.profile_read().items():
+                        lib_ms[k] += v
+                c.record()
+                torch.cuda.synchronize()
+                hess_ms += a.elapsed_time(b)
+                dev_ms += a.elapsed_time(c)
+                del inputs, fused
+            wall_s = time.perf_counter() - wall0
+            hess_flops = n_layers * sum(float(n_tokens) * d * (d + 1)
+                                        for d in workloads.DECODER_7B_INPUTS.values())
+            fl = {k: 0.0 for k in ("factor", "column_loop", "lazy_update", "loss")}
+            for _, r, d, _ in shapes:
+                for k, v in gptq_flops(r, d, 128).items():
+                    fl[k] += n_layers * v
+            st = gptq_stage_table(hess_flops, hess_ms, lib_ms, fl, pk, clock_mhz,
+                                  n_tokens=4 * n_layers * n_tokens)
+            res[f"g{g}_act_order_{'on' if ao else 'off'}"] = {
+                "layers": n_layers, "tokens_per_input": n_tokens, "weights": n_layers * n_w,
+                "device_s": dev_ms / 1e3, "wall_s": wall_s,
+                "layers_per_s": n_layers / (dev_ms / 1e3),
+                "weights_per_s": n_layers * n_w / (dev_ms / 1e3),
+                "launches": gptq.launch_count() - launches0,
+                "mean_loss": {k: float(np.mean(v)) for k, v in losses.items()},
+                "stages": st}
+            del outs
+    finally:
+        gptq.profile_enable(False)
+        del hs, ws
+        torch.cuda.empty_cache()
+    return res
 
 
 def run_ours(args):
@@ -390,14 +547,6 @@ def run_ours(args):
         for k, v in gptq.profile_read().items():
             lib_stage_tot[k] += v
     gptq.profile_enable(False)
-    rtn_stack = None if args.no_rtn_stack else rtn_stack_measure(gptq, device)
-    decoder = None
-    if not args.no_decoder_layer:
-        try:
-            decoder = decoder_layer_measure(gptq, device)
-        except Exception as exc:                      # reported in the line, never fatal
-            decoder = {"error": f"{type(exc).__name__}: {exc}"[:300]}
-
     K = args.steps
     total_ms_max = max_over_ranks(total_ms, distributed, device)
     ms_per_step = total_ms_max / K
@@ -405,66 +554,44 @@ def run_ours(args):
     value = job_value(world, K, weights_per_step, total_ms_max)
 
     hess_ms = stage_tot["hessian"] / K
-    gptq_ms = stage_tot["gptq"] / K
     rtn_ms = stage_tot["rtn"] / K
     lib_ms = {k: v / K for k, v in lib_stage_tot.items()}
     d, n, d_out = wl.d_in, wl.n_tokens, wl.d_out
 
     # ---- per-stage roofline ----
     clock_mhz = (clocks or {}).get("sm_mhz") or peaks.get("clocks_under_load", {}).get("sm_mhz_median", 1312.0)
-    fp32_peak_tf = N_SM * FP32_LANES_PER_SM * 2 * clock_mhz * 1e6 / 1e12
-    tc_peak = peaks["bf16_tflops"]                       # fp16 MMA runs at the bf16 rate
-    tf32_peak = tc_peak * TF32_PER_BF16                  # nominal dense tf32 : bf16 ratio
+    pk = peaks_for(peaks, clock_mhz)
+    tc_peak = pk["tensor"]
     hess_flops = float(n) * d * (d + 1)                  # symmetric 2·XᵀX
     hess_tf = hess_flops / (hess_ms / 1e3) / 1e12
-    chol_flops = d ** 3 / 3.0
-    trtri_flops = d ** 3 / 3.0
-    col_flops = float(d_out) * d * wl.block_size         # d_out·d·B/2 FMAs
-    lazy_flops = 2.0 * d_out * sum(wl.block_size * max(0, d - j0 - wl.block_size)
-                                   for j0 in range(0, d, wl.block_size))
     w_f16 = wl.w_dtype == "f16"
-    loss_flops = float(d_out) * d * (d + 1) if w_f16 else 2.0 * d_out * d * d
+    stages = gptq_stage_table(hess_flops, hess_ms, lib_ms, gptq_flops(d_out, d, wl.block_size, w_f16),
+                              pk, clock_mhz, w_f16, n, d)
     rtn_bytes = d_out * d * (2 + (0.5 if wl.bits == 4 else 1.0)) + d_out * (d // wl.group_size) * 4
+    stages["rtn"] = {"ms": rtn_ms, "bound": "hbm", "gbs": rtn_bytes / (rtn_ms / 1e3) / 1e9,
+                     "frac": rtn_bytes / (rtn_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+                     "note": "one call on this layer's W (90 MB, inside L2) right after a "
+                             "synchronising call: includes the host submission gap; see "
+                             "rtn_7b_stack"}
 
-    def stage(ms, bound, flops=None, peak=None, note=None):
-        out = {"ms": ms, "bound": bound}
-        if flops is not None and ms > 0:
-            out["tflops"] = flops / (ms / 1e3) / 1e12
-            out["peak_tflops"] = peak
-            out["frac"] = out["tflops"] / peak
-        if note:
-            out["peak_note"] = note
-        return out
-
-    tf32x3 = f"tf32 = {TF32_PER_BF16} x measured bf16, / 3 MMA passes (3xTF32)"
-    stages = {
-        "hessian": dict(stage(hess_ms, "tensor", hess_flops, tc_peak, "measured bf16 dense burst"),
-                        calib_tokens_per_s=n / (hess_ms / 1e3)),
-        "prepare": {"ms": lib_ms["prepare"]},
-        "factor": stage(lib_ms["factor"], "tensor", chol_flops + trtri_flops, tf32_peak / 3,
-                        tf32x3 + "; Cholesky and triangular inverse, overlapped on two streams"),
-        "images": {"ms": lib_ms["images"]},
-        "column_loop": dict(stage(lib_ms["column_loop"], "alu", col_flops, fp32_peak_tf,
-                                  f"FFMA 148 SM x 128 lanes x 2 at the sampled {clock_mhz:.0f} MHz"),
-                            us_per_column_step=lib_ms["column_loop"] * 1e3 / d),
-        "lazy_update": stage(lib_ms["lazy_update"], "tensor", lazy_flops, tf32_peak / 3, tf32x3),
-        "assemble": {"ms": lib_ms["assemble"]},
-        "loss": stage(lib_ms["loss"], "tensor", loss_flops,
-                      tc_peak if w_f16 else tf32_peak / 3,
-                      "Gram matrix WᵀW on the fp16 path; measured bf16 dense burst" if w_f16
-                      else tf32x3),
-        "rtn": {"ms": rtn_ms, "bound": "hbm", "gbs": rtn_bytes / (rtn_ms / 1e3) / 1e9,
-                "frac": rtn_bytes / (rtn_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
-                "note": "one call on this layer's W (90 MB, inside L2) right after a synchronising "
-                        "call: includes the host submission gap; see rtn_7b_stack"},
-    }
-    if decoder is not None:
-        stages["gptq_7b_decoder_layer"] = decoder
+    # ---- outside the timed steps (1 GPU only): RTN over a 7B stack, every config, the stack ----
+    extras = world == 1
+    rtn_stack = None if (args.no_rtn_stack or not extras) else rtn_stack_measure(gptq, device)
     if rtn_stack is not None:
         stages["rtn_7b_stack"] = dict(rtn_stack, bound="hbm",
                                       frac=rtn_stack["gbs"] / peaks["hbm_gbs"],
                                       note="INT4 g128 RTN over a 7B decoder stack's 224 matrices "
                                            "(6.48e9 fp16 weights), outside the timed step")
+    configs = None
+    if extras and not args.no_configs:
+        configs = configs_measure(gptq, device, flush, peaks, clock_mhz)
+    stack = None
+    if extras and not args.no_stack:
+        try:
+            stack = stack_measure(gptq, device, peaks, clock_mhz, n_layers=args.stack_layers)
+        except Exception as exc:                      # reported in the line, never fatal
+            stack = {"error": f"{type(exc).__name__}: {exc}"[:300]}
+            torch.cuda.empty_cache()
 
     # the dominant kernel (largest stage) carries the roofline object
     traffic, _ = ncu_traffic("hessian_pair_kernel_mlp_up_7b.md", "hessian.cu")
@@ -474,7 +601,7 @@ def run_ours(args):
             "peak_note": "measured bf16 dense burst (fp16 MMA runs at the bf16 rate); of measured"
             if peaks["source"] == "measured" else "fallback"}
     # (the 7B-stack RTN measurement runs outside the step and does not compete)
-    dom = max((k for k in stages if k not in ("rtn_7b_stack", "gptq_7b_decoder_layer")
+    dom = max((k for k in stages if k != "rtn_7b_stack"
                and ("frac" in stages[k] or k == "hessian")),
               key=lambda k: stages[k]["ms"])
     if dom != "hessian":
@@ -506,6 +633,8 @@ def run_ours(args):
         "calib_tokens_per_s": world * n / (hess_ms / 1e3),
         "layer_loss": step.loss,
         "stages": stages,
+        "configs": configs,
+        "stack_7b": stack,
         "roofline": roof,
         "clocks": clocks,
         "gpu_launches": launches,
@@ -691,8 +820,11 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-rtn-stack", action="store_true",
                     help="skip the RTN measurement over a 7B decoder stack (13 GB of weights)")
-    ap.add_argument("--no-decoder-layer", action="store_true",
-                    help="skip the GPTQ measurement over one 7B decoder layer (about 10 GB)")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the timed lines of the other layer workloads")
+    ap.add_argument("--no-stack", action="store_true",
+                    help="skip GPTQ over a full 7B decoder stack (4 variants)")
+    ap.add_argument("--stack-layers", type=int, default=32)
     ap.add_argument("--ncu-case", choices=("hessian", "gptq", "rtn"),
                     help="run one small case for an ncu capture and exit (no JSON line)")
     args = ap.parse_args(argv)

@@ -36,7 +36,7 @@ Rows of W are independent given H, so both accept ``rows`` to run a subset of ro
 import numpy as np
 
 from .factor import damp, damping, upper_chol_of_inverse, upper_chol_of_inverse_reversed
-from .quantizer import group_params, quantize, dequantize
+from .quantizer import group_params, group_params_sym, quantize, dequantize
 
 
 def act_order_perm(H):
@@ -61,14 +61,17 @@ def _prepare(W, H, percdamp, act_order, rows, need_hd=True):
     return W, W[:, perm].copy(), perm, Hd, lam
 
 
-def _assemble(codes_p, What_p, scales, zeros, perm, group_size):
+def _assemble(codes_p, What_p, scales, zeros, perm, group_size, static_groups=False):
     d_out, d_in = codes_p.shape
     codes = np.empty_like(codes_p)
     codes[:, perm] = codes_p
     What = np.empty_like(What_p)
     What[:, perm] = What_p
     g_idx = np.empty(d_in, dtype=np.int64)
-    g_idx[perm] = np.arange(d_in) // group_size
+    if static_groups:
+        g_idx[:] = np.arange(d_in) // group_size
+    else:
+        g_idx[perm] = np.arange(d_in) // group_size
     return dict(codes=codes, scales=scales, zeros=zeros, g_idx=g_idx, perm=perm, What=What)
 
 
@@ -77,28 +80,53 @@ def _check_args(d_in, bits, group_size, block_size=None):
         raise ValueError("bits must be in [2, 8]")
     if group_size <= 0 or d_in % group_size:
         raise ValueError("d_in must be a multiple of group_size")
-    if block_size is not None and (block_size <= 0 or block_size % group_size):
+    # one group per row (per-channel) has no group boundary inside a block
+    if block_size is not None and (block_size <= 0 or
+                                   (block_size % group_size and group_size != d_in)):
         raise ValueError("block_size must be a multiple of group_size")
 
 
-def gptq_obs_ref(W, H, bits, group_size, percdamp=0.01, act_order=False, rows=None):
-    """Unblocked reference: OBS update with the inverse over the remaining columns."""
+def _params_fn(sym):
+    return group_params_sym if sym else group_params
+
+
+def static_group_params(W0, bits, group_size, sym=False):
+    """Scale and zero of every group of the ORIGINAL weights in the original column order
+    (groups of ``group_size`` consecutive original columns), as static groups fix them before
+    any column is quantized. Returns fp64 arrays [rows, d_in/group_size]."""
+    W0 = np.asarray(W0, dtype=np.float64)
+    d_out, d_in = W0.shape
+    Wg = W0.reshape(d_out, d_in // group_size, group_size)
+    return _params_fn(sym)(Wg.min(axis=2), Wg.max(axis=2), 2 ** bits - 1)
+
+
+def gptq_obs_ref(W, H, bits, group_size, percdamp=0.01, act_order=False, rows=None,
+                 sym=False, static_groups=False):
+    """Unblocked reference: OBS update with the inverse over the remaining columns. The
+    quantizer variants are those of ``gptq_blocked_ref``."""
     d_in = np.asarray(H).shape[0]
     _check_args(d_in, bits, group_size)
     maxq = 2 ** bits - 1
     _, Wp, perm, Hd, _ = _prepare(W, H, percdamp, act_order, rows)
     d_out = Wp.shape[0]
+    params = _params_fn(sym)
     Hinv = np.linalg.inv(Hd)                       # inverse over F = all columns
     codes = np.zeros((d_out, d_in), dtype=np.int64)
     What = np.zeros((d_out, d_in))
-    scales = np.zeros((d_out, d_in // group_size))
-    zeros = np.zeros((d_out, d_in // group_size))
+    if static_groups:
+        scales, zeros = static_group_params(np.asarray(W, np.float64)[rows] if rows is not None
+                                            else W, bits, group_size, sym)
+        col_group = perm // group_size
+    else:
+        scales = np.zeros((d_out, d_in // group_size))
+        zeros = np.zeros((d_out, d_in // group_size))
+        col_group = np.arange(d_in) // group_size
     for q in range(d_in):
-        if q % group_size == 0:
+        if not static_groups and q % group_size == 0:
             grp = Wp[:, q:q + group_size]
-            s, z = group_params(grp.min(axis=1), grp.max(axis=1), maxq)
+            s, z = params(grp.min(axis=1), grp.max(axis=1), maxq)
             scales[:, q // group_size], zeros[:, q // group_size] = s, z
-        s, z = scales[:, q // group_size], zeros[:, q // group_size]
+        s, z = scales[:, col_group[q]], zeros[:, col_group[q]]
         w = Wp[:, q].copy()
         codes[:, q] = quantize(w, s, z, maxq)
         What[:, q] = dequantize(codes[:, q], s, z)
@@ -107,15 +135,22 @@ def gptq_obs_ref(W, H, bits, group_size, percdamp=0.01, act_order=False, rows=No
         Wp[:, q] = What[:, q]
         # remove column q from F: inverse of H restricted to F \ {q}
         Hinv = Hinv - np.outer(Hinv[:, q], Hinv[q, :]) / Hinv[q, q]
-    return _assemble(codes, What, scales, zeros, perm, group_size)
+    return _assemble(codes, What, scales, zeros, perm, group_size, static_groups)
 
 
 def gptq_blocked_ref(W, H, bits, group_size, block_size=128, percdamp=0.01, act_order=False,
-                     rows=None, U=None, trace=False):
+                     rows=None, U=None, trace=False, sym=False, static_groups=False):
     """Blocked reference with lazy batch updates, driven by U (UᵀU = H_d⁻¹).
 
     ``U`` may be passed in when it was already computed by ``prepare_u`` for the same
     (H, percdamp, act_order); rows of W are processed independently either way.
+
+    Quantizer variants: ``sym`` takes the symmetric quantizer (``quantizer.group_params_sym``);
+    ``group_size == d_in`` is one group per row (per-channel), whose scale and zero come from
+    the whole row before its first column is quantized; ``static_groups`` fixes every group's
+    scale and zero from the original weights, groups of consecutive ORIGINAL columns, before
+    any column is quantized, and each column then uses the group of its original position
+    (g_idx[c] = c // group_size, scales indexed by that group), whatever order act_order gives.
 
     With ``trace`` the result also holds the values each rounding decision was taken on, in
     the processing order: ``pre`` [d_out, d_in], the compensated weight of every column just
@@ -129,6 +164,7 @@ def gptq_blocked_ref(W, H, bits, group_size, block_size=128, percdamp=0.01, act_
     if U is None:
         U = upper_chol_of_inverse(Hd)
     d_out = Wp.shape[0]
+    params = _params_fn(sym)
     codes = np.zeros((d_out, d_in), dtype=np.int64)
     What = np.zeros((d_out, d_in))
     scales = np.zeros((d_out, d_in // group_size))
@@ -137,18 +173,28 @@ def gptq_blocked_ref(W, H, bits, group_size, block_size=128, percdamp=0.01, act_
         pre = np.zeros((d_out, d_in))
         steps = np.zeros((d_out, d_in // group_size))
         zquots = np.zeros((d_out, d_in // group_size))
+    if static_groups:
+        W0 = np.empty_like(Wp)
+        W0[:, perm] = Wp                          # the original weights, original order
+        G0 = W0.reshape(d_out, d_in // group_size, group_size)
+        s0, z0, step0, zquot0 = params(G0.min(axis=2), G0.max(axis=2), maxq, trace=True)
+        scales[:], zeros[:] = s0, z0
+        if trace:
+            steps[:], zquots[:] = step0, zquot0
+        col_group = perm // group_size            # the group of each processing position
+    else:
+        col_group = np.arange(d_in) // group_size
     for j0 in range(0, d_in, block_size):
         j1 = min(j0 + block_size, d_in)
         Err = np.zeros((d_out, j1 - j0))
         for q in range(j0, j1):
-            if q % group_size == 0:
+            if not static_groups and q % group_size == 0:
                 grp = Wp[:, q:q + group_size]
-                s, z, step, zquot = group_params(grp.min(axis=1), grp.max(axis=1), maxq,
-                                                 trace=True)
+                s, z, step, zquot = params(grp.min(axis=1), grp.max(axis=1), maxq, trace=True)
                 scales[:, q // group_size], zeros[:, q // group_size] = s, z
                 if trace:
                     steps[:, q // group_size], zquots[:, q // group_size] = step, zquot
-            s, z = scales[:, q // group_size], zeros[:, q // group_size]
+            s, z = scales[:, col_group[q]], zeros[:, col_group[q]]
             w = Wp[:, q].copy()
             if trace:
                 pre[:, q] = w
@@ -159,7 +205,7 @@ def gptq_blocked_ref(W, H, bits, group_size, block_size=128, percdamp=0.01, act_
             Wp[:, q] = What[:, q]
             Err[:, q - j0] = err
         Wp[:, j1:] -= Err @ U[j0:j1, j1:]          # lazy batch update of all later columns
-    out = _assemble(codes, What, scales, zeros, perm, group_size)
+    out = _assemble(codes, What, scales, zeros, perm, group_size, static_groups)
     out["lam"] = lam
     if trace:
         out.update(pre=pre, step=steps, zquot=zquots, codes_p=codes)

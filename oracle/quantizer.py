@@ -64,6 +64,26 @@ def group_params(xmin, xmax, maxq, trace=False):
     return scale, zero
 
 
+def group_params_sym(xmin, xmax, maxq, trace=False):
+    """(scale, zero) of the symmetric quantizer for groups with the given minima and maxima.
+
+    0539edu.com/news/6111416 §2.3: a symmetric quantizer fixes the zero point at 0, so
+    q = round(x/scale). Reading: the range is [-m, m] with m = max(|min|, |max|), split into
+    maxq steps like the asymmetric range: scale = 2m/maxq rounded up to fp16 (1 for an all-zero
+    group). Codes stay unsigned: the zero point 0 of the signed code is stored as the code
+    offset 2**(bits-1) = (maxq + 1)/2, so q = clamp(rint(w/scale) + (maxq+1)/2, 0, maxq) and
+    |w - ŵ| <= scale/2 still holds for every entry.
+    """
+    m = np.maximum(np.abs(np.asarray(xmin, dtype=np.float64)),
+                   np.abs(np.asarray(xmax, dtype=np.float64)))
+    step = 2.0 * m / maxq
+    scale = np.where(m == 0.0, 1.0, fp16_round_up(step))
+    zero = np.full_like(scale, (maxq + 1) // 2, dtype=np.float64)
+    if trace:
+        return scale, zero, step, np.full_like(scale, np.nan)
+    return scale, zero
+
+
 def quantize(w, scale, zero, maxq):
     """Integer codes q = clamp(rint(w/scale) + zero, 0, maxq) (fp64 in, int64 out)."""
     w = np.asarray(w, dtype=np.float64)

@@ -13,20 +13,81 @@ packed form holds two codes per byte, the even column in the low nibble.
 
 import numpy as np
 
-from .quantizer import group_params, quantize, dequantize
+from .quantizer import group_params, group_params_sym, quantize, dequantize
 
 
-def rtn_minmax(W, bits, group_size):
-    """Return (codes int64 [d_out, d_in], scales fp64, zeros fp64 [d_out, d_in/g])."""
+def rtn_minmax(W, bits, group_size, sym=False):
+    """Return (codes int64 [d_out, d_in], scales fp64, zeros fp64 [d_out, d_in/g]).
+    ``sym`` takes the symmetric quantizer (0539edu.com §2.3) instead of the asymmetric one."""
     W = np.asarray(W, dtype=np.float64)
     d_out, d_in = W.shape
     if d_in % group_size:
         raise ValueError("d_in must be a multiple of group_size")
     maxq = 2 ** bits - 1
     Wg = W.reshape(d_out, d_in // group_size, group_size)
-    scale, zero = group_params(Wg.min(axis=2), Wg.max(axis=2), maxq)
+    params = group_params_sym if sym else group_params
+    scale, zero = params(Wg.min(axis=2), Wg.max(axis=2), maxq)
     q = quantize(Wg, scale[..., None], zero[..., None], maxq)
     return q.reshape(d_out, d_in), scale, zero
+
+
+def clip_ratios(min_ratio=0.5, step=0.05):
+    """The clip grid of gtnt.cn/news/115337 §3 (awq_clip): ratios of the block's amax from 1
+    down to min_ratio (default 0.5) in steps of `step` (default 0.05), largest first:
+    ρ_i = 1 − i·step, i = 0 … round((1 − min_ratio)/step)."""
+    n = int(round((1.0 - min_ratio) / step)) + 1
+    return np.array([1.0 - i * step for i in range(n)])
+
+
+def rtn_clip_search(W, bits, group_size, H=None, sym=False, min_ratio=0.5, step=0.05):
+    """Group RTN with a clip search per group (gtnt.cn §3: search each quantization block's
+    clip bound c in [amax·min_ratio, amax], amax = max |w| of the block, truncating the
+    weights to [-c, c] before their min-max scale is taken).
+
+    For each group and each grid ratio ρ (``clip_ratios(min_ratio, step)``), c = ρ·amax; the group's weights
+    are clamped to [-c, c] and quantized with the scale and zero of the clamped group; the
+    criterion is the group's share of the layer output error, d·H_gg·d with d = w − ŵ (the
+    original weights minus the reconstruction) and H_gg the group's diagonal block of
+    H = 2XᵀX; without H it is the weight error d·d. The smallest criterion wins, ties to the
+    larger ratio (less clipping).
+
+    Returns (codes [d_out, d_in], scales, zeros [d_out, d_in/g], ratio index [d_out, d_in/g],
+    criteria [grid points, d_out, d_in/g])."""
+    W = np.asarray(W, dtype=np.float64)
+    d_out, d_in = W.shape
+    if d_in % group_size:
+        raise ValueError("d_in must be a multiple of group_size")
+    maxq = 2 ** bits - 1
+    ng = d_in // group_size
+    Wg = W.reshape(d_out, ng, group_size)
+    amax = np.max(np.abs(Wg), axis=2)
+    params = group_params_sym if sym else group_params
+    if H is not None:
+        H = np.asarray(H, dtype=np.float64)
+        Hb = np.stack([H[k * group_size:(k + 1) * group_size, k * group_size:(k + 1) * group_size]
+                       for k in range(ng)])
+    ratios = clip_ratios(min_ratio, step)
+    crit = np.empty((len(ratios), d_out, ng))
+    cand = []
+    for i, rho in enumerate(ratios):
+        c = rho * amax
+        Wc = np.clip(Wg, -c[..., None], c[..., None])
+        s, z = params(Wc.min(axis=2), Wc.max(axis=2), maxq)
+        q = quantize(Wc, s[..., None], z[..., None], maxq)
+        D = Wg - dequantize(q, s[..., None], z[..., None])
+        if H is None:
+            crit[i] = np.sum(D * D, axis=2)
+        else:
+            crit[i] = np.einsum("rkg,kgh,rkh->rk", D, Hb, D)
+        cand.append((q, s, z))
+    best = np.argmin(crit, axis=0)                # first index among equal minima
+    codes = np.empty((d_out, ng, group_size), dtype=np.int64)
+    scales = np.empty((d_out, ng))
+    zeros = np.empty((d_out, ng))
+    for i, (q, s, z) in enumerate(cand):
+        m = best == i
+        codes[m], scales[m], zeros[m] = q[m], s[m], z[m]
+    return codes.reshape(d_out, d_in), scales, zeros, best, crit
 
 
 def rtn_dequant(codes, scales, zeros, group_size):

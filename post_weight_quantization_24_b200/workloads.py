@@ -84,6 +84,14 @@ DECODER_7B_LINEARS = (
     ("down_proj", 4096, 11008, "down_in"),
 )
 DECODER_7B_INPUTS = {"attn_in": 4096, "o_in": 4096, "mlp_in": 4096, "down_in": 11008}
+# The same layer with the linears that read one input stacked row-wise (q;k;v and gate;up), as
+# fused projections store them: (name, parts, d_in, input).
+DECODER_7B_FUSED = (
+    ("qkv_proj", ("q_proj", "k_proj", "v_proj"), 4096, "attn_in"),
+    ("o_proj", ("o_proj",), 4096, "o_in"),
+    ("gate_up_proj", ("gate_proj", "up_proj"), 4096, "mlp_in"),
+    ("down_proj", ("down_proj",), 11008, "down_in"),
+)
 
 _TID_W, _TID_W_OUTLIER, _TID_X, _TID_X_SCALE, _TID_X_OUTLIER = 1, 2, 3, 4, 5
 
@@ -150,3 +158,30 @@ def correlated_activations(n: int, d: int, rank: int = 4, seed: int = 0,
     M = torch.eye(d) + 0.9 * (A @ A.T) / np.sqrt(rank) + 0.05 * torch.randn(d, d, generator=g)
     Z = torch.randn(n, d, generator=g)
     return (Z @ M).to(torch.float16).to(device)
+
+
+def make_decoder_layer(layer: int, n_tokens: int, device="cpu", seed_base: int = 1000):
+    """One synthetic 7B decoder layer of a stack: its four distinct inputs (n_tokens each, the
+    7B activation recipe) and its weights (the 7B weight recipe, fp16), with the linears that
+    read one input stacked row-wise. Every tensor has its own seed, distinct per layer.
+    Returns (inputs: {input name: X}, fused: [(name, W, input name)])."""
+    base = WORKLOADS["mlp_up_7b"]
+    seed0 = seed_base + 64 * layer
+    inputs = {}
+    for idx, (name, d) in enumerate(DECODER_7B_INPUTS.items()):
+        inputs[name] = make_activations(base.replace(d_in=d, n_tokens=n_tokens),
+                                        device=device, seed=seed0 + idx)
+    shapes = {name: (d_out, d_in) for name, d_out, d_in, _ in DECODER_7B_LINEARS}
+    order = [name for name, _, _, _ in DECODER_7B_LINEARS]
+    fused = []
+    for name, parts, d_in, src in DECODER_7B_FUSED:
+        rows = sum(shapes[p][0] for p in parts)
+        W = torch.empty(rows, d_in, dtype=torch.float16, device=device)
+        r0 = 0
+        for p in parts:
+            d_out = shapes[p][0]
+            W[r0:r0 + d_out] = make_weights(base.replace(d_out=d_out, d_in=d_in), device=device,
+                                            seed=seed0 + 8 + order.index(p))
+            r0 += d_out
+        fused.append((name, W, src))
+    return inputs, fused
