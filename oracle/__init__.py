@@ -32,6 +32,7 @@ Modules:
              output assembly
   loss       layer reconstruction loss tr(ΔHΔᵀ)/tr(WHWᵀ)
   w4a16      the W4A16 layer that consumes the output: fp16 reconstruction and X·Ŵᵀ
+  awq        AWQ-lite: activation-aware channel scales, grid search over α
   sequential layer-by-layer GPTQ of a stack of MLP blocks, each layer's Hessian from the
              outputs of the already-quantized layers before it
 
@@ -39,4 +40,4 @@ Every function is pinned by a ``-m "not gpu"`` test in ``tests/test_oracle_*.py`
 something other than itself (worked example, closed forms, brute force, invariants).
 """
 
-from . import quantizer, rtn, hessian, factor, gptq, loss, w4a16, sequential  # noqa: F401
+from . import quantizer, rtn, hessian, factor, gptq, loss, w4a16, sequential, awq  # noqa: F401
