@@ -153,6 +153,30 @@ gptq_status gptq_quantize_layer(const void* W, int w_dtype, int d_out, int d_in,
                                 int32_t* g_idx, int32_t* perm, float* loss,
                                 void* workspace, size_t workspace_bytes, void* stream);
 
+/* gptq_quantize_layer with the quantizer variants (same arguments, plus two switches, same
+ * workspace size). gptq_quantize_layer is this call with sym = 0 and static_groups = 0.
+ *   sym            1: the symmetric quantizer of 0539edu.com §2.3 (zero point fixed at 0,
+ *                  q = round(x/scale)): scale = 2*max|w|/(2^bits-1) rounded up to fp16 over the
+ *                  group, and the signed zero stored as the code offset 2^(bits-1), so
+ *                  code = clamp(rint(w/scale) + 2^(bits-1), 0, 2^bits-1) and zeros hold
+ *                  2^(bits-1).
+ *   static_groups  1: every group's scale and zero are fixed from the ORIGINAL weights, groups
+ *                  of group_size consecutive original columns, before any column is quantized;
+ *                  each column uses the group of its original position, whatever order
+ *                  act_order processes it in: g_idx[c] = c / group_size and scales/zeros are
+ *                  indexed by that group (the inference-time gather of GPTQ deep-dive §3.3
+ *                  then reads contiguous groups).
+ *   group_size == d_in  one group per row (per-channel): its scale and zero come from the
+ *                  whole original row before its first column is quantized; block_size is then
+ *                  free (any multiple of 8 up to 128).
+ * Errors: as gptq_quantize_layer; ARG also for sym or static_groups outside {0, 1}. */
+gptq_status gptq_quantize_layer_ex(const void* W, int w_dtype, int d_out, int d_in,
+                                   const float* H, int bits, int group_size, int block_size,
+                                   float percdamp, int act_order, int sym, int static_groups,
+                                   uint8_t* codes, uint16_t* scales, uint16_t* zeros,
+                                   int32_t* g_idx, int32_t* perm, float* loss,
+                                   void* workspace, size_t workspace_bytes, void* stream);
+
 /* No-allocation form of gptq_quantize_layer, with the same arguments except the workspace.
  * The pages have no counterpart; this is an integration aid. It is for callers that may not
  * allocate device memory when they quantize: runtimes that reserved almost all of the GPU for
@@ -206,6 +230,126 @@ gptq_status gptq_inverse_factor(const float* H, int d_in, float percdamp, int ac
 gptq_status rtn_minmax_quantize(const void* W, int w_dtype, int d_out, int d_in, int bits,
                                 int group_size, uint8_t* packed, uint16_t* scales,
                                 uint16_t* zeros, void* stream);
+
+/* Group RTN with a clip search per group (gtnt.cn §3, awq_clip: each quantization block's clip
+ * bound c is searched in [amax * min_ratio, amax], amax = max |w| of the block, truncating the
+ * weights to [-c, c] before their min-max scale is taken).
+ *   For ratios rho_i = 1 - i*step, i = 0 .. round((1 - min_ratio)/step) (the pages' defaults
+ *   min_ratio = 0.5, step = 0.05: 11 ratios), c = rho_i * amax; the group's weights are clamped
+ *   to [-c, c] and quantized with the scale and zero of the clamped group (sym selects the
+ *   symmetric quantizer). The criterion is the group's share of the layer output error,
+ *   d * H_gg * d with d = w - What (original weights minus the reconstruction) and H_gg the
+ *   group's diagonal block of H = 2 X^T X; with H = NULL it is the weight error d.d. The smallest
+ *   criterion wins, ties to the larger ratio. For the chosen ratio the codes, scales and zeros
+ *   equal the fp64 definition bit for bit; the criterion is accumulated in fp32.
+ *   W        device [d_out x d_in], fp16 or fp32.  d_in: a multiple of group_size.
+ *   group_size  16, 32, 64 or 128.
+ *   H        device fp32 [d_in x d_in], upper triangle read, 16-byte aligned; or NULL.
+ *   min_ratio in (0, 1], step > 0, at most 64 grid points.
+ *   packed, scales, zeros  as rtn_minmax_quantize.
+ *   ratio_idx device uint8 [d_out x d_in/group_size] (index i of the chosen ratio), or NULL.
+ * Asynchronous. Errors: ARG, CUDA, UNSUPPORTED. */
+gptq_status rtn_clip_search(const void* W, int w_dtype, int d_out, int d_in, int bits,
+                            int group_size, int sym, const float* H, double min_ratio,
+                            double step, uint8_t* packed, uint16_t* scales, uint16_t* zeros,
+                            uint8_t* ratio_idx, void* stream);
+
+/* rtn_minmax_quantize with the symmetric quantizer as an option (sym = 1: zero point fixed,
+ * see gptq_quantize_layer_ex; sym = 0 is rtn_minmax_quantize). Same layouts and errors. */
+gptq_status rtn_quantize_ex(const void* W, int w_dtype, int d_out, int d_in, int bits,
+                            int group_size, int sym, uint8_t* packed, uint16_t* scales,
+                            uint16_t* zeros, void* stream);
+
+/* ------------------------------------------------------------------------------------------
+ * The W4A16 layer that serves the quantized weights (0539edu.com §3.2, §5.2: 4-bit weights,
+ * fp16 activations; GPTQ deep-dive §3.3: with desc_act the groups of the columns are scattered
+ * and inference gathers them):
+ *   Y = fp16(X * What^T + R),  What[r][c] = fp16(scale[r][k] * (code[r][c] - zero[r][k])),
+ * fp32 accumulation on the tensor cores (tcgen05 kind::f16), k the group of column c.
+ * The act_order gather is done on both sides of the contraction: w4a16_pack stores the codes in
+ * the processing order of `perm` (so every group is again a run of group_size consecutive
+ * columns, as the scales of gptq_quantize_layer are indexed), and w4a16_linear with the same
+ * perm gathers the columns of X into the workspace before the GEMM. Without act_order (or with
+ * static groups, whose g_idx is c / group_size) pass perm = NULL to both.
+ * ------------------------------------------------------------------------------------------ */
+
+/* packed[r][p/2] = codes[r][perm[p]] (codes[r][p] if perm is NULL), even p in the low nibble.
+ *   codes   device uint8 [d_out x d_in] (gptq_quantize_layer's output, original order).
+ *   perm    device int32 [d_in] or NULL.   packed: device uint8 [d_out x d_in/2].
+ * Asynchronous. Errors: ARG (d_in odd), CUDA, UNSUPPORTED. */
+gptq_status w4a16_pack(const uint8_t* codes, int d_out, int d_in, const int32_t* perm,
+                       uint8_t* packed, void* stream);
+
+/* Workspace bytes of w4a16_linear: n_tokens * d_in * 2 with a perm (the gathered X), else 0. */
+size_t w4a16_linear_workspace(int64_t n_tokens, int d_in, int has_perm);
+
+/* Y = fp16(X * What^T + R).
+ *   X        device fp16 [n_tokens x d_in], 16-byte aligned; 1 <= n_tokens < 2^31.
+ *   d_in     a multiple of 64, <= 65536.   d_out: a multiple of 8.
+ *   packed   device uint8 [d_out x d_in/2] from w4a16_pack (same perm), 16-byte aligned.
+ *   scales, zeros  device fp16 [d_out x d_in/group_size]: group p / group_size of processing
+ *            position p.   group_size: a multiple of 8 dividing d_in.
+ *   perm     device int32 [d_in] or NULL (see w4a16_pack).
+ *   R        device fp16 [n_tokens x d_out] or NULL (a residual added before the rounding; may
+ *            be the same buffer as Y).
+ *   Y        device fp16 [n_tokens x d_out], 16-byte aligned.
+ *   workspace device, >= w4a16_linear_workspace(n_tokens, d_in, perm != NULL) bytes (may be
+ *            NULL without perm).
+ *   status_dev device int or NULL: set to GPTQ_ERR_TIMEOUT if a bounded wait gave up.
+ * Asynchronous. Errors: ARG, WORKSPACE, CUDA, UNSUPPORTED. */
+gptq_status w4a16_linear(const void* X, int64_t n_tokens, int d_in, const uint8_t* packed,
+                         const uint16_t* scales, const uint16_t* zeros, int group_size,
+                         int d_out, const int32_t* perm, const void* R, void* Y,
+                         void* workspace, size_t workspace_bytes, int* status_dev,
+                         void* stream);
+
+/* ------------------------------------------------------------------------------------------
+ * AWQ-lite (gtnt.cn §3, awq_lite; 0539edu.com §3.2): per-input-channel scales
+ * s = x_mean^alpha / w_mean^(1-alpha) searched over alpha = 0, step, ..., 1 by the layer's
+ * output error, with group min-max RTN as the quantizer. The weights of channel c are
+ * multiplied by s_c before quantization and its activations are to be divided by s_c (folded
+ * into the preceding layer), which leaves the layer's output unchanged before quantization.
+ * ------------------------------------------------------------------------------------------ */
+
+/* sums[c] += sum over rows of |X[r][c]| in fp64 (accumulates over calibration batches; zero
+ * sums first). X device fp16 or fp32 [n x d] row-major; sums device fp64 [d].
+ * Asynchronous. Errors: ARG, CUDA, UNSUPPORTED. */
+gptq_status gptq_channel_abs_sum(const void* X, int w_dtype, int64_t n, int d, double* sums,
+                                 void* stream);
+
+/* Workspace bytes of awq_lite_search (0 for invalid arguments). */
+size_t awq_lite_workspace(int d_out, int d_in, double alpha_step);
+
+/* The grid search, for fp16 W [d_out x d_in] (so that W * s is exact):
+ *   x_mean_c = x_abs_sum[c] / n_tokens (x_abs_sum from gptq_channel_abs_sum, device fp64 [d_in]);
+ *   w_mean_c = mean over rows of |W[r][c]|;
+ *   for alpha_i = i * alpha_step, i = 0 .. round(1/alpha_step):
+ *     s_c = fp16(x_mean_c^alpha / w_mean_c^(1-alpha)), 1 where x_mean_c or w_mean_c is 0 or the
+ *     fp16 value is not positive and finite;
+ *     L_i = tr(D H D^T), D = W - RTN(W * s) / s (RTN: group min-max, sym as in rtn_quantize_ex);
+ *   best = argmin L_i (ties to the smaller alpha).
+ *   H        device fp32 [d_in x d_in], FULL symmetric (as gptq_hessian_get writes it), H = 2X^T X.
+ *   packed, scales, zeros  the RTN of W * s_best (layouts of rtn_minmax_quantize).
+ *   s_out    device fp16 [d_in] (s_best) or NULL.
+ *   losses   host double [round(1/alpha_step) + 1] or NULL (L_i, fp32-accurate).
+ *   best     host int or NULL.
+ *   workspace device, >= awq_lite_workspace(d_out, d_in, alpha_step) bytes, 256-byte aligned.
+ * Synchronises `stream` once to choose alpha. Errors: ARG (also fp32 W), WORKSPACE, CUDA,
+ * TIMEOUT, UNSUPPORTED. */
+gptq_status awq_lite_search(const void* W, int w_dtype, int d_out, int d_in,
+                            const double* x_abs_sum, int64_t n_tokens, const float* H, int bits,
+                            int group_size, int sym, double alpha_step, uint8_t* packed,
+                            uint16_t* scales, uint16_t* zeros, uint16_t* s_out,
+                            double* losses, int* best, void* workspace, size_t workspace_bytes,
+                            void* stream);
+
+/* The gate of a gated MLP block between its two quantized projections (layer-by-layer GPTQ
+ * of a block stack, gtnt.cn §4: the down projection's Hessian comes from these activations):
+ * A[t][j] = fp16(silu(GU[t][j]) * GU[t][d_ff + j]), silu(g) = g / (1 + e^-g) in fp32.
+ *   GU  device fp16 [n_tokens x 2*d_ff] (gate outputs, then up outputs, per row).
+ *   A   device fp16 [n_tokens x d_ff].   d_ff: a multiple of 8; both 16-byte aligned.
+ * Asynchronous. Errors: ARG, CUDA, UNSUPPORTED. */
+gptq_status gptq_silu_mul(const void* GU, int64_t n_tokens, int d_ff, void* A, void* stream);
 
 /* ------------------------------------------------------------------------------------------
  * Stage timing. When enabled, gptq_quantize_layer records CUDA events around each stage on

@@ -22,7 +22,8 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libgptq_b200.so")
-SOURCES = ("api.cu", "rtn.cu", "hessian.cu", "factor.cu", "gptq.cu", "noalloc.cu", "tcgemm.cu")
+SOURCES = ("api.cu", "rtn.cu", "rtn_clip.cu", "hessian.cu", "factor.cu", "gptq.cu", "noalloc.cu",
+           "tcgemm.cu", "w4a16.cu", "awq.cu")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O3",
                 "--expt-relaxed-constexpr", "-I" + os.path.join(ROOT, "include")]

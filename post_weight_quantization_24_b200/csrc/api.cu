@@ -290,15 +290,32 @@ gptq_status gptq_quantize_layer(const void* W, int w_dtype, int d_out, int d_in,
                                 float percdamp, int act_order, uint8_t* codes, uint16_t* scales,
                                 uint16_t* zeros, int32_t* g_idx, int32_t* perm, float* loss,
                                 void* workspace, size_t workspace_bytes, void* stream) {
+    return gptq_quantize_layer_ex(W, w_dtype, d_out, d_in, H, bits, group_size, block_size,
+                                  percdamp, act_order, 0, 0, codes, scales, zeros, g_idx, perm,
+                                  loss, workspace, workspace_bytes, stream);
+}
+
+gptq_status gptq_quantize_layer_ex(const void* W, int w_dtype, int d_out, int d_in,
+                                   const float* H, int bits, int group_size, int block_size,
+                                   float percdamp, int act_order, int sym, int static_groups,
+                                   uint8_t* codes, uint16_t* scales, uint16_t* zeros,
+                                   int32_t* g_idx, int32_t* perm, float* loss, void* workspace,
+                                   size_t workspace_bytes, void* stream) {
     // ---- argument checks (no launch on failure) ----
     if (!W || !H || !codes || !scales || !zeros || !g_idx || !workspace) return GPTQ_ERR_ARG;
     if (w_dtype != GPTQ_DTYPE_F16 && w_dtype != GPTQ_DTYPE_F32) return GPTQ_ERR_ARG;
     if (d_out < 1 || d_in < 8 || d_in > 65536 || d_in % 8) return GPTQ_ERR_ARG;
     if (bits < 2 || bits > 8) return GPTQ_ERR_ARG;
     if (group_size < 1 || d_in % group_size) return GPTQ_ERR_ARG;
-    if (block_size < 8 || block_size > 128 || block_size % 8 || block_size % group_size)
+    const bool per_channel = group_size == d_in;
+    if (block_size < 8 || block_size > 128 || block_size % 8 ||
+        (block_size % group_size && !per_channel))
         return GPTQ_ERR_ARG;
     if (!(percdamp >= 0.0f) || act_order < 0 || act_order > 1) return GPTQ_ERR_ARG;
+    if (sym < 0 || sym > 1 || static_groups < 0 || static_groups > 1) return GPTQ_ERR_ARG;
+    // grids fixed before the column loop: every group of the original weights (static
+    // groups), or the whole row (per-channel)
+    const int preset = (static_groups || per_channel) ? 1 : 0;
     if (!aligned16(W) || !aligned16(H) || !aligned16(codes) ||
         (reinterpret_cast<uintptr_t>(workspace) & 255))
         return GPTQ_ERR_ARG;
@@ -320,6 +337,9 @@ gptq_status gptq_quantize_layer(const void* W, int w_dtype, int d_out, int d_in,
     GPTQ_TRY(act_order_launch(H, d_in, act_order, ws.perm, ws.invperm, s));
     GPTQ_TRY(gather_h_launch(H, d_in, ws.perm, ws.st, 1, ws.A, status, s));
     GPTQ_TRY(gather_w_launch(W, w_dtype, d_out, d_in, ws.perm, ws.Wk, status, s));
+    if (preset)
+        GPTQ_TRY(group_grid_launch(W, w_dtype, d_out, d_in, group_size, bits, sym, scales, zeros,
+                                   s));
     tm.end();
     // ---- stage 1: U with U^T U = H_d^-1 (factor and inverse overlap on two streams) ----
     tm.begin(1);
@@ -348,8 +368,9 @@ gptq_status gptq_quantize_layer(const void* W, int w_dtype, int d_out, int d_in,
             float* err_lo = ws.ErrLo + (j0 - s0);
             tm.begin(3);
             GPTQ_TRY(gptq_block_launch(ws.Wk, d_out, d_in, j0, bw, ws.P, ws.Dinv, group_size,
-                                       bits, codes_p, scales, zeros, err_hi, err_lo, kSuperCols,
-                                       &ws.st->err_sq, status, s));
+                                       bits, sym, preset ? ws.perm : nullptr, codes_p, scales,
+                                       zeros, err_hi, err_lo, kSuperCols, &ws.st->err_sq, status,
+                                       s));
             tm.end();
             tm.begin(4);
             GPTQ_TRY(lazy_update_launch(ws.Wk, d_out, d_in, j0, j1, j1, s1, ws.X, ws.A, err_hi,
@@ -364,13 +385,13 @@ gptq_status gptq_quantize_layer(const void* W, int w_dtype, int d_out, int d_in,
     // ---- stage 5: outputs in the original column order ----
     tm.begin(5);
     GPTQ_TRY(assemble_launch(codes_p, d_out, d_in, ws.perm, ws.invperm, group_size, act_order,
-                             codes, g_idx, perm, s));
+                             preset, codes, g_idx, perm, s));
     tm.end();
     // ---- stage 6: reconstruction loss ----
     if (loss) {
         tm.begin(6);
         GPTQ_TRY(loss_launch(W, w_dtype, d_out, d_in, H, ws.perm, codes_p, scales, zeros,
-                             group_size, ws.Wk, ws.A, ws.st, s));
+                             group_size, preset, ws.Wk, ws.A, ws.st, s));
         tm.end();
     }
     DevState host{};
@@ -421,13 +442,20 @@ gptq_status gptq_inverse_factor(const float* H, int d_in, float percdamp, int ac
 gptq_status rtn_minmax_quantize(const void* W, int w_dtype, int d_out, int d_in, int bits,
                                 int group_size, uint8_t* packed, uint16_t* scales,
                                 uint16_t* zeros, void* stream) {
+    return rtn_quantize_ex(W, w_dtype, d_out, d_in, bits, group_size, 0, packed, scales, zeros,
+                           stream);
+}
+
+gptq_status rtn_quantize_ex(const void* W, int w_dtype, int d_out, int d_in, int bits,
+                            int group_size, int sym, uint8_t* packed, uint16_t* scales,
+                            uint16_t* zeros, void* stream) {
     if (!W || !packed || !scales || !zeros) return GPTQ_ERR_ARG;
     if (w_dtype != GPTQ_DTYPE_F16 && w_dtype != GPTQ_DTYPE_F32) return GPTQ_ERR_ARG;
     if (d_out < 1 || d_in < 8 || d_in % 8 || bits < 2 || bits > 8) return GPTQ_ERR_ARG;
-    if (group_size < 1 || d_in % group_size) return GPTQ_ERR_ARG;
+    if (group_size < 1 || d_in % group_size || sym < 0 || sym > 1) return GPTQ_ERR_ARG;
     if (!aligned16(W) || !aligned16(packed)) return GPTQ_ERR_ARG;
     GPTQ_TRY(check_device());
-    return rtn_launch(W, w_dtype, d_out, d_in, bits, group_size, packed, scales, zeros,
+    return rtn_launch(W, w_dtype, d_out, d_in, bits, group_size, sym, packed, scales, zeros,
                       static_cast<cudaStream_t>(stream));
 }
 

@@ -39,7 +39,7 @@ constexpr int PH = 16;                       // block columns per window phase
 constexpr int NPH = MAXB / PH;
 constexpr int WARPS = 2;
 constexpr int THREADS = WARPS * 32;          // one row per thread
-constexpr int SMEM = MAXB * MAXB * 4 + MAXB * 4 + NPH * 8;
+constexpr int SMEM = MAXB * MAXB * 4 + MAXB * 4 + NPH * 8 + MAXB * 4;   // + grid indices
 }  // namespace gr
 
 // img[R][k] = U[R][R+1+k] while R+1+k stays inside R's block (else 0); rdiag[R] = 1/U[R][R]
@@ -71,7 +71,10 @@ struct RowCtx {
     float* Err;           // tf32 hi and lo parts of the errors (the lazy update's operand)
     float* ErrLo;
     QParams P;
-    int next_gs;          // block column of the next group start
+    int next_gs;          // block column of the next group start (grids found in the loop)
+    bool sym;             // symmetric quantizer
+    const int* pidx;      // preset grids: grid index of each block column (else nullptr)
+    int cur_k;            // preset grids: the grid P holds
     float e0, e1, e2, e3; // errors of the last four columns (e0 newest)
     uint32_t qword;       // their codes, oldest in the low byte
     double esq;           // this row's sum of squared OBS errors
@@ -82,7 +85,17 @@ __device__ __forceinline__ void rows_phase(float (&w)[gr::MAXB], int p0, RowCtx&
     const int i_end = min(p0 + gr::PH, x.bw);
 #pragma unroll 1
     for (int i = p0; i < i_end; ++i) {
-        if (i == x.next_gs) {
+        if (x.pidx) {
+            // preset grids (per-channel, static groups): this column's grid, from the outputs
+            const int k = x.pidx[i];
+            if (k != x.cur_k) {
+                x.cur_k = k;
+                if (x.row_ok) {
+                    const int64_t gi = x.r * x.n_groups_row + k;
+                    x.P = stored_params(x.scales[gi], x.zeros[gi]);
+                }
+            }
+        } else if (i == x.next_gs) {
             // group [i, i+g): min/max of its current weights, w[0..g)
             x.next_gs += x.g;
             float mn = w[0], mx = w[0];
@@ -97,7 +110,7 @@ __device__ __forceinline__ void rows_phase(float (&w)[gr::MAXB], int p0, RowCtx&
                     }
                 }
             }
-            x.P = group_params(mn, mx, x.maxq);
+            x.P = group_params_any(mn, mx, x.maxq, x.sym);
             if (x.row_ok) {
                 const int64_t gi = x.r * x.n_groups_row + (x.j0 + i) / x.g;
                 x.scales[gi] = half_bits(x.P.scale);
@@ -160,20 +173,25 @@ __device__ __forceinline__ bool rows_phases(float (&w)[gr::MAXB], RowCtx& x, uin
 
 __global__ void __launch_bounds__(gr::THREADS, 3) gptq_rows_kernel(
     const float* __restrict__ Wk, int d_out, int d_in, int j0, int bw,
-    const float* __restrict__ img, const float* __restrict__ rdiag, int g, int bits,
-    uint8_t* __restrict__ codes_p, uint16_t* __restrict__ scales, uint16_t* __restrict__ zeros,
-    float* __restrict__ Err, float* __restrict__ ErrLo, int err_ld, double* err_sq, int* status) {
+    const float* __restrict__ img, const float* __restrict__ rdiag, int g, int bits, int sym,
+    const int* __restrict__ preset_perm, uint8_t* __restrict__ codes_p,
+    uint16_t* __restrict__ scales, uint16_t* __restrict__ zeros, float* __restrict__ Err,
+    float* __restrict__ ErrLo, int err_ld, double* err_sq, int* status) {
     if (status_bad(status)) return;
     extern __shared__ __align__(128) unsigned char rows_smem[];
     float* Us = reinterpret_cast<float*>(rows_smem);
     float* rd = Us + gr::MAXB * gr::MAXB;
     uint64_t* bars = reinterpret_cast<uint64_t*>(rd + gr::MAXB);
+    int* pidx = reinterpret_cast<int*>(bars + gr::NPH);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
     if (tid == 0) {
         for (int p = 0; p < gr::NPH; ++p) mbar_init(&bars[p], 1);
         fence_mbar_init();
     }
+    // preset grids: the grid of block column i is the group of its original column
+    if (preset_perm)
+        for (int i = tid; i < bw; i += gr::THREADS) pidx[i] = preset_perm[j0 + i] / g;
     __syncthreads();
     if (warp == 0 && lane < gr::NPH) {
         // image rows [16p, 16p+16) of the block arrive on barrier p (+ the diagonal on 0)
@@ -197,6 +215,9 @@ __global__ void __launch_bounds__(gr::THREADS, 3) gptq_rows_kernel(
     x.codes_p = codes_p; x.scales = scales; x.zeros = zeros; x.Err = Err; x.ErrLo = ErrLo;
     x.P.scale = 1.f; x.P.zero = 0.f; x.P.inv_scale = 1.f;
     x.next_gs = 0;   // j0 is a multiple of g
+    x.sym = sym != 0;
+    x.pidx = preset_perm ? pidx : nullptr;
+    x.cur_k = -1;
     x.e0 = x.e1 = x.e2 = x.e3 = 0.f;
     x.qword = 0u;
     x.esq = 0.0;
@@ -227,9 +248,10 @@ __global__ void __launch_bounds__(gr::THREADS, 3) gptq_rows_kernel(
 static bool g_rows_attr_set = false;
 
 gptq_status gptq_block_launch(float* Wk, int d_out, int d_in, int j0, int bw, const float* img,
-                              const float* rdiag, int group_size, int bits, uint8_t* codes_p,
-                              uint16_t* scales, uint16_t* zeros, float* Err, float* ErrLo,
-                              int err_ld, double* err_sq, int* status, cudaStream_t s) {
+                              const float* rdiag, int group_size, int bits, int sym,
+                              const int* preset_perm, uint8_t* codes_p, uint16_t* scales,
+                              uint16_t* zeros, float* Err, float* ErrLo, int err_ld,
+                              double* err_sq, int* status, cudaStream_t s) {
     if (!g_rows_attr_set) {
         GPTQ_CUDA_TRY(cudaFuncSetAttribute(gptq_rows_kernel,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -238,8 +260,64 @@ gptq_status gptq_block_launch(float* Wk, int d_out, int d_in, int j0, int bw, co
     }
     const int grid = (d_out + gr::THREADS - 1) / gr::THREADS;
     gptq_rows_kernel<<<grid, gr::THREADS, gr::SMEM, s>>>(Wk, d_out, d_in, j0, bw, img, rdiag,
-                                                        group_size, bits, codes_p, scales, zeros,
-                                                        Err, ErrLo, err_ld, err_sq, status);
+                                                        group_size, bits, sym, preset_perm,
+                                                        codes_p, scales, zeros, Err, ErrLo,
+                                                        err_ld, err_sq, status);
+    GPTQ_LAUNCHED();
+    return GPTQ_OK;
+}
+
+// Preset grids: the scale and zero of every group of the ORIGINAL weights in the original
+// column order (static groups; one group per row for per-channel), before any column is
+// quantized. One warp per (row, group): lane-strided min/max, a warp reduction, and the
+// group's scalars in fp64 as the column loop computes them.
+template <typename T>
+__global__ void __launch_bounds__(256) group_grid_kernel(const T* __restrict__ W, int d_out,
+                                                         int d_in, int g, int bits, int sym,
+                                                         uint16_t* __restrict__ scales,
+                                                         uint16_t* __restrict__ zeros) {
+    const int maxq = (1 << bits) - 1;
+    const int ng = d_in / g;
+    const int64_t n_units = static_cast<int64_t>(d_out) * ng;
+    const int lane = threadIdx.x & 31;
+    const int64_t wstride = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+    for (int64_t u = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+         u < n_units; u += wstride) {
+        const int64_t r = u / ng;
+        const int k = static_cast<int>(u - r * ng);
+        const T* w = W + r * d_in + static_cast<int64_t>(k) * g;
+        float mn = static_cast<float>(w[0]), mx = mn;
+        for (int i = lane; i < g; i += 32) {
+            const float v = static_cast<float>(w[i]);
+            mn = fminf(mn, v);
+            mx = fmaxf(mx, v);
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        }
+        if (lane == 0) {
+            const QParams p = group_params_any(mn, mx, maxq, sym != 0);
+            scales[u] = half_bits(p.scale);
+            zeros[u] = half_bits(p.zero);
+        }
+    }
+}
+
+gptq_status group_grid_launch(const void* W, int w_dtype, int d_out, int d_in, int group_size,
+                              int bits, int sym, uint16_t* scales, uint16_t* zeros,
+                              cudaStream_t s) {
+    const int64_t units = static_cast<int64_t>(d_out) * (d_in / group_size);
+    const int blocks = static_cast<int>(std::max<int64_t>(
+        1, std::min<int64_t>((units + 7) / 8, static_cast<int64_t>(num_sms()) * 16)));
+    if (w_dtype == GPTQ_DTYPE_F16)
+        group_grid_kernel<__half><<<blocks, 256, 0, s>>>(static_cast<const __half*>(W), d_out,
+                                                         d_in, group_size, bits, sym, scales,
+                                                         zeros);
+    else
+        group_grid_kernel<float><<<blocks, 256, 0, s>>>(static_cast<const float*>(W), d_out, d_in,
+                                                        group_size, bits, sym, scales, zeros);
     GPTQ_LAUNCHED();
     return GPTQ_OK;
 }
@@ -263,11 +341,11 @@ gptq_status lazy_update_launch(float* Wk, int d_out, int d_in, int k0, int k1, i
 // codes[r][c] = codes_p[r][invperm[c]]; g_idx[c] = invperm[c] / g; perm_out = perm
 __global__ void assemble_kernel(const uint8_t* __restrict__ codes_p, int d_out, int d_in,
                                 const int* __restrict__ perm, const int* __restrict__ invperm,
-                                int g, int act_order, uint8_t* __restrict__ codes,
+                                int g, int act_order, int preset, uint8_t* __restrict__ codes,
                                 int32_t* __restrict__ g_idx, int32_t* __restrict__ perm_out) {
     const int t0 = blockIdx.x * blockDim.x + threadIdx.x, stride = gridDim.x * blockDim.x;
     for (int c = t0; c < d_in; c += stride) {
-        g_idx[c] = invperm[c] / g;
+        g_idx[c] = (preset ? c : invperm[c]) / g;
         if (perm_out) perm_out[c] = perm[c];
     }
     if (!act_order) return;
@@ -279,12 +357,11 @@ __global__ void assemble_kernel(const uint8_t* __restrict__ codes_p, int d_out, 
 }
 
 gptq_status assemble_launch(const uint8_t* codes_p, int d_out, int d_in, const int* perm,
-                            const int* invperm, int group_size, int act_order, uint8_t* codes,
-                            int32_t* g_idx, int32_t* perm_out, cudaStream_t s) {
+                            const int* invperm, int group_size, int act_order, int preset,
+                            uint8_t* codes, int32_t* g_idx, int32_t* perm_out, cudaStream_t s) {
     const int blocks = std::max(1, std::min(std::max(d_out, (d_in + 255) / 256), num_sms() * 16));
-    assemble_kernel<<<blocks, 256, 0, s>>>(codes_p, d_out, d_in, perm, invperm,
-                                                       group_size, act_order, codes, g_idx,
-                                                       perm_out);
+    assemble_kernel<<<blocks, 256, 0, s>>>(codes_p, d_out, d_in, perm, invperm, group_size,
+                                           act_order, preset, codes, g_idx, perm_out);
     GPTQ_LAUNCHED();
     return GPTQ_OK;
 }
@@ -294,7 +371,7 @@ template <typename T>
 __global__ void __launch_bounds__(256) delta_sq_kernel(
     const T* __restrict__ W, int d_out, int d_in, const int* __restrict__ perm,
     const uint8_t* __restrict__ codes_p, const uint16_t* __restrict__ scales,
-    const uint16_t* __restrict__ zeros, int g, double* out) {
+    const uint16_t* __restrict__ zeros, int g, int preset, double* out) {
     const int ng = d_in / g;
     const float inv_g = 1.0f / static_cast<float>(g);
     double acc = 0.0;
@@ -302,10 +379,13 @@ __global__ void __launch_bounds__(256) delta_sq_kernel(
         const int64_t row = static_cast<int64_t>(r) * d_in;
         float part = 0.0f;
         for (int p = threadIdx.x; p < d_in; p += blockDim.x) {
-            // p / g from a float quotient, corrected by one either way (p < 2^17)
-            int q = __float2int_rz(static_cast<float>(p) * inv_g);
-            if (q * g > p) --q;
-            else if ((q + 1) * g <= p) ++q;
+            // the grid of processing position p: group of p, or with preset grids the group
+            // of its original column; the quotient from a float one, corrected by one either
+            // way (< 2^17)
+            const int c = preset ? perm[p] : p;
+            int q = __float2int_rz(static_cast<float>(c) * inv_g);
+            if (q * g > c) --q;
+            else if ((q + 1) * g <= c) ++q;
             const int64_t gi = static_cast<int64_t>(r) * ng + q;
             const float s = __half2float(__ushort_as_half(scales[gi]));
             const float z = __half2float(__ushort_as_half(zeros[gi]));
@@ -369,17 +449,17 @@ __global__ void __launch_bounds__(256) upper_dot_kernel(const float* __restrict_
 // fp16) takes the tf32x3 GEMM route: tr(W H W^T) with W and H in the processing order.
 gptq_status loss_launch(const void* W, int w_dtype, int d_out, int d_in, const float* H,
                         const int* perm, const uint8_t* codes_p, const uint16_t* scales,
-                        const uint16_t* zeros, int group_size, float* Wk, float* Hp,
+                        const uint16_t* zeros, int group_size, int preset, float* Wk, float* Hp,
                         DevState* st, cudaStream_t s) {
     const int blocks = std::min(d_out, num_sms() * 8);
     if (w_dtype == GPTQ_DTYPE_F16)
         delta_sq_kernel<__half><<<blocks, 256, 0, s>>>(static_cast<const __half*>(W), d_out,
                                                        d_in, perm, codes_p, scales, zeros,
-                                                       group_size, &st->delta_sq);
+                                                       group_size, preset, &st->delta_sq);
     else
         delta_sq_kernel<float><<<blocks, 256, 0, s>>>(static_cast<const float*>(W), d_out, d_in,
                                                       perm, codes_p, scales, zeros, group_size,
-                                                      &st->delta_sq);
+                                                      preset, &st->delta_sq);
     GPTQ_LAUNCHED();
     if (w_dtype == GPTQ_DTYPE_F16) {
         float* G = Hp;

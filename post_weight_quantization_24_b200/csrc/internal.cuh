@@ -21,7 +21,7 @@ constexpr int kSuperCols = 512;   // columns whose errors are collected before t
 
 // rtn.cu
 gptq_status rtn_launch(const void* W, int w_dtype, int d_out, int d_in, int bits,
-                       int group_size, uint8_t* out, uint16_t* scales, uint16_t* zeros,
+                       int group_size, int sym, uint8_t* out, uint16_t* scales, uint16_t* zeros,
                        cudaStream_t s);
 
 // hessian.cu
@@ -53,22 +53,30 @@ gptq_status factor_stall_set(int on);
 // img[R][k] = U[R][R+1+k] inside R's block of block_size columns (else 0); rdiag[R] = 1/U[R][R].
 gptq_status column_images_launch(const float* U, int d, int block_size, float* img, float* rdiag,
                                  cudaStream_t s);
-// The column loop of the block [j0, j0+bw), with img/rdiag as column_images_launch writes them
+// The column loop of the block [j0, j0+bw), with img/rdiag as column_images_launch writes them.
+// sym: symmetric quantizer. preset_perm != nullptr: the grids are preset in scales/zeros and
+// processing position p uses grid preset_perm[p] / group_size (else each group's grid is found
+// at its first column and written there).
 gptq_status gptq_block_launch(float* Wk, int d_out, int d_in, int j0, int bw, const float* img,
-                              const float* rdiag, int group_size, int bits, uint8_t* codes_p,
-                              uint16_t* scales, uint16_t* zeros, float* Err, float* ErrLo,
-                              int err_ld, double* err_sq, int* status, cudaStream_t s);
+                              const float* rdiag, int group_size, int bits, int sym,
+                              const int* preset_perm, uint8_t* codes_p, uint16_t* scales,
+                              uint16_t* zeros, float* Err, float* ErrLo, int err_ld,
+                              double* err_sq, int* status, cudaStream_t s);
+// Preset grids of the original weights: scales/zeros [d_out x d_in/group_size]
+gptq_status group_grid_launch(const void* W, int w_dtype, int d_out, int d_in, int group_size,
+                              int bits, int sym, uint16_t* scales, uint16_t* zeros,
+                              cudaStream_t s);
 // W[:, c0:c1] -= Err[:, 0:k1-k0] * U[k0:k1, c0:c1], both operands given as tf32 hi/lo parts
 gptq_status lazy_update_launch(float* Wk, int d_out, int d_in, int k0, int k1, int c0, int c1,
                                const float* U_hi, const float* U_lo, const float* Err_hi,
                                const float* Err_lo, int err_ld, const int* status,
                                cudaStream_t s);
 gptq_status assemble_launch(const uint8_t* codes_p, int d_out, int d_in, const int* perm,
-                            const int* invperm, int group_size, int act_order, uint8_t* codes,
-                            int32_t* g_idx, int32_t* perm_out, cudaStream_t s);
+                            const int* invperm, int group_size, int act_order, int preset,
+                            uint8_t* codes, int32_t* g_idx, int32_t* perm_out, cudaStream_t s);
 gptq_status loss_launch(const void* W, int w_dtype, int d_out, int d_in, const float* H,
                         const int* perm, const uint8_t* codes_p, const uint16_t* scales,
-                        const uint16_t* zeros, int group_size, float* Wk, float* Hp,
+                        const uint16_t* zeros, int group_size, int preset, float* Wk, float* Hp,
                         DevState* st, cudaStream_t s);
 
 }  // namespace gq

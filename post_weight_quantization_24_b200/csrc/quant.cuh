@@ -74,6 +74,33 @@ __device__ __forceinline__ QParams group_params(float xmin, float xmax, int maxq
     return p;
 }
 
+// The symmetric quantizer (0539edu.com §2.3: zero point fixed at 0, q = round(x/scale)): the
+// range is [-m, m], m = max(|xmin|, |xmax|), split into maxq steps, scale = smallest fp16 >=
+// 2m/maxq (1 for an all-zero group), and the signed zero 0 is stored as the code offset
+// (maxq + 1)/2, so code = clamp(rint(w/scale) + (maxq + 1)/2, 0, maxq).
+__device__ __forceinline__ QParams group_params_sym(float xmin, float xmax, int maxq) {
+    const double m = fmax(fabs(static_cast<double>(xmin)), fabs(static_cast<double>(xmax)));
+    const double s = (m == 0.0) ? 1.0 : fp16_ceil(2.0 * m / static_cast<double>(maxq));
+    QParams p;
+    p.scale = static_cast<float>(s);
+    p.zero = static_cast<float>((maxq + 1) / 2);
+    p.inv_scale = __frcp_rn(p.scale);
+    return p;
+}
+
+__device__ __forceinline__ QParams group_params_any(float xmin, float xmax, int maxq, bool sym) {
+    return sym ? group_params_sym(xmin, xmax, maxq) : group_params(xmin, xmax, maxq);
+}
+
+// A stored grid (fp16 scale and zero bit patterns) as the quantizer uses it.
+__device__ __forceinline__ QParams stored_params(uint16_t scale_bits, uint16_t zero_bits) {
+    QParams p;
+    p.scale = __half2float(__ushort_as_half(scale_bits));
+    p.zero = __half2float(__ushort_as_half(zero_bits));
+    p.inv_scale = __frcp_rn(p.scale);
+    return p;
+}
+
 // The same, kept out of line: for loops that reach it rarely (once per group) and would
 // otherwise carry one inlined copy of the fp64 sequence per unrolled iteration.
 static __device__ __noinline__ QParams group_params_call(float xmin, float xmax, int maxq) {

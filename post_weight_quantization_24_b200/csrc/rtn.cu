@@ -46,7 +46,7 @@ struct Load8<float> {
 // in [1, 32]. All loads of an iteration are issued before any arithmetic.
 template <typename T, int E, int TPG>
 __global__ void __launch_bounds__(256) rtn_kernel(const T* __restrict__ W, int64_t n_chunks,
-                                                  int bits, uint8_t* __restrict__ out,
+                                                  int bits, int sym, uint8_t* __restrict__ out,
                                                   uint16_t* __restrict__ scales,
                                                   uint16_t* __restrict__ zeros) {
     const int maxq = (1 << bits) - 1;
@@ -77,7 +77,7 @@ __global__ void __launch_bounds__(256) rtn_kernel(const T* __restrict__ W, int64
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
         }
         if (!ok) continue;
-        const QParams p = group_params(mn, mx, maxq);
+        const QParams p = group_params_any(mn, mx, maxq, sym != 0);
         int q[E];
 #pragma unroll
         for (int i = 0; i < E; ++i) q[i] = quant_code(v[i], p, maxq);
@@ -187,7 +187,7 @@ __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_gr
 // patterns and are packed with byte permutes. Chunk indices are 32-bit (the launcher checks).
 template <int TPG, bool INT4>
 __global__ void __launch_bounds__(rp::THREADS, 3) rtn_f16_kernel(const __half* __restrict__ W,
-                                                                int n_chunks, int bits,
+                                                                int n_chunks, int bits, int sym,
                                                                 uint8_t* __restrict__ out,
                                                                 uint16_t* __restrict__ scales,
                                                                 uint16_t* __restrict__ zeros) {
@@ -240,7 +240,7 @@ __global__ void __launch_bounds__(rp::THREADS, 3) rtn_f16_kernel(const __half* _
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
         }
         if (t >= n_chunks) continue;
-        const QParams p = group_params_stream(mn, mx, maxq);
+        const QParams p = sym ? group_params_sym(mn, mx, maxq) : group_params_stream(mn, mx, maxq);
         // m = fma(w, 1/scale, zero + 1.5 * 2^23): the product is exact inside the fma and the
         // single rounding (ulp 1 at 1.5 * 2^23) rounds w/scale + zero to the nearest integer,
         // half to even, leaving it in the low mantissa bits. Every w lies inside the group's
@@ -295,7 +295,7 @@ __global__ void __launch_bounds__(rp::THREADS, 3) rtn_f16_kernel(const __half* _
 }
 
 template <int TPG, bool INT4>
-static gptq_status launch_rtn_f16(const __half* W, int64_t n, int bits, uint8_t* out,
+static gptq_status launch_rtn_f16(const __half* W, int64_t n, int bits, int sym, uint8_t* out,
                                   uint16_t* scales, uint16_t* zeros, cudaStream_t s) {
     static bool attr = false;
     if (!attr) {
@@ -309,22 +309,24 @@ static gptq_status launch_rtn_f16(const __half* W, int64_t n, int bits, uint8_t*
     const int64_t want = (n_wit + rp::WARPS - 1) / rp::WARPS;
     const unsigned grid = static_cast<unsigned>(
         std::max<int64_t>(1, std::min<int64_t>(want, 3 * static_cast<int64_t>(num_sms()))));
-    rtn_f16_kernel<TPG, INT4><<<grid, rp::THREADS, rp::SMEM, s>>>(W, n_chunks, bits, out, scales, zeros);
+    rtn_f16_kernel<TPG, INT4><<<grid, rp::THREADS, rp::SMEM, s>>>(W, n_chunks, bits, sym, out,
+                                                                  scales, zeros);
     GPTQ_LAUNCHED();
     return GPTQ_OK;
 }
 
 template <int TPG>
-static gptq_status launch_rtn_f16_bits(const __half* W, int64_t n, int bits, uint8_t* out,
-                                       uint16_t* scales, uint16_t* zeros, cudaStream_t s) {
-    return bits == 4 ? launch_rtn_f16<TPG, true>(W, n, bits, out, scales, zeros, s)
-                     : launch_rtn_f16<TPG, false>(W, n, bits, out, scales, zeros, s);
+static gptq_status launch_rtn_f16_bits(const __half* W, int64_t n, int bits, int sym,
+                                       uint8_t* out, uint16_t* scales, uint16_t* zeros,
+                                       cudaStream_t s) {
+    return bits == 4 ? launch_rtn_f16<TPG, true>(W, n, bits, sym, out, scales, zeros, s)
+                     : launch_rtn_f16<TPG, false>(W, n, bits, sym, out, scales, zeros, s);
 }
 
 // Any group size: one thread per group.
 template <typename T>
 __global__ void rtn_generic_kernel(const T* __restrict__ W, int64_t n_groups, int group_size,
-                                   int bits, uint8_t* __restrict__ out,
+                                   int bits, int sym, uint8_t* __restrict__ out,
                                    uint16_t* __restrict__ scales, uint16_t* __restrict__ zeros) {
     const int maxq = (1 << bits) - 1;
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
@@ -337,7 +339,7 @@ __global__ void rtn_generic_kernel(const T* __restrict__ W, int64_t n_groups, in
             mn = fminf(mn, x);
             mx = fmaxf(mx, x);
         }
-        const QParams p = group_params(mn, mx, maxq);
+        const QParams p = group_params_any(mn, mx, maxq, sym != 0);
         for (int i = 0; i < group_size; ++i) {
             const int64_t e = gi * group_size + i;
             const int q = quant_code(static_cast<float>(w[i]), p, maxq);
@@ -357,17 +359,17 @@ __global__ void rtn_generic_kernel(const T* __restrict__ W, int64_t n_groups, in
 }
 
 template <typename T>
-static gptq_status launch_rtn(const T* W, int64_t n, int group_size, int bits, uint8_t* out,
-                              uint16_t* scales, uint16_t* zeros, cudaStream_t s) {
+static gptq_status launch_rtn(const T* W, int64_t n, int group_size, int bits, int sym,
+                              uint8_t* out, uint16_t* scales, uint16_t* zeros, cudaStream_t s) {
     const int sms = num_sms();
     const bool pow2 = (group_size & (group_size - 1)) == 0;
     if (std::is_same<T, __half>::value && pow2 && group_size >= 32 && group_size <= 256 &&
         n / rp::E < (int64_t(1) << 31) - 64) {
         const __half* Wh = reinterpret_cast<const __half*>(W);
-        if (group_size == 32) GPTQ_TRY(launch_rtn_f16_bits<1>(Wh, n, bits, out, scales, zeros, s));
-        else if (group_size == 64) GPTQ_TRY(launch_rtn_f16_bits<2>(Wh, n, bits, out, scales, zeros, s));
-        else if (group_size == 128) GPTQ_TRY(launch_rtn_f16_bits<4>(Wh, n, bits, out, scales, zeros, s));
-        else GPTQ_TRY(launch_rtn_f16_bits<8>(Wh, n, bits, out, scales, zeros, s));
+        if (group_size == 32) GPTQ_TRY(launch_rtn_f16_bits<1>(Wh, n, bits, sym, out, scales, zeros, s));
+        else if (group_size == 64) GPTQ_TRY(launch_rtn_f16_bits<2>(Wh, n, bits, sym, out, scales, zeros, s));
+        else if (group_size == 128) GPTQ_TRY(launch_rtn_f16_bits<4>(Wh, n, bits, sym, out, scales, zeros, s));
+        else GPTQ_TRY(launch_rtn_f16_bits<8>(Wh, n, bits, sym, out, scales, zeros, s));
         return GPTQ_OK;
     } else if (group_size % 8 == 0 && group_size <= 256 && pow2) {
         // 16 weights per thread when the group allows it, else 8
@@ -380,14 +382,14 @@ static gptq_status launch_rtn(const T* W, int64_t n, int group_size, int bits, u
         const dim3 grid(static_cast<unsigned>(blocks)), block(256);
         if (E == 16) {
             switch (group_size / 16) {
-                case 1: rtn_kernel<T, 16, 1><<<grid, block, 0, s>>>(W, n_chunks, bits, out, scales, zeros); break;
-                case 2: rtn_kernel<T, 16, 2><<<grid, block, 0, s>>>(W, n_chunks, bits, out, scales, zeros); break;
-                case 4: rtn_kernel<T, 16, 4><<<grid, block, 0, s>>>(W, n_chunks, bits, out, scales, zeros); break;
-                case 8: rtn_kernel<T, 16, 8><<<grid, block, 0, s>>>(W, n_chunks, bits, out, scales, zeros); break;
-                default: rtn_kernel<T, 16, 16><<<grid, block, 0, s>>>(W, n_chunks, bits, out, scales, zeros); break;
+                case 1: rtn_kernel<T, 16, 1><<<grid, block, 0, s>>>(W, n_chunks, bits, sym, out, scales, zeros); break;
+                case 2: rtn_kernel<T, 16, 2><<<grid, block, 0, s>>>(W, n_chunks, bits, sym, out, scales, zeros); break;
+                case 4: rtn_kernel<T, 16, 4><<<grid, block, 0, s>>>(W, n_chunks, bits, sym, out, scales, zeros); break;
+                case 8: rtn_kernel<T, 16, 8><<<grid, block, 0, s>>>(W, n_chunks, bits, sym, out, scales, zeros); break;
+                default: rtn_kernel<T, 16, 16><<<grid, block, 0, s>>>(W, n_chunks, bits, sym, out, scales, zeros); break;
             }
         } else {
-            rtn_kernel<T, 8, 1><<<grid, block, 0, s>>>(W, n_chunks, bits, out, scales, zeros);
+            rtn_kernel<T, 8, 1><<<grid, block, 0, s>>>(W, n_chunks, bits, sym, out, scales, zeros);
         }
     } else {
         const int64_t n_groups = n / group_size;
@@ -397,20 +399,22 @@ static gptq_status launch_rtn(const T* W, int64_t n, int group_size, int bits, u
         if (blocks > cap) blocks = cap;
         if (blocks < 1) blocks = 1;
         rtn_generic_kernel<T><<<static_cast<unsigned>(blocks), 128, 0, s>>>(
-            W, n_groups, group_size, bits, out, scales, zeros);
+            W, n_groups, group_size, bits, sym, out, scales, zeros);
     }
     GPTQ_LAUNCHED();
     return GPTQ_OK;
 }
 
 gptq_status rtn_launch(const void* W, int w_dtype, int d_out, int d_in, int bits,
-                       int group_size, uint8_t* out, uint16_t* scales, uint16_t* zeros,
+                       int group_size, int sym, uint8_t* out, uint16_t* scales, uint16_t* zeros,
                        cudaStream_t s) {
     const int64_t n = static_cast<int64_t>(d_out) * d_in;
     if (n == 0) return GPTQ_OK;
     if (w_dtype == GPTQ_DTYPE_F16)
-        return launch_rtn(static_cast<const __half*>(W), n, group_size, bits, out, scales, zeros, s);
-    return launch_rtn(static_cast<const float*>(W), n, group_size, bits, out, scales, zeros, s);
+        return launch_rtn(static_cast<const __half*>(W), n, group_size, bits, sym, out, scales,
+                          zeros, s);
+    return launch_rtn(static_cast<const float*>(W), n, group_size, bits, sym, out, scales, zeros,
+                      s);
 }
 
 }  // namespace gq

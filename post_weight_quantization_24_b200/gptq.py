@@ -63,6 +63,20 @@ _SIGNATURES = {
     "gptq_inverse_factor_workspace": ([_I], _SZ),
     "gptq_inverse_factor": ([_P, _I, _F, _I, _P, _P, _P, _SZ, _P], _I),
     "rtn_minmax_quantize": ([_P, _I, _I, _I, _I, _I, _P, _P, _P, _P], _I),
+    "gptq_quantize_layer_ex": ([_P, _I, _I, _I, _P, _I, _I, _I, _F, _I, _I, _I, _P, _P, _P, _P,
+                                _P, ctypes.POINTER(_F), _P, _SZ, _P], _I),
+    "rtn_quantize_ex": ([_P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P], _I),
+    "rtn_clip_search": ([_P, _I, _I, _I, _I, _I, _I, _P, ctypes.c_double, ctypes.c_double, _P,
+                         _P, _P, _P, _P], _I),
+    "w4a16_pack": ([_P, _I, _I, _P, _P, _P], _I),
+    "w4a16_linear_workspace": ([_I64, _I, _I], _SZ),
+    "w4a16_linear": ([_P, _I64, _I, _P, _P, _P, _I, _I, _P, _P, _P, _P, _SZ, _P, _P], _I),
+    "gptq_silu_mul": ([_P, _I64, _I, _P, _P], _I),
+    "gptq_channel_abs_sum": ([_P, _I, _I64, _I, _P, _P], _I),
+    "awq_lite_workspace": ([_I, _I, ctypes.c_double], _SZ),
+    "awq_lite_search": ([_P, _I, _I, _I, _P, _I64, _P, _I, _I, _I, ctypes.c_double, _P, _P, _P,
+                         _P, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_I), _P, _SZ, _P],
+                        _I),
     "gptq_quantize_layer_noalloc": ([_P, _I, _I, _I, _P, _I, _I, _I, _F, _I, _P, _P, _P, _P, _P,
                                      ctypes.POINTER(_F), _P], _I),
     "gptq_profile_enable": ([_I], None),
@@ -202,11 +216,13 @@ def quantize_layer_workspace(d_out: int, d_in: int, block_size: int = 128) -> in
 def quantize_layer(W: torch.Tensor, H: torch.Tensor, bits: int = 4, group_size: int = 128,
                    block_size: int = 128, percdamp: float = 0.01, act_order: bool = False,
                    compute_loss: bool = False, workspace: torch.Tensor | None = None,
-                   out: dict | None = None) -> dict:
+                   out: dict | None = None, sym: bool = False,
+                   static_groups: bool = False) -> dict:
     """GPTQ-quantize W [d_out, d_in] (fp16/fp32) with Hessian H [d_in, d_in] (upper read).
 
     Returns dict(codes uint8 [d_out, d_in] original order, scales/zeros fp16 [d_out, d_in/g],
-    g_idx int32 [d_in], perm int32 [d_in], loss float | None).
+    g_idx int32 [d_in], perm int32 [d_in], loss float | None). ``sym``, ``static_groups`` and
+    group_size == d_in (per-channel) select the quantizer variants of gptq_quantize_layer_ex.
     """
     _require_cuda(W, "W")
     _require_cuda(H, "H")
@@ -225,13 +241,14 @@ def quantize_layer(W: torch.Tensor, H: torch.Tensor, bits: int = 4, group_size: 
         nbytes = quantize_layer_workspace(d_out, d_in, block_size)
         workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=dev)
     loss = ctypes.c_float(float("nan"))
-    st = lib().gptq_quantize_layer(
+    st = lib().gptq_quantize_layer_ex(
         W.data_ptr(), _dtype_code(W), d_out, d_in, H.data_ptr(), bits, group_size, block_size,
-        float(percdamp), int(bool(act_order)), out["codes"].data_ptr(), out["scales"].data_ptr(),
-        out["zeros"].data_ptr(), out["g_idx"].data_ptr(), _ptr(out.get("perm")),
+        float(percdamp), int(bool(act_order)), int(bool(sym)), int(bool(static_groups)),
+        out["codes"].data_ptr(), out["scales"].data_ptr(), out["zeros"].data_ptr(),
+        out["g_idx"].data_ptr(), _ptr(out.get("perm")),
         ctypes.byref(loss) if compute_loss else None, workspace.data_ptr(),
         workspace.numel(), _stream())
-    _check(st, "gptq_quantize_layer")
+    _check(st, "gptq_quantize_layer_ex")
     res = dict(out)
     res["loss"] = float(loss.value) if compute_loss else None
     return res
@@ -289,10 +306,11 @@ def inverse_factor(H: torch.Tensor, percdamp: float = 0.01, act_order: bool = Fa
 # RTN
 # ------------------------------------------------------------------------------------------
 def rtn_minmax_quantize(W: torch.Tensor, bits: int = 4, group_size: int = 128,
-                        out: tuple | None = None):
+                        out: tuple | None = None, sym: bool = False):
     """Group min-max RTN of W [d_out, d_in] -> (packed uint8, scales fp16, zeros fp16).
 
     bits == 4: packed is [d_out, d_in/2] (even column in the low nibble); else [d_out, d_in].
+    ``sym`` takes the symmetric quantizer (rtn_quantize_ex).
     """
     _require_cuda(W, "W")
     d_out, d_in = W.shape
@@ -303,11 +321,123 @@ def rtn_minmax_quantize(W: torch.Tensor, bits: int = 4, group_size: int = 128,
         out = (packed, torch.empty(d_out, ng, dtype=torch.float16, device=dev),
                torch.empty(d_out, ng, dtype=torch.float16, device=dev))
     packed, scales, zeros = out
-    st = lib().rtn_minmax_quantize(W.data_ptr(), _dtype_code(W), d_out, d_in, bits, group_size,
-                                   packed.data_ptr(), scales.data_ptr(), zeros.data_ptr(),
-                                   _stream())
-    _check(st, "rtn_minmax_quantize")
+    st = lib().rtn_quantize_ex(W.data_ptr(), _dtype_code(W), d_out, d_in, bits, group_size,
+                               int(bool(sym)), packed.data_ptr(), scales.data_ptr(),
+                               zeros.data_ptr(), _stream())
+    _check(st, "rtn_quantize_ex")
     return packed, scales, zeros
+
+
+def rtn_clip_search(W: torch.Tensor, bits: int = 4, group_size: int = 128,
+                    H: torch.Tensor | None = None, sym: bool = False, min_ratio: float = 0.5,
+                    step: float = 0.05):
+    """Group RTN with a clip search per group (criterion d·H_gg·d, or d·d without H) ->
+    (packed uint8, scales fp16, zeros fp16, ratio index uint8 [d_out, d_in/g])."""
+    _require_cuda(W, "W")
+    d_out, d_in = W.shape
+    dev = W.device
+    ng = d_in // group_size if group_size > 0 and d_in % group_size == 0 else 1
+    packed = torch.empty(d_out, d_in // 2 if bits == 4 else d_in, dtype=torch.uint8, device=dev)
+    scales = torch.empty(d_out, ng, dtype=torch.float16, device=dev)
+    zeros = torch.empty(d_out, ng, dtype=torch.float16, device=dev)
+    ridx = torch.empty(d_out, ng, dtype=torch.uint8, device=dev)
+    if H is not None:
+        _require_cuda(H, "H")
+        if H.dtype != torch.float32 or H.shape != (d_in, d_in):
+            raise ValueError("H must be fp32 [d_in, d_in]")
+    st = lib().rtn_clip_search(W.data_ptr(), _dtype_code(W), d_out, d_in, bits, group_size,
+                               int(bool(sym)), _ptr(H), float(min_ratio), float(step),
+                               packed.data_ptr(), scales.data_ptr(), zeros.data_ptr(),
+                               ridx.data_ptr(), _stream())
+    _check(st, "rtn_clip_search")
+    return packed, scales, zeros, ridx
+
+
+# ------------------------------------------------------------------------------------------
+# W4A16 layer
+# ------------------------------------------------------------------------------------------
+def w4a16_pack(codes: torch.Tensor, perm: torch.Tensor | None = None) -> torch.Tensor:
+    """INT4 codes [d_out, d_in] (original order) -> packed [d_out, d_in/2] in perm's order."""
+    _require_cuda(codes, "codes")
+    d_out, d_in = codes.shape
+    packed = torch.empty(d_out, d_in // 2, dtype=torch.uint8, device=codes.device)
+    _check(lib().w4a16_pack(codes.data_ptr(), d_out, d_in, _ptr(perm), packed.data_ptr(),
+                            _stream()), "w4a16_pack")
+    return packed
+
+
+def w4a16_linear(X: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor,
+                 zeros: torch.Tensor, group_size: int = 128, perm: torch.Tensor | None = None,
+                 R: torch.Tensor | None = None, out: torch.Tensor | None = None,
+                 workspace: torch.Tensor | None = None,
+                 status: torch.Tensor | None = None) -> torch.Tensor:
+    """Y = fp16(X·Ŵᵀ + R) for fp16 X [n, d_in] and packed INT4 weights [d_out, d_in/2]."""
+    _require_cuda(X, "X")
+    n, d_in = X.shape
+    d_out = packed.shape[0]
+    if out is None:
+        out = torch.empty(n, d_out, dtype=torch.float16, device=X.device)
+    nb = int(lib().w4a16_linear_workspace(n, d_in, int(perm is not None)))
+    if perm is not None and (workspace is None or workspace.numel() < nb):
+        workspace = torch.empty(nb, dtype=torch.uint8, device=X.device)
+    st = lib().w4a16_linear(X.data_ptr(), n, d_in, packed.data_ptr(), scales.data_ptr(),
+                            zeros.data_ptr(), group_size, d_out, _ptr(perm), _ptr(R),
+                            out.data_ptr(), _ptr(workspace),
+                            0 if workspace is None else workspace.numel(), _ptr(status),
+                            _stream())
+    _check(st, "w4a16_linear")
+    return out
+
+
+def channel_abs_sum(X: torch.Tensor, sums: torch.Tensor | None = None) -> torch.Tensor:
+    """sums[c] += Σ_t |X[t, c]| (fp64 [d]); a new zeroed buffer when `sums` is None."""
+    _require_cuda(X, "X")
+    n, d = X.shape
+    if sums is None:
+        sums = torch.zeros(d, dtype=torch.float64, device=X.device)
+    _check(lib().gptq_channel_abs_sum(X.data_ptr(), _dtype_code(X), n, d, sums.data_ptr(),
+                                      _stream()), "gptq_channel_abs_sum")
+    return sums
+
+
+def awq_lite_search(W: torch.Tensor, x_abs_sum: torch.Tensor, n_tokens: int, H: torch.Tensor,
+                    bits: int = 4, group_size: int = 128, sym: bool = False,
+                    alpha_step: float = 0.1) -> dict:
+    """AWQ-lite grid search (H full symmetric). Returns dict(packed, scales, zeros, s (fp16
+    [d_in]), losses (list), best (index), alpha)."""
+    _require_cuda(W, "W")
+    _require_cuda(H, "H")
+    d_out, d_in = W.shape
+    dev = W.device
+    ng = d_in // group_size
+    n_alpha = int(round(1.0 / alpha_step)) + 1
+    packed = torch.empty(d_out, d_in // 2 if bits == 4 else d_in, dtype=torch.uint8, device=dev)
+    scales = torch.empty(d_out, ng, dtype=torch.float16, device=dev)
+    zeros = torch.empty(d_out, ng, dtype=torch.float16, device=dev)
+    s_out = torch.empty(d_in, dtype=torch.float16, device=dev)
+    ws = torch.empty(max(1, int(lib().awq_lite_workspace(d_out, d_in, float(alpha_step)))),
+                     dtype=torch.uint8, device=dev)
+    losses = (ctypes.c_double * n_alpha)()
+    best = ctypes.c_int(-1)
+    st = lib().awq_lite_search(W.data_ptr(), _dtype_code(W), d_out, d_in, x_abs_sum.data_ptr(),
+                               int(n_tokens), H.data_ptr(), bits, group_size, int(bool(sym)),
+                               float(alpha_step), packed.data_ptr(), scales.data_ptr(),
+                               zeros.data_ptr(), s_out.data_ptr(), losses, ctypes.byref(best),
+                               ws.data_ptr(), ws.numel(), _stream())
+    _check(st, "awq_lite_search")
+    return dict(packed=packed, scales=scales, zeros=zeros, s=s_out, losses=list(losses),
+                best=int(best.value), alpha=int(best.value) * alpha_step)
+
+
+def silu_mul(GU: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+    """A = fp16(silu(gate)·up) for GU fp16 [n, 2·d_ff] (gate outputs, then up outputs)."""
+    _require_cuda(GU, "GU")
+    n, two = GU.shape
+    if out is None:
+        out = torch.empty(n, two // 2, dtype=torch.float16, device=GU.device)
+    _check(lib().gptq_silu_mul(GU.data_ptr(), n, two // 2, out.data_ptr(), _stream()),
+           "gptq_silu_mul")
+    return out
 
 
 # ------------------------------------------------------------------------------------------

@@ -79,10 +79,11 @@ def _fp16_below(s):
 
 def window_from_h_sensitivity(W, H, bits, g, B, percdamp, act_order, ref_trace, rows,
                               U_pert=None, H_pert=None, route="textbook", rel=1e-5,
-                              safety=2.0):
+                              safety=2.0, **variant):
     """The tie window eps (see the module docstring), from the oracle run on H and on a
     perturbed H over the sampled ``rows``. ``ref_trace`` is the oracle's traced result for
-    those rows on H. Returns (eps, detail)."""
+    those rows on H; ``variant`` are the quantizer switches of ``gptq_blocked_ref``.
+    Returns (eps, detail)."""
     if U_pert is None:
         if H_pert is None:
             H_pert = perturbed_hessian(H, rel)
@@ -90,7 +91,7 @@ def window_from_h_sensitivity(W, H, bits, g, B, percdamp, act_order, ref_trace, 
     if H_pert is None:
         H_pert = perturbed_hessian(H, rel)
     alt = ogptq.gptq_blocked_ref(W, H_pert, bits, g, B, percdamp, act_order, rows=rows,
-                                 U=U_pert, trace=True)
+                                 U=U_pert, trace=True, **variant)
     first, _ = first_divergence(ref_trace["codes_p"], alt["codes_p"], ref_trace["scales"],
                                 ref_trace["zeros"], alt["scales"], alt["zeros"], g)
     moved = np.flatnonzero(alt["perm"] != ref_trace["perm"])
@@ -98,7 +99,10 @@ def window_from_h_sensitivity(W, H, bits, g, B, percdamp, act_order, ref_trace, 
         # a perturbation that reorders act_order's keys changes the columns from the first
         # moved position on: compare only the positions before it
         first = np.minimum(first, int(moved[0]))
-    gi = np.arange(ref_trace["pre"].shape[1]) // g
+    if variant.get("static_groups"):
+        gi = np.asarray(ref_trace["perm"]) // g
+    else:
+        gi = np.arange(ref_trace["pre"].shape[1]) // g
     s_col = ref_trace["scales"][:, gi]
     dev = np.abs(ref_trace["pre"] - alt["pre"]) / s_col
     mask = np.arange(dev.shape[1])[None, :] < first[:, None]
@@ -109,12 +113,15 @@ def window_from_h_sensitivity(W, H, bits, g, B, percdamp, act_order, ref_trace, 
     return safety * eps_meas, detail
 
 
-def near_tie_report(codes, scales, zeros, perm, ref_trace, g, bits, eps, rows=None):
+def near_tie_report(codes, scales, zeros, perm, ref_trace, g, bits, eps, rows=None,
+                    static_groups=False):
     """Check every row of a GPU result against the oracle's traced result (same rows).
 
     codes: GPU codes [rows, d] in the ORIGINAL column order; scales/zeros [rows, d/g]; perm the
-    GPU's processing order (must equal the oracle's). Returns a dict of statistics; the
-    parity criterion is ``bad_origin == 0``."""
+    GPU's processing order (must equal the oracle's). With static groups every grid is fixed
+    from the original weights before the first column, so a grid difference is the row's
+    first divergence. Returns a dict of statistics; the parity criterion is
+    ``bad_origin == 0``."""
     maxq = 2 ** bits - 1
     codes = np.asarray(codes).astype(np.int64)
     cg = codes[:, perm]
@@ -124,13 +131,19 @@ def near_tie_report(codes, scales, zeros, perm, ref_trace, g, bits, eps, rows=No
     so, zo = ref_trace["scales"], ref_trace["zeros"]
     first, kind = first_divergence(cg, co, sg, zg, so, zo, g)
     d = cg.shape[1]
+    if static_groups:
+        grid_diff = np.any((sg != so) | (zg != zo), axis=1)
+        kind = np.where(grid_diff, "param", kind)
+        k_static = np.where(grid_diff, ((sg != so) | (zg != zo)).argmax(1), 0)
+        first = np.where(grid_diff, 0, first)
     diff = cg - co
     bad_rows = []
     for r in np.flatnonzero(first < d):
         q = int(first[r])
-        k = q // g
+        k = int(k_static[r]) if static_groups and kind[r] == "param" else q // g
         if kind[r] == "code":
-            t = ref_trace["pre"][r, q] / so[r, k]
+            kk = int(perm[q]) // g if static_groups else k
+            t = ref_trace["pre"][r, q] / so[r, kk]
             ok = _code_tie_dist(t) <= eps
             why = dict(t=float(t), dist=float(_code_tie_dist(t)))
         else:
@@ -145,7 +158,7 @@ def near_tie_report(codes, scales, zeros, perm, ref_trace, g, bits, eps, rows=No
         if not ok:
             bad_rows.append(dict(row=int(r if rows is None else rows[r]), col=q,
                                  kind=str(kind[r]), **why))
-    gi = np.arange(d) // g
+    gi = (np.asarray(perm) // g) if static_groups else np.arange(d) // g
     t_all = ref_trace["pre"] / so[:, gi]
     n_near = int(np.sum(_code_tie_dist(t_all) <= eps))
     hist = {int(k): int(v) for k, v in zip(*np.unique(diff, return_counts=True))}

@@ -60,19 +60,21 @@ def rel_fro_blocked(Hg, Href, block=4096):
 
 
 def oracle_ref(Wn, Href, bits, g, B, act_order, percdamp=0.01, rows=None, U=None,
-               route="textbook", n_window_rows=64, U_pert=None, H_pert=None):
-    """The oracle's traced result, and the tie window derived from its sensitivity to H."""
+               route="textbook", n_window_rows=64, U_pert=None, H_pert=None, **variant):
+    """The oracle's traced result, and the tie window derived from its sensitivity to H.
+    ``variant``: the quantizer switches (sym, static_groups) of gptq_blocked_ref."""
     if U is None:
         _, U = ogptq.prepare_u(Href, percdamp, act_order, route=route)
     ref = ogptq.gptq_blocked_ref(Wn, Href, bits, g, B, percdamp, act_order, rows=rows, U=U,
-                                 trace=True)
+                                 trace=True, **variant)
     n = ref["codes"].shape[0]
     sel = np.sort(np.random.default_rng(1).choice(n, min(n_window_rows, n), replace=False))
     sub = {k: ref[k][sel] for k in ("pre", "codes_p", "scales", "zeros", "step", "zquot")}
     sub["perm"] = ref["perm"]
     wrows = sel if rows is None else np.asarray(rows)[sel]
     eps, detail = window_from_h_sensitivity(Wn, Href, bits, g, B, percdamp, act_order, sub,
-                                            wrows, U_pert=U_pert, H_pert=H_pert, route=route)
+                                            wrows, U_pert=U_pert, H_pert=H_pert, route=route,
+                                            **variant)
     return ref, eps, detail
 
 
@@ -86,21 +88,22 @@ def gpu_what(codes, scales, zeros, g_idx):
     return scales[:, g_idx].astype(np.float64) * (codes.astype(np.float64) - zeros[:, g_idx])
 
 
-def check_near_ties(out, ref, g, bits, eps, detail, rows=None):
+def check_near_ties(out, ref, g, bits, eps, detail, rows=None, static_groups=False):
     codes, sc, zr, perm = gpu_outputs(out, rows)
     assert np.array_equal(perm, ref["perm"])
-    rep = near_tie_report(codes, sc, zr, perm, ref, g, bits, eps, rows=rows)
+    rep = near_tie_report(codes, sc, zr, perm, ref, g, bits, eps, rows=rows,
+                          static_groups=static_groups)
     log_parity(window=detail, **rep)
     assert rep["bad_origin"] == 0, rep["bad_examples"]
     return rep
 
 
-def check_outputs(out, ref, Wn, Href, g, bits, eps, detail, max_diff=1):
+def check_outputs(out, ref, Wn, Href, g, bits, eps, detail, max_diff=1, static_groups=False):
     """Small and medium cases: strict one-level mismatches, plus the near-tie origin of every
     differing row."""
     assert np.array_equal(out["perm"].cpu().numpy(), ref["perm"])
     assert np.array_equal(out["g_idx"].cpu().numpy(), ref["g_idx"])
-    rep = check_near_ties(out, ref, g, bits, eps, detail)
+    rep = check_near_ties(out, ref, g, bits, eps, detail, static_groups=static_groups)
     assert rep["agree"] >= 0.99, rep
     if max_diff is not None:
         assert rep["max_abs_diff"] <= max_diff, rep
@@ -128,14 +131,14 @@ def full_size_checks(out, ref, Wn, Href, Hg, g, bits, eps, detail):
     return rep
 
 
-def run_case(lib, W, X, bits, g, B, act_order, percdamp=0.01):
+def run_case(lib, W, X, bits, g, B, act_order, percdamp=0.01, **variant):
     H = gpu_hessian(lib, X)
     out = lib.quantize_layer(W, H, bits=bits, group_size=g, block_size=B, percdamp=percdamp,
-                             act_order=act_order, compute_loss=True)
+                             act_order=act_order, compute_loss=True, **variant)
     torch.cuda.synchronize()
     Wn = W.float().cpu().numpy().astype(np.float64)
     Href = ohess.hessian(X.cpu().numpy())
-    ref, eps, detail = oracle_ref(Wn, Href, bits, g, B, act_order, percdamp)
+    ref, eps, detail = oracle_ref(Wn, Href, bits, g, B, act_order, percdamp, **variant)
     return out, ref, Wn, Href, H, eps, detail
 
 
