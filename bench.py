@@ -413,6 +413,112 @@ def configs_measure(gptq, device, flush, peaks, clock_mhz, steps=3, warmup=3):
     return res
 
 
+def _events():
+    return torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+
+def w4a16_measure(gptq, device, peaks, n_tokens=16384, d_in=4096, d_out=22016, reps=5):
+    """The W4A16 layer on the 7B MLP-in shape (gate;up stacked: 22016 x 4096, INT4 g128) over
+    16384 tokens, with and without the act_order gather. Algorithmic flops 2·n·d_out·d_in."""
+    wl = workloads.WORKLOADS["mlp_up_7b"]
+    W = workloads.make_weights(wl.replace(d_out=d_out, d_in=d_in), device=device)
+    packed, scales, zeros = gptq.rtn_minmax_quantize(W, 4, 128)
+    X = workloads.make_activations(wl.replace(d_in=d_in, n_tokens=n_tokens), device=device)
+    Y = torch.empty(n_tokens, d_out, dtype=torch.float16, device=device)
+    perm = torch.randperm(d_in, device=device).to(torch.int32)
+    ws = torch.empty(gptq.lib().w4a16_linear_workspace(n_tokens, d_in, 1), dtype=torch.uint8,
+                     device=device)
+    out = {}
+    flops = 2.0 * n_tokens * d_out * d_in
+    for name, pm in (("plain", None), ("act_order_gather", perm)):
+        for _ in range(2):
+            gptq.w4a16_linear(X, packed, scales, zeros, 128, perm=pm, out=Y, workspace=ws)
+        a, b = _events()
+        a.record()
+        for _ in range(reps):
+            gptq.w4a16_linear(X, packed, scales, zeros, 128, perm=pm, out=Y, workspace=ws)
+        b.record()
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b) / reps
+        tf = flops / (ms / 1e3) / 1e12
+        out[name] = {"ms": ms, "tflops": tf, "bound": "tensor", "peak_tflops": peaks["bf16_tflops"],
+                     "frac": tf / peaks["bf16_tflops"]}
+    out["workload"] = (f"X {n_tokens}x{d_in} fp16, W {d_out}x{d_in} INT4 g128 (7B gate;up), "
+                       "fp32 accumulate, fp16 out")
+    del W, X, Y, ws
+    torch.cuda.empty_cache()
+    return out
+
+
+def sequential_measure(gptq, device, peaks, n_blocks=2, n_tokens=65536, d=4096, d_ff=11008):
+    """Layer-by-layer GPTQ of `n_blocks` 7B-shaped gated-MLP blocks (gate;up 22016 x 4096,
+    down 4096 x 11008, INT4 g128), each layer's Hessian from the W4A16 outputs of the layers
+    before it, over 65536 calibration tokens."""
+    from post_weight_quantization_24_b200 import sequential
+    g = torch.Generator(device=device).manual_seed(77)
+    blocks = []
+    for _ in range(n_blocks):
+        f = lambda r, c: (0.02 * torch.randn(r, c, generator=g, device=device)).to(torch.float16)
+        blocks.append((f(d_ff, d), f(d_ff, d), f(d, d_ff)))
+    X0 = workloads.make_activations(workloads.WORKLOADS["mlp_up_7b"].replace(
+        d_in=d, n_tokens=n_tokens, seed=78), device=device)
+    sequential.quantize_mlp_stack(X0, blocks[:1])            # warm-up (one block)
+    torch.cuda.synchronize()
+    timings = {}
+    a, b = _events()
+    a.record()
+    _, recs = sequential.quantize_mlp_stack(X0, blocks, timings=timings)
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b)
+    w4_flops = n_blocks * 2.0 * n_tokens * (2 * d_ff * d + d * d_ff)
+    h_flops = n_blocks * float(n_tokens) * (d * (d + 1) + d_ff * (d_ff + 1))
+    out = {"blocks": n_blocks, "tokens": n_tokens, "ms": ms,
+           "layers_per_s": 2 * n_blocks / (ms / 1e3),
+           "weights_per_s": n_blocks * 3 * d * d_ff / (ms / 1e3),
+           "stage_ms": timings,
+           "w4a16_frac": w4_flops / (timings.get("w4a16", 1e-9) / 1e3) / 1e12 / peaks["bf16_tflops"],
+           "hessian_frac": h_flops / (timings.get("hessian", 1e-9) / 1e3) / 1e12 / peaks["bf16_tflops"],
+           "losses": {r["name"]: r["loss"] for r in recs},
+           "workload": f"{n_blocks} gated-MLP blocks d={d} d_ff={d_ff}, {n_tokens} tokens, INT4 g128"}
+    del blocks, X0, recs
+    torch.cuda.empty_cache()
+    return out
+
+
+def awq_clip_measure(gptq, device, peaks, reps=3):
+    """AWQ-lite (11 alphas) and the RTN clip search (11 ratios, H criterion) on the mlp_up_7b
+    weights, H from 65536 tokens of its activations."""
+    wl = workloads.WORKLOADS["mlp_up_7b"]
+    W = workloads.make_weights(wl, device=device)
+    X = workloads.make_activations(wl.replace(n_tokens=65536), device=device)
+    h = gptq.Hessian(wl.d_in)
+    h.accumulate(X)
+    H = h.get()
+    sums = gptq.channel_abs_sum(X)
+    res = {}
+    for name, fn in (("awq_lite", lambda: gptq.awq_lite_search(W, sums, X.shape[0], H)),
+                     ("rtn_clip_search", lambda: gptq.rtn_clip_search(W, 4, 128, H=H))):
+        fn()
+        torch.cuda.synchronize()
+        a, b = _events()
+        a.record()
+        for _ in range(reps):
+            r = fn()
+        b.record()
+        torch.cuda.synchronize()
+        res[name] = {"ms": a.elapsed_time(b) / reps}
+        if name == "awq_lite":
+            res[name]["alpha"] = r["alpha"]
+            d, n_a = wl.d_in, len(r["losses"])
+            fl = n_a * 2.0 * wl.d_out * d * d       # the loss GEMMs, fp32-equivalent
+            res[name]["loss_gemm_tflops_equiv"] = fl / (res[name]["ms"] / 1e3) / 1e12
+    res["workload"] = "W 11008x4096 fp16 INT4 g128; H over 65536 tokens"
+    del W, X, H, h
+    torch.cuda.empty_cache()
+    return res
+
+
 def stack_measure(gptq, device, peaks, clock_mhz, n_layers=32, n_tokens=131072,
                   variants=((128, False), (128, True), (64, False), (64, True))):
     """GPTQ over a full 7B-shaped decoder stack, end to end: for each of `n_layers` layers,
@@ -585,6 +691,16 @@ def run_ours(args):
     configs = None
     if extras and not args.no_configs:
         configs = configs_measure(gptq, device, flush, peaks, clock_mhz)
+    more = {}
+    if extras and not args.no_configs:
+        for key, fn in (("w4a16", lambda: w4a16_measure(gptq, device, peaks)),
+                        ("sequential_mlp_7b", lambda: sequential_measure(gptq, device, peaks)),
+                        ("awq_clip", lambda: awq_clip_measure(gptq, device, peaks))):
+            try:
+                more[key] = fn()
+            except Exception as exc:                  # reported in the line, never fatal
+                more[key] = {"error": f"{type(exc).__name__}: {exc}"[:300]}
+                torch.cuda.empty_cache()
     stack = None
     if extras and not args.no_stack:
         try:
@@ -635,6 +751,7 @@ def run_ours(args):
         "stages": stages,
         "configs": configs,
         "stack_7b": stack,
+        "next_rows": more or None,
         "roofline": roof,
         "clocks": clocks,
         "gpu_launches": launches,
@@ -740,13 +857,21 @@ def oracle_sample(W_np, X_np, wl, n_tok, n_rows, n_rtn_rows, seed=0):
     return full, measured, detail
 
 
+# One oracle sample definition for both the cpu_baseline leg and the reference arm: the
+# Hessian over the first 4096 tokens, the full factorisation (d_in = 4096), GPTQ and the loss
+# on 64 rows, RTN on 1024 rows; each part is then scaled to the full layer.
+SAMPLE = dict(n_tok=4096, n_rows=64, n_rtn_rows=1024)
+THREAD_NOTE = ("numpy/LAPACK with its BLAS threads for the matrix products and factorisation; "
+               "the oracle's column loop itself is a Python loop of numpy vector steps on one "
+               "thread")
+
+
 def cpu_baseline(step, wl):
-    X_np = step.X[:8192].cpu().numpy()
+    X_np = step.X[:SAMPLE["n_tok"]].cpu().numpy()
     W_np = step.W.float().cpu().numpy()
-    full, measured, detail = oracle_sample(W_np, X_np, wl, n_tok=8192, n_rows=128,
-                                           n_rtn_rows=2048)
+    full, measured, detail = oracle_sample(W_np, X_np, wl, **SAMPLE)
     return {"value": wl.d_out * wl.d_in / full, "unit": UNIT, "cores": _blas_threads(),
-            "kind": "oracle", "sample": detail}
+            "kind": "oracle", "sample": detail + "; " + THREAD_NOTE}
 
 
 def run_reference(args):
@@ -756,10 +881,10 @@ def run_reference(args):
     wl = workloads.WORKLOADS[args.workload]
     # the same generator recipe on the CPU (bounded: only what the sample touches)
     W = workloads.make_weights(wl, device="cpu").float().numpy()
-    X = workloads.make_activations(wl, device="cpu", n_tokens=2048).numpy()
+    X = workloads.make_activations(wl, device="cpu", n_tokens=SAMPLE["n_tok"]).numpy()
     fulls, measured = [], 0.0
     for i in range(args.warmup + args.steps):
-        full, m, detail = oracle_sample(W, X, wl, n_tok=2048, n_rows=32, n_rtn_rows=512, seed=i)
+        full, m, detail = oracle_sample(W, X, wl, seed=i, **SAMPLE)
         if i >= args.warmup:
             fulls.append(full)
             measured += m
@@ -774,7 +899,7 @@ def run_reference(args):
                                   f"X {wl.n_tokens}x{wl.d_in} fp16, INT{wl.bits} g{wl.group_size} "
                                   f"B{wl.block_size} percdamp {wl.percdamp}"},
            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                            "sample": detail + f"; {args.steps} timed samples"},
+                            "sample": detail + f"; {args.steps} timed samples; " + THREAD_NOTE},
            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(res), flush=True)
 

@@ -43,27 +43,35 @@ def damp(H, percdamp):
     return Hd, lam
 
 
+def _cholesky_lower(A):
+    """L lower triangular with A = L Lᵀ (LAPACK potrf); NotPositiveDefinite otherwise."""
+    try:
+        return scipy.linalg.cholesky(A, lower=True, check_finite=False)
+    except np.linalg.LinAlgError as exc:
+        raise NotPositiveDefinite(str(exc)) from exc
+
+
+def _inverse_lower(L):
+    """L⁻¹ for a lower-triangular L (LAPACK trtri)."""
+    Linv, info = scipy.linalg.lapack.dtrtri(L, lower=1)
+    if info != 0:
+        raise NotPositiveDefinite(f"singular triangular factor (info={info})")
+    return np.tril(Linv)
+
+
 def upper_chol_of_inverse(Hd):
     """U upper triangular with UᵀU = Hd⁻¹, by Cholesky → explicit inverse → Cholesky."""
     Hd = np.asarray(Hd, dtype=np.float64)
-    try:
-        L = np.linalg.cholesky(Hd)
-    except np.linalg.LinAlgError as exc:
-        raise NotPositiveDefinite(str(exc)) from exc
-    Linv = scipy.linalg.solve_triangular(L, np.eye(Hd.shape[0]), lower=True)
+    L = _cholesky_lower(Hd)
+    Linv = _inverse_lower(L)
     Hinv = Linv.T @ Linv
     Hinv = 0.5 * (Hinv + Hinv.T)
-    C = np.linalg.cholesky(Hinv)          # Hinv = C Cᵀ, C lower
+    C = _cholesky_lower(Hinv)             # Hinv = C Cᵀ, C lower
     return C.T                            # U = Cᵀ: UᵀU = C Cᵀ
 
 
 def upper_chol_of_inverse_reversed(Hd):
     """U = P · L⁻¹ · P with P H_d P = L Lᵀ and P the index reversal."""
     Hd = np.asarray(Hd, dtype=np.float64)
-    A = Hd[::-1, ::-1]
-    try:
-        L = np.linalg.cholesky(A)
-    except np.linalg.LinAlgError as exc:
-        raise NotPositiveDefinite(str(exc)) from exc
-    Linv = scipy.linalg.solve_triangular(L, np.eye(Hd.shape[0]), lower=True)
-    return Linv[::-1, ::-1].copy()
+    L = _cholesky_lower(np.ascontiguousarray(Hd[::-1, ::-1]))
+    return _inverse_lower(L)[::-1, ::-1].copy()

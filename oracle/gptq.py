@@ -55,7 +55,7 @@ def _prepare(W, H, percdamp, act_order, rows, need_hd=True):
     d_in = H.shape[0]
     perm = act_order_perm(H) if act_order else np.arange(d_in)
     if need_hd:
-        Hd, lam = damp(H[np.ix_(perm, perm)], percdamp)
+        Hd, lam = damp(H[np.ix_(perm, perm)] if act_order else H, percdamp)
     else:
         Hd, lam = None, damping(H, percdamp)
     return W, W[:, perm].copy(), perm, Hd, lam
@@ -222,7 +222,7 @@ def prepare_u(H, percdamp=0.01, act_order=False, route="textbook"):
     """
     H = np.asarray(H, dtype=np.float64)
     perm = act_order_perm(H) if act_order else np.arange(H.shape[0])
-    Hd, _ = damp(H[np.ix_(perm, perm)], percdamp)
+    Hd, _ = damp(H[np.ix_(perm, perm)] if act_order else H, percdamp)
     if route == "reversed":
         return perm, upper_chol_of_inverse_reversed(Hd)
     if route != "textbook":

@@ -12,16 +12,24 @@ H because the damping is relative to mean(diag H)). Accumulation is additive ove
 """
 
 import numpy as np
+import scipy.linalg
 
 
 def hessian(X, chunk=8192):
-    """H = 2·Σ_t x_t x_tᵀ in fp64 for X of shape [n_tokens, d_in] (any float dtype)."""
+    """H = 2·Σ_t x_t x_tᵀ in fp64 for X of shape [n_tokens, d_in] (any float dtype).
+
+    Each chunk of tokens is added with the BLAS symmetric rank-k update (one triangle of
+    XᵀX, the other is its mirror), accumulated in fp64."""
     X = np.asarray(X)
     n, d = X.shape
-    H = np.zeros((d, d), dtype=np.float64)
+    S = np.zeros((d, d), dtype=np.float64, order="F")
     for t0 in range(0, n, chunk):
         Xc = X[t0:t0 + chunk].astype(np.float64)
-        H += Xc.T @ Xc
+        # S (upper triangle) += Xcᵀ·Xc; Xc.T is a Fortran-ordered d x chunk view
+        S = scipy.linalg.blas.dsyrk(1.0, Xc.T, beta=1.0, c=S, trans=0, lower=0,
+                                    overwrite_c=1)
+    H = S + S.T                           # the lower triangle of S is zero
+    H[np.diag_indices(d)] -= np.diag(S)   # the diagonal was counted twice (exact)
     return 2.0 * H
 
 
