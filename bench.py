@@ -109,7 +109,8 @@ def barrier(distributed: bool):
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap,"
+              "timestamp")
 
     def __init__(self, device_index: int):
         self.proc = None
@@ -121,36 +122,57 @@ class ClockSampler:
             sel = []
         self.sel = sel
 
-    def start(self):
+    def start(self, wait_s: float = 5.0):
+        """Start sampling every 20 ms and wait (up to wait_s) for the first sample, so that the
+        sampler is running before the timed region begins."""
         fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
         os.close(fd)
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100", *self.sel], stdout=open(self.path, "w"),
+                 "-lms", "20", *self.sel], stdout=open(self.path, "w"),
                 stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
+            return
+        t0 = time.time()
+        while time.time() - t0 < wait_s and os.path.getsize(self.path) == 0:
+            time.sleep(0.01)
 
-    def stop(self):
+    def mark(self):
+        """Wall-clock marks of the timed region (the samples' timestamps are wall clock)."""
+        return time.time()
+
+    def stop(self, t_begin=None, t_end=None):
         if self.proc is None:
             return None
+        time.sleep(0.05)
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
-        rows = []
+        rows, inside = [], []
         for line in open(self.path):
             parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
+            if len(parts) < 10:
                 continue
             try:
-                rows.append(dict(sm=float(parts[1]), smax=float(parts[2]), power=float(parts[3]),
-                                 hw=parts[5], hwt=parts[6], swt=parts[7], swp=parts[8]))
+                row = dict(sm=float(parts[1]), smax=float(parts[2]), power=float(parts[3]),
+                           hw=parts[5], hwt=parts[6], swt=parts[7], swp=parts[8])
             except ValueError:
                 continue
+            rows.append(row)
+            try:
+                import datetime
+                ts = datetime.datetime.strptime(parts[9], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                if t_begin is not None and t_begin - 0.05 <= ts <= t_end + 0.05:
+                    inside.append(row)
+            except ValueError:
+                pass
         os.unlink(self.path)
+        if inside:
+            rows = inside
         if not rows:
             return None
         busy = [r for r in rows if r["power"] > 250.0] or rows
@@ -164,6 +186,7 @@ class ClockSampler:
                 "sm_max_mhz": max(r["smax"] for r in rows),
                 "power_w_max": max(r["power"] for r in rows),
                 "samples": len(rows), "samples_under_load": len(busy),
+                "samples_in_timed_region": len(inside),
                 "reasons": sorted(reasons)}
 
 
@@ -627,6 +650,7 @@ def run_ours(args):
     barrier(distributed)
     torch.cuda.synchronize()
     sampler.start()
+    t_mark0 = sampler.mark()
     launches0 = gptq.launch_count()
     t_wall0 = time.perf_counter()
     for _ in range(args.steps):
@@ -642,7 +666,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     wall_s = time.perf_counter() - t_wall0
     launches = gptq.launch_count() - launches0
-    clocks = sampler.stop()
+    clocks = sampler.stop(t_mark0, sampler.mark())
     barrier(distributed)
     # the library's per-stage breakdown, from as many further steps with its stage events on
     gptq.profile_enable(True)
@@ -928,6 +952,10 @@ def run_ncu_case(name: str):
         W = workloads.make_weights(wl, device="cuda")
         for _ in range(3):
             gptq.rtn_minmax_quantize(W, 4, 128)
+    elif name == "rtn_big":                      # 4 layers of 7B weights: 153600 x 4096 fp16
+        W = workloads.make_weights(wl.replace(d_out=4 * (4 * 4096 + 2 * 11008)), device="cuda")
+        for _ in range(3):                       # (1.26 GB, ten times L2)
+            gptq.rtn_minmax_quantize(W, 4, 128)
     else:
         raise SystemExit(f"unknown ncu case {name}")
     torch.cuda.synchronize()
@@ -950,7 +978,7 @@ def main(argv=None):
     ap.add_argument("--no-stack", action="store_true",
                     help="skip GPTQ over a full 7B decoder stack (4 variants)")
     ap.add_argument("--stack-layers", type=int, default=32)
-    ap.add_argument("--ncu-case", choices=("hessian", "gptq", "rtn"),
+    ap.add_argument("--ncu-case", choices=("hessian", "gptq", "rtn", "rtn_big"),
                     help="run one small case for an ncu capture and exit (no JSON line)")
     args = ap.parse_args(argv)
     if args.ncu_case:

@@ -343,6 +343,13 @@ gptq_status awq_lite_search(const void* W, int w_dtype, int d_out, int d_in,
                             double* losses, int* best, void* workspace, size_t workspace_bytes,
                             void* stream);
 
+/* The unit-weight RMS pre-norm of a block (the input of its gate/up projections):
+ * Y[t] = fp16(X[t] / sqrt(mean(X[t]^2) + eps)), fp32 sum of squares.
+ *   X, Y device fp16 [n_tokens x d], 16-byte aligned (may not overlap); d a multiple of 8.
+ * Asynchronous. Errors: ARG, CUDA, UNSUPPORTED. */
+gptq_status gptq_rms_norm(const void* X, int64_t n_tokens, int d, float eps, void* Y,
+                          void* stream);
+
 /* The gate of a gated MLP block between its two quantized projections (layer-by-layer GPTQ
  * of a block stack, gtnt.cn §4: the down projection's Hessian comes from these activations):
  * A[t][j] = fp16(silu(GU[t][j]) * GU[t][d_ff + j]), silu(g) = g / (1 + e^-g) in fp32.

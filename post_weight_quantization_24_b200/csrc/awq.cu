@@ -61,8 +61,10 @@ __global__ void awq_scales_kernel(const double* __restrict__ x_sum, double x_cou
     const int i = blockIdx.y;
     if (c >= d || i >= n_alpha) return;
     const double xm = x_sum[c] / x_count, wm = w_sum[c] / w_count;
-    const double a = i * alpha_step;
-    const double v = pow(xm, a) / pow(wm, 1.0 - a);
+    // alpha = i*step and 1 - alpha rounded on their own, as the grid is defined (no fused
+    // multiply-add)
+    const double a = __dmul_rn(static_cast<double>(i), alpha_step);
+    const double v = pow(xm, a) / pow(wm, __dsub_rn(1.0, a));
     const float h = __half2float(__double2half(v));
     const bool ok = xm > 0.0 && wm > 0.0 && isfinite(h) && h > 0.0f;
     s[static_cast<int64_t>(i) * d + c] = ok ? h : 1.0f;

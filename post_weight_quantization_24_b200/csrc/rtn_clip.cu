@@ -77,6 +77,13 @@ __device__ __forceinline__ int clip_code(float w, double c, float cf, const QPar
     return clip_code_slow(w, c, p, maxq);
 }
 
+// c = (1 - i*step) * amax with each operation rounded on its own, as the ratio grid is defined
+// (a fused multiply-add would round 1 - i*step once and move c; e.g. 1 - 7*0.05 is
+// 0.6499999999999999 with two roundings and 0.65 with one)
+__device__ __forceinline__ double clip_bound(int i, double step, double amax) {
+    return __dmul_rn(__dsub_rn(1.0, __dmul_rn(static_cast<double>(i), step)), amax);
+}
+
 template <int G, typename T>
 __global__ void __launch_bounds__(rc::ROWS, 1) rtn_clip_kernel(
     const T* __restrict__ W, int d_out, int d_in, int bits, int sym, const float* __restrict__ H,
@@ -118,7 +125,7 @@ __global__ void __launch_bounds__(rc::ROWS, 1) rtn_clip_kernel(
     float best = 0.0f;
     int best_i = 0;
     for (int gi = 0; gi < n_grid; ++gi) {
-        const double c = (1.0 - gi * step) * amax;
+        const double c = clip_bound(gi, step, amax);
         const float cf = __double2float_rd(c);
         const QParams p = range_params(fmax(static_cast<double>(mn), -c),
                                        fmin(static_cast<double>(mx), c), maxq, sym != 0);
@@ -159,7 +166,7 @@ __global__ void __launch_bounds__(rc::ROWS, 1) rtn_clip_kernel(
     }
 
     // the chosen ratio's codes, grid and index
-    const double c = (1.0 - best_i * step) * amax;
+    const double c = clip_bound(best_i, step, amax);
     const float cf = __double2float_rd(c);
     const QParams p = range_params(fmax(static_cast<double>(mn), -c),
                                    fmin(static_cast<double>(mx), c), maxq, sym != 0);

@@ -387,6 +387,45 @@ __global__ void __launch_bounds__(256) silu_mul_kernel(const __half* __restrict_
     }
 }
 
+// Y[t] = fp16(X[t] / sqrt(mean(X[t]^2) + eps)) per row (the unit-weight RMS pre-norm of a
+// block): one warp per row, fp32 sum of squares over 16-byte chunks, IEEE sqrt and division.
+__global__ void __launch_bounds__(256) rms_norm_kernel(const __half* __restrict__ X, int64_t n,
+                                                       int d, float eps, __half* __restrict__ Y) {
+    const int lane = threadIdx.x & 31;
+    const int64_t wstride = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+    for (int64_t t = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+         t < n; t += wstride) {
+        const uint4* row = reinterpret_cast<const uint4*>(X + t * d);
+        float ss = 0.0f;
+        for (int c = lane; c < d / 8; c += 32) {
+            const uint4 v = row[c];
+            const __half2* h = reinterpret_cast<const __half2*>(&v);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float2 f = __half22float2(h[i]);
+                ss = fmaf(f.x, f.x, ss);
+                ss = fmaf(f.y, f.y, ss);
+            }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+        const float r = sqrtf(ss / static_cast<float>(d) + eps);
+        uint4* out = reinterpret_cast<uint4*>(Y + t * d);
+        for (int c = lane; c < d / 8; c += 32) {
+            const uint4 v = row[c];
+            const __half2* h = reinterpret_cast<const __half2*>(&v);
+            uint32_t o[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float2 f = __half22float2(h[i]);
+                const __half2 q = __floats2half2_rn(f.x / r, f.y / r);
+                o[i] = *reinterpret_cast<const uint32_t*>(&q);
+            }
+            out[c] = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+    }
+}
+
 static int g_wq_attr = 0;
 
 gptq_status w4a16_launch(const __half* X, int64_t n, int d_in, const uint8_t* packed,
@@ -446,6 +485,15 @@ gptq_status w4a16_pack_launch(const uint8_t* codes, int d_out, int d_in, const i
     return GPTQ_OK;
 }
 
+gptq_status rms_norm_launch(const __half* X, int64_t n, int d, float eps, __half* Y,
+                            cudaStream_t s) {
+    const int blocks = static_cast<int>(std::max<int64_t>(
+        1, std::min<int64_t>((n + 7) / 8, static_cast<int64_t>(num_sms()) * 16)));
+    rms_norm_kernel<<<blocks, 256, 0, s>>>(X, n, d, eps, Y);
+    GPTQ_LAUNCHED();
+    return GPTQ_OK;
+}
+
 gptq_status silu_mul_launch(const __half* GU, int64_t n, int d_ff, __half* A, cudaStream_t s) {
     const int64_t total = n * (d_ff / 8);
     const int blocks = static_cast<int>(std::max<int64_t>(
@@ -466,6 +514,16 @@ gptq_status gptq_silu_mul(const void* GU, int64_t n_tokens, int d_ff, void* A, v
     GPTQ_TRY(gq::check_device());
     return gq::silu_mul_launch(static_cast<const __half*>(GU), n_tokens, d_ff,
                                static_cast<__half*>(A), static_cast<cudaStream_t>(stream));
+}
+
+gptq_status gptq_rms_norm(const void* X, int64_t n_tokens, int d, float eps, void* Y,
+                          void* stream) {
+    if (!X || !Y || n_tokens < 1 || d < 8 || d % 8 || !(eps >= 0.0f)) return GPTQ_ERR_ARG;
+    if ((reinterpret_cast<uintptr_t>(X) & 15) || (reinterpret_cast<uintptr_t>(Y) & 15))
+        return GPTQ_ERR_ARG;
+    GPTQ_TRY(gq::check_device());
+    return gq::rms_norm_launch(static_cast<const __half*>(X), n_tokens, d, eps,
+                               static_cast<__half*>(Y), static_cast<cudaStream_t>(stream));
 }
 
 size_t w4a16_linear_workspace(int64_t n_tokens, int d_in, int has_perm) {

@@ -72,6 +72,7 @@ _SIGNATURES = {
     "w4a16_linear_workspace": ([_I64, _I, _I], _SZ),
     "w4a16_linear": ([_P, _I64, _I, _P, _P, _P, _I, _I, _P, _P, _P, _P, _SZ, _P, _P], _I),
     "gptq_silu_mul": ([_P, _I64, _I, _P, _P], _I),
+    "gptq_rms_norm": ([_P, _I64, _I, _F, _P, _P], _I),
     "gptq_channel_abs_sum": ([_P, _I, _I64, _I, _P, _P], _I),
     "awq_lite_workspace": ([_I, _I, ctypes.c_double], _SZ),
     "awq_lite_search": ([_P, _I, _I, _I, _P, _I64, _P, _I, _I, _I, ctypes.c_double, _P, _P, _P,
@@ -427,6 +428,17 @@ def awq_lite_search(W: torch.Tensor, x_abs_sum: torch.Tensor, n_tokens: int, H: 
     _check(st, "awq_lite_search")
     return dict(packed=packed, scales=scales, zeros=zeros, s=s_out, losses=list(losses),
                 best=int(best.value), alpha=int(best.value) * alpha_step)
+
+
+def rms_norm(X: torch.Tensor, eps: float = 1e-6, out: torch.Tensor | None = None) -> torch.Tensor:
+    """Y = fp16(x / sqrt(mean(x²) + eps)) per row of fp16 X [n, d] (unit-weight RMS norm)."""
+    _require_cuda(X, "X")
+    n, d = X.shape
+    if out is None:
+        out = torch.empty_like(X)
+    _check(lib().gptq_rms_norm(X.data_ptr(), n, d, float(eps), out.data_ptr(), _stream()),
+           "gptq_rms_norm")
+    return out
 
 
 def silu_mul(GU: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:

@@ -2,11 +2,12 @@
 of the already-quantized layers before it (gtnt.cn/news/115337 §4: Hessians from calibration
 forward passes, layers quantized in order; hncyxsy.com/news/243429 §3.1 step 4).
 
-Block: X_{b+1} = X_b + down(silu(gate(X_b)) ⊙ up(X_b)), the gated MLP of the 7B decoder shapes
-with a residual (attention left out). Per block, in order:
-  1. H = 2·X_bᵀX_b (tensor-core Hessian);
+Block: N_b = rms_norm(X_b), X_{b+1} = X_b + down(silu(gate(N_b)) ⊙ up(N_b)), the gated MLP of
+the 7B decoder shapes with its unit-weight RMS pre-norm and a residual (attention left out). Per
+block, in order:
+  1. N_b = rms_norm(X_b), H = 2·N_bᵀN_b (tensor-core Hessian);
   2. GPTQ of the row-stacked gate;up weights (one Hessian, one factorisation);
-  3. the W4A16 layer on X_b with the quantized gate;up -> G;U, then A = silu(G)·U;
+  3. the W4A16 layer on N_b with the quantized gate;up -> G;U, then A = silu(G)·U;
   4. H = 2·AᵀA, GPTQ of down;
   5. X_{b+1} = X_b + the W4A16 layer on A with the quantized down (residual added before the
      fp16 rounding).
@@ -38,7 +39,7 @@ def quantize_mlp_stack(X0: torch.Tensor, blocks, bits: int = 4, group_size: int 
 
     Returns (final activations fp16 [n, d], per-layer records dict(name, codes, scales, zeros,
     g_idx, perm, packed, loss)). With `timings` (a dict), CUDA-event milliseconds per step kind
-    are added to it: hessian, gptq, w4a16, silu."""
+    are added to it: norm, hessian, gptq, w4a16, silu."""
     if bits != 4:
         raise ValueError("the W4A16 layer serves 4-bit codes")
     X = X0
@@ -59,14 +60,17 @@ def quantize_mlp_stack(X0: torch.Tensor, blocks, bits: int = 4, group_size: int 
                              gptq.quantize_layer_workspace(d, d_ff, block_size)),
                          dtype=torch.uint8, device=X.device)
         mark("start")
+        Nx = gptq.rms_norm(X)
+        mark("norm")
         h1 = gptq.Hessian(d)
-        h1.accumulate(X)
+        h1.accumulate(Nx)
         mark("hessian")
         o1 = _quantize_and_pack(W_gu, h1.raw(), bits, group_size, block_size, percdamp,
                                 act_order, ws)
         mark("gptq")
-        GU = gptq.w4a16_linear(X, o1["packed"], o1["scales"], o1["zeros"], group_size,
+        GU = gptq.w4a16_linear(Nx, o1["packed"], o1["scales"], o1["zeros"], group_size,
                                perm=o1["perm_gather"])
+        del Nx
         mark("w4a16")
         A = gptq.silu_mul(GU)
         del GU

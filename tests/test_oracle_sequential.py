@@ -37,6 +37,15 @@ def test_silu_closed_forms():
     assert np.array_equal(s, exact.astype(np.float16).astype(np.float64))
 
 
+def test_rms_norm_closed_forms():
+    X = np.array([[3.0, 4.0], [0.0, 0.0], [-2.0, 2.0]], dtype=np.float16)
+    Nx = sequential.rms_norm(X)
+    # rms of (3, 4) is sqrt(12.5): outputs 3/sqrt(12.5), 4/sqrt(12.5); an all-zero row stays 0
+    assert np.allclose(Nx[0], np.array([3, 4]) / np.sqrt(12.5 + 1e-6), rtol=1e-3)
+    assert np.array_equal(Nx[1], [0.0, 0.0])
+    assert np.allclose(np.mean(Nx[2] ** 2), 1.0, rtol=1e-3)
+
+
 def test_eight_bit_stack_follows_the_float_stack():
     X, blocks = _stack()
     Xq, recs = sequential.sequential_mlp_stack(X, blocks, bits=8, group_size=32, block_size=32)
@@ -64,6 +73,7 @@ def test_quantization_error_propagates_to_later_hessians():
     # with 8-bit layers the down projection's Hessian is close to the float forward's
     Wg, Wu, _ = blocks[0]
     Xf = np.asarray(X, np.float64)
+    Xf = Xf / np.sqrt(np.mean(Xf * Xf, axis=1, keepdims=True) + sequential.RMS_EPS)
     G, U = Xf @ Wg.T, Xf @ Wu.T
     Af = G / (1 + np.exp(-G)) * U
     Hf = hessian.hessian(Af)
