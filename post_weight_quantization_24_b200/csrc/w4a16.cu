@@ -54,6 +54,7 @@ constexpr uint32_t IDESC = (1u << 4) | (static_cast<uint32_t>(BN >> 3) << 17) |
 
 struct WqParams {
     int n_tok, d_in, d_out, g, ng;
+    int g_shift;          // log2(g) when g is a power of two, else -1
     int n_mt, n_nt, n_kb;
     long long n_tiles;
     const uint16_t* scales;
@@ -242,7 +243,8 @@ __global__ void __launch_bounds__(wq::THREADS, 1)
                 uint8_t* brow = sa + wq::OFF_B + row_off;
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
-                    const int k = (kb * wq::BK + 8 * c) / p.g;
+                    const int col = kb * wq::BK + 8 * c;
+                    const int k = p.g_shift >= 0 ? (col >> p.g_shift) : col / p.g;
                     if (k != cur_k) {
                         cur_k = k;
                         if (row_ok) {
@@ -458,6 +460,9 @@ gptq_status w4a16_launch(const __half* X, int64_t n, int d_in, const uint8_t* pa
     p.d_out = d_out;
     p.g = g;
     p.ng = d_in / g;
+    p.g_shift = -1;
+    for (int sft = 3; sft < 17; ++sft)
+        if ((1 << sft) == g) p.g_shift = sft;
     p.n_mt = static_cast<int>((n + wq::BM - 1) / wq::BM);
     p.n_nt = (d_out + wq::BN - 1) / wq::BN;
     p.n_kb = d_in / wq::BK;
