@@ -5,6 +5,9 @@ Sources
   * 0539edu.com/news/6111416 §4.2: with fp16 scale and zero per group, 4-bit storage costs
     4 + 32/group_size bits per weight (4.25 / 4.5 / 5 at 128 / 64 / 32).
   * hncyxsy.com/news/243429 §1.2: RTN rounds every weight independently, with no compensation.
+  * gtnt.cn/news/115337 §3 (awq_clip) and bhfrc.com/news/5741 §4.3: the range can be clipped
+    before the min-max scale is taken, by a searched ratio of the block's absolute maximum or
+    by a percentile (99.99 %) or a fixed absolute range.
 
 Layout: W is [d_out, d_in] (PyTorch Linear layout); groups are ``group_size`` consecutive
 input columns of one row. scales and zeros are [d_out, d_in/group_size]. For 4-bit codes the
@@ -88,6 +91,54 @@ def rtn_clip_search(W, bits, group_size, H=None, sym=False, min_ratio=0.5, step=
         m = best == i
         codes[m], scales[m], zeros[m] = q[m], s[m], z[m]
     return codes.reshape(d_out, d_in), scales, zeros, best, crit
+
+
+def group_quantile(v_sorted, frac):
+    """The frac-quantile of each group's values (last axis, sorted ascending), by linear
+    interpolation between the order statistics around position frac·(g − 1), every operation
+    in fp64 and rounded on its own: h = frac·(g − 1), k = floor(h), t = h − k,
+    q = v[k] + t·(v[k+1] − v[k]) (q = v[g−1] at the top)."""
+    v = np.asarray(v_sorted, dtype=np.float64)
+    g = v.shape[-1]
+    h = float(frac) * float(g - 1)
+    k = int(np.floor(h))
+    if k >= g - 1:
+        return v[..., g - 1].copy()
+    t = h - k
+    return v[..., k] + t * (v[..., k + 1] - v[..., k])
+
+
+def rtn_range_clip(W, bits, group_size, percentile=100.0, abs_range=0.0, sym=False):
+    """Group RTN of clipped weights (bhfrc.com/news/5741 §4.3: instead of the group's extreme
+    values, take a percentile of its values such as 99.99 %, or an absolute range such as
+    [-10, 10], and truncate what lies outside before the min-max range is formed).
+
+    Per group: lo and hi are the (1 − p) and p quantiles of its weights (``group_quantile``,
+    p = percentile/100; percentile 100 gives the min and the max); with abs_range a > 0 they
+    are further limited to [−a, a]. The weights are clamped to [lo, hi] and quantized with the
+    quantizer of the range [lo, hi] (widened to contain 0, or symmetric with
+    m = max(|lo|, |hi|)). Returns (codes [d_out, d_in], scales, zeros [d_out, d_in/g],
+    lo, hi [d_out, d_in/g])."""
+    W = np.asarray(W, dtype=np.float64)
+    d_out, d_in = W.shape
+    if d_in % group_size:
+        raise ValueError("d_in must be a multiple of group_size")
+    if not (50.0 <= percentile <= 100.0) or abs_range < 0:
+        raise ValueError("percentile must lie in [50, 100] and abs_range >= 0")
+    maxq = 2 ** bits - 1
+    Wg = W.reshape(d_out, d_in // group_size, group_size)
+    v = np.sort(Wg, axis=2)
+    p = percentile / 100.0
+    hi = group_quantile(v, p)
+    lo = group_quantile(v, 1.0 - p)
+    if abs_range > 0:
+        lo = np.maximum(lo, -abs_range)
+        hi = np.minimum(hi, abs_range)
+    Wc = np.clip(Wg, lo[..., None], hi[..., None])
+    params = group_params_sym if sym else group_params
+    scale, zero = params(lo, hi, maxq)
+    q = quantize(Wc, scale[..., None], zero[..., None], maxq)
+    return q.reshape(d_out, d_in), scale, zero, lo, hi
 
 
 def rtn_dequant(codes, scales, zeros, group_size):

@@ -414,31 +414,24 @@ gptq_status side_streams(SideStreams** out) {
 }
 }  // namespace
 
-// Blocked right-looking Cholesky of A and the blocked triangular inverse X = L^-1, then
-// U = reverse(X), in outer panels of kOuterCols columns factored by 128-wide steps.
+// Blocked right-looking Cholesky of A with one step of lookahead, and the blocked triangular
+// inverse X = L^-1, then U = reverse(X).
 //
-// Main stream, outer panel [K0, E), for each 128-column step [k0, e) inside it:
-//   diag(k0)    L11 and its inverse Dinv (one CTA)
-//   trsm(k0)    L21 = A21 Dinv^T for all rows below, in place
-//   inner(k0)   A[e:, e:E] -= L21 L21[0:E-e]^T: the panel's own later columns only
-// then, once per outer panel (K = E - K0 in both updates, so the trailing matrix is read and
-// written once per kOuterCols columns instead of once per 128):
-//   next(P)     A[E:, E:E2] -= L[E:, K0:E] L[E:E2, K0:E]^T, the next panel's columns (main
-//               stream, after rest(P-1), the only other writer of those columns)
-//   rest(P)     A[E2:, E2:] -= L[E2:, K0:E] L[E2:, K0:E]^T (lower tiles), on the side stream
-// Side stream, after the panel is factored, the inverse's rows of the panel:
-//   X[k0:e, 0:e] = Dinv X[k0:e, 0:e] (in place) and X[e:E, 0:e] -= L[e:E, k0:e] X[k0:e, 0:e]
-//   per 128-column step, then X[E:, 0:E] -= L[E:, K0:E] X[K0:E, 0:E] once (K = E - K0).
-// The side stream's GEMMs leave as many SMs free as the main stream's kernels of the next
-// panel have CTAs (one per 128 rows below it; at most half the GPU), so the chain of diagonal
-// blocks does not wait for an SM.
-constexpr int kOuterCols = 512;
-
+// Main stream, panel m (columns k0 .. e-1, e = k0 + nbc; rem = d - e rows below):
+//   diag(m)   L11 and its inverse Dinv_m (one CTA)
+//   trsm(m)   L21 = A21 Dinv_m^T, in place (each output tile is the input tile it reads)
+//   next(m)   the trailing update of panel m+1's columns only: A[e:, e:e+128] -= L21 L21^T
+// Side stream, after trsm(m):
+//   rest(m)   the rest of the trailing update: A[e+128:, e+128:] -= L21' L21'^T (lower tiles)
+//   inv(m)    X[k0:e, 0:e] = Dinv_m X[k0:e, 0:e] (in place), X[e:, 0:e] -= L21 X[k0:e, 0:e]
+// next(m) waits for rest(m-1), the only other writer of its columns; diag(m+1) and trsm(m+1)
+// need only next(m), so rest(m) and inv(m) overlap them. The side stream's GEMMs leave as many
+// SMs free as the main stream's kernels of the next panel have CTAs (one, or one per 128 rows
+// below it; at most half the GPU), so the chain of diagonal blocks does not wait for an SM.
 gptq_status factor_inverse_launch(float* A, int d, float* Dinv, float* X, int* status,
                                   cudaStream_t s) {
     const int nb = kCholBlock;
     static_assert(kCholBlock == pd::NB, "diagonal-block kernel is written for 128-wide panels");
-    static_assert(kOuterCols % kCholBlock == 0, "outer panels are whole 128-column steps");
     const int smem = pd::SMEM;
     if (g_potrf_smem != smem) {
         GPTQ_CUDA_TRY(cudaFuncSetAttribute(potrf_diag_kernel,
@@ -455,74 +448,65 @@ gptq_status factor_inverse_launch(float* A, int d, float* Dinv, float* X, int* s
     GPTQ_CUDA_TRY(cudaStreamWaitEvent(t2, ss->fork, 0));
     // Everything below is enqueued on both streams; on an error the side stream is joined
     // back before returning, so a capture of `s` stays well formed.
-    auto gemm = [&](int M, int N, int K, float alpha, float beta, const float* Am, int lda,
-                    const float* Bm, int ldb, bool b_kmajor, float* C, int lower, int max_ctas,
-                    cudaStream_t st) -> gptq_status {
-        if (M <= 0 || N <= 0 || K <= 0) return GPTQ_OK;
-        TcGemmArgs g{};
-        g.M = M; g.N = N; g.K = K; g.alpha = alpha; g.beta = beta;
-        g.A = Am; g.lda = lda; g.B = Bm; g.ldb = ldb; g.C = C; g.ldc = d;
-        g.lower_only = lower; g.status = status; g.max_ctas = max_ctas;
-        return tcgemm_launch(g, b_kmajor, TC_EPI_STORE, true, true, st);
-    };
     auto body = [&]() -> gptq_status {
         GPTQ_CUDA_TRY(cudaMemsetAsync(X, 0, static_cast<size_t>(d) * d * 4, t2));
         set_identity_kernel<<<(d + 255) / 256, 256, 0, t2>>>(X, d);
         GPTQ_LAUNCHED();
-        bool rest_pending = false;
-        for (int K0 = 0; K0 < d; K0 += kOuterCols) {
-            const int E = std::min(K0 + kOuterCols, d);
-            const int rem_panel = d - E;
-            // SMs kept free for the main stream while this panel's side work runs: the next
-            // panel's diag takes one, its trsm and updates one per 128 rows below
-            const int reserve = std::min(sms / 2, std::max(1, (rem_panel + nb - 1) / nb));
+        const int nbl = (d + nb - 1) / nb;
+        for (int m = 0; m < nbl; ++m) {
+            const int k0 = m * nb, nbc = std::min(nb, d - k0), e = k0 + nbc, rem = d - e;
+            float* Dm = Dinv + static_cast<int64_t>(m) * nb * nb;
+            float* A21 = A + static_cast<int64_t>(e) * d + k0;
+            // SMs kept free for the main stream while this panel's side work runs: diag(m+1)
+            // takes one, trsm(m+1) and next(m+1) one per 128 rows below panel m+1
+            const int reserve = std::min(sms / 2, std::max(1, (rem + nb - 1) / nb));
             const int side_ctas = std::max(1, sms - reserve);
-            // ---- main: factor the panel's columns in 128-wide steps ----
-            for (int k0 = K0; k0 < E; k0 += nb) {
-                const int m = k0 / nb, nbc = std::min(nb, d - k0), e = k0 + nbc, rem = d - e;
-                float* Dm = Dinv + static_cast<int64_t>(m) * nb * nb;
-                float* A21 = A + static_cast<int64_t>(e) * d + k0;
-                potrf_diag_kernel<<<1, pd::THREADS, smem, s>>>(A, d, k0, nbc, Dm, status);
-                GPTQ_LAUNCHED();
-                // A21 = A21 * Dinv^T, in place (each output tile is the input tile it reads)
-                GPTQ_TRY(gemm(rem, nbc, nbc, 1.f, 0.f, A21, d, Dm, nb, true, A21, 0, 0, s));
-                // the panel's own later columns: A[e:, e:E] -= A21 A21[0:E-e]^T
-                GPTQ_TRY(gemm(rem, E - e, nbc, -1.f, 1.f, A21, d, A21, d, true,
-                              A + static_cast<int64_t>(e) * d + e, 1, 0, s));
-            }
-            GPTQ_CUDA_TRY(cudaEventRecord(ss->trsm, s));        // the panel's L is complete
-            GPTQ_CUDA_TRY(cudaStreamWaitEvent(t2, ss->trsm, 0));
-            const float* Lp = A + static_cast<int64_t>(E) * d + K0;   // L[E:, K0:E]
-            if (rem_panel > 0) {
-                const int E2 = std::min(E + kOuterCols, d);
-                // next panel's columns, after rest(P-1), the other writer of those columns
-                if (rest_pending) GPTQ_CUDA_TRY(cudaStreamWaitEvent(s, ss->rest, 0));
-                GPTQ_TRY(gemm(rem_panel, E2 - E, E - K0, -1.f, 1.f, Lp, d, Lp, d, true,
-                              A + static_cast<int64_t>(E) * d + E, 1, 0, s));
-                // the rest of the trailing matrix on the side stream
-                if (E2 < d) {
-                    const float* Lr = Lp + static_cast<int64_t>(E2 - E) * d;
-                    GPTQ_TRY(gemm(d - E2, d - E2, E - K0, -1.f, 1.f, Lr, d, Lr, d, true,
-                                  A + static_cast<int64_t>(E2) * d + E2, 1, side_ctas, t2));
+            potrf_diag_kernel<<<1, pd::THREADS, smem, s>>>(A, d, k0, nbc, Dm, status);
+            GPTQ_LAUNCHED();
+            if (rem > 0) {
+                TcGemmArgs t{};  // A21 = A21 * Dinv_m^T
+                t.M = rem; t.N = nbc; t.K = nbc; t.alpha = 1.f; t.beta = 0.f;
+                t.A = A21; t.lda = d; t.B = Dm; t.ldb = nb; t.C = A21; t.ldc = d;
+                t.status = status;
+                GPTQ_TRY(tcgemm_launch(t, true, TC_EPI_STORE, true, true, s));
+                GPTQ_CUDA_TRY(cudaEventRecord(ss->trsm, s));
+                // next(m) after rest(m-1): the event's last record is still rest(m-1)'s
+                if (m > 0) GPTQ_CUDA_TRY(cudaStreamWaitEvent(s, ss->rest, 0));
+                TcGemmArgs u{};  // A[e:, e:e+128] -= A21 A21[0:128]^T
+                u.M = rem; u.N = std::min(nb, rem); u.K = nbc; u.alpha = -1.f; u.beta = 1.f;
+                u.A = A21; u.lda = d; u.B = A21; u.ldb = d;
+                u.C = A + static_cast<int64_t>(e) * d + e; u.ldc = d;
+                u.lower_only = 1; u.status = status;
+                GPTQ_TRY(tcgemm_launch(u, true, TC_EPI_STORE, true, true, s));
+                GPTQ_CUDA_TRY(cudaStreamWaitEvent(t2, ss->trsm, 0));
+                if (rem > nb) {
+                    const float* A21r = A21 + static_cast<int64_t>(nb) * d;
+                    TcGemmArgs r{};  // A[e+128:, e+128:] -= A21' A21'^T (lower tiles)
+                    r.M = rem - nb; r.N = rem - nb; r.K = nbc; r.alpha = -1.f; r.beta = 1.f;
+                    r.A = A21r; r.lda = d; r.B = A21r; r.ldb = d;
+                    r.C = A + static_cast<int64_t>(e + nb) * d + (e + nb); r.ldc = d;
+                    r.lower_only = 1; r.status = status; r.max_ctas = side_ctas;
+                    GPTQ_TRY(tcgemm_launch(r, true, TC_EPI_STORE, true, true, t2));
                 }
                 GPTQ_CUDA_TRY(cudaEventRecord(ss->rest, t2));
-                rest_pending = true;
+            } else {
+                GPTQ_CUDA_TRY(cudaEventRecord(ss->trsm, s));
+                GPTQ_CUDA_TRY(cudaStreamWaitEvent(t2, ss->trsm, 0));
             }
-            // ---- side: the inverse's rows of the panel, then their effect on the rows below
-            for (int k0 = K0; k0 < E; k0 += nb) {
-                const int m = k0 / nb, nbc = std::min(nb, d - k0), e = k0 + nbc;
-                float* Dm = Dinv + static_cast<int64_t>(m) * nb * nb;
-                float* Xk = X + static_cast<int64_t>(k0) * d;
-                // X[k0:e, 0:e] = Dinv * X[k0:e, 0:e], in place
-                GPTQ_TRY(gemm(nbc, e, nbc, 1.f, 0.f, Dm, nb, Xk, d, false, Xk, 0, side_ctas, t2));
-                // X[e:E, 0:e] -= L[e:E, k0:e] * X[k0:e, 0:e]
-                GPTQ_TRY(gemm(E - e, e, nbc, -1.f, 1.f, A + static_cast<int64_t>(e) * d + k0, d,
-                              Xk, d, false, X + static_cast<int64_t>(e) * d, 0, side_ctas, t2));
+            float* Xk = X + static_cast<int64_t>(k0) * d;
+            TcGemmArgs v{};  // X[k0:e, 0:e] = Dinv_m * X[k0:e, 0:e], in place
+            v.M = nbc; v.N = e; v.K = nbc; v.alpha = 1.f; v.beta = 0.f;
+            v.A = Dm; v.lda = nb; v.B = Xk; v.ldb = d; v.C = Xk; v.ldc = d;
+            v.status = status; v.max_ctas = side_ctas;
+            GPTQ_TRY(tcgemm_launch(v, false, TC_EPI_STORE, true, true, t2));
+            if (rem > 0) {
+                TcGemmArgs w{};  // X[e:, 0:e] -= L21 * X[k0:e, 0:e]
+                w.M = rem; w.N = e; w.K = nbc; w.alpha = -1.f; w.beta = 1.f;
+                w.A = A21; w.lda = d; w.B = Xk; w.ldb = d;
+                w.C = X + static_cast<int64_t>(e) * d; w.ldc = d;
+                w.status = status; w.max_ctas = side_ctas;
+                GPTQ_TRY(tcgemm_launch(w, false, TC_EPI_STORE, true, true, t2));
             }
-            // X[E:, 0:E] -= L[E:, K0:E] * X[K0:E, 0:E]
-            GPTQ_TRY(gemm(rem_panel, E, E - K0, -1.f, 1.f, Lp, d,
-                          X + static_cast<int64_t>(K0) * d, d, false,
-                          X + static_cast<int64_t>(E) * d, 0, side_ctas, t2));
         }
         const int64_t half = static_cast<int64_t>(d) * d / 2;
         const int blocks =

@@ -179,81 +179,12 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-// Packed pairs of fp32 values (two lanes of one 64-bit register pair) for the f32x2 arithmetic
-// of sm_100: one instruction applies the operation to both values, each rounded on its own.
-__device__ __forceinline__ unsigned long long f2_pack(float lo, float hi) {
-    return (static_cast<unsigned long long>(__float_as_uint(hi)) << 32) | __float_as_uint(lo);
-}
-__device__ __forceinline__ float f2_lo(unsigned long long v) {
-    return __uint_as_float(static_cast<uint32_t>(v));
-}
-__device__ __forceinline__ float f2_hi(unsigned long long v) {
-    return __uint_as_float(static_cast<uint32_t>(v >> 32));
-}
-__device__ __forceinline__ unsigned long long f2_fma(unsigned long long a, unsigned long long b,
-                                                     unsigned long long c) {
-    unsigned long long d;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-    return d;
-}
-__device__ __forceinline__ unsigned long long f2_sub(unsigned long long a, unsigned long long b) {
-    unsigned long long d;
-    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
-__device__ __forceinline__ unsigned long long f2_add(unsigned long long a, unsigned long long b) {
-    unsigned long long d;
-    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
-
-// The two fp16 values of a 32-bit word as fp32 values scaled by 2^-112 (exactly): the fp16
-// sign goes to bit 31 and its exponent and mantissa bits, shifted up by 13, become an fp32
-// exponent and mantissa with the exponent bias 15 read as 127, i.e. a factor 2^-112. fp16
-// subnormals become fp32 subnormals (exact; this file is compiled without flush-to-zero).
-// Integer operations only, so the conversion does not occupy the conversion pipe.
-__device__ __forceinline__ unsigned long long half2_bits_scaled(uint32_t u) {
-    const uint32_t lo = ((u << 13) & 0x0FFFE000u) | ((u << 16) & 0x80000000u);
-    const uint32_t hi = ((u >> 3) & 0x0FFFE000u) | (u & 0x80000000u);
-    return (static_cast<unsigned long long>(hi) << 32) | lo;
-}
-
-// The exact path for one lane's chunk of the ring stage (its 16-byte pieces 4L .. 4L+3 at their
-// swizzled positions), kept out of line: the fast path reaches it rarely.
-__device__ __forceinline__ int ring_chunk(int c) { return c ^ ((c >> 3) & 7); }
-__device__ __noinline__ void rtn_chunk_exact_ring(const uint8_t* stage, int lane, QParams p,
-                                                  int bits, uint8_t* __restrict__ out,
-                                                  int64_t t) {
-    __half w[32];
-#pragma unroll
-    for (int h = 0; h < 4; ++h) {
-        const uint4 v = *reinterpret_cast<const uint4*>(stage + 16 * ring_chunk(4 * lane + h));
-        const __half* hv = reinterpret_cast<const __half*>(&v);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) w[8 * h + i] = hv[i];
-    }
-    rtn_chunk_exact(w, p, bits, out, t);
-}
-
 // fp16 weights, power-of-two groups of 32..256: a lane quantizes 32 consecutive weights
 // (TPG = group_size / 32 lanes per group). Each warp streams its 2 KB per iteration through a
 // 4-stage shared-memory ring with per-lane async copies (coalesced: lane L copies bytes
 // 16L + 512h), keeping three iterations in flight while it computes one, which is what keeps
-// enough bytes outstanding to run at HBM speed. The ring stores 16-byte chunk c at chunk
-// position c ^ ((c >> 3) & 7), so that both the copies (lane L: chunks L + 32h) and the reads
-// (lane L: its own chunks 4L .. 4L+3) touch eight different 16-byte bank groups per eight lanes.
-//
-// Codes are decided by two roundings that bracket the exact quotient: with inv ~ 1/scale
-// (relative error below 2^-22), inv_- = inv(1 - 2^-20) < 1/scale < inv_+ = inv(1 + 2^-20), so
-// w*inv_- and w*inv_+ (exact products inside the fused multiply-add) lie on either side of
-// w/scale. m_+- = rint(w*inv_+- + zero + 1.5*2^23) rounds at ulp 1 (magic number); where the two
-// agree for every weight of the lane's chunk, no half-integer lies between them, so that
-// integer is rint(w/scale) + zero exactly (and lies in [0, maxq]: every w is inside its group's
-// range); otherwise (about 3e-5 of the weights, near a rounding boundary) the chunk is redone on
-// the exact path. The weights enter as fp32 values scaled by 2^-112 (half2_bits_scaled) and the
-// factor 2^112 is folded, exactly, into inv_+-. Both roundings of a pair of weights take one
-// f32x2 fused multiply-add each. Codes come out as float bit patterns and are packed with byte
-// permutes. Chunk indices are 32-bit (the launcher checks).
+// enough bytes outstanding to run at HBM speed. Codes come out of the rounding as float bit
+// patterns and are packed with byte permutes. Chunk indices are 32-bit (the launcher checks).
 template <int TPG, bool INT4>
 __global__ void __launch_bounds__(rp::THREADS, 3) rtn_f16_kernel(const __half* __restrict__ W,
                                                                 int n_chunks, int bits, int sym,
@@ -271,11 +202,11 @@ __global__ void __launch_bounds__(rp::THREADS, 3) rtn_f16_kernel(const __half* _
     auto issue = [&](int wi, int st) {
         if (wi < n_wit) {
             const uint8_t* src = wbytes + static_cast<int64_t>(wi) * rp::STAGE_BYTES + 16 * lane;
-            uint8_t* dst = ring + st * rp::STAGE_BYTES;
+            uint8_t* dst = ring + st * rp::STAGE_BYTES + 16 * lane;
             const int valid = min(32, n_chunks - wi * 32) * (2 * rp::E) - 16 * lane;   // bytes
 #pragma unroll
             for (int h = 0; h < 4; ++h)
-                if (512 * h < valid) cp_async16(dst + 16 * ring_chunk(lane + 32 * h), src + 512 * h);
+                if (512 * h < valid) cp_async16(dst + 512 * h, src + 512 * h);
         }
         cp_async_commit();
     };
@@ -288,12 +219,11 @@ __global__ void __launch_bounds__(rp::THREADS, 3) rtn_f16_kernel(const __half* _
         cp_async_wait<rp::STAGES - 1>();
         __syncwarp();     // this iteration's 2 KB, copied by all lanes, is in shared memory
         const int t = wi * 32 + lane;
-        const uint8_t* stage = ring + st * rp::STAGE_BYTES;
+        const uint4* mine = reinterpret_cast<const uint4*>(ring + st * rp::STAGE_BYTES + 64 * lane);
         st = (st + 1) & (rp::STAGES - 1);
         uint4 raw[4];
 #pragma unroll
-        for (int h = 0; h < 4; ++h)      // (lanes past the end hold stale data, unused)
-            raw[h] = *reinterpret_cast<const uint4*>(stage + 16 * ring_chunk(4 * lane + h));
+        for (int h = 0; h < 4; ++h) raw[h] = mine[h];   // (lanes past the end hold stale data, unused)
         // group min/max on the fp16 pairs (exact: the fp16 -> fp32 conversion is monotone)
         const __half2* hp = reinterpret_cast<const __half2*>(raw);
         __half2 mn2 = __hmin2(hp[0], hp[1]), mx2 = __hmax2(hp[0], hp[1]);
@@ -311,35 +241,36 @@ __global__ void __launch_bounds__(rp::THREADS, 3) rtn_f16_kernel(const __half* _
         }
         if (t >= n_chunks) continue;
         const QParams p = sym ? group_params_sym(mn, mx, maxq) : group_params_stream(mn, mx, maxq);
+        // m = fma(w, 1/scale, zero + 1.5 * 2^23): the product is exact inside the fma and the
+        // single rounding (ulp 1 at 1.5 * 2^23) rounds w/scale + zero to the nearest integer,
+        // half to even, leaving it in the low mantissa bits. Every w lies inside the group's
+        // range, so the rounded value is within 3.1e-5 of the exact w/scale + zero (1/scale is
+        // within 2^-23). A second fma gives the residual r = w/scale + zero - code; if every |r|
+        // stays 6e-5 clear of 1/2, every code is the exact rounding and lies in [0, maxq] (no
+        // clamp); otherwise the chunk is redone on the exact path.
         constexpr float kMagic = 12582912.0f;                  // 1.5 * 2^23
         const float C = p.zero + kMagic;                         // exact: zero is an integer
-        // 2^112 * inv * (1 +- 2^-20); scales below 2^-14 (inv above 2^14, where 2^112 * inv
-        // could overflow) take the exact path
-        const bool fast = p.inv_scale < 16384.0f;
-        const float inv_up = p.inv_scale * 5.192296858534828e33f * (1.0f + 9.5367431640625e-7f);
-        const float inv_dn = p.inv_scale * 5.192296858534828e33f * (1.0f - 9.5367431640625e-7f);
-        const unsigned long long INVP = f2_pack(inv_up, inv_up), INVM = f2_pack(inv_dn, inv_dn);
-        const unsigned long long CC = f2_pack(C, C);
-        const uint32_t* wu = reinterpret_cast<const uint32_t*>(raw);
-        unsigned long long mp[16];
-        unsigned long long acc = 0ull;
+        float m[32];
+        float dev = 0.0f;
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-            const unsigned long long x = half2_bits_scaled(wu[i]);
-            mp[i] = f2_fma(x, INVP, CC);
-            const unsigned long long mm = f2_fma(x, INVM, CC);
-            acc = f2_add(acc, f2_sub(mp[i], mm));
+            const float2 f = __half22float2(hp[i]);
+            m[2 * i] = fmaf(f.x, p.inv_scale, C);
+            m[2 * i + 1] = fmaf(f.y, p.inv_scale, C);
+            const float r0 = fmaf(f.x, p.inv_scale, C - m[2 * i]);      // C - m is exact
+            const float r1 = fmaf(f.y, p.inv_scale, C - m[2 * i + 1]);
+            dev = fmaxf(dev, fmaxf(fabsf(r0), fabsf(r1)));
         }
-        if (!fast || f2_lo(acc) != 0.0f || f2_hi(acc) != 0.0f) {
-            // rare: a code near a rounding boundary (or a tiny scale); redo the chunk exactly
-            rtn_chunk_exact_ring(stage, lane, p, bits, out, t);
+        if (dev > 0.5f - 6.0e-5f) {
+            // rare: a code within 6e-5 of a rounding boundary; redo the chunk on the exact path
+            rtn_chunk_exact(reinterpret_cast<const __half*>(mine), p, bits, out, t);
         } else if (INT4) {
             // byte b holds codes 2b (low nibble) and 2b+1: (M + q0) + 16 q1 has q0 + 16 q1 in its
             // low byte (exact: all values are integers below 2^24)
             uint32_t by[16];
 #pragma unroll
             for (int b = 0; b < 16; ++b)
-                by[b] = __float_as_uint(fmaf(f2_hi(mp[b]) - kMagic, 16.0f, f2_lo(mp[b])));
+                by[b] = __float_as_uint(fmaf(m[2 * b + 1] - kMagic, 16.0f, m[2 * b]));
             uint32_t word[4];
 #pragma unroll
             for (int w4 = 0; w4 < 4; ++w4)
@@ -351,8 +282,8 @@ __global__ void __launch_bounds__(rp::THREADS, 3) rtn_f16_kernel(const __half* _
             uint32_t word[8];
 #pragma unroll
             for (int w4 = 0; w4 < 8; ++w4)
-                word[w4] = __byte_perm(__byte_perm(__float_as_uint(f2_lo(mp[2 * w4])), __float_as_uint(f2_hi(mp[2 * w4])), 0x0040),
-                                       __byte_perm(__float_as_uint(f2_lo(mp[2 * w4 + 1])), __float_as_uint(f2_hi(mp[2 * w4 + 1])), 0x0040), 0x5410);
+                word[w4] = __byte_perm(__byte_perm(__float_as_uint(m[4 * w4]), __float_as_uint(m[4 * w4 + 1]), 0x0040),
+                                       __byte_perm(__float_as_uint(m[4 * w4 + 2]), __float_as_uint(m[4 * w4 + 3]), 0x0040), 0x5410);
             __stcs(reinterpret_cast<uint4*>(out) + 2 * t, make_uint4(word[0], word[1], word[2], word[3]));
             __stcs(reinterpret_cast<uint4*>(out) + 2 * t + 1, make_uint4(word[4], word[5], word[6], word[7]));
         }

@@ -208,3 +208,70 @@ def test_clip_search_without_h_is_weight_mse():
     b = rtn.rtn_clip_search(W, 4, 16, H=np.eye(32))
     assert np.array_equal(a[3], b[3]) and np.allclose(a[4], b[4], rtol=1e-12, atol=0)
     assert np.any(a[3] > 0)               # the outlier groups do get clipped
+
+
+# ---------------------------------------------------- percentile / fixed-range clipping -------
+def test_group_quantile_worked_example_and_library():
+    """The interpolation between order statistics: [1, 2, 3, 4, 10] at 0.9 sits at position
+    0.9·4 = 3.6, so 4 + 0.6·(10 − 4) = 7.6; at 0.1 at 0.4: 1 + 0.4·1 = 1.4. The 0 and 1
+    quantiles are the min and the max, and positions that are whole numbers give the order
+    statistic itself. It agrees with numpy's default ("linear") quantile to rounding."""
+    v = np.array([[1.0, 2.0, 3.0, 4.0, 10.0]])
+    assert abs(rtn.group_quantile(v, 0.9)[0] - 7.6) < 1e-14
+    assert abs(rtn.group_quantile(v, 0.1)[0] - 1.4) < 1e-14
+    assert rtn.group_quantile(v, 1.0)[0] == 10.0 and rtn.group_quantile(v, 0.0)[0] == 1.0
+    assert rtn.group_quantile(v, 0.5)[0] == 3.0 and rtn.group_quantile(v, 0.75)[0] == 4.0
+    rng = np.random.default_rng(5)
+    x = np.sort(rng.standard_normal((300, 128)), axis=1)
+    for p in (0.9999, 0.999, 0.99, 0.9, 0.5, 0.0001):
+        q = rtn.group_quantile(x, p)
+        ref = np.quantile(x, p, axis=1)
+        # (rounding relative to the interpolated values, which may cancel towards 0)
+        assert np.all(np.abs(q - ref) <= 4 * np.spacing(np.max(np.abs(x), axis=1))), p
+        assert np.all(q >= x[:, :1].T[0]) and np.all(q <= x[:, -1])
+
+
+@pytest.mark.parametrize("sym", [False, True])
+def test_range_clip_without_clipping_is_plain_rtn(sym):
+    W = _weights(12, 128, 11)
+    c, s, z = rtn.rtn_minmax(W, 4, 32, sym=sym)
+    for kw in (dict(), dict(abs_range=float(np.max(np.abs(W))))):
+        codes, scales, zeros, lo, hi = rtn.rtn_range_clip(W, 4, 32, sym=sym, **kw)
+        assert np.array_equal(codes, c) and np.array_equal(scales, s)
+        assert np.array_equal(zeros, z)
+
+
+@pytest.mark.parametrize("sym", [False, True])
+@pytest.mark.parametrize("percentile,abs_range", [(99.99, 0.0), (99.0, 0.0), (90.0, 0.0),
+                                                  (100.0, 0.02), (99.9, 0.05)])
+def test_range_clip_codes_are_the_nearest_level_of_the_clamped_weight(sym, percentile,
+                                                                      abs_range):
+    """Brute force: every code is the nearest level of the clamped weight (ties to the even
+    quotient), values beyond a bound take the bound's code, |clip(w) − ŵ| <= scale/2, and the
+    bounds are the quantiles (limited by the absolute range)."""
+    bits, g = 4, 16
+    maxq = 2 ** bits - 1
+    W = _weights(9, 64, 12)
+    codes, scales, zeros, lo, hi = rtn.rtn_range_clip(W, bits, g, percentile, abs_range, sym)
+    Wg = W.reshape(9, 4, g)
+    v = np.sort(Wg, axis=2)
+    p = percentile / 100.0
+    exp_hi, exp_lo = rtn.group_quantile(v, p), rtn.group_quantile(v, 1.0 - p)
+    if abs_range > 0:
+        exp_hi, exp_lo = np.minimum(exp_hi, abs_range), np.maximum(exp_lo, -abs_range)
+    assert np.array_equal(hi, exp_hi) and np.array_equal(lo, exp_lo)
+    wc = np.clip(Wg, lo[..., None], hi[..., None])
+    s, z = scales[..., None], zeros[..., None]
+    levels = np.arange(maxq + 1)
+    recon = s[..., None] * (levels - z[..., None])               # [r, k, 1, levels]
+    dist = np.abs(wc[..., None] - recon)
+    q = codes.reshape(9, 4, g)
+    got = np.take_along_axis(dist, q[..., None], axis=3)[..., 0]
+    assert np.all(got <= dist.min(axis=3) + 1e-18)
+    assert np.all(np.abs(wc - s * (q - z)) <= s / 2 + 1e-18)
+    clipped = (Wg > hi[..., None]) | (Wg < lo[..., None])
+    if percentile < 100.0:
+        assert clipped.any()
+    bound = np.where(Wg > hi[..., None], hi[..., None], lo[..., None])
+    q_bound = quantizer.quantize(bound, s, z, maxq)
+    assert np.array_equal(q[clipped], q_bound[clipped])
