@@ -762,14 +762,10 @@ def run_ours(args):
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic",
-        "config": {"workload": f"{wl.name}: W {d_out}x{d} {wl.w_dtype}, X {n}x{d} fp16 "
-                               f"(lognormal channel scales, outliers), INT{wl.bits} g{wl.group_size} "
-                               f"B{wl.block_size} percdamp {wl.percdamp} act_order {wl.act_order}",
-                   "per_rank": "one independent layer per GPU (seed = rank)",
-                   "l2": "X (2.1 GB) larger than L2, plus a 512 MB L2 flush between steps",
-                   "arithmetic": "Hessian and loss Gram matrix fp16 x fp16 -> fp32 on tcgen05; "
-                                 "factorisation and lazy update fp32 as 3xTF32 on tcgen05; "
-                                 "column loop fp32 FFMA; group scalars fp64"},
+        "config": workload_config(wl),
+        "arithmetic": "Hessian and loss Gram matrix fp16 x fp16 -> fp32 on tcgen05; "
+                      "factorisation and lazy update fp32 as 3xTF32 on tcgen05; "
+                      "column loop fp32 FFMA; group scalars fp64",
         "calib_tokens_per_s": world * n / (hess_ms / 1e3),
         "layer_loss": step.loss,
         "stages": stages,
@@ -789,6 +785,17 @@ def run_ours(args):
     if distributed:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+def workload_config(wl):
+    """The `config` object of both arms' lines: the same workload, named the same way."""
+    d_out, d, n = wl.d_out, wl.d_in, wl.n_tokens
+    return {"workload": f"{wl.name}: W {d_out}x{d} {wl.w_dtype}, X {n}x{d} fp16 "
+                        f"(lognormal channel scales, outliers), INT{wl.bits} g{wl.group_size} "
+                        f"B{wl.block_size} percdamp {wl.percdamp} act_order {wl.act_order}",
+            "per_rank": "one independent layer per GPU (seed = rank)",
+            "l2": f"X ({n * d * 2 / 1e9:.1f} GB) larger than L2, plus a 512 MB L2 flush "
+                  f"between steps"}
 
 
 def run_e2e(step, gptq, args, distributed, device, world):
@@ -919,9 +926,7 @@ def run_reference(args):
            "warmup": args.warmup, "ms_per_step": full * 1e3, "higher_is_better": True,
            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
            "impl": "reference",
-           "config": {"workload": f"{wl.name}: W {wl.d_out}x{wl.d_in} {wl.w_dtype}, "
-                                  f"X {wl.n_tokens}x{wl.d_in} fp16, INT{wl.bits} g{wl.group_size} "
-                                  f"B{wl.block_size} percdamp {wl.percdamp}"},
+           "config": workload_config(wl),
            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                             "sample": detail + f"; {args.steps} timed samples; " + THREAD_NOTE},
            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -952,6 +957,13 @@ def run_ncu_case(name: str):
         W = workloads.make_weights(wl, device="cuda")
         for _ in range(3):
             gptq.rtn_minmax_quantize(W, 4, 128)
+    elif name == "w4a16":                        # X 16384 x 4096, W 22016 x 4096 INT4; 3 launches
+        W = workloads.make_weights(wl.replace(d_out=22016), device="cuda")
+        packed, scales, zeros = gptq.rtn_minmax_quantize(W, 4, 128)
+        X = workloads.make_activations(wl.replace(n_tokens=16384), device="cuda")
+        Y = torch.empty(16384, 22016, dtype=torch.float16, device="cuda")
+        for _ in range(3):
+            gptq.w4a16_linear(X, packed, scales, zeros, 128, out=Y)
     elif name == "rtn_big":                      # 4 layers of 7B weights: 153600 x 4096 fp16
         W = workloads.make_weights(wl.replace(d_out=4 * (4 * 4096 + 2 * 11008)), device="cuda")
         for _ in range(3):                       # (1.26 GB, ten times L2)
@@ -978,7 +990,7 @@ def main(argv=None):
     ap.add_argument("--no-stack", action="store_true",
                     help="skip GPTQ over a full 7B decoder stack (4 variants)")
     ap.add_argument("--stack-layers", type=int, default=32)
-    ap.add_argument("--ncu-case", choices=("hessian", "gptq", "rtn", "rtn_big"),
+    ap.add_argument("--ncu-case", choices=("hessian", "gptq", "rtn", "rtn_big", "w4a16"),
                     help="run one small case for an ncu capture and exit (no JSON line)")
     args = ap.parse_args(argv)
     if args.ncu_case:

@@ -24,9 +24,10 @@
  *     them. No call allocates device memory except gptq_hessian_create.
  *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream). Work is
  *     ordered on it. Calls are not thread-safe on the same handle or workspace.
- *   - gptq_quantize_layer and gptq_inverse_factor also run part of the factorisation on a
- *     second stream that the library owns (one per device). It is forked from `stream` and
- *     joined back to it by events inside the call, so the call stays ordered on `stream`.
+ *   - gptq_quantize_layer and gptq_inverse_factor also run part of the factorisation (and
+ *     gptq_quantize_layer part of its far lazy updates) on a second stream that the library
+ *     owns (one per device). It is forked from `stream` and joined back to it by events inside
+ *     the call, so the call stays ordered on `stream`.
  *   - One process drives one GPU. The library sets its kernels' shared-memory limits once per
  *     process, on the device current at the first call; a process that switches devices
  *     between calls is not supported (launches on the second device fail with CUDA).
@@ -188,7 +189,7 @@ gptq_status gptq_quantize_layer_ex(const void* W, int w_dtype, int d_out, int d_
  * that reserves its memory pools at start-up should make one call before reserving them.
  *   - Layers whose gptq_quantize_layer_workspace(d_out, d_in, block_size) exceeds 32 MiB are
  *     rejected with GPTQ_ERR_WORKSPACE before anything is launched. For example, d_in = 1024
- *     fits up to d_out = 2615 and d_in = 512 up to d_out = 4646; d_in = 4096 does not fit.
+ *     fits up to d_out = 1811 and d_in = 512 up to d_out = 2876; d_in = 4096 does not fit.
  *   - No cudaMalloc, cudaFree or other allocating call is made.
  *   - The first call on each device looks up the array's device address (cudaGetSymbolAddress
  *     with that device current). Make that first call before any stream capture on the device.
@@ -253,6 +254,25 @@ gptq_status rtn_clip_search(const void* W, int w_dtype, int d_out, int d_in, int
                             int group_size, int sym, const float* H, double min_ratio,
                             double step, uint8_t* packed, uint16_t* scales, uint16_t* zeros,
                             uint8_t* ratio_idx, void* stream);
+
+/* Group RTN of clipped weights (bhfrc.com §4.3: instead of the extreme values, take a
+ * percentile of the values, such as 99.99 %, or a fixed absolute range, such as [-10, 10], and
+ * truncate what lies outside before the min-max range is formed).
+ *   Per group: hi = the p-quantile and lo = the (1 - p)-quantile of its weights,
+ *   p = percentile / 100; a q-quantile is v[k] + t * (v[k+1] - v[k]) with v the group sorted
+ *   ascending, h = q * (group_size - 1), k = floor(h), t = h - k (v[group_size-1] when k is the
+ *   last position), every operation rounded on its own in fp64. With abs_range > 0, lo and hi
+ *   are further limited to [-abs_range, abs_range]. The weights are clamped to [lo, hi] and
+ *   quantized with the quantizer of the range [lo, hi] (asymmetric: widened to contain 0;
+ *   symmetric with sym = 1: m = max(|lo|, |hi|)). percentile = 100 and abs_range = 0 give
+ *   rtn_quantize_ex. Codes, scales and zeros equal that fp64 definition bit for bit.
+ *   W        device [d_out x d_in], fp16 or fp32, finite.  d_in: a multiple of group_size.
+ *   group_size  16, 32, 64 or 128.   percentile in [50, 100].   abs_range >= 0 (0: none).
+ *   packed, scales, zeros  as rtn_minmax_quantize.
+ * Asynchronous. Errors: ARG, CUDA, UNSUPPORTED. */
+gptq_status rtn_range_clip(const void* W, int w_dtype, int d_out, int d_in, int bits,
+                           int group_size, int sym, double percentile, double abs_range,
+                           uint8_t* packed, uint16_t* scales, uint16_t* zeros, void* stream);
 
 /* rtn_minmax_quantize with the symmetric quantizer as an option (sym = 1: zero point fixed,
  * see gptq_quantize_layer_ex; sym = 0 is rtn_minmax_quantize). Same layouts and errors. */

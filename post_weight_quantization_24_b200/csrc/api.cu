@@ -134,8 +134,8 @@ struct Workspace {
     float* A;        // d^2: damped, permuted, reversed H -> Cholesky factor; later undamped Hp
     float* X;        // d^2: L^-1, then U
     float* Wk;       // d_out x d_in working weights (processing order)
-    float* Err;      // d_out x kSuperCols errors of the current super-block (tf32 hi part)
-    float* ErrLo;    // d_out x kSuperCols (tf32 lo part)
+    float* Err[2];   // d_out x kSuperCols errors of a super-block (tf32 hi part), two buffers:
+    float* ErrLo[2]; // a super-block's far update may still read one while the next fills the other
     uint8_t* codes_p;// d_out x d_in codes in processing order
     float* P;        // d x 128: the column loop's images of U's diagonal blocks
     float* Dinv;     // ceil(d/128) x 128 x 128 inverses of the Cholesky diagonal blocks
@@ -158,8 +158,10 @@ static Workspace layout(void* base, int d_out, int d_in) {
     w.A = reinterpret_cast<float*>(take(d * d * 4));
     w.X = reinterpret_cast<float*>(take(d * d * 4));
     w.Wk = reinterpret_cast<float*>(take(static_cast<size_t>(d_out) * d * 4));
-    w.Err = reinterpret_cast<float*>(take(static_cast<size_t>(d_out) * kSuperCols * 4));
-    w.ErrLo = reinterpret_cast<float*>(take(static_cast<size_t>(d_out) * kSuperCols * 4));
+    for (int b = 0; b < 2; ++b) {
+        w.Err[b] = reinterpret_cast<float*>(take(static_cast<size_t>(d_out) * kSuperCols * 4));
+        w.ErrLo[b] = reinterpret_cast<float*>(take(static_cast<size_t>(d_out) * kSuperCols * 4));
+    }
     w.codes_p = take(static_cast<size_t>(d_out) * d);
     w.P = reinterpret_cast<float*>(take(d * kCholBlock * 4));
     w.Dinv = reinterpret_cast<float*>(take(nbl * kCholBlock * kCholBlock * 4));
@@ -359,29 +361,72 @@ gptq_status gptq_quantize_layer_ex(const void* W, int w_dtype, int d_out, int d_
     // kSuperCols columns) are kept; after each block only the rest of its super-block is
     // updated, and the columns beyond the super-block get one update per super-block. Every
     // column still receives the compensation of all earlier columns before it is quantized.
+    // The far update of super-block S is split in two: the next super-block's columns on the
+    // caller's stream (its column loop needs them next), and all later columns on the library's
+    // second stream, where it runs on the SMs the next column loop leaves free. The main stream
+    // waits for that rest before it next writes those columns; the errors alternate between
+    // two buffers so the rest can read S's errors while S+1 records its own.
     const int super = block_size * std::max(1, kSuperCols / block_size);
-    for (int s0 = 0; s0 < d_in; s0 += super) {
-        const int s1 = std::min(s0 + super, d_in);
-        for (int j0 = s0; j0 < s1; j0 += block_size) {
-            const int bw = std::min(block_size, s1 - j0), j1 = j0 + bw;
-            float* err_hi = ws.Err + (j0 - s0);
-            float* err_lo = ws.ErrLo + (j0 - s0);
-            tm.begin(3);
-            GPTQ_TRY(gptq_block_launch(ws.Wk, d_out, d_in, j0, bw, ws.P, ws.Dinv, group_size,
-                                       bits, sym, preset ? ws.perm : nullptr, codes_p, scales,
-                                       zeros, err_hi, err_lo, kSuperCols, &ws.st->err_sq, status,
-                                       s));
-            tm.end();
-            tm.begin(4);
-            GPTQ_TRY(lazy_update_launch(ws.Wk, d_out, d_in, j0, j1, j1, s1, ws.X, ws.A, err_hi,
-                                        err_lo, kSuperCols, status, s));
-            tm.end();
-        }
-        tm.begin(4);
-        GPTQ_TRY(lazy_update_launch(ws.Wk, d_out, d_in, s0, s1, s1, d_in, ws.X, ws.A, ws.Err,
-                                    ws.ErrLo, kSuperCols, status, s));
-        tm.end();
+    const int side_ctas = num_sms() - gptq_rows_ctas(d_out);
+    const bool overlap = side_ctas >= 16 && d_in > 2 * super;
+    // while the overlap runs, the caller's stream keeps its GEMMs on the SMs the second stream
+    // leaves free, so that every CTA of a persistent launch is resident at once
+    const int main_ctas = overlap ? num_sms() - side_ctas : 0;
+    std::unique_lock<std::mutex> side_lock(side_streams_mutex(), std::defer_lock);
+    SideStreams* ss = nullptr;
+    if (overlap) {
+        side_lock.lock();
+        GPTQ_TRY(side_streams(&ss));
+        GPTQ_CUDA_TRY(cudaEventRecord(ss->aux1, s));
+        GPTQ_CUDA_TRY(cudaStreamWaitEvent(ss->side, ss->aux1, 0));
     }
+    auto column_stage = [&]() -> gptq_status {
+        bool rest_pending = false;
+        for (int s0 = 0, sb = 0; s0 < d_in; s0 += super, ++sb) {
+            const int s1 = std::min(s0 + super, d_in);
+            const int s2 = std::min(s1 + super, d_in);
+            float* Eh = ws.Err[sb & 1];
+            float* El = ws.ErrLo[sb & 1];
+            for (int j0 = s0; j0 < s1; j0 += block_size) {
+                const int bw = std::min(block_size, s1 - j0), j1 = j0 + bw;
+                float* err_hi = Eh + (j0 - s0);
+                float* err_lo = El + (j0 - s0);
+                tm.begin(3);
+                GPTQ_TRY(gptq_block_launch(ws.Wk, d_out, d_in, j0, bw, ws.P, ws.Dinv, group_size,
+                                           bits, sym, preset ? ws.perm : nullptr, codes_p,
+                                           scales, zeros, err_hi, err_lo, kSuperCols,
+                                           &ws.st->err_sq, status, s));
+                tm.end();
+                tm.begin(4);
+                GPTQ_TRY(lazy_update_launch(ws.Wk, d_out, d_in, j0, j1, j1, s1, ws.X, ws.A,
+                                            err_hi, err_lo, kSuperCols, status, s, main_ctas));
+                tm.end();
+            }
+            tm.begin(4);
+            if (rest_pending) GPTQ_CUDA_TRY(cudaStreamWaitEvent(s, ss->aux2, 0));
+            GPTQ_TRY(lazy_update_launch(ws.Wk, d_out, d_in, s0, s1, s1, overlap ? s2 : d_in,
+                                        ws.X, ws.A, Eh, El, kSuperCols, status, s, main_ctas));
+            tm.end();
+            if (overlap && s2 < d_in) {
+                GPTQ_CUDA_TRY(cudaEventRecord(ss->aux1, s));      // S's errors are complete
+                GPTQ_CUDA_TRY(cudaStreamWaitEvent(ss->side, ss->aux1, 0));
+                GPTQ_TRY(lazy_update_launch(ws.Wk, d_out, d_in, s0, s1, s2, d_in, ws.X, ws.A, Eh,
+                                            El, kSuperCols, status, ss->side, side_ctas));
+                GPTQ_CUDA_TRY(cudaEventRecord(ss->aux2, ss->side));
+                rest_pending = true;
+            }
+        }
+        return GPTQ_OK;
+    };
+    const gptq_status crc = column_stage();
+    if (overlap) {
+        // join the second stream back, also after an error, so a capture of `s` stays formed
+        const cudaError_t e1 = cudaEventRecord(ss->join, ss->side);
+        const cudaError_t e2 = cudaStreamWaitEvent(s, ss->join, 0);
+        side_lock.unlock();
+        if (crc == GPTQ_OK && (e1 != cudaSuccess || e2 != cudaSuccess)) return GPTQ_ERR_CUDA;
+    }
+    GPTQ_TRY(crc);
     // ---- stage 5: outputs in the original column order ----
     tm.begin(5);
     GPTQ_TRY(assemble_launch(codes_p, d_out, d_in, ws.perm, ws.invperm, group_size, act_order,

@@ -391,13 +391,12 @@ __global__ void reverse_inplace_kernel(float* X, int64_t half) {
 // Per device: a second stream and the events that order the two streams. The enqueue of one
 // factorisation holds the mutex, so the events are never recorded by two sequences at once.
 namespace {
-struct SideStreams {
-    cudaStream_t side = nullptr;
-    cudaEvent_t fork = nullptr, trsm = nullptr, rest = nullptr, join = nullptr;
-};
 constexpr int kMaxDevices = 64;
 SideStreams g_side[kMaxDevices];
 std::mutex g_side_mu;
+}  // namespace
+
+std::mutex& side_streams_mutex() { return g_side_mu; }
 
 gptq_status side_streams(SideStreams** out) {
     int dev = 0;
@@ -406,13 +405,12 @@ gptq_status side_streams(SideStreams** out) {
     SideStreams& ss = g_side[dev];
     if (!ss.side) {
         GPTQ_CUDA_TRY(cudaStreamCreateWithFlags(&ss.side, cudaStreamNonBlocking));
-        for (cudaEvent_t* e : {&ss.fork, &ss.trsm, &ss.rest, &ss.join})
+        for (cudaEvent_t* e : {&ss.fork, &ss.trsm, &ss.rest, &ss.join, &ss.aux1, &ss.aux2})
             GPTQ_CUDA_TRY(cudaEventCreateWithFlags(e, cudaEventDisableTiming));
     }
     *out = &ss;
     return GPTQ_OK;
 }
-}  // namespace
 
 // Blocked right-looking Cholesky of A with one step of lookahead, and the blocked triangular
 // inverse X = L^-1, then U = reverse(X).

@@ -37,7 +37,7 @@ namespace gr {
 constexpr int MAXB = 128;                    // widest block handled in one launch
 constexpr int PH = 16;                       // block columns per window phase
 constexpr int NPH = MAXB / PH;
-constexpr int WARPS = 2;
+constexpr int WARPS = 4;
 constexpr int THREADS = WARPS * 32;          // one row per thread
 constexpr int SMEM = MAXB * MAXB * 4 + MAXB * 4 + NPH * 8 + MAXB * 4;   // + grid indices
 }  // namespace gr
@@ -171,7 +171,7 @@ __device__ __forceinline__ bool rows_phases(float (&w)[gr::MAXB], RowCtx& x, uin
     return true;
 }
 
-__global__ void __launch_bounds__(gr::THREADS, 3) gptq_rows_kernel(
+__global__ void __launch_bounds__(gr::THREADS, 2) gptq_rows_kernel(
     const float* __restrict__ Wk, int d_out, int d_in, int j0, int bw,
     const float* __restrict__ img, const float* __restrict__ rdiag, int g, int bits, int sym,
     const int* __restrict__ preset_perm, uint8_t* __restrict__ codes_p,
@@ -324,17 +324,19 @@ gptq_status group_grid_launch(const void* W, int w_dtype, int d_out, int d_in, i
 
 // W[:, c0:c1] -= Err[:, 0:k1-k0] * U[k0:k1, c0:c1]  (3xTF32 on the tensor cores, with both
 // operands split into tf32 hi/lo once: U after the factorisation, Err by the column loop)
+int gptq_rows_ctas(int d_out) { return (d_out + gr::THREADS - 1) / gr::THREADS; }
+
 gptq_status lazy_update_launch(float* Wk, int d_out, int d_in, int k0, int k1, int c0, int c1,
                                const float* U_hi, const float* U_lo, const float* Err_hi,
                                const float* Err_lo, int err_ld, const int* status,
-                               cudaStream_t s) {
+                               cudaStream_t s, int max_ctas) {
     if (c1 <= c0 || k1 <= k0) return GPTQ_OK;
     const int64_t boff = static_cast<int64_t>(k0) * d_in + c0;
     TcGemmArgs a{};
     a.M = d_out; a.N = c1 - c0; a.K = k1 - k0; a.alpha = -1.f; a.beta = 1.f;
     a.A = Err_hi; a.A_lo = Err_lo; a.lda = err_ld;
     a.B = U_hi + boff; a.B_lo = U_lo + boff; a.ldb = d_in;
-    a.C = Wk + c0; a.ldc = d_in; a.status = status;
+    a.C = Wk + c0; a.ldc = d_in; a.status = status; a.max_ctas = max_ctas;
     return tcgemm_presplit_launch(a, s);
 }
 

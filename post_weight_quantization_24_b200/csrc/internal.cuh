@@ -1,9 +1,22 @@
 // Declarations shared between the library's translation units.
 #pragma once
 
+#include <mutex>
+
 #include "common.cuh"
 
 namespace gq {
+
+// The library's second stream on the current device and the events that order it with the
+// caller's stream (created on first use; one set per device). Hold side_streams_mutex() while
+// enqueuing work that uses them.
+struct SideStreams {
+    cudaStream_t side = nullptr;
+    cudaEvent_t fork = nullptr, trsm = nullptr, rest = nullptr, join = nullptr;
+    cudaEvent_t aux1 = nullptr, aux2 = nullptr;
+};
+std::mutex& side_streams_mutex();
+gptq_status side_streams(SideStreams** out);
 
 // Per-call device state at the head of the quantizer workspace (zeroed at the start of a call).
 struct DevState {
@@ -70,7 +83,9 @@ gptq_status group_grid_launch(const void* W, int w_dtype, int d_out, int d_in, i
 gptq_status lazy_update_launch(float* Wk, int d_out, int d_in, int k0, int k1, int c0, int c1,
                                const float* U_hi, const float* U_lo, const float* Err_hi,
                                const float* Err_lo, int err_ld, const int* status,
-                               cudaStream_t s);
+                               cudaStream_t s, int max_ctas = 0);
+// CTAs of one column-loop launch for d_out rows
+int gptq_rows_ctas(int d_out);
 gptq_status assemble_launch(const uint8_t* codes_p, int d_out, int d_in, const int* perm,
                             const int* invperm, int group_size, int act_order, int preset,
                             uint8_t* codes, int32_t* g_idx, int32_t* perm_out, cudaStream_t s);

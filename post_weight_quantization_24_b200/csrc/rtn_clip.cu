@@ -19,6 +19,7 @@
 // so for a given ratio the codes, scales and zeros equal the fp64 definition bit for bit; the
 // criterion itself is fp32.
 #include <algorithm>
+#include <cmath>
 
 #include "internal.cuh"
 #include "quant.cuh"
@@ -228,7 +229,177 @@ gptq_status rtn_clip_launch(const void* W, int w_dtype, int d_out, int d_in, int
                          step, out, scales, zeros, ratio_idx, s);
 }
 
+// ---------------------------------------------------------------------------------------
+// Percentile and fixed-range clipping (bhfrc.com/news/5741 §4.3: take a percentile of the
+// values, such as 99.99 %, or an absolute range, such as [-10, 10], instead of the extreme
+// values, and truncate what lies outside). Per group: lo and hi are the (1 - p) and p
+// quantiles of its values, each interpolated linearly between the two order statistics around
+// position frac * (g - 1) (q = v[k] + t * (v[k+1] - v[k]), every operation rounded on its own
+// in fp64); with a fixed range a > 0 they are limited to [-a, a]. The weights are clamped to
+// [lo, hi] and quantized with the quantizer of that range.
+//
+// Kernel: the clip search's layout (one CTA per group and 128 rows, the group transposed in
+// shared memory, one thread per row). Each thread finds the four order statistics it needs by
+// counting, for every value of its row's group, the values below it (index order breaks ties),
+// which costs g^2 comparisons per row and group and no sort.
+// ---------------------------------------------------------------------------------------
+struct RangeClipArgs {
+    int kl, kh;          // order-statistic positions of the lower and upper quantile
+    double tl, th;       // their interpolation weights
+    double abs_range;    // 0: no fixed range
+};
+
+// Code of w under the clamp to [lo, hi] and the grid p: clamped weights are quantized at the
+// bound in fp64 (lo and hi are fp64 values), the others by the exact rounding of quant_code.
+__device__ __noinline__ int range_code_slow(float w, double lo, double hi, QParams p, int maxq) {
+    const double wd = static_cast<double>(w);
+    if (wd > hi || wd < lo) {
+        const double q = rint((wd > hi ? hi : lo) / static_cast<double>(p.scale)) +
+                         static_cast<double>(p.zero);
+        return static_cast<int>(fmin(fmax(q, 0.0), static_cast<double>(maxq)));
+    }
+    return quant_code(w, p, maxq);
+}
+
+// Fast path: lof < w < hif (the bounds rounded inwards to fp32, so w is not clamped) and
+// w/scale clear of a rounding boundary by more than the error of its fp32 quotient.
+__device__ __forceinline__ int range_code(float w, double lo, double hi, float lof, float hif,
+                                          const QParams& p, int maxq) {
+    const float t = w * p.inv_scale;
+    const float k = rintf(t);
+    if (w > lof && w < hif && fabsf(t - k) <= 0.5f - fabsf(t) * 3.0e-7f - 1.0e-30f)
+        return static_cast<int>(fminf(fmaxf(k + p.zero, 0.0f), static_cast<float>(maxq)));
+    return range_code_slow(w, lo, hi, p, maxq);
+}
+
+__device__ __forceinline__ double lerp_rn(double v0, double v1, double t) {
+    return __dadd_rn(v0, __dmul_rn(t, __dsub_rn(v1, v0)));
+}
+
+template <int G, typename T>
+__global__ void __launch_bounds__(rc::ROWS) rtn_range_kernel(
+    const T* __restrict__ W, int d_out, int d_in, int bits, int sym, RangeClipArgs a,
+    uint8_t* __restrict__ out, uint16_t* __restrict__ scales, uint16_t* __restrict__ zeros) {
+    extern __shared__ __align__(16) float range_smem[];
+    float* Wt = range_smem;                   // [G][WS]: Wt[j][t] = W[r0 + t][k0 + j]
+    const int t = threadIdx.x;
+    const int k = blockIdx.x, r0 = blockIdx.y * rc::ROWS;
+    const int64_t k0 = static_cast<int64_t>(k) * G;
+    const int maxq = (1 << bits) - 1;
+    for (int rr = 0; rr < rc::ROWS; ++rr) {
+        const int r = r0 + rr;
+        for (int j = t; j < G; j += rc::ROWS)
+            Wt[j * rc::WS + rr] = r < d_out ? static_cast<float>(W[static_cast<int64_t>(r) * d_in + k0 + j]) : 0.0f;
+    }
+    __syncthreads();
+    const int r = r0 + t;
+    if (r >= d_out) return;
+
+    // the order statistics at positions kl, kl + 1, kh, kh + 1 (clamped to g - 1)
+    const int pl0 = a.kl, pl1 = min(a.kl + 1, G - 1), ph0 = a.kh, ph1 = min(a.kh + 1, G - 1);
+    float vl0 = 0.f, vl1 = 0.f, vh0 = 0.f, vh1 = 0.f;
+#pragma unroll 1
+    for (int j = 0; j < G; ++j) {
+        const float vj = Wt[j * rc::WS + t];
+        int rank = 0;
+#pragma unroll 8
+        for (int i = 0; i < G; ++i) {
+            const float vi = Wt[i * rc::WS + t];
+            rank += (vi < vj || (vi == vj && i < j)) ? 1 : 0;
+        }
+        if (rank == pl0) vl0 = vj;
+        if (rank == pl1) vl1 = vj;
+        if (rank == ph0) vh0 = vj;
+        if (rank == ph1) vh1 = vj;
+    }
+    double lo = a.kl >= G - 1 ? static_cast<double>(vl0)
+                              : lerp_rn(static_cast<double>(vl0), static_cast<double>(vl1), a.tl);
+    double hi = a.kh >= G - 1 ? static_cast<double>(vh0)
+                              : lerp_rn(static_cast<double>(vh0), static_cast<double>(vh1), a.th);
+    if (a.abs_range > 0.0) {
+        lo = fmax(lo, -a.abs_range);
+        hi = fmin(hi, a.abs_range);
+    }
+    const float lof = __double2float_ru(lo), hif = __double2float_rd(hi);
+    const QParams p = range_params(lo, hi, maxq, sym != 0);
+    if (bits == 4) {
+        uint8_t* o = out + static_cast<int64_t>(r) * (d_in / 2) + k0 / 2;
+        for (int j = 0; j < G; j += 2) {
+            const int q0 = range_code(Wt[j * rc::WS + t], lo, hi, lof, hif, p, maxq);
+            const int q1 = range_code(Wt[(j + 1) * rc::WS + t], lo, hi, lof, hif, p, maxq);
+            o[j / 2] = static_cast<uint8_t>(q0 | (q1 << 4));
+        }
+    } else {
+        uint8_t* o = out + static_cast<int64_t>(r) * d_in + k0;
+        for (int j = 0; j < G; ++j)
+            o[j] = static_cast<uint8_t>(range_code(Wt[j * rc::WS + t], lo, hi, lof, hif, p, maxq));
+    }
+    const int64_t gidx = static_cast<int64_t>(r) * (d_in / G) + k;
+    scales[gidx] = half_bits(p.scale);
+    zeros[gidx] = half_bits(p.zero);
+}
+
+template <int G, typename T>
+static gptq_status launch_range(const T* W, int d_out, int d_in, int bits, int sym,
+                                const RangeClipArgs& a, uint8_t* out, uint16_t* scales,
+                                uint16_t* zeros, cudaStream_t s) {
+    const int smem = G * rc::WS * 4;
+    GPTQ_CUDA_TRY(cudaFuncSetAttribute(rtn_range_kernel<G, T>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    const dim3 grid(d_in / G, (d_out + rc::ROWS - 1) / rc::ROWS);
+    rtn_range_kernel<G, T><<<grid, rc::ROWS, smem, s>>>(W, d_out, d_in, bits, sym, a, out,
+                                                        scales, zeros);
+    GPTQ_LAUNCHED();
+    return GPTQ_OK;
+}
+
+template <typename T>
+static gptq_status range_dispatch(const T* W, int d_out, int d_in, int bits, int g, int sym,
+                                  const RangeClipArgs& a, uint8_t* out, uint16_t* scales,
+                                  uint16_t* zeros, cudaStream_t s) {
+    switch (g) {
+        case 16: return launch_range<16>(W, d_out, d_in, bits, sym, a, out, scales, zeros, s);
+        case 32: return launch_range<32>(W, d_out, d_in, bits, sym, a, out, scales, zeros, s);
+        case 64: return launch_range<64>(W, d_out, d_in, bits, sym, a, out, scales, zeros, s);
+        case 128: return launch_range<128>(W, d_out, d_in, bits, sym, a, out, scales, zeros, s);
+        default: return GPTQ_ERR_ARG;
+    }
+}
+
 }  // namespace gq
+
+extern "C" gptq_status rtn_range_clip(const void* W, int w_dtype, int d_out, int d_in, int bits,
+                                      int group_size, int sym, double percentile,
+                                      double abs_range, uint8_t* packed, uint16_t* scales,
+                                      uint16_t* zeros, void* stream) {
+    if (!W || !packed || !scales || !zeros) return GPTQ_ERR_ARG;
+    if (w_dtype != GPTQ_DTYPE_F16 && w_dtype != GPTQ_DTYPE_F32) return GPTQ_ERR_ARG;
+    if (d_out < 1 || d_in < 16 || bits < 2 || bits > 8 || sym < 0 || sym > 1) return GPTQ_ERR_ARG;
+    if (group_size != 16 && group_size != 32 && group_size != 64 && group_size != 128)
+        return GPTQ_ERR_ARG;
+    if (d_in % group_size) return GPTQ_ERR_ARG;
+    if (!(percentile >= 50.0 && percentile <= 100.0) || !(abs_range >= 0.0) ||
+        std::isinf(abs_range))
+        return GPTQ_ERR_ARG;
+    // the quantile positions, each operation rounded on its own (as the definition reads)
+    const double p = percentile / 100.0;
+    const double q_lo = 1.0 - p;
+    const double gm1 = static_cast<double>(group_size - 1);
+    const double h_hi = p * gm1, h_lo = q_lo * gm1;
+    gq::RangeClipArgs a;
+    a.kh = static_cast<int>(std::floor(h_hi));
+    a.kl = static_cast<int>(std::floor(h_lo));
+    a.th = h_hi - a.kh;
+    a.tl = h_lo - a.kl;
+    a.abs_range = abs_range;
+    GPTQ_TRY(gq::check_device());
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (w_dtype == GPTQ_DTYPE_F16)
+        return gq::range_dispatch(static_cast<const __half*>(W), d_out, d_in, bits, group_size,
+                                  sym, a, packed, scales, zeros, s);
+    return gq::range_dispatch(static_cast<const float*>(W), d_out, d_in, bits, group_size, sym,
+                              a, packed, scales, zeros, s);
+}
 
 extern "C" gptq_status rtn_clip_search(const void* W, int w_dtype, int d_out, int d_in,
                                        int bits, int group_size, int sym, const float* H,

@@ -91,6 +91,9 @@ __global__ void __launch_bounds__(tg::THREADS, 1)
                   const __grid_constant__ CUtensorMap alomap,
                   const __grid_constant__ CUtensorMap blomap, const TcParams p) {
     static_assert(!PRE || (SPLIT_A && SPLIT_B), "pre-split operands come in hi/lo pairs");
+    // pre-split operands need no converter warps: the epilogue warps follow warp 1 directly
+    // (warps 2..5 take TMEM lane quarters 2, 3, 0, 1, as warps 10..13 do)
+    constexpr int EPI0 = PRE ? 2 : tg::EPI_WARP0;
     if (status_bad(p.a.status)) return;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -238,7 +241,7 @@ __global__ void __launch_bounds__(tg::THREADS, 1)
             if (!mbar_wait(drained, 0)) set_status(status, GPTQ_ERR_TIMEOUT);
         }
         __syncwarp();
-    } else if (warp < tg::EPI_WARP0) {
+    } else if (warp < EPI0) {
         // ---------------- converters: fp32 -> tf32 hi (in place) + lo ----------------
         if constexpr (!PRE) {   // (pre-split operands arrive ready for the MMA)
             const int ct = (warp - 2) * 32 + lane;   // 0..255
@@ -304,7 +307,7 @@ __global__ void __launch_bounds__(tg::THREADS, 1)
         // ---------------- epilogue ----------------
         const int q = warp & 3;
         const uint32_t t_lane = static_cast<uint32_t>(32 * q) << 16;
-        float* stage_buf = epi_smem + (warp - tg::EPI_WARP0) * 2 * (tg::EPI_BUF / 4);
+        float* stage_buf = epi_smem + (warp - EPI0) * 2 * (tg::EPI_BUF / 4);
         double dot = 0.0;
         int lt = 0, nbulk = 0;
         bool stop = false;
@@ -401,8 +404,9 @@ static gptq_status launch_variant(const CUtensorMap& am, const CUtensorMap& bm,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, tg::SMEM));
         attr = true;
     }
-    tcgemm_kernel<B_K, EPI, SA, SB, PRE><<<grid, tg::THREADS, tg::SMEM, s>>>(am, bm, cm, alom,
-                                                                             blom, p);
+    constexpr int threads = PRE ? 6 * 32 : tg::THREADS;
+    tcgemm_kernel<B_K, EPI, SA, SB, PRE><<<grid, threads, tg::SMEM, s>>>(am, bm, cm, alom, blom,
+                                                                         p);
     GPTQ_LAUNCHED();
     return GPTQ_OK;
 }

@@ -68,6 +68,8 @@ _SIGNATURES = {
     "rtn_quantize_ex": ([_P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P], _I),
     "rtn_clip_search": ([_P, _I, _I, _I, _I, _I, _I, _P, ctypes.c_double, ctypes.c_double, _P,
                          _P, _P, _P, _P], _I),
+    "rtn_range_clip": ([_P, _I, _I, _I, _I, _I, _I, ctypes.c_double, ctypes.c_double, _P, _P,
+                        _P, _P], _I),
     "w4a16_pack": ([_P, _I, _I, _P, _P, _P], _I),
     "w4a16_linear_workspace": ([_I64, _I, _I], _SZ),
     "w4a16_linear": ([_P, _I64, _I, _P, _P, _P, _I, _I, _P, _P, _P, _P, _SZ, _P, _P], _I),
@@ -352,6 +354,25 @@ def rtn_clip_search(W: torch.Tensor, bits: int = 4, group_size: int = 128,
                                ridx.data_ptr(), _stream())
     _check(st, "rtn_clip_search")
     return packed, scales, zeros, ridx
+
+
+def rtn_range_clip(W: torch.Tensor, bits: int = 4, group_size: int = 128,
+                   percentile: float = 99.99, abs_range: float = 0.0, sym: bool = False):
+    """Group RTN of the weights clipped to each group's (100 - percentile)/percentile
+    quantiles, limited to [-abs_range, abs_range] when abs_range > 0 ->
+    (packed uint8, scales fp16, zeros fp16)."""
+    _require_cuda(W, "W")
+    d_out, d_in = W.shape
+    dev = W.device
+    ng = d_in // group_size if group_size > 0 and d_in % group_size == 0 else 1
+    packed = torch.empty(d_out, d_in // 2 if bits == 4 else d_in, dtype=torch.uint8, device=dev)
+    scales = torch.empty(d_out, ng, dtype=torch.float16, device=dev)
+    zeros = torch.empty(d_out, ng, dtype=torch.float16, device=dev)
+    st = lib().rtn_range_clip(W.data_ptr(), _dtype_code(W), d_out, d_in, bits, group_size,
+                              int(bool(sym)), float(percentile), float(abs_range),
+                              packed.data_ptr(), scales.data_ptr(), zeros.data_ptr(), _stream())
+    _check(st, "rtn_range_clip")
+    return packed, scales, zeros
 
 
 # ------------------------------------------------------------------------------------------

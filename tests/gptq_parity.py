@@ -17,8 +17,11 @@ The criterion applied here, per row, in the processing order:
 
 The window is derived, not chosen: it is the largest move of any pre-rounding value (in units
 of its group's scale) that a perturbation of H at the Hessian tolerance causes in the oracle
-itself, measured on sampled rows before their own first divergence, times a safety factor of
-2. The perturbation moves every entry of H by 1e-5 of its value with a random sign (so its
+itself, measured before each row's own first divergence, times a safety factor of 2. The rows
+it is measured on are a random sample plus every row in which the two results differ, i.e.
+every row the criterion is applied to: a maximum taken over a small random sample alone
+misses the tail of the rows' sensitivities (a layer's rows differ in their outlier weights
+and in how far their compensation reaches). The perturbation moves every entry of H by 1e-5 of its value with a random sign (so its
 relative Frobenius norm is the tolerance, 1e-5). That is five times the GPU's measured error
 on the diagonal (about 2e-6, a truncation bias of the tensor cores' accumulation) and far above
 its error on the off-diagonal entries, whose fp32 partial sums have random signs; the GPU's
@@ -79,17 +82,22 @@ def _fp16_below(s):
 
 def window_from_h_sensitivity(W, H, bits, g, B, percdamp, act_order, ref_trace, rows,
                               U_pert=None, H_pert=None, route="textbook", rel=1e-5,
-                              safety=2.0, **variant):
+                              safety=2.0, cache=None, **variant):
     """The tie window eps (see the module docstring), from the oracle run on H and on a
-    perturbed H over the sampled ``rows``. ``ref_trace`` is the oracle's traced result for
-    those rows on H; ``variant`` are the quantizer switches of ``gptq_blocked_ref``.
-    Returns (eps, detail)."""
+    perturbed H over the ``rows``. ``ref_trace`` is the oracle's traced result for those rows
+    on H; ``variant`` are the quantizer switches of ``gptq_blocked_ref``. ``cache`` (a dict),
+    if given, keeps the perturbed H and its factor for a later call. Returns (eps, detail)."""
+    if cache is not None:
+        H_pert = cache.get("H_pert", H_pert)
+        U_pert = cache.get("U_pert", U_pert)
     if U_pert is None:
         if H_pert is None:
             H_pert = perturbed_hessian(H, rel)
         _, U_pert = ogptq.prepare_u(H_pert, percdamp, act_order, route=route)
     if H_pert is None:
         H_pert = perturbed_hessian(H, rel)
+    if cache is not None:
+        cache["H_pert"], cache["U_pert"] = H_pert, U_pert
     alt = ogptq.gptq_blocked_ref(W, H_pert, bits, g, B, percdamp, act_order, rows=rows,
                                  U=U_pert, trace=True, **variant)
     first, _ = first_divergence(ref_trace["codes_p"], alt["codes_p"], ref_trace["scales"],

@@ -59,22 +59,42 @@ def rel_fro_blocked(Hg, Href, block=4096):
     return float(np.sqrt(num / den))
 
 
+MAX_WINDOW_ROWS = 1024   # bound on the rows the window is measured on (oracle time)
+
+
+def _window(ref, local_rows):
+    """The tie window measured on the given rows of the oracle's traced result ``ref`` (indices
+    into its rows), with the context ``oracle_ref`` stored in it."""
+    ctx = ref["_window"]
+    local_rows = np.asarray(local_rows, dtype=np.int64)
+    sub = {k: ref[k][local_rows] for k in ("pre", "codes_p", "scales", "zeros", "step", "zquot")}
+    sub["perm"] = ref["perm"]
+    wrows = local_rows if ctx["rows"] is None else np.asarray(ctx["rows"])[local_rows]
+    return window_from_h_sensitivity(ctx["W"], ctx["H"], ctx["bits"], ctx["g"], ctx["B"],
+                                     ctx["percdamp"], ctx["act_order"], sub, wrows,
+                                     route=ctx["route"], cache=ctx["cache"], **ctx["variant"])
+
+
 def oracle_ref(Wn, Href, bits, g, B, act_order, percdamp=0.01, rows=None, U=None,
                route="textbook", n_window_rows=64, U_pert=None, H_pert=None, **variant):
-    """The oracle's traced result, and the tie window derived from its sensitivity to H.
-    ``variant``: the quantizer switches (sym, static_groups) of gptq_blocked_ref."""
+    """The oracle's traced result, and the tie window derived from its sensitivity to H on a
+    random sample of rows (``check_near_ties`` measures it again with every differing row
+    added). ``variant``: the quantizer switches (sym, static_groups) of gptq_blocked_ref."""
     if U is None:
         _, U = ogptq.prepare_u(Href, percdamp, act_order, route=route)
     ref = ogptq.gptq_blocked_ref(Wn, Href, bits, g, B, percdamp, act_order, rows=rows, U=U,
                                  trace=True, **variant)
     n = ref["codes"].shape[0]
     sel = np.sort(np.random.default_rng(1).choice(n, min(n_window_rows, n), replace=False))
-    sub = {k: ref[k][sel] for k in ("pre", "codes_p", "scales", "zeros", "step", "zquot")}
-    sub["perm"] = ref["perm"]
-    wrows = sel if rows is None else np.asarray(rows)[sel]
-    eps, detail = window_from_h_sensitivity(Wn, Href, bits, g, B, percdamp, act_order, sub,
-                                            wrows, U_pert=U_pert, H_pert=H_pert, route=route,
-                                            **variant)
+    cache = {}
+    if H_pert is not None:
+        cache["H_pert"] = H_pert
+    if U_pert is not None:
+        cache["U_pert"] = U_pert
+    ref["_window"] = dict(W=Wn, H=Href, bits=bits, g=g, B=B, percdamp=percdamp,
+                          act_order=act_order, rows=rows, route=route, variant=variant,
+                          cache=cache, sample=sel)
+    eps, detail = _window(ref, sel)
     return ref, eps, detail
 
 
@@ -91,6 +111,17 @@ def gpu_what(codes, scales, zeros, g_idx):
 def check_near_ties(out, ref, g, bits, eps, detail, rows=None, static_groups=False):
     codes, sc, zr, perm = gpu_outputs(out, rows)
     assert np.array_equal(perm, ref["perm"])
+    if "_window" in ref:
+        # measure the window again on the random sample plus every row that differs
+        differ = np.flatnonzero(
+            np.any(codes != ref["codes"], axis=1) | np.any(sc != ref["scales"], axis=1) |
+            np.any(zr != ref["zeros"], axis=1))
+        extra = np.setdiff1d(differ, ref["_window"]["sample"])
+        if extra.size:
+            wr = np.union1d(ref["_window"]["sample"], extra)[:MAX_WINDOW_ROWS]
+            eps2, detail2 = _window(ref, wr)
+            detail = dict(detail2, sample_eps=eps, sample_rows=detail["rows"])
+            eps = max(eps, eps2)
     rep = near_tie_report(codes, sc, zr, perm, ref, g, bits, eps, rows=rows,
                           static_groups=static_groups)
     log_parity(window=detail, **rep)

@@ -124,3 +124,40 @@ def test_clip_search_matches_oracle(cuda_lib, with_h, bits, g, sym):
     cm = np.repeat(same, g, axis=1)
     assert np.array_equal(codes[cm], c_ref[cm])
     assert np.any(best > 0)                  # some groups really are clipped
+
+
+@pytest.mark.parametrize("dtype", [torch.float16, torch.float32])
+@pytest.mark.parametrize("bits,g,percentile,abs_range,sym", [
+    (4, 128, 99.99, 0.0, False), (4, 128, 99.0, 0.0, True), (3, 64, 95.0, 0.0, False),
+    (4, 32, 100.0, 0.03, False), (2, 16, 90.0, 0.05, True), (8, 128, 99.9, 0.0, False),
+    (4, 16, 50.0, 0.0, False), (4, 64, 100.0, 0.0, False)])
+def test_range_clip_bit_exact(cuda_lib, dtype, bits, g, percentile, abs_range, sym):
+    """Percentile / fixed-range clipping: codes, scales and zeros equal the oracle's bit for
+    bit (ragged row count, outlier columns, ties of equal values inside a group)."""
+    W = _w(333, 1024, seed=int(percentile * 10) + g + bits, dtype=dtype)
+    W[5, :g] = W[5, 0]                        # a constant group: every rank is a tie
+    W[7, g:2 * g] = torch.round(W[7, g:2 * g] * 50) / 50   # many equal values
+    packed, scales, zeros = cuda_lib.rtn_range_clip(W, bits, g, percentile, abs_range, sym)
+    torch.cuda.synchronize()
+    c_ref, s_ref, z_ref, _, _ = ortn.rtn_range_clip(W.float().cpu().numpy().astype(np.float64),
+                                                    bits, g, percentile, abs_range, sym)
+    assert np.array_equal(_unpack(packed, bits), c_ref)
+    assert np.array_equal(scales.float().cpu().numpy().astype(np.float64), s_ref)
+    assert np.array_equal(zeros.float().cpu().numpy().astype(np.float64), z_ref)
+
+
+def test_range_clip_full_size_and_no_clip_is_rtn(cuda_lib):
+    """The timed layer's W (11008 x 4096 fp16) at the page's 99.99 %: bit-exact; and with
+    nothing clipped the result is the plain RTN kernel's."""
+    wl = workloads.WORKLOADS["mlp_up_7b"]
+    W = workloads.make_weights(wl, device="cuda")
+    packed, scales, zeros = cuda_lib.rtn_range_clip(W, 4, 128, 99.99)
+    p2, s2, z2 = cuda_lib.rtn_range_clip(W, 4, 128, 100.0)
+    p3, s3, z3 = cuda_lib.rtn_minmax_quantize(W, 4, 128)
+    torch.cuda.synchronize()
+    c_ref, s_ref, z_ref, _, _ = ortn.rtn_range_clip(W.float().cpu().numpy().astype(np.float64),
+                                                    4, 128, 99.99)
+    assert np.array_equal(_unpack(packed, 4), c_ref)
+    assert np.array_equal(scales.float().cpu().numpy().astype(np.float64), s_ref)
+    assert np.array_equal(zeros.float().cpu().numpy().astype(np.float64), z_ref)
+    assert torch.equal(p2, p3) and torch.equal(s2, s3) and torch.equal(z2, z3)
