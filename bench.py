@@ -566,6 +566,17 @@ def stack_measure(gptq, device, peaks, clock_mhz, n_layers=32, n_tokens=131072,
     res = {}
     gptq.profile_enable(True)
     try:
+        # one untimed layer per setting first: module loading and one-time kernel set-up
+        inputs, fused = workloads.make_decoder_layer(n_layers, n_tokens, device=device)
+        for k, X in inputs.items():
+            hs[k].reset()
+            hs[k].accumulate(X)
+        for g, ao in variants:
+            for name, W, src in fused:
+                gptq.quantize_layer(W, hs[src].raw(), bits=4, group_size=g, block_size=128,
+                                    act_order=ao, compute_loss=True, workspace=ws)
+        del inputs, fused
+        torch.cuda.synchronize()
         for g, ao in variants:
             outs = {name: dict(codes=torch.empty(r, d, dtype=torch.uint8, device=device),
                                scales=torch.empty(r, d // g, dtype=torch.float16, device=device),
@@ -964,6 +975,13 @@ def run_ncu_case(name: str):
         Y = torch.empty(16384, 22016, dtype=torch.float16, device="cuda")
         for _ in range(3):
             gptq.w4a16_linear(X, packed, scales, zeros, 128, out=Y)
+    elif name == "factor":                       # d = 11008 (mlp_down_7b's H), 2 calls
+        wd = workloads.WORKLOADS["mlp_down_7b"]
+        X = workloads.make_activations(wd.replace(n_tokens=4096), device="cuda")
+        h = gptq.Hessian(wd.d_in)
+        h.accumulate(X)
+        for _ in range(2):
+            gptq.inverse_factor(h.raw(), act_order=True)
     elif name == "rtn_big":                      # 4 layers of 7B weights: 153600 x 4096 fp16
         W = workloads.make_weights(wl.replace(d_out=4 * (4 * 4096 + 2 * 11008)), device="cuda")
         for _ in range(3):                       # (1.26 GB, ten times L2)
@@ -990,7 +1008,7 @@ def main(argv=None):
     ap.add_argument("--no-stack", action="store_true",
                     help="skip GPTQ over a full 7B decoder stack (4 variants)")
     ap.add_argument("--stack-layers", type=int, default=32)
-    ap.add_argument("--ncu-case", choices=("hessian", "gptq", "rtn", "rtn_big", "w4a16"),
+    ap.add_argument("--ncu-case", choices=("hessian", "gptq", "rtn", "rtn_big", "w4a16", "factor"),
                     help="run one small case for an ncu capture and exit (no JSON line)")
     args = ap.parse_args(argv)
     if args.ncu_case:

@@ -189,7 +189,7 @@ gptq_status gptq_quantize_layer_ex(const void* W, int w_dtype, int d_out, int d_
  * that reserves its memory pools at start-up should make one call before reserving them.
  *   - Layers whose gptq_quantize_layer_workspace(d_out, d_in, block_size) exceeds 32 MiB are
  *     rejected with GPTQ_ERR_WORKSPACE before anything is launched. For example, d_in = 1024
- *     fits up to d_out = 1811 and d_in = 512 up to d_out = 2876; d_in = 4096 does not fit.
+ *     fits up to d_out = 1653 and d_in = 512 up to d_out = 2779; d_in = 4096 does not fit.
  *   - No cudaMalloc, cudaFree or other allocating call is made.
  *   - The first call on each device looks up the array's device address (cudaGetSymbolAddress
  *     with that device current). Make that first call before any stream capture on the device.

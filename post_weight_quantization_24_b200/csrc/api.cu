@@ -139,6 +139,7 @@ struct Workspace {
     uint8_t* codes_p;// d_out x d_in codes in processing order
     float* P;        // d x 128: the column loop's images of U's diagonal blocks
     float* Dinv;     // ceil(d/128) x 128 x 128 inverses of the Cholesky diagonal blocks
+    float* F;        // 4 x d x 128: the factorisation's split panels (two L21 lo, X_top hi, lo)
     int* perm;
     int* invperm;
     size_t bytes;
@@ -165,6 +166,7 @@ static Workspace layout(void* base, int d_out, int d_in) {
     w.codes_p = take(static_cast<size_t>(d_out) * d);
     w.P = reinterpret_cast<float*>(take(d * kCholBlock * 4));
     w.Dinv = reinterpret_cast<float*>(take(nbl * kCholBlock * kCholBlock * 4));
+    w.F = reinterpret_cast<float*>(take(4 * d * kCholBlock * 4));
     w.perm = reinterpret_cast<int*>(take(d * 4));
     w.invperm = reinterpret_cast<int*>(take(d * 4));
     w.bytes = off;
@@ -345,7 +347,7 @@ gptq_status gptq_quantize_layer_ex(const void* W, int w_dtype, int d_out, int d_
     tm.end();
     // ---- stage 1: U with U^T U = H_d^-1 (factor and inverse overlap on two streams) ----
     tm.begin(1);
-    GPTQ_TRY(factor_inverse_launch(ws.A, d_in, ws.Dinv, ws.X, status, s));
+    GPTQ_TRY(factor_inverse_launch(ws.A, d_in, ws.Dinv, ws.X, ws.F, status, s));
     tm.end();
     // ---- stage 2: the forms of U that the column loop and the lazy updates read ----
     uint8_t* codes_p = act_order ? ws.codes_p : codes;
@@ -367,8 +369,11 @@ gptq_status gptq_quantize_layer_ex(const void* W, int w_dtype, int d_out, int d_
     // waits for that rest before it next writes those columns; the errors alternate between
     // two buffers so the rest can read S's errors while S+1 records its own.
     const int super = block_size * std::max(1, kSuperCols / block_size);
+    constexpr int kMinSideCtas = 64;
     const int side_ctas = num_sms() - gptq_rows_ctas(d_out);
-    const bool overlap = side_ctas >= 16 && d_in > 2 * super;
+    // (the 3xTF32 GEMM needs most of the GPU to pay: with fewer free SMs than this the far
+    // update on the side would outlast the column loop it hides behind)
+    const bool overlap = side_ctas >= kMinSideCtas && d_in > 2 * super;
     // while the overlap runs, the caller's stream keeps its GEMMs on the SMs the second stream
     // leaves free, so that every CTA of a persistent launch is resident at once
     const int main_ctas = overlap ? num_sms() - side_ctas : 0;
@@ -471,7 +476,7 @@ gptq_status gptq_inverse_factor(const float* H, int d_in, float percdamp, int ac
     GPTQ_TRY(diag_stats_launch(H, d_in, static_cast<double>(percdamp), ws.st, s));
     GPTQ_TRY(act_order_launch(H, d_in, act_order, ws.perm, ws.invperm, s));
     GPTQ_TRY(gather_h_launch(H, d_in, ws.perm, ws.st, 1, ws.A, status, s));
-    GPTQ_TRY(factor_inverse_launch(ws.A, d_in, ws.Dinv, ws.X, status, s));
+    GPTQ_TRY(factor_inverse_launch(ws.A, d_in, ws.Dinv, ws.X, ws.F, status, s));
     GPTQ_CUDA_TRY(cudaMemcpyAsync(U, ws.X, static_cast<size_t>(d_in) * d_in * 4,
                                   cudaMemcpyDeviceToDevice, s));
     if (perm)

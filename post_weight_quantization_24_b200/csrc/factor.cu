@@ -412,6 +412,10 @@ gptq_status side_streams(SideStreams** out) {
     return GPTQ_OK;
 }
 
+#ifndef GPTQ_FACTOR_RESERVE_DIV
+#define GPTQ_FACTOR_RESERVE_DIV 16  // at most sms / this many SMs kept free for the main stream
+#endif
+
 // Blocked right-looking Cholesky of A with one step of lookahead, and the blocked triangular
 // inverse X = L^-1, then U = reverse(X).
 //
@@ -420,13 +424,19 @@ gptq_status side_streams(SideStreams** out) {
 //   trsm(m)   L21 = A21 Dinv_m^T, in place (each output tile is the input tile it reads)
 //   next(m)   the trailing update of panel m+1's columns only: A[e:, e:e+128] -= L21 L21^T
 // Side stream, after trsm(m):
+//   split(m)  L21 into tf32 hi and lo parts (Lhi, Llo: rows of 128)
 //   rest(m)   the rest of the trailing update: A[e+128:, e+128:] -= L21' L21'^T (lower tiles)
-//   inv(m)    X[k0:e, 0:e] = Dinv_m X[k0:e, 0:e] (in place), X[e:, 0:e] -= L21 X[k0:e, 0:e]
+//   inv(m)    X[k0:e, 0:e] = Dinv_m X[k0:e, 0:e] (in place), split into Thi/Tlo, then
+//             X[e:, 0:e] -= L21 X[k0:e, 0:e]
 // next(m) waits for rest(m-1), the only other writer of its columns; diag(m+1) and trsm(m+1)
-// need only next(m), so rest(m) and inv(m) overlap them. The side stream's GEMMs leave as many
-// SMs free as the main stream's kernels of the next panel have CTAs (one, or one per 128 rows
-// below it; at most half the GPU), so the chain of diagonal blocks does not wait for an SM.
-gptq_status factor_inverse_launch(float* A, int d, float* Dinv, float* X, int* status,
+// need only next(m), so the side stream's work overlaps them. The side stream's GEMMs (the
+// bulk of the flops) take operands split once per panel and run without converter warps;
+// the main stream's chain stays as short as it can be.
+// The side stream gets most of the GPU: its GEMMs leave as many SMs free as the main stream's
+// kernels of the next panel have CTAs, but at most a sixteenth of the GPU (measured: 13.5
+// against 17.1 ms at d = 11008 and 174 against 270 ms at d = 28672 when half the GPU was kept
+// free; no change at d = 4096).
+gptq_status factor_inverse_launch(float* A, int d, float* Dinv, float* X, float* F, int* status,
                                   cudaStream_t s) {
     const int nb = kCholBlock;
     static_assert(kCholBlock == pd::NB, "diagonal-block kernel is written for 128-wide panels");
@@ -441,6 +451,11 @@ gptq_status factor_inverse_launch(float* A, int d, float* Dinv, float* X, int* s
     GPTQ_TRY(side_streams(&ss));
     cudaStream_t t2 = ss->side;
     const int sms = num_sms();
+    // F: L21's hi and lo parts (d x 128 each, indexed by row), then T hi and lo (128 x d each)
+    float* Lhi = F;
+    float* Llo = F + static_cast<int64_t>(d) * nb;
+    float* Thi = F + 2 * static_cast<int64_t>(d) * nb;
+    float* Tlo = Thi + static_cast<int64_t>(d) * nb;
 
     GPTQ_CUDA_TRY(cudaEventRecord(ss->fork, s));
     GPTQ_CUDA_TRY(cudaStreamWaitEvent(t2, ss->fork, 0));
@@ -455,9 +470,12 @@ gptq_status factor_inverse_launch(float* A, int d, float* Dinv, float* X, int* s
             const int k0 = m * nb, nbc = std::min(nb, d - k0), e = k0 + nbc, rem = d - e;
             float* Dm = Dinv + static_cast<int64_t>(m) * nb * nb;
             float* A21 = A + static_cast<int64_t>(e) * d + k0;
+            float* L21hi = Lhi + static_cast<int64_t>(e) * nb;
+            float* L21lo = Llo + static_cast<int64_t>(e) * nb;
             // SMs kept free for the main stream while this panel's side work runs: diag(m+1)
             // takes one, trsm(m+1) and next(m+1) one per 128 rows below panel m+1
-            const int reserve = std::min(sms / 2, std::max(1, (rem + nb - 1) / nb));
+            const int reserve =
+                std::min(sms / GPTQ_FACTOR_RESERVE_DIV, std::max(1, (rem + nb - 1) / nb));
             const int side_ctas = std::max(1, sms - reserve);
             potrf_diag_kernel<<<1, pd::THREADS, smem, s>>>(A, d, k0, nbc, Dm, status);
             GPTQ_LAUNCHED();
@@ -477,14 +495,18 @@ gptq_status factor_inverse_launch(float* A, int d, float* Dinv, float* X, int* s
                 u.lower_only = 1; u.status = status;
                 GPTQ_TRY(tcgemm_launch(u, true, TC_EPI_STORE, true, true, s));
                 GPTQ_CUDA_TRY(cudaStreamWaitEvent(t2, ss->trsm, 0));
+                // (the previous panel's readers of Lhi/Llo ran earlier on this stream)
+                GPTQ_TRY(tcgemm_split_launch(A21, L21hi, L21lo, rem, nbc, d, false, t2, nb, nb));
                 if (rem > nb) {
-                    const float* A21r = A21 + static_cast<int64_t>(nb) * d;
+                    const float* Lrhi = L21hi + static_cast<int64_t>(nb) * nb;
+                    const float* Lrlo = L21lo + static_cast<int64_t>(nb) * nb;
                     TcGemmArgs r{};  // A[e+128:, e+128:] -= A21' A21'^T (lower tiles)
                     r.M = rem - nb; r.N = rem - nb; r.K = nbc; r.alpha = -1.f; r.beta = 1.f;
-                    r.A = A21r; r.lda = d; r.B = A21r; r.ldb = d;
+                    r.A = Lrhi; r.lda = nb; r.A_lo = Lrlo;
+                    r.B = Lrhi; r.ldb = nb; r.B_lo = Lrlo;
                     r.C = A + static_cast<int64_t>(e + nb) * d + (e + nb); r.ldc = d;
                     r.lower_only = 1; r.status = status; r.max_ctas = side_ctas;
-                    GPTQ_TRY(tcgemm_launch(r, true, TC_EPI_STORE, true, true, t2));
+                    GPTQ_TRY(tcgemm_presplit_launch(r, t2, true));
                 }
                 GPTQ_CUDA_TRY(cudaEventRecord(ss->rest, t2));
             } else {
@@ -498,12 +520,14 @@ gptq_status factor_inverse_launch(float* A, int d, float* Dinv, float* X, int* s
             v.status = status; v.max_ctas = side_ctas;
             GPTQ_TRY(tcgemm_launch(v, false, TC_EPI_STORE, true, true, t2));
             if (rem > 0) {
+                GPTQ_TRY(tcgemm_split_launch(Xk, Thi, Tlo, nbc, e, d, false, t2));
                 TcGemmArgs w{};  // X[e:, 0:e] -= L21 * X[k0:e, 0:e]
                 w.M = rem; w.N = e; w.K = nbc; w.alpha = -1.f; w.beta = 1.f;
-                w.A = A21; w.lda = d; w.B = Xk; w.ldb = d;
+                w.A = L21hi; w.lda = nb; w.A_lo = L21lo;
+                w.B = Thi; w.ldb = d; w.B_lo = Tlo;
                 w.C = X + static_cast<int64_t>(e) * d; w.ldc = d;
                 w.status = status; w.max_ctas = side_ctas;
-                GPTQ_TRY(tcgemm_launch(w, false, TC_EPI_STORE, true, true, t2));
+                GPTQ_TRY(tcgemm_presplit_launch(w, t2, false));
             }
         }
         const int64_t half = static_cast<int64_t>(d) * d / 2;

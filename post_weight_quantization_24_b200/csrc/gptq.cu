@@ -37,7 +37,10 @@ namespace gr {
 constexpr int MAXB = 128;                    // widest block handled in one launch
 constexpr int PH = 16;                       // block columns per window phase
 constexpr int NPH = MAXB / PH;
-constexpr int WARPS = 4;
+#ifndef GPTQ_ROWS_WARPS
+#define GPTQ_ROWS_WARPS 2
+#endif
+constexpr int WARPS = GPTQ_ROWS_WARPS;       // rows (warps of 32) per CTA
 constexpr int THREADS = WARPS * 32;          // one row per thread
 constexpr int SMEM = MAXB * MAXB * 4 + MAXB * 4 + NPH * 8 + MAXB * 4;   // + grid indices
 }  // namespace gr
@@ -171,7 +174,7 @@ __device__ __forceinline__ bool rows_phases(float (&w)[gr::MAXB], RowCtx& x, uin
     return true;
 }
 
-__global__ void __launch_bounds__(gr::THREADS, 2) gptq_rows_kernel(
+__global__ void __launch_bounds__(gr::THREADS, gr::WARPS <= 2 ? 3 : 2) gptq_rows_kernel(
     const float* __restrict__ Wk, int d_out, int d_in, int j0, int bw,
     const float* __restrict__ img, const float* __restrict__ rdiag, int g, int bits, int sym,
     const int* __restrict__ preset_perm, uint8_t* __restrict__ codes_p,

@@ -55,8 +55,9 @@ gptq_status gather_w_launch(const void* W, int w_dtype, int d_out, int d_in, con
                             float* Wk, int* status, cudaStream_t s);
 // In-place lower Cholesky factor L of A (lda = d), the inverses of its diagonal blocks in Dinv
 // (ceil(d/nb) blocks of nb x nb, row-major, zero above the diagonal), and U = reverse(L^-1) in
-// X. Uses a second stream of its own, forked from and joined back to s.
-gptq_status factor_inverse_launch(float* A, int d, float* Dinv, float* X, int* status,
+// X. F is scratch of 4 x d x 128 floats (the tf32 hi/lo parts of one panel of L and of one
+// panel of rows of L^-1). Uses a second stream of its own, forked from and joined back to s.
+gptq_status factor_inverse_launch(float* A, int d, float* Dinv, float* X, float* F, int* status,
                                   cudaStream_t s);
 // Test switch: the diagonal-block kernel waits on a barrier nothing arrives at (bounded).
 gptq_status factor_stall_set(int on);

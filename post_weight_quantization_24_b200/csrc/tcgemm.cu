@@ -434,20 +434,27 @@ static gptq_status check_args(const TcGemmArgs& a, int epi) {
     return GPTQ_OK;
 }
 
-static gptq_status encode_a(CUtensorMap* m, const float* A, const TcGemmArgs& a) {
+static gptq_status encode_a(CUtensorMap* m, const float* A, const TcGemmArgs& a, int lda) {
     return encode_tensor_map_2d(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, const_cast<float*>(A), a.K,
-                                a.M, static_cast<uint64_t>(a.lda) * 4, 32, 128,
+                                a.M, static_cast<uint64_t>(lda) * 4, 32, 128,
                                 CU_TENSOR_MAP_SWIZZLE_128B);
 }
+static gptq_status encode_a(CUtensorMap* m, const float* A, const TcGemmArgs& a) {
+    return encode_a(m, A, a, a.lda);
+}
 
-static gptq_status encode_b(CUtensorMap* m, const float* B, const TcGemmArgs& a, bool b_kmajor) {
+static gptq_status encode_b(CUtensorMap* m, const float* B, const TcGemmArgs& a, bool b_kmajor,
+                            int ldb) {
     if (b_kmajor)
         return encode_tensor_map_2d(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, const_cast<float*>(B),
-                                    a.K, a.N, static_cast<uint64_t>(a.ldb) * 4, 32, 128,
+                                    a.K, a.N, static_cast<uint64_t>(ldb) * 4, 32, 128,
                                     CU_TENSOR_MAP_SWIZZLE_128B);
     return encode_tensor_map_2d(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, const_cast<float*>(B), a.N,
-                                a.K, static_cast<uint64_t>(a.ldb) * 4, 32, 32,
+                                a.K, static_cast<uint64_t>(ldb) * 4, 32, 32,
                                 CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B);
+}
+static gptq_status encode_b(CUtensorMap* m, const float* B, const TcGemmArgs& a, bool b_kmajor) {
+    return encode_b(m, B, a, b_kmajor, a.ldb);
 }
 
 static gptq_status encode_c(CUtensorMap* m, const TcGemmArgs& a) {
@@ -494,27 +501,34 @@ gptq_status tcgemm_launch(const TcGemmArgs& a, bool b_kmajor, int epi, bool spli
                : launch_split<false, TC_EPI_DOT>(am, bm, cm, p, grid, split_a, split_b, s);
 }
 
-gptq_status tcgemm_presplit_launch(const TcGemmArgs& a, cudaStream_t s) {
+gptq_status tcgemm_presplit_launch(const TcGemmArgs& a, cudaStream_t s, bool b_kmajor) {
     if (a.M <= 0 || a.N <= 0 || a.K <= 0) return GPTQ_OK;
     GPTQ_TRY(check_args(a, TC_EPI_STORE));
+    const int lda_lo = a.lda_lo > 0 ? a.lda_lo : a.lda;
+    const int ldb_lo = a.ldb_lo > 0 ? a.ldb_lo : a.ldb;
     if (!a.A_lo || !a.B_lo || (reinterpret_cast<uintptr_t>(a.A_lo) & 15) ||
-        (reinterpret_cast<uintptr_t>(a.B_lo) & 15))
+        (reinterpret_cast<uintptr_t>(a.B_lo) & 15) || lda_lo % 4 || ldb_lo % 4)
         return GPTQ_ERR_ARG;
     CUtensorMap am, bm, cm, alom, blom;
     GPTQ_TRY(encode_a(&am, a.A, a));
-    GPTQ_TRY(encode_a(&alom, a.A_lo, a));
-    GPTQ_TRY(encode_b(&bm, a.B, a, false));
-    GPTQ_TRY(encode_b(&blom, a.B_lo, a, false));
+    GPTQ_TRY(encode_a(&alom, a.A_lo, a, lda_lo));
+    GPTQ_TRY(encode_b(&bm, a.B, a, b_kmajor));
+    GPTQ_TRY(encode_b(&blom, a.B_lo, a, b_kmajor, ldb_lo));
     GPTQ_TRY(encode_c(&cm, a));
     int grid;
     const TcParams p = make_params(a, grid);
+    if (b_kmajor)
+        return launch_variant<true, TC_EPI_STORE, true, true, true>(am, bm, cm, alom, blom, p,
+                                                                    grid, s);
     return launch_variant<false, TC_EPI_STORE, true, true, true>(am, bm, cm, alom, blom, p, grid, s);
 }
 
 __global__ void tf32_split_kernel(const float* src, float* hi, float* __restrict__ lo, int rows,
-                                  int cols, int ld, int upper) {
+                                  int cols, int ld, int ld_hi, int ld_lo, int upper) {
     for (int r = blockIdx.x; r < rows; r += gridDim.x) {
         const int64_t row = static_cast<int64_t>(r) * ld;
+        const int64_t row_hi = static_cast<int64_t>(r) * ld_hi;
+        const int64_t row_lo = static_cast<int64_t>(r) * ld_lo;
         for (int c = (upper ? (r & ~3) : 0) + 4 * static_cast<int>(threadIdx.x); c < cols;
              c += 4 * blockDim.x) {
             const float4 x = *reinterpret_cast<const float4*>(src + row + c);
@@ -523,18 +537,22 @@ __global__ void tf32_split_kernel(const float* src, float* hi, float* __restrict
             h.y = tf32_rna(x.y); l.y = tf32_rna(x.y - h.y);
             h.z = tf32_rna(x.z); l.z = tf32_rna(x.z - h.z);
             h.w = tf32_rna(x.w); l.w = tf32_rna(x.w - h.w);
-            *reinterpret_cast<float4*>(hi + row + c) = h;
-            *reinterpret_cast<float4*>(lo + row + c) = l;
+            *reinterpret_cast<float4*>(hi + row_hi + c) = h;
+            *reinterpret_cast<float4*>(lo + row_lo + c) = l;
         }
     }
 }
 
 gptq_status tcgemm_split_launch(const float* src, float* hi, float* lo, int rows, int cols, int ld,
-                                bool upper, cudaStream_t s) {
+                                bool upper, cudaStream_t s, int ld_hi, int ld_lo) {
     if (rows <= 0 || cols <= 0) return GPTQ_OK;
-    if (cols % 4 || ld % 4) return GPTQ_ERR_ARG;
+    if (ld_hi <= 0) ld_hi = ld;
+    if (ld_lo <= 0) ld_lo = ld;
+    if (cols % 4 || ld % 4 || ld_hi % 4 || ld_lo % 4 || (upper && (ld_lo != ld || ld_hi != ld)))
+        return GPTQ_ERR_ARG;
     const int blocks = std::min(rows, num_sms() * 8);
-    tf32_split_kernel<<<blocks, 256, 0, s>>>(src, hi, lo, rows, cols, ld, upper ? 1 : 0);
+    tf32_split_kernel<<<blocks, 256, 0, s>>>(src, hi, lo, rows, cols, ld, ld_hi, ld_lo,
+                                             upper ? 1 : 0);
     GPTQ_LAUNCHED();
     return GPTQ_OK;
 }

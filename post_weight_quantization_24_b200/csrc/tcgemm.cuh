@@ -31,9 +31,11 @@ struct TcGemmArgs {
     int lower_only;   // skip output tiles entirely above the diagonal
     const int* status;  // optional: skip all work when *status != 0; receives TIMEOUT
     // Pre-split operands (tcgemm_presplit_launch): A and B hold the tf32 hi parts, A_lo and
-    // B_lo the lo parts, with the layouts and strides of A and B.
+    // B_lo the lo parts, with the layouts of A and B and the strides lda_lo, ldb_lo (0: lda,
+    // ldb).
     const float* A_lo;
     const float* B_lo;
+    int lda_lo, ldb_lo;
     int max_ctas;     // > 0: launch at most this many CTAs (leaves SMs to concurrent work)
 };
 
@@ -44,13 +46,15 @@ gptq_status tcgemm_launch(const TcGemmArgs& a, bool b_kmajor, int epi, bool spli
                           cudaStream_t s);
 
 // C = alpha*A*B + beta*C (store epilogue) with both operands already split into tf32 hi and lo
-// (hi = tf32_rna(x), lo = tf32_rna(x - hi), as tcgemm_split_launch writes them); B MN-major.
-// Operands reused by many tiles are split once instead of in every tile.
-gptq_status tcgemm_presplit_launch(const TcGemmArgs& a, cudaStream_t s);
+// (hi = tf32_rna(x), lo = tf32_rna(x - hi), as tcgemm_split_launch writes them); B MN-major,
+// or K-major with b_kmajor. Operands reused by many tiles are split once instead of in every
+// tile, and the kernel runs without converter warps.
+gptq_status tcgemm_presplit_launch(const TcGemmArgs& a, cudaStream_t s, bool b_kmajor = false);
 
 // hi[i][j] = tf32_rna(x), lo[i][j] = tf32_rna(x - hi) for x = src[i][j], j0(i) <= j < cols,
-// j0(i) = upper ? i & ~3 : 0 (rows of stride ld; hi may alias src)
+// j0(i) = upper ? i & ~3 : 0 (src rows of stride ld, hi and lo rows of strides ld_hi, ld_lo;
+// 0 means ld; hi may alias src)
 gptq_status tcgemm_split_launch(const float* src, float* hi, float* lo, int rows, int cols, int ld,
-                                bool upper, cudaStream_t s);
+                                bool upper, cudaStream_t s, int ld_hi = 0, int ld_lo = 0);
 
 }  // namespace gq

@@ -91,7 +91,7 @@ def test_workspace_sizes(L):
         nbl = (d_in + 127) // 128
         expect = (r256(40) + 2 * r256(d_in * d_in * 4) + r256(d_out * d_in * 4)
                   + 4 * r256(d_out * 512 * 4) + r256(d_out * d_in) + r256(d_in * 128 * 4)
-                  + r256(nbl * 128 * 128 * 4) + 2 * r256(d_in * 4))
+                  + r256(nbl * 128 * 128 * 4) + r256(4 * d_in * 128 * 4) + 2 * r256(d_in * 4))
         assert L.gptq_quantize_layer_workspace(d_out, d_in, 128) == expect
     assert L.gptq_quantize_layer_workspace(0, 512, 128) == 0
 
