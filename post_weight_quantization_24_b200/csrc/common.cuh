@@ -31,6 +31,30 @@
 
 namespace gq {
 
+// Programmatic dependent launch. A kernel launched with launch_pdl may be scheduled as soon as
+// every CTA of the previous kernel in its stream has exited, before that kernel's completion
+// and memory flush are processed; pdl_wait() (the first statement of such a kernel) holds its
+// threads until the previous kernel has completed and its writes are visible. Without the
+// launch attribute pdl_wait() returns at once. This hides the launch latency between the short
+// kernels of the factorisation's and the column loop's chains.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t s, Args... args) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // ~2 s at the B200's highest SM clock: every spin on an mbarrier gives up after this many
 // cycles and records GPTQ_ERR_TIMEOUT instead of hanging the device.
 constexpr long long kWaitLimitCycles = 4000000000LL;

@@ -290,6 +290,7 @@ __global__ void __launch_bounds__(pd::THREADS, 1) potrf_diag_kernel(float* __res
                                                                    int k0, int nbc,
                                                                    float* __restrict__ Dinv,
                                                                    int* status) {
+    pdl_wait();
     if (status_bad(status)) return;
     extern __shared__ __align__(16) float sm[];
     float* Lsh = sm;                          // [NB][LS]
@@ -477,7 +478,8 @@ gptq_status factor_inverse_launch(float* A, int d, float* Dinv, float* X, float*
             const int reserve =
                 std::min(sms / GPTQ_FACTOR_RESERVE_DIV, std::max(1, (rem + nb - 1) / nb));
             const int side_ctas = std::max(1, sms - reserve);
-            potrf_diag_kernel<<<1, pd::THREADS, smem, s>>>(A, d, k0, nbc, Dm, status);
+            GPTQ_CUDA_TRY(launch_pdl(potrf_diag_kernel, dim3(1), dim3(pd::THREADS), smem, s, A, d,
+                                     k0, nbc, Dm, status));
             GPTQ_LAUNCHED();
             if (rem > 0) {
                 TcGemmArgs t{};  // A21 = A21 * Dinv_m^T

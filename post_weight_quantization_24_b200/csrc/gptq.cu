@@ -180,6 +180,7 @@ __global__ void __launch_bounds__(gr::THREADS, gr::WARPS <= 2 ? 3 : 2) gptq_rows
     const int* __restrict__ preset_perm, uint8_t* __restrict__ codes_p,
     uint16_t* __restrict__ scales, uint16_t* __restrict__ zeros, float* __restrict__ Err,
     float* __restrict__ ErrLo, int err_ld, double* err_sq, int* status) {
+    pdl_wait();
     if (status_bad(status)) return;
     extern __shared__ __align__(128) unsigned char rows_smem[];
     float* Us = reinterpret_cast<float*>(rows_smem);
@@ -262,10 +263,9 @@ gptq_status gptq_block_launch(float* Wk, int d_out, int d_in, int j0, int bw, co
         g_rows_attr_set = true;
     }
     const int grid = (d_out + gr::THREADS - 1) / gr::THREADS;
-    gptq_rows_kernel<<<grid, gr::THREADS, gr::SMEM, s>>>(Wk, d_out, d_in, j0, bw, img, rdiag,
-                                                        group_size, bits, sym, preset_perm,
-                                                        codes_p, scales, zeros, Err, ErrLo,
-                                                        err_ld, err_sq, status);
+    GPTQ_CUDA_TRY(launch_pdl(gptq_rows_kernel, dim3(grid), dim3(gr::THREADS), gr::SMEM, s, Wk,
+                             d_out, d_in, j0, bw, img, rdiag, group_size, bits, sym, preset_perm,
+                             codes_p, scales, zeros, Err, ErrLo, err_ld, err_sq, status));
     GPTQ_LAUNCHED();
     return GPTQ_OK;
 }

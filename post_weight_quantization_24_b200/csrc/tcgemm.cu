@@ -90,6 +90,7 @@ __global__ void __launch_bounds__(tg::THREADS, 1)
                   const __grid_constant__ CUtensorMap cmap,
                   const __grid_constant__ CUtensorMap alomap,
                   const __grid_constant__ CUtensorMap blomap, const TcParams p) {
+    pdl_wait();
     static_assert(!PRE || (SPLIT_A && SPLIT_B), "pre-split operands come in hi/lo pairs");
     // pre-split operands need no converter warps: the epilogue warps follow warp 1 directly
     // (warps 2..5 take TMEM lane quarters 2, 3, 0, 1, as warps 10..13 do)
@@ -405,8 +406,8 @@ static gptq_status launch_variant(const CUtensorMap& am, const CUtensorMap& bm,
         attr = true;
     }
     constexpr int threads = PRE ? 6 * 32 : tg::THREADS;
-    tcgemm_kernel<B_K, EPI, SA, SB, PRE><<<grid, threads, tg::SMEM, s>>>(am, bm, cm, alom, blom,
-                                                                         p);
+    GPTQ_CUDA_TRY(launch_pdl(tcgemm_kernel<B_K, EPI, SA, SB, PRE>, dim3(grid), dim3(threads),
+                             tg::SMEM, s, am, bm, cm, alom, blom, p));
     GPTQ_LAUNCHED();
     return GPTQ_OK;
 }
@@ -525,6 +526,7 @@ gptq_status tcgemm_presplit_launch(const TcGemmArgs& a, cudaStream_t s, bool b_k
 
 __global__ void tf32_split_kernel(const float* src, float* hi, float* __restrict__ lo, int rows,
                                   int cols, int ld, int ld_hi, int ld_lo, int upper) {
+    pdl_wait();
     for (int r = blockIdx.x; r < rows; r += gridDim.x) {
         const int64_t row = static_cast<int64_t>(r) * ld;
         const int64_t row_hi = static_cast<int64_t>(r) * ld_hi;
@@ -551,8 +553,8 @@ gptq_status tcgemm_split_launch(const float* src, float* hi, float* lo, int rows
     if (cols % 4 || ld % 4 || ld_hi % 4 || ld_lo % 4 || (upper && (ld_lo != ld || ld_hi != ld)))
         return GPTQ_ERR_ARG;
     const int blocks = std::min(rows, num_sms() * 8);
-    tf32_split_kernel<<<blocks, 256, 0, s>>>(src, hi, lo, rows, cols, ld, ld_hi, ld_lo,
-                                             upper ? 1 : 0);
+    GPTQ_CUDA_TRY(launch_pdl(tf32_split_kernel, dim3(blocks), dim3(256), 0, s, src, hi, lo, rows,
+                             cols, ld, ld_hi, ld_lo, upper ? 1 : 0));
     GPTQ_LAUNCHED();
     return GPTQ_OK;
 }

@@ -10,17 +10,22 @@
 // the same perm (gather_cols_kernel) before the GEMM. The contraction does not depend on the
 // order of its terms, so this is the g_idx formulation.
 //
-// GEMM kernel (persistent, one CTA per SM, output tiles of 128 tokens x 256 channels,
-// k-blocks of 64 input channels, 3-stage ring):
-//   warp 0      TMA producer: the X tile (128 x 64 fp16, 128-byte swizzle) and the packed
-//               codes of the tile's 256 rows (256 x 32 bytes) per k-block.
-//   warps 2-9   dequantisers: thread j expands row j's 64 codes with the row's scale and zero
-//               (fp16 arithmetic: (1024 + q) - (1024 + z) is exact, times the scale is the one
-//               rounding of the exact product) and writes them into the B tile in the 128-byte
-//               swizzled K-major layout the MMA reads, then fences and signals the stage.
-//   warp 1      TMEM allocator and MMA issuer: per k-block 4 x tcgen05.mma kind::f16
-//               M128 N256 K16 into one of two 256-column TMEM accumulators.
+// GEMM kernel (persistent, one CTA per SM, output tiles of 256 tokens x 128 channels,
+// k-blocks of 64 input channels, 4-stage ring):
+//   warp 0      TMA producer: the X tile (two 128 x 64 fp16 boxes, 128-byte swizzle) and the
+//               packed codes of the tile's 128 rows (128 x 32 bytes) per k-block.
+//   warps 2-9   dequantisers: threads 2r and 2r+1 expand row r's 64 codes (32 each) with its
+//               scale and zero (fp16 arithmetic: (1024 + q) - (1024 + z) is exact, times the
+//               scale is the one rounding of the exact product) and write them into the B tile
+//               in the 128-byte swizzled K-major layout the MMA reads, then fence and signal
+//               the stage.
+//   warp 1      TMEM allocator and MMA issuer: per k-block 2 x 4 tcgen05.mma kind::f16
+//               M128 N128 K16, one group per 128-token half of the tile, both reading the same
+//               expanded weight tile, into one of two 256-column TMEM accumulator pairs.
 //   warps 10-13 epilogue: tcgen05.ld, + R, fp16, vector stores.
+// Each expanded weight tile serves 256 tokens, so a weight is expanded n/256 times: the
+// expansion, not the tensor pipe, bounds this kernel (half as many expansions as with
+// 128-token tiles).
 // Tiles run in bands of 8 token tiles with the token tile varying fastest, so the CTAs that run
 // together share the same weight tiles and activation rows in L2. Every mbarrier wait is
 // bounded; on timeout the kernel records GPTQ_ERR_TIMEOUT, drains its copies and MMAs, frees
@@ -33,23 +38,27 @@
 namespace gq {
 
 namespace wq {
-constexpr int BM = 128, BN = 256, BK = 64, STAGES = 3;
-constexpr int A_BYTES = BM * BK * 2;                 // 16 KB
-constexpr int B_BYTES = BN * BK * 2;                 // 32 KB
-constexpr int C_BYTES = BN * BK / 2;                 // 8 KB packed codes
+constexpr int BM = 256, MS = 128, BN = 128, BK = 64, STAGES = 4;
+constexpr int A_SUB = MS * BK * 2;                   // 16 KB: one 128-token half
+constexpr int A_BYTES = BM * BK * 2;                 // 32 KB
+constexpr int B_BYTES = BN * BK * 2;                 // 16 KB
+constexpr int C_BYTES = BN * BK / 2;                 // 4 KB packed codes
 constexpr int OFF_B = A_BYTES;
 constexpr int OFF_C = A_BYTES + B_BYTES;
-constexpr int STAGE = A_BYTES + B_BYTES + C_BYTES;   // 56 KB, A and B 1024-aligned
-constexpr int DQ_WARPS = 8;
+constexpr int STAGE = A_BYTES + B_BYTES + C_BYTES;   // 52 KB, A and B 1024-aligned
+constexpr int DQ_WARPS = BN / 16;                    // two threads per weight row
 constexpr int EPI_WARP0 = 2 + DQ_WARPS;
 constexpr int THREADS = (EPI_WARP0 + 4) * 32;        // 448
 constexpr int BAR_BYTES = 256;
 constexpr int SMEM = 1024 + STAGES * STAGE + BAR_BYTES;
-constexpr uint32_t TMEM_COLS = 512;
+constexpr int ACC_COLS = (BM / MS) * BN;             // 256: one tile's two accumulators
+constexpr uint32_t TMEM_COLS = 512;                  // two tiles in flight
 constexpr int BAND = 8;
-// kind::f16: fp16 A and B, fp32 D, both operands K-major
+// kind::f16: fp16 A and B, fp32 D, both operands K-major, M128 N128
 constexpr uint32_t IDESC = (1u << 4) | (static_cast<uint32_t>(BN >> 3) << 17) |
-                           (static_cast<uint32_t>(BM >> 4) << 24);
+                           (static_cast<uint32_t>(MS >> 4) << 24);
+static_assert(2 * ACC_COLS <= static_cast<int>(TMEM_COLS), "two tiles of accumulators");
+static_assert(SMEM <= 227 * 1024, "shared memory");
 }  // namespace wq
 
 struct WqParams {
@@ -152,6 +161,7 @@ __global__ void __launch_bounds__(wq::THREADS, 1)
                     uint8_t* sa = smem + st * wq::STAGE;
                     mbar_arrive_expect_tx(&full[st], wq::A_BYTES + wq::C_BYTES);
                     tma_load_2d(sa, &xmap, &full[st], kb * wq::BK, m0);
+                    tma_load_2d(sa + wq::A_SUB, &xmap, &full[st], kb * wq::BK, m0 + wq::MS);
                     tma_load_2d(sa + wq::OFF_C, &cmap, &full[st], kb * (wq::BK / 2), n0);
                 }
             }
@@ -178,7 +188,7 @@ __global__ void __launch_bounds__(wq::THREADS, 1)
                     break;
                 }
                 tc_fence_after();
-                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * wq::BN);
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * wq::ACC_COLS);
                 for (int kb = 0; kb < p.n_kb; ++kb, ++it) {
                     const int st = it % wq::STAGES;
                     const uint32_t par = (it / wq::STAGES) & 1;
@@ -191,9 +201,13 @@ __global__ void __launch_bounds__(wq::THREADS, 1)
 #pragma unroll
                     for (int kk = 0; kk < wq::BK / 16; ++kk) {
                         // K-major rows of 128 B; a k-step of 16 fp16 is 32 B along the row
-                        const uint64_t ad = umma_desc_sw128(s0 + kk * 32, 16, 1024);
                         const uint64_t bd = umma_desc_sw128(s0 + wq::OFF_B + kk * 32, 16, 1024);
-                        umma_f16(d_tmem, ad, bd, wq::IDESC, (kb > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+                        for (int h = 0; h < wq::BM / wq::MS; ++h) {
+                            const uint64_t ad = umma_desc_sw128(s0 + h * wq::A_SUB + kk * 32, 16, 1024);
+                            umma_f16(d_tmem + static_cast<uint32_t>(h * wq::BN), ad, bd, wq::IDESC,
+                                     (kb > 0 || kk > 0) ? 1u : 0u);
+                        }
                     }
                     umma_commit(&empty[st]);
                 }
@@ -210,21 +224,39 @@ __global__ void __launch_bounds__(wq::THREADS, 1)
         }
         __syncwarp();
     } else if (warp < wq::EPI_WARP0) {
-        // ---------------- dequantisers: thread j expands weight row n0 + j ----------------
-        const int j = (warp - 2) * 32 + lane;                    // 0..255
-        const uint32_t row_off = static_cast<uint32_t>((j >> 3) * 1024 + (j & 7) * 128);
+        // ---------- dequantisers: two threads per weight row, 32 codes each ----------
+        const int j = (warp - 2) * 32 + lane;                    // 0 .. 2*BN-1
+        const int jr = j >> 1, hsel = j & 1;                     // row of the tile, half
+        const uint32_t row_off = static_cast<uint32_t>((jr >> 3) * 1024 + (jr & 7) * 128);
+        // one group per k-block when groups are whole multiples of it: one scale and zero per
+        // k-block, fetched a k-block ahead
+        const bool one_group = (p.g % wq::BK) == 0;
         int it = 0;
         bool stop = false;
         for (long long t = blockIdx.x; t < p.n_tiles && !stop; t += gridDim.x) {
             int m0, n0;
             if (!wq_tile(p, t, m0, n0)) continue;
-            const int r = n0 + j;
+            const int r = n0 + jr;
             const bool row_ok = r < p.d_out;
             const int64_t srow = static_cast<int64_t>(row_ok ? r : 0) * p.ng;
             int cur_k = -1;
             __half2 s2 = __float2half2_rn(0.0f), z2 = __float2half2_rn(1024.0f);
+            uint16_t s_next = 0, z_next = 0;
+            if (one_group && row_ok) {
+                s_next = __ldg(p.scales + srow);
+                z_next = __ldg(p.zeros + srow);
+            }
             for (int kb = 0; kb < p.n_kb; ++kb, ++it) {
                 const int st = it % wq::STAGES;
+                if (one_group) {
+                    s2 = __half2half2(__ushort_as_half(s_next));
+                    z2 = __half2half2(__hadd(__float2half_rn(1024.0f), __ushort_as_half(z_next)));
+                    const int kn = ((kb + 1) * wq::BK) / p.g;         // next k-block's group
+                    if (row_ok && kb + 1 < p.n_kb) {
+                        s_next = __ldg(p.scales + srow + kn);
+                        z_next = __ldg(p.zeros + srow + kn);
+                    }
+                }
                 int ok = 1;
                 if (lane == 0) ok = mbar_wait(&full[st], (it / wq::STAGES) & 1) ? 1 : 0;
                 ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -237,25 +269,27 @@ __global__ void __launch_bounds__(wq::THREADS, 1)
                     break;
                 }
                 uint8_t* sa = smem + st * wq::STAGE;
-                const uint4* crow = reinterpret_cast<const uint4*>(sa + wq::OFF_C + j * 32);
-                const uint4 c0 = crow[0], c1 = crow[1];
-                const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+                const uint4 cv = *reinterpret_cast<const uint4*>(sa + wq::OFF_C + j * 16);
+                const uint32_t cw[4] = {cv.x, cv.y, cv.z, cv.w};
                 uint8_t* brow = sa + wq::OFF_B + row_off;
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const int col = kb * wq::BK + 8 * c;
-                    const int k = p.g_shift >= 0 ? (col >> p.g_shift) : col / p.g;
-                    if (k != cur_k) {
-                        cur_k = k;
-                        if (row_ok) {
-                            const __half s = __ushort_as_half(__ldg(p.scales + srow + k));
-                            const __half z = __ushort_as_half(__ldg(p.zeros + srow + k));
-                            s2 = __half2half2(s);
-                            z2 = __half2half2(__hadd(__float2half_rn(1024.0f), z));
+                for (int i = 0; i < 4; ++i) {
+                    const int c = 4 * hsel + i;                       // 8-column chunk
+                    if (!one_group) {
+                        const int col = kb * wq::BK + 8 * c;
+                        const int k = p.g_shift >= 0 ? (col >> p.g_shift) : col / p.g;
+                        if (k != cur_k) {
+                            cur_k = k;
+                            if (row_ok) {
+                                const __half sh = __ushort_as_half(__ldg(p.scales + srow + k));
+                                const __half zh = __ushort_as_half(__ldg(p.zeros + srow + k));
+                                s2 = __half2half2(sh);
+                                z2 = __half2half2(__hadd(__float2half_rn(1024.0f), zh));
+                            }
                         }
                     }
-                    const uint4 v = row_ok ? dequant8(cw[c], z2, s2) : make_uint4(0u, 0u, 0u, 0u);
-                    *reinterpret_cast<uint4*>(brow + ((c ^ (j & 7)) << 4)) = v;
+                    const uint4 v = row_ok ? dequant8(cw[i], z2, s2) : make_uint4(0u, 0u, 0u, 0u);
+                    *reinterpret_cast<uint4*>(brow + ((c ^ (jr & 7)) << 4)) = v;
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
@@ -285,24 +319,27 @@ __global__ void __launch_bounds__(wq::THREADS, 1)
                 break;
             }
             tc_fence_after();
-            const int row = m0 + 32 * q + lane;
-            const bool row_ok = row < p.n_tok;
 #pragma unroll 1
-            for (int c = 0; c < wq::BN / 32; ++c) {
+            for (int hc = 0; hc < (wq::BM / wq::MS) * (wq::BN / 32); ++hc) {
+                const int h = hc / (wq::BN / 32), c = hc % (wq::BN / 32);
+                const int row = m0 + h * wq::MS + 32 * q + lane;
+                const bool row_ok = row < p.n_tok;
                 uint32_t v[32];
-                tmem_ld_32x32b_x32(tmem_base + t_lane + static_cast<uint32_t>(b * wq::BN + 32 * c), v);
+                tmem_ld_32x32b_x32(tmem_base + t_lane +
+                                       static_cast<uint32_t>(b * wq::ACC_COLS + h * wq::BN + 32 * c),
+                                   v);
                 tmem_ld_wait();
                 const int col0 = n0 + 32 * c;
                 if (!row_ok || col0 >= p.d_out) continue;
                 const int64_t off = static_cast<int64_t>(row) * p.d_out + col0;
 #pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                    if (col0 + 8 * h >= p.d_out) break;
+                for (int u = 0; u < 4; ++u) {
+                    if (col0 + 8 * u >= p.d_out) break;
                     float f[8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[8 * h + e]);
+                    for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[8 * u + e]);
                     if (p.R) {
-                        const uint4 rv = *reinterpret_cast<const uint4*>(p.R + off + 8 * h);
+                        const uint4 rv = *reinterpret_cast<const uint4*>(p.R + off + 8 * u);
                         const __half2* rh = reinterpret_cast<const __half2*>(&rv);
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
@@ -317,7 +354,7 @@ __global__ void __launch_bounds__(wq::THREADS, 1)
                         const __half2 hv = __floats2half2_rn(f[2 * e], f[2 * e + 1]);
                         o[e] = *reinterpret_cast<const uint32_t*>(&hv);
                     }
-                    *reinterpret_cast<uint4*>(p.Y + off + 8 * h) = make_uint4(o[0], o[1], o[2], o[3]);
+                    *reinterpret_cast<uint4*>(p.Y + off + 8 * u) = make_uint4(o[0], o[1], o[2], o[3]);
                 }
             }
             tc_fence_before();
@@ -448,7 +485,7 @@ gptq_status w4a16_launch(const __half* X, int64_t n, int d_in, const uint8_t* pa
     }
     CUtensorMap xmap, cmap;
     GPTQ_TRY(encode_tensor_map_2d(&xmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, const_cast<__half*>(A),
-                                  d_in, n, static_cast<uint64_t>(d_in) * 2, wq::BK, wq::BM,
+                                  d_in, n, static_cast<uint64_t>(d_in) * 2, wq::BK, wq::MS,
                                   CU_TENSOR_MAP_SWIZZLE_128B));
     GPTQ_TRY(encode_tensor_map_2d(&cmap, CU_TENSOR_MAP_DATA_TYPE_UINT8,
                                   const_cast<uint8_t*>(packed), d_in / 2, d_out,
