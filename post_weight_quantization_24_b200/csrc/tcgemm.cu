@@ -41,8 +41,15 @@ constexpr int EPI_BUF = 32 * 32 * 4;                // 4 KB: 32 rows x 32 fp32
 constexpr int EPI_BYTES = 4 * 2 * EPI_BUF;           // 4 warps, double-buffered
 constexpr int BAR_BYTES = 256;
 constexpr int SMEM = 1024 + STAGES * STAGE + EPI_BYTES + BAR_BYTES;
-constexpr uint32_t TMEM_COLS = 256;
+constexpr uint32_t TMEM_COLS = 512;                  // two chunk accumulators + the sum
 constexpr int BAND = 16;                             // m-tiles per raster band (L2 reuse)
+// Promoted accumulation: the tensor cores' fp32 accumulation truncates, so a long K-chain
+// drifts; K is cut into chunks of PROMO_KB k-blocks (128), each accumulated in TMEM from zero,
+// and the chunks are summed with round-to-nearest fp32 additions by the epilogue: into a
+// third TMEM region for the store epilogue (read, add, store back, 32 columns at a time), and
+// straight into the dot for the dot epilogue.
+constexpr int PROMO_KB = 4;
+constexpr uint32_t SUM_COL = 2 * BN;                 // the running sum's TMEM columns
 }  // namespace tg
 
 // kind::tf32 instruction descriptor: A, B tf32 (format 2), D f32, A K-major, B K- or MN-major
@@ -95,6 +102,9 @@ __global__ void __launch_bounds__(tg::THREADS, 1)
     // pre-split operands need no converter warps: the epilogue warps follow warp 1 directly
     // (warps 2..5 take TMEM lane quarters 2, 3, 0, 1, as warps 10..13 do)
     constexpr int EPI0 = PRE ? 2 : tg::EPI_WARP0;
+    // accumulation chunks of the tile's K (a K of at most 128 is one chunk)
+    const int ckb = tg::PROMO_KB;
+    const int n_chunks = (p.n_kb + ckb - 1) / ckb;
     if (status_bad(p.a.status)) return;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -188,11 +198,12 @@ __global__ void __launch_bounds__(tg::THREADS, 1)
         // ---------------- MMA issuer ----------------
         if (lane == 0) {
             constexpr uint32_t IDESC = umma_idesc_tf32(tg::BM, tg::BN, !B_K);
-            int it = 0, lt = 0;
+            int it = 0, lt = 0;   // lt counts accumulation chunks
             bool ok = true;
             for (long long t = blockIdx.x; ok && t < p.n_tiles && !*abort_flag; t += gridDim.x) {
                 int m0, n0;
                 if (!tc_tile(p, t, m0, n0)) continue;
+              for (int ch = 0; ok && ch < n_chunks; ++ch) {
                 const int b = lt & 1;
                 if (!mbar_wait(&acc_empty[b], ((lt >> 1) & 1) ^ 1)) {
                     ok = false;
@@ -200,7 +211,8 @@ __global__ void __launch_bounds__(tg::THREADS, 1)
                 }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * tg::BN);
-                for (int kb = 0; kb < p.n_kb; ++kb, ++it) {
+                const int kb_first = ch * ckb, kb_end = min(p.n_kb, kb_first + ckb);
+                for (int kb = kb_first; kb < kb_end; ++kb, ++it) {
                     const int st = it % tg::STAGES;
                     if (!mbar_wait(PRE ? &full[st] : &conv[st], (it / tg::STAGES) & 1)) {
                         ok = false;
@@ -224,7 +236,7 @@ __global__ void __launch_bounds__(tg::THREADS, 1)
                             b_hi = umma_desc_sw128_32b(s0 + tg::OFF_B + kk * 1024, 4096, 512);
                             b_lo = umma_desc_sw128_32b(s0 + tg::OFF_B_LO + kk * 1024, 4096, 512);
                         }
-                        umma_tf32(d_tmem, a_hi, b_hi, IDESC, (kb > 0 || kk > 0) ? 1u : 0u);
+                        umma_tf32(d_tmem, a_hi, b_hi, IDESC, (kb > kb_first || kk > 0) ? 1u : 0u);
                         if (SPLIT_B) umma_tf32(d_tmem, a_hi, b_lo, IDESC, 1u);
                         if (SPLIT_A) umma_tf32(d_tmem, a_lo, b_hi, IDESC, 1u);
                     }
@@ -233,6 +245,7 @@ __global__ void __launch_bounds__(tg::THREADS, 1)
                 if (!ok) break;
                 umma_commit(&acc_full[b]);
                 ++lt;
+              }
             }
             if (!ok) {
                 set_status(status, GPTQ_ERR_TIMEOUT);
@@ -312,9 +325,32 @@ __global__ void __launch_bounds__(tg::THREADS, 1)
         double dot = 0.0;
         int lt = 0, nbulk = 0;
         bool stop = false;
+        // stage one 32 x 32 piece (this warp's rows, 32 columns) with the 128-byte swizzle of
+        // the C map and send it out with a TMA store or reduce-add
+        auto store_piece = [&](const float* v, int col0, int row0) {
+            float* buf = stage_buf + (nbulk & 1) * (tg::EPI_BUF / 4);
+            if (lane == 0) bulk_wait_read<1>();
+            __syncwarp();
+            float4* rowp = reinterpret_cast<float4*>(buf + lane * 32);
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                rowp[j ^ (lane & 7)] = make_float4(p.a.alpha * v[4 * j], p.a.alpha * v[4 * j + 1],
+                                                   p.a.alpha * v[4 * j + 2], p.a.alpha * v[4 * j + 3]);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                if (p.beta_one) tma_reduce_add_2d(&cmap, buf, col0, row0);
+                else tma_store_2d(&cmap, buf, col0, row0);
+                bulk_commit();
+            }
+            ++nbulk;
+        };
         for (long long t = blockIdx.x; t < p.n_tiles && !stop; t += gridDim.x) {
             int m0, n0;
             if (!tc_tile(p, t, m0, n0)) continue;
+            const int row0 = m0 + 32 * q;
+            const int row = row0 + lane;
+          for (int ch = 0; ch < n_chunks && !stop; ++ch) {
             const int b = lt & 1;
             int ok = 1;
             if (lane == 0) ok = mbar_wait(&acc_full[b], (lt >> 1) & 1) ? 1 : 0;
@@ -328,8 +364,39 @@ __global__ void __launch_bounds__(tg::THREADS, 1)
                 break;
             }
             tc_fence_after();
-            const int row0 = m0 + 32 * q;
-            const int row = row0 + lane;
+            if constexpr (EPI == TC_EPI_STORE) {
+                if (n_chunks > 1) {
+                    const bool last = ch == n_chunks - 1;
+                    // sum += this chunk, 32 columns at a time; the last chunk goes out instead
+#pragma unroll 1
+                    for (int c = 0; c < tg::BN / 32; ++c) {
+                        const uint32_t cc = static_cast<uint32_t>(32 * c);
+                        uint32_t r[32], a[32];
+                        tmem_ld_32x32b_x32(tmem_base + t_lane + static_cast<uint32_t>(b * tg::BN) + cc, r);
+                        if (ch > 0) tmem_ld_32x32b_x32(tmem_base + t_lane + tg::SUM_COL + cc, a);
+                        tmem_ld_wait();
+                        if (ch > 0) {
+#pragma unroll
+                            for (int i = 0; i < 32; ++i)
+                                r[i] = __float_as_uint(__uint_as_float(a[i]) + __uint_as_float(r[i]));
+                        }
+                        if (!last) {
+                            tmem_st_32x32b_x32(tmem_base + t_lane + tg::SUM_COL + cc, r);
+                        } else if (row0 < p.a.M && n0 + 32 * c < p.a.N) {   // warp-uniform
+                            float v[32];
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+                            store_piece(v, n0 + 32 * c, row0);
+                        }
+                    }
+                    if (!last) tmem_st_wait();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&acc_empty[b]);
+                    ++lt;
+                    continue;
+                }
+            }
 #pragma unroll 1
             for (int c = 0; c < tg::BN / 32; ++c) {
                 uint32_t r[32];
@@ -338,25 +405,10 @@ __global__ void __launch_bounds__(tg::THREADS, 1)
                 const int col0 = n0 + 32 * c;
                 if (row0 >= p.a.M || col0 >= p.a.N) continue;       // warp-uniform
                 if (EPI == TC_EPI_STORE) {
-                    // stage this warp's 32 x 32 piece with the 128-byte swizzle of the C map
-                    float* buf = stage_buf + (nbulk & 1) * (tg::EPI_BUF / 4);
-                    if (lane == 0) bulk_wait_read<1>();
-                    __syncwarp();
-                    float4* rowp = reinterpret_cast<float4*>(buf + lane * 32);
+                    float v[32];
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        rowp[j ^ (lane & 7)] = make_float4(
-                            p.a.alpha * __uint_as_float(r[4 * j]), p.a.alpha * __uint_as_float(r[4 * j + 1]),
-                            p.a.alpha * __uint_as_float(r[4 * j + 2]), p.a.alpha * __uint_as_float(r[4 * j + 3]));
-                    }
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) {
-                        if (p.beta_one) tma_reduce_add_2d(&cmap, buf, col0, row0);
-                        else tma_store_2d(&cmap, buf, col0, row0);
-                        bulk_commit();
-                    }
-                    ++nbulk;
+                    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+                    store_piece(v, col0, row0);
                 } else if (row < p.a.M) {
                     const float* dp = p.a.D + static_cast<int64_t>(row) * p.a.ldd + col0;
                     float part = 0.0f;
@@ -377,6 +429,7 @@ __global__ void __launch_bounds__(tg::THREADS, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&acc_empty[b]);
             ++lt;
+          }
         }
         if (EPI == TC_EPI_STORE) {
             if (lane == 0) bulk_wait_all();

@@ -14,8 +14,8 @@
 // k-blocks of 64 input channels, 4-stage ring):
 //   warp 0      TMA producer: the X tile (two 128 x 64 fp16 boxes, 128-byte swizzle) and the
 //               packed codes of the tile's 128 rows (128 x 32 bytes) per k-block.
-//   warps 2-9   dequantisers: threads 2r and 2r+1 expand row r's 64 codes (32 each) with its
-//               scale and zero (fp16 arithmetic: (1024 + q) - (1024 + z) is exact, times the
+//   warps 2-9   dequantisers: threads 2r and 2r+1 expand row r's 64 codes (32 each; a build
+//               option splits a row over four threads) with its scale and zero (fp16 arithmetic: (1024 + q) - (1024 + z) is exact, times the
 //               scale is the one rounding of the exact product) and write them into the B tile
 //               in the 128-byte swizzled K-major layout the MMA reads, then fence and signal
 //               the stage.
@@ -46,9 +46,14 @@ constexpr int C_BYTES = BN * BK / 2;                 // 4 KB packed codes
 constexpr int OFF_B = A_BYTES;
 constexpr int OFF_C = A_BYTES + B_BYTES;
 constexpr int STAGE = A_BYTES + B_BYTES + C_BYTES;   // 52 KB, A and B 1024-aligned
-constexpr int DQ_WARPS = BN / 16;                    // two threads per weight row
+#ifndef GPTQ_W4_TPR
+#define GPTQ_W4_TPR 2
+#endif
+constexpr int TPR = GPTQ_W4_TPR;                     // expanding threads per weight row (2, 4)
+constexpr int DQ_WARPS = BN * TPR / 32;
+static_assert(TPR == 2 || TPR == 4, "a thread expands 32 or 16 codes of its row");
 constexpr int EPI_WARP0 = 2 + DQ_WARPS;
-constexpr int THREADS = (EPI_WARP0 + 4) * 32;        // 448
+constexpr int THREADS = (EPI_WARP0 + 4) * 32;        // 448 (TPR 2), 704 (TPR 4)
 constexpr int BAR_BYTES = 256;
 constexpr int SMEM = 1024 + STAGES * STAGE + BAR_BYTES;
 constexpr int ACC_COLS = (BM / MS) * BN;             // 256: one tile's two accumulators
@@ -224,12 +229,13 @@ __global__ void __launch_bounds__(wq::THREADS, 1)
         }
         __syncwarp();
     } else if (warp < wq::EPI_WARP0) {
-        // ---------- dequantisers: two threads per weight row, 32 codes each ----------
-        const int j = (warp - 2) * 32 + lane;                    // 0 .. 2*BN-1
-        const int jr = j >> 1, hsel = j & 1;                     // row of the tile, half
+        // ---------- dequantisers: TPR threads per weight row, 64/TPR codes each ----------
+        constexpr int TPR = wq::TPR, CPT = 8 / TPR;              // 8-column chunks per thread
+        const int j = (warp - 2) * 32 + lane;                    // 0 .. TPR*BN-1
+        const int jr = j / TPR, hsel = j % TPR;                  // row of the tile, part
         const uint32_t row_off = static_cast<uint32_t>((jr >> 3) * 1024 + (jr & 7) * 128);
         // one group per k-block when groups are whole multiples of it: one scale and zero per
-        // k-block, fetched a k-block ahead
+        // k-block, fetched a k-block ahead. Rows past d_out keep scale 0 and expand to zeros.
         const bool one_group = (p.g % wq::BK) == 0;
         int it = 0;
         bool stop = false;
@@ -269,12 +275,18 @@ __global__ void __launch_bounds__(wq::THREADS, 1)
                     break;
                 }
                 uint8_t* sa = smem + st * wq::STAGE;
-                const uint4 cv = *reinterpret_cast<const uint4*>(sa + wq::OFF_C + j * 16);
-                const uint32_t cw[4] = {cv.x, cv.y, cv.z, cv.w};
+                uint32_t cw[CPT];
+                if constexpr (CPT == 4) {
+                    const uint4 cv = *reinterpret_cast<const uint4*>(sa + wq::OFF_C + j * 16);
+                    cw[0] = cv.x; cw[1] = cv.y; cw[2] = cv.z; cw[3] = cv.w;
+                } else {
+                    const uint2 cv = *reinterpret_cast<const uint2*>(sa + wq::OFF_C + j * 8);
+                    cw[0] = cv.x; cw[1] = cv.y;
+                }
                 uint8_t* brow = sa + wq::OFF_B + row_off;
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int c = 4 * hsel + i;                       // 8-column chunk
+                for (int i = 0; i < CPT; ++i) {
+                    const int c = CPT * hsel + i;                     // 8-column chunk
                     if (!one_group) {
                         const int col = kb * wq::BK + 8 * c;
                         const int k = p.g_shift >= 0 ? (col >> p.g_shift) : col / p.g;
@@ -288,8 +300,7 @@ __global__ void __launch_bounds__(wq::THREADS, 1)
                             }
                         }
                     }
-                    const uint4 v = row_ok ? dequant8(cw[i], z2, s2) : make_uint4(0u, 0u, 0u, 0u);
-                    *reinterpret_cast<uint4*>(brow + ((c ^ (jr & 7)) << 4)) = v;
+                    *reinterpret_cast<uint4*>(brow + ((c ^ (jr & 7)) << 4)) = dequant8(cw[i], z2, s2);
                 }
                 fence_proxy_async_smem();
                 __syncwarp();

@@ -212,6 +212,43 @@ def test_identity_hessian_is_rtn_bit_exact(cuda_lib, dtype, act_order):
     assert np.array_equal(rtn_codes, codes)
 
 
+def test_smallest_layer_matches_oracle(cuda_lib):
+    """The smallest layer the call accepts: one output row, d_in = 8, one 8-column group and
+    one 8-column block."""
+    wl = workloads.WORKLOADS["mlp_up_7b"].replace(d_out=1, d_in=8, n_tokens=64, seed=8)
+    W = workloads.make_weights(wl, device="cuda")
+    X = workloads.make_activations(wl, device="cuda")
+    out, ref, Wn, Href, _, eps, detail = run_case(cuda_lib, W, X, 4, 8, 8, True)
+    check_outputs(out, ref, Wn, Href, 8, 4, eps, detail)
+
+
+@pytest.mark.slow
+def test_largest_width_identity_hessian_is_rtn(cuda_lib):
+    """d_in = 65536, the largest width the call accepts (H and the factor's two d x d buffers
+    hold 4.3e9 entries each, past 32-bit indexing): with H = c·I the result is RTN's bit for
+    bit, so every stage runs at that size against a definition the oracle fixes exactly."""
+    d, d_out = 65536, 48
+    wl = workloads.WORKLOADS["mlp_up_7b"].replace(d_out=d_out, d_in=d)
+    W = workloads.make_weights(wl, device="cuda")
+    H = torch.zeros(d, d, device="cuda")
+    H.diagonal().fill_(5.0)
+    out = cuda_lib.quantize_layer(W, H, bits=4, group_size=128, act_order=False,
+                                  compute_loss=True)
+    del H
+    packed, scales, zeros = cuda_lib.rtn_minmax_quantize(W, 4, 128)
+    torch.cuda.synchronize()
+    codes, s_ref, z_ref = ortn.rtn_minmax(W.float().cpu().numpy().astype(np.float64), 4, 128)
+    assert np.array_equal(out["codes"].cpu().numpy(), codes)
+    assert np.array_equal(ortn.unpack_int4(packed.cpu().numpy()), codes)
+    assert np.array_equal(out["scales"].float().cpu().numpy().astype(np.float64), s_ref)
+    assert np.array_equal(out["zeros"].float().cpu().numpy().astype(np.float64), z_ref)
+    # the loss of RTN under H = c·I: ||W - What||^2 / ||W||^2
+    Wn = W.float().cpu().numpy().astype(np.float64)
+    D = Wn - ortn.rtn_dequant(codes, s_ref, z_ref, 128)
+    l_ref = float(np.sum(D * D) / np.sum(Wn * Wn))
+    assert abs(out["loss"] - l_ref) <= 1e-4 * l_ref, (out["loss"], l_ref)
+
+
 def test_correlated_inputs(cuda_lib):
     """Strongly correlated channels (not one of the named workloads): compensation is large, so
     a legitimate near-tie flip upstream can move later codes of its row by more than one
