@@ -139,7 +139,7 @@ struct Workspace {
     uint8_t* codes_p;// d_out x d_in codes in processing order
     float* P;        // d x 128: the column loop's images of U's diagonal blocks
     float* Dinv;     // ceil(d/128) x 128 x 128 inverses of the Cholesky diagonal blocks
-    float* F;        // 4 x d x 128: the factorisation's split panels (two L21 lo, X_top hi, lo)
+    float* F;        // 4 x d x 128 (512 from kOuterMinD on): the factorisation's split panels
     int* perm;
     int* invperm;
     size_t bytes;
@@ -166,7 +166,8 @@ static Workspace layout(void* base, int d_out, int d_in) {
     w.codes_p = take(static_cast<size_t>(d_out) * d);
     w.P = reinterpret_cast<float*>(take(d * kCholBlock * 4));
     w.Dinv = reinterpret_cast<float*>(take(nbl * kCholBlock * kCholBlock * 4));
-    w.F = reinterpret_cast<float*>(take(4 * d * kCholBlock * 4));
+    w.F = reinterpret_cast<float*>(
+        take(4 * d * static_cast<size_t>(factor_panel_cols(static_cast<int>(d))) * 4));
     w.perm = reinterpret_cast<int*>(take(d * 4));
     w.invperm = reinterpret_cast<int*>(take(d * 4));
     w.bytes = off;

@@ -539,7 +539,120 @@ gptq_status factor_inverse_launch(float* A, int d, float* Dinv, float* X, float*
         GPTQ_LAUNCHED();
         return GPTQ_OK;
     };
-    const gptq_status rc = body();
+    // Wide layers: outer panels of kOuterCols columns. The main stream factors a panel's
+    // columns in 128-wide steps, each step's solve updating only the panel's own later columns;
+    // once per panel it updates the next panel's columns (K = 512) after the previous panel's
+    // rest. The second stream splits the panel's L once and applies the rest of the trailing
+    // update and the inverse's bulk update with K = 512 (a quarter of the passes over the
+    // d x d matrices); the inverse's rows of the panel itself are done in 128-wide steps.
+    auto body_outer = [&]() -> gptq_status {
+        const int op = kOuterCols;
+        float* Phi = F;
+        float* Plo = F + static_cast<int64_t>(d) * op;
+        float* Thi = F + 2 * static_cast<int64_t>(d) * op;
+        float* Tlo = F + 3 * static_cast<int64_t>(d) * op;
+        GPTQ_CUDA_TRY(cudaMemsetAsync(X, 0, static_cast<size_t>(d) * d * 4, t2));
+        set_identity_kernel<<<(d + 255) / 256, 256, 0, t2>>>(X, d);
+        GPTQ_LAUNCHED();
+        for (int K0 = 0; K0 < d; K0 += op) {
+            const int E = std::min(K0 + op, d), wP = E - K0, remP = d - E;
+            const int reserve =
+                std::min(sms / GPTQ_FACTOR_RESERVE_DIV, std::max(1, (remP + nb - 1) / nb));
+            const int side_ctas = std::max(1, sms - reserve);
+            // ---- main: the panel's columns in 128-wide steps ----
+            for (int k0 = K0; k0 < E; k0 += nb) {
+                const int m = k0 / nb, nbc = std::min(nb, d - k0), e = k0 + nbc, rem = d - e;
+                float* Dm = Dinv + static_cast<int64_t>(m) * nb * nb;
+                float* A21 = A + static_cast<int64_t>(e) * d + k0;
+                GPTQ_CUDA_TRY(launch_pdl(potrf_diag_kernel, dim3(1), dim3(pd::THREADS), smem, s,
+                                         A, d, k0, nbc, Dm, status));
+                GPTQ_LAUNCHED();
+                if (rem == 0) continue;
+                TcGemmArgs t{};  // A21 = A21 * Dinv_m^T
+                t.M = rem; t.N = nbc; t.K = nbc; t.alpha = 1.f; t.beta = 0.f;
+                t.A = A21; t.lda = d; t.B = Dm; t.ldb = nb; t.C = A21; t.ldc = d;
+                t.status = status;
+                GPTQ_TRY(tcgemm_launch(t, true, TC_EPI_STORE, true, true, s));
+                if (E > e) {
+                    TcGemmArgs u{};  // the panel's own later columns: A[e:, e:E] -= A21 A21[0:E-e]^T
+                    u.M = rem; u.N = E - e; u.K = nbc; u.alpha = -1.f; u.beta = 1.f;
+                    u.A = A21; u.lda = d; u.B = A21; u.ldb = d;
+                    u.C = A + static_cast<int64_t>(e) * d + e; u.ldc = d;
+                    u.lower_only = 1; u.status = status;
+                    GPTQ_TRY(tcgemm_launch(u, true, TC_EPI_STORE, true, true, s));
+                }
+            }
+            GPTQ_CUDA_TRY(cudaEventRecord(ss->trsm, s));      // the panel's L is complete
+            const float* Lp = A + static_cast<int64_t>(E) * d + K0;   // L[E:, K0:E]
+            if (remP > 0) {
+                const int E2 = std::min(E + op, d);
+                // the next panel's columns, after the previous panel's rest (their other writer)
+                if (K0 > 0) GPTQ_CUDA_TRY(cudaStreamWaitEvent(s, ss->rest, 0));
+                TcGemmArgs u{};  // A[E:, E:E2] -= L[E:, K0:E] L[E:E2, K0:E]^T
+                u.M = remP; u.N = E2 - E; u.K = wP; u.alpha = -1.f; u.beta = 1.f;
+                u.A = Lp; u.lda = d; u.B = Lp; u.ldb = d;
+                u.C = A + static_cast<int64_t>(E) * d + E; u.ldc = d;
+                u.lower_only = 1; u.status = status;
+                GPTQ_TRY(tcgemm_launch(u, true, TC_EPI_STORE, true, true, s));
+            }
+            // ---- side: split the panel, the rest of the trailing update, the inverse ----
+            GPTQ_CUDA_TRY(cudaStreamWaitEvent(t2, ss->trsm, 0));
+            if (remP > 0) {
+                const int E2 = std::min(E + op, d);
+                float* Ph = Phi + static_cast<int64_t>(E) * op;   // rows E.. of the panel
+                float* Pl = Plo + static_cast<int64_t>(E) * op;
+                GPTQ_TRY(tcgemm_split_launch(Lp, Ph, Pl, remP, wP, d, false, t2, op, op));
+                if (E2 < d) {
+                    const int64_t off = static_cast<int64_t>(E2 - E) * op;
+                    TcGemmArgs r{};  // A[E2:, E2:] -= L[E2:, K0:E] L[E2:, K0:E]^T (lower tiles)
+                    r.M = d - E2; r.N = d - E2; r.K = wP; r.alpha = -1.f; r.beta = 1.f;
+                    r.A = Ph + off; r.lda = op; r.A_lo = Pl + off;
+                    r.B = Ph + off; r.ldb = op; r.B_lo = Pl + off;
+                    r.C = A + static_cast<int64_t>(E2) * d + E2; r.ldc = d;
+                    r.lower_only = 1; r.status = status; r.max_ctas = side_ctas;
+                    GPTQ_TRY(tcgemm_presplit_launch(r, t2, true));
+                }
+            }
+            GPTQ_CUDA_TRY(cudaEventRecord(ss->rest, t2));
+            for (int k0 = K0; k0 < E; k0 += nb) {
+                const int m = k0 / nb, nbc = std::min(nb, d - k0), e = k0 + nbc;
+                float* Dm = Dinv + static_cast<int64_t>(m) * nb * nb;
+                float* Xk = X + static_cast<int64_t>(k0) * d;
+                TcGemmArgs v{};  // X[k0:e, 0:e] = Dinv_m * X[k0:e, 0:e], in place
+                v.M = nbc; v.N = e; v.K = nbc; v.alpha = 1.f; v.beta = 0.f;
+                v.A = Dm; v.lda = nb; v.B = Xk; v.ldb = d; v.C = Xk; v.ldc = d;
+                v.status = status; v.max_ctas = side_ctas;
+                GPTQ_TRY(tcgemm_launch(v, false, TC_EPI_STORE, true, true, t2));
+                if (E > e) {
+                    TcGemmArgs w{};  // X[e:E, 0:e] -= L[e:E, k0:e] * X[k0:e, 0:e]
+                    w.M = E - e; w.N = e; w.K = nbc; w.alpha = -1.f; w.beta = 1.f;
+                    w.A = A + static_cast<int64_t>(e) * d + k0; w.lda = d;
+                    w.B = Xk; w.ldb = d; w.C = X + static_cast<int64_t>(e) * d; w.ldc = d;
+                    w.status = status; w.max_ctas = side_ctas;
+                    GPTQ_TRY(tcgemm_launch(w, false, TC_EPI_STORE, true, true, t2));
+                }
+            }
+            if (remP > 0) {
+                float* XP = X + static_cast<int64_t>(K0) * d;      // X[K0:E, 0:E]
+                GPTQ_TRY(tcgemm_split_launch(XP, Thi, Tlo, wP, E, d, false, t2));
+                TcGemmArgs w{};  // X[E:, 0:E] -= L[E:, K0:E] * X[K0:E, 0:E]
+                w.M = remP; w.N = E; w.K = wP; w.alpha = -1.f; w.beta = 1.f;
+                w.A = Phi + static_cast<int64_t>(E) * op; w.lda = op;
+                w.A_lo = Plo + static_cast<int64_t>(E) * op;
+                w.B = Thi; w.ldb = d; w.B_lo = Tlo;
+                w.C = X + static_cast<int64_t>(E) * d; w.ldc = d;
+                w.status = status; w.max_ctas = side_ctas;
+                GPTQ_TRY(tcgemm_presplit_launch(w, t2, false));
+            }
+        }
+        const int64_t half = static_cast<int64_t>(d) * d / 2;
+        const int blocks =
+            static_cast<int>(std::min<int64_t>((half + 255) / 256, num_sms() * 16));
+        reverse_inplace_kernel<<<blocks, 256, 0, t2>>>(X, half);
+        GPTQ_LAUNCHED();
+        return GPTQ_OK;
+    };
+    const gptq_status rc = d >= kOuterMinD ? body_outer() : body();
     const cudaError_t e1 = cudaEventRecord(ss->join, t2);
     const cudaError_t e2 = cudaStreamWaitEvent(s, ss->join, 0);
     if (rc != GPTQ_OK) return rc;

@@ -30,6 +30,16 @@ struct DevState {
 };
 
 constexpr int kCholBlock = 128;   // panel width of the blocked Cholesky / triangular inverse
+// From this width on, the factorisation applies its trailing and inverse updates once per
+// outer panel of kOuterCols columns (K = 512, accumulated in 128-deep chunks) instead of once
+// per 128 columns: a quarter of the passes over the d x d matrices.
+#ifndef GPTQ_OUTER_MIN_D
+#define GPTQ_OUTER_MIN_D 16384
+#endif
+constexpr int kOuterMinD = GPTQ_OUTER_MIN_D;
+constexpr int kOuterCols = 512;
+// Width of the factorisation's split panels (the scratch F is 4 x d x this many floats).
+inline int factor_panel_cols(int d) { return d >= kOuterMinD ? kOuterCols : kCholBlock; }
 constexpr int kSuperCols = 512;   // columns whose errors are collected before the far update
 
 // rtn.cu
@@ -55,8 +65,8 @@ gptq_status gather_w_launch(const void* W, int w_dtype, int d_out, int d_in, con
                             float* Wk, int* status, cudaStream_t s);
 // In-place lower Cholesky factor L of A (lda = d), the inverses of its diagonal blocks in Dinv
 // (ceil(d/nb) blocks of nb x nb, row-major, zero above the diagonal), and U = reverse(L^-1) in
-// X. F is scratch of 4 x d x 128 floats (the tf32 hi/lo parts of one panel of L and of one
-// panel of rows of L^-1). Uses a second stream of its own, forked from and joined back to s.
+// X. F is scratch of 4 x d x factor_panel_cols(d) floats (the tf32 hi/lo parts of one panel of
+// L and of one panel of rows of L^-1). Uses a second stream of its own, forked from and joined back to s.
 gptq_status factor_inverse_launch(float* A, int d, float* Dinv, float* X, float* F, int* status,
                                   cudaStream_t s);
 // Test switch: the diagonal-block kernel waits on a barrier nothing arrives at (bounded).

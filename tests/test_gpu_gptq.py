@@ -316,6 +316,62 @@ def test_inverse_factor_4096(cuda_lib, act_order):
 
 
 @pytest.mark.slow
+@pytest.mark.parametrize("act_order", [False, True])
+def test_inverse_factor_outer_panels(cuda_lib, act_order):
+    """d = 16768: wide enough for the outer-panel factorisation (updates with K = 512 once per
+    512 columns), with a ragged last outer panel of 384 columns. Oracle: the reversal route in
+    fp64. Same bound as above; the residual is taken on 64 sampled columns and the condition
+    number by Lanczos (the dense forms would take minutes at this size)."""
+    from scipy.sparse.linalg import LinearOperator, eigsh
+    d = 16768
+    wl = workloads.WORKLOADS["mlp_up_7b"].replace(d_in=d, n_tokens=20000, seed=6)
+    X = workloads.make_activations(wl, device="cuda")
+    H = gpu_hessian(cuda_lib, X)
+    U, perm = cuda_lib.inverse_factor(H, 0.01, act_order)
+    Ug = U.cpu().numpy().astype(np.float64)
+    del U, H
+    Href = ohess.hessian(X.cpu().numpy())
+    del X
+    perm_ref = ogptq.act_order_perm(Href) if act_order else np.arange(d)
+    perm_gpu = perm.cpu().numpy().astype(np.int64)
+    moved = np.flatnonzero(perm_gpu != perm_ref)
+    log_parity(perm_positions_moved=int(moved.size))
+    if moved.size:
+        # act_order's own near ties (as in the mlp_down_7b test): diag(H) entries within the H
+        # tolerance of each other may come out in either order; the factor is then compared
+        # for the GPU's processing order
+        dg_h = np.diag(Href)
+        gap = np.abs(dg_h[perm_gpu[moved]] - dg_h[perm_ref[moved]]) / dg_h[perm_ref[moved]]
+        assert np.all(gap <= 4 * H_TOL), gap
+        perm_ref = perm_gpu
+    Hd, _ = ofac.damp(Href[np.ix_(perm_ref, perm_ref)], 0.01)
+    Uref = ofac.upper_chol_of_inverse_reversed(Hd)
+    del Href
+    dg = np.sqrt(np.diag(Uref))
+    max_scaled = 0.0
+    for i0 in range(0, d, 2048):
+        blk = np.abs(Ug[i0:i0 + 2048] - Uref[i0:i0 + 2048]) / np.outer(dg[i0:i0 + 2048], dg)
+        max_scaled = max(max_scaled, float(np.max(blk)))
+    cols = np.sort(np.random.default_rng(2).choice(d, 64, replace=False))
+    E = Ug.T @ (Ug @ Hd[:, cols])
+    E[cols, np.arange(64)] -= 1.0
+    resid = float(np.max(np.abs(E)))
+    sc = 1.0 / np.sqrt(np.diag(Hd))
+    Hs = Hd * sc[:, None]
+    Hs *= sc[None, :]
+    lmax = eigsh(Hs, k=1, which="LA", return_eigenvectors=False, tol=1e-3)[0]
+    # the largest eigenvalue of Hs^-1 = S^-1 U^T U S^-1 (U the oracle's factor) is 1/lambda_min
+    inv = LinearOperator((d, d), dtype=np.float64,
+                         matvec=lambda v: (Uref.T @ (Uref @ (v.ravel() / sc))) / sc)
+    lmin = 1.0 / eigsh(inv, k=1, which="LA", return_eigenvectors=False, tol=1e-3)[0]
+    err = dict(max_scaled=max_scaled, residual=resid, kappa_scaled=float(lmax / lmin))
+    log_parity(**err)
+    bound = 8.0 * np.sqrt(d) * err["kappa_scaled"] * U_EPS
+    assert max_scaled <= bound, (err, bound)
+    assert resid <= bound, (err, bound)
+
+
+@pytest.mark.slow
 def test_full_size_mlp_up_7b(cuda_lib):
     """The timed workload: W 11008x4096 fp16, X 262144x4096, INT4 g128 B128, all rows."""
     wl = workloads.WORKLOADS["mlp_up_7b"]
