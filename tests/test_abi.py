@@ -89,9 +89,10 @@ def test_workspace_sizes(L):
         return (b + 255) // 256 * 256
     for d_out, d_in in ((512, 512), (11008, 4096), (4096, 11008), (3, 8)):
         nbl = (d_in + 127) // 128
+        panel = 512 if d_in >= 9216 else 128      # the factorisation's split-panel width
         expect = (r256(40) + 2 * r256(d_in * d_in * 4) + r256(d_out * d_in * 4)
                   + 4 * r256(d_out * 512 * 4) + r256(d_out * d_in) + r256(d_in * 128 * 4)
-                  + r256(nbl * 128 * 128 * 4) + r256(4 * d_in * 128 * 4) + 2 * r256(d_in * 4))
+                  + r256(nbl * 128 * 128 * 4) + r256(4 * d_in * panel * 4) + 2 * r256(d_in * 4))
         assert L.gptq_quantize_layer_workspace(d_out, d_in, 128) == expect
     assert L.gptq_quantize_layer_workspace(0, 512, 128) == 0
 

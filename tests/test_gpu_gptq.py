@@ -318,7 +318,7 @@ def test_inverse_factor_4096(cuda_lib, act_order):
 @pytest.mark.slow
 @pytest.mark.parametrize("act_order", [False, True])
 def test_inverse_factor_outer_panels(cuda_lib, act_order):
-    """d = 16768: wide enough for the outer-panel factorisation (updates with K = 512 once per
+    """d = 16768: wide enough for the outer-panel factorisation (from d = 9216 on) (updates with K = 512 once per
     512 columns), with a ragged last outer panel of 384 columns. Oracle: the reversal route in
     fp64. Same bound as above; the residual is taken on 64 sampled columns and the condition
     number by Lanczos (the dense forms would take minutes at this size)."""
