@@ -183,108 +183,155 @@ gptq_status gather_w_launch(const void* W, int w_dtype, int d_out, int d_in, con
 // ---------------------------------------------------------------------------------------
 // blocked Cholesky
 // ---------------------------------------------------------------------------------------
-// ---- diagonal block: one CTA factors the 128 x 128 block A[k0:, k0:] and inverts its factor.
-// Pass 1 (factor) is right-looking elimination with one thread per row. At step c every
-// thread has published its current column-c entry a_ic; by symmetry the pivot row's entries
-// a_cm are the published a_mc, so the column is all a step needs. Thread i then applies
-// a_im -= (a_ic / a_cc) a_mc to its row and records L[i][c] = a_ic / sqrt(a_cc).
-// Pass 2 (inverse) gives thread i column i of L^-1 by forward substitution against the
-// recorded columns of L: x_m -= L[m][c] * x_c / L[c][c], with x_c / L[c][c] = (L^-1)[c][i].
-// In both passes a thread's values sit in a register window that moves down one position
-// per step (position p holds matrix index c + p), so the running step is always position 0
-// and every register index is a compile-time constant; the window narrows in phases of 16
-// steps. In pass 1 a thread computes its next column entry first, publishes it and arrives
-// on the next step's mbarrier before it sweeps the rest of its row, so the exchange of one
-// step overlaps the arithmetic of the previous one (three column buffers, one mbarrier
-// each). Pass 2 needs no synchronisation. Rows and columns beyond the matrix edge are padded
-// with the identity.
+// ---- diagonal block: one CTA of 512 threads factors the 128 x 128 block A[k0:, k0:] and
+// inverts its factor, blocked in four sub-panels of 32 columns (right-looking):
+//   for k = 0..3 (b = 32k):
+//     factor   one warp: L_kk = chol(A_kk) and I_kk = L_kk^-1, 32 steps in registers
+//     solve    L_rk = A_rk I_kk^T for the row blocks r below (all threads)
+//     update   A_ij -= L_ik L_jk^T for the trailing lower blocks (all threads)
+//   inverse    X = L^-1 by block forward substitution, column blocks in parallel:
+//              W_ij = sum_{m<i} L_im X_mj accumulated right-looking, X_ij = -I_ii W_ij
+// In the factor warp, lane i holds row i of A_kk and column i of I_kk. At step c the pivot
+// a_cc is broadcast, lane i forms L[i][c] = a_ic / sqrt(a_cc) and its inverse column entry
+// y_c = w_c / L_cc, then applies the rank-1 update to its row (a_im -= L[i][c] L[m][c]) and
+// the substitution update to its inverse column (w_m -= L[m][c] y_c); both updates take the
+// same broadcast L[m][c]. Lane c+1 computes the next pivot first, so the chain from one
+// pivot to the next is a reciprocal square root, two multiply-adds and one shuffle.
+// The block products run on 2 x 4 register tiles per thread, 128 threads per 32 x 32 block.
+// Rows and columns beyond the matrix edge are padded with the identity.
 namespace pd {
-constexpr int NB = 128, THREADS = NB, PH = 16, NBUF = 3;
-constexpr int LS = NB + 4;          // Lsh row stride: Lsh[c][m - c + 3] = L[m][c], m >= c
-constexpr int CB = NB + 8;          // published column: cb[i - c + 3] = a_ic of step c
-// + rs[c]; NBUF exchange mbarriers and one that nothing arrives at (the stall test below)
-constexpr int SMEM = (NB * LS + NBUF * CB + NB) * 4 + (NBUF + 1) * 8;
+constexpr int NB = 128, SB = 32, NSB = NB / SB, THREADS = 512;
+constexpr int LD = NB + 4;          // row stride (floats) of S, X and LT: 16-byte rows, and
+                                    // consecutive rows start four banks apart
+constexpr int ILD = SB + 4;         // row stride of IkT
+// S [NB][LD]: the block, overwritten by L; X [NB][LD]: L^-1 (its blocks below the diagonal
+// hold the partial sums W until they are final); LT [SB][LD]: the current sub-panel's L_rk,
+// transposed; IkT [SB][ILD]: I_kk transposed; lbuf [2][SB]: the factor warp's column
+// exchange; then the stall-test mbarrier
+constexpr int SMEM_FLOATS = 2 * NB * LD + SB * LD + SB * ILD + 2 * SB;
+constexpr int SMEM = SMEM_FLOATS * 4 + 16;
 constexpr long long STALL_LIMIT_CYCLES = 2000000;   // about 1 ms
 }  // namespace pd
 
 // Test switch for the bounded-wait path (set by gptq_test_stall_factor): when nonzero, every
 // thread of the diagonal-block kernel first waits on an mbarrier that nothing arrives at. The
 // wait gives up after STALL_LIMIT_CYCLES, the kernel records GPTQ_ERR_TIMEOUT and returns, and
-// the rest of the factorisation skips its work on the status word. The kernel's barriers are
-// fed by its own threads' arrivals only; no copy or MMA is in flight when it gives up.
+// the rest of the factorisation skips its work on the status word. No copy or MMA is in
+// flight when it gives up.
 __device__ int g_factor_stall = 0;
 
-__device__ __forceinline__ float rcp_approx(float x) {
-    float r;
-    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
-    return r;
-}
-
-__device__ __forceinline__ float rsqrt_approx(float x) {
+// 1/sqrt(x): the hardware estimate refined by one Newton-Raphson step r' = r (1 + (1 - x r^2)/2)
+__device__ __forceinline__ float rsqrt_nr(float x) {
     float r;
     asm("rsqrt.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
-    return r;
+    const float e = fmaf(-(x * r), r, 1.0f);
+    return fmaf(0.5f * r, e, r);
 }
 
-template <int W>
-__device__ __forceinline__ bool potrf_factor_phase(float (&w)[pd::NB], int q, int i, float* Lsh,
-                                                   float* cb, uint64_t* mb, float* rs, bool& bad) {
-#pragma unroll 1
-    for (int c = q * pd::PH; c < (q + 1) * pd::PH; ++c) {
-        const int b = c % pd::NBUF, nb = (c + 1) % pd::NBUF;
-        if (!mbar_wait(&mb[b], (c / pd::NBUF) & 1)) return false;
-        const float* buf = cb + b * pd::CB;
-        const float* col = buf + 4;          // col[k] = a_{c+1+k, c}
-        if ((i | 31) >= c) {                 // this warp still has a row at or below the pivot
-            const float p = buf[3];
-            const float t = w[0] * rcp_approx(p);
-            // the next step's column entry first: publish it, then sweep the rest of the row
-            const float nw0 = fmaf(-t, col[0], w[1]);
-            if (i > c) cb[nb * pd::CB + i - c + 2] = nw0;
-            mbar_arrive(&mb[nb]);
-            const float rsp = rsqrt_approx(p);
-            if (i >= c) Lsh[c * pd::LS + i - c + 3] = (i == c) ? p * rsp : w[0] * rsp;
-            if (i == c) {
-                rs[c] = rsp;
-                if (!(p > 0.0f) || !isfinite(p)) bad = true;
-            }
-            w[0] = nw0;
+// One warp: L_kk and I_kk of the 32 x 32 block at S[b:, b:]. Writes L_kk (zeros above the
+// diagonal) back into S, I_kk into X's diagonal block and, transposed, into IkT. Returns
+// true on a pivot that is not a positive normal number. Each step's column L[:, c] is
+// exchanged through lbuf (two buffers: a lane writes step c+2's column only after every lane
+// has passed step c+1's __syncwarp, so after it has read step c's); the pivot goes by shuffle.
+__device__ __forceinline__ bool potrf32_warp(float* S, float* X, float* IkT, float* lbuf, int b,
+                                            int lane) {
+    constexpr unsigned FULL = 0xffffffffu;
+    float dr[pd::SB], w[pd::SB];
+    const float4* src = reinterpret_cast<const float4*>(S + (b + lane) * pd::LD + b);
 #pragma unroll
-            for (int k4 = 0; k4 < W; k4 += 4) {
-                const float4 v = *reinterpret_cast<const float4*>(col + k4);
-                const float vv[4] = {v.x, v.y, v.z, v.w};
+    for (int q = 0; q < pd::SB / 4; ++q) {
+        const float4 v = src[q];
+        dr[4 * q] = v.x; dr[4 * q + 1] = v.y; dr[4 * q + 2] = v.z; dr[4 * q + 3] = v.w;
+    }
 #pragma unroll
-                for (int u = 0; u < 4; ++u)
-                    if (k4 + u >= 1 && k4 + u + 1 < W) w[k4 + u] = fmaf(-t, vv[u], w[k4 + u + 1]);
+    for (int m = 0; m < pd::SB; ++m) w[m] = (m == lane) ? 1.0f : 0.0f;
+    bool bad = false;
+    float p = __shfl_sync(FULL, dr[0], 0);
+#pragma unroll
+    for (int c = 0; c < pd::SB; ++c) {
+        bad = bad || !(p >= 1.17549435e-38f && p <= 3.40282347e38f);
+        const float r = rsqrt_nr(p);                       // 1 / L_cc
+        const float l = (lane >= c) ? dr[c] * r : 0.0f;     // L[lane][c]
+        const float y = w[c] * r;                           // I_kk[c][lane]
+        dr[c] = l;
+        w[c] = y;
+        if (c + 1 == pd::SB) break;
+        float* lb = lbuf + (c & 1) * pd::SB;
+        lb[lane] = l;
+        p = __shfl_sync(FULL, fmaf(-l, l, dr[c + 1]), c + 1);
+        __syncwarp();
+#pragma unroll
+        for (int m4 = (c + 1) & ~3; m4 < pd::SB; m4 += 4) {
+            const float4 v = *reinterpret_cast<const float4*>(lb + m4);   // L[m4 .. m4+3][c]
+            const float lv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                if (m4 + u <= c) continue;
+                dr[m4 + u] = fmaf(-l, lv[u], dr[m4 + u]);
+                w[m4 + u] = fmaf(-lv[u], y, w[m4 + u]);
             }
-            w[W - 1] = 0.0f;
-        } else {
-            mbar_arrive(&mb[nb]);
         }
     }
-    return true;
+    float4* dst = reinterpret_cast<float4*>(S + (b + lane) * pd::LD + b);
+    float4* idst = reinterpret_cast<float4*>(IkT + lane * pd::ILD);
+#pragma unroll
+    for (int q = 0; q < pd::SB / 4; ++q) {
+        dst[q] = make_float4(dr[4 * q], dr[4 * q + 1], dr[4 * q + 2], dr[4 * q + 3]);
+        idst[q] = make_float4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+    }
+#pragma unroll
+    for (int c = 0; c < pd::SB; ++c) X[(b + c) * pd::LD + b + lane] = w[c];
+    return bad;
 }
 
-template <int W>
-__device__ __forceinline__ void potrf_inverse_phase(float (&w)[pd::NB], int q, int i, int nbc,
-                                                    const float* Lsh, const float* rs,
-                                                    float* __restrict__ Dinv) {
-#pragma unroll 1
-    for (int c = q * pd::PH; c < (q + 1) * pd::PH; ++c) {
-        const float t2 = w[0] * rs[c];       // (L^-1)[c][i]
-        Dinv[c * pd::NB + i] = (c < nbc && i < nbc) ? t2 : 0.0f;
-        const float* col = Lsh + c * pd::LS + 4;   // col[k] = L[c+1+k][c]
+// acc[h][q] += sum_m P[ti + 16h][m] Q[m][4 tj + q], m < 32 (P, Q row-major, 16-byte rows)
+__device__ __forceinline__ void block_mma32(const float* P, int ldp, const float* Q, int ldq,
+                                            int ti, int tj, float (&acc)[2][4]) {
 #pragma unroll
-        for (int k4 = 0; k4 < W; k4 += 4) {
-            const float4 v = *reinterpret_cast<const float4*>(col + k4);
-            const float vv[4] = {v.x, v.y, v.z, v.w};
+    for (int m4 = 0; m4 < pd::SB; m4 += 4) {
+        const float4 a0 = *reinterpret_cast<const float4*>(P + ti * ldp + m4);
+        const float4 a1 = *reinterpret_cast<const float4*>(P + (ti + 16) * ldp + m4);
+        const float av[2][4] = {{a0.x, a0.y, a0.z, a0.w}, {a1.x, a1.y, a1.z, a1.w}};
 #pragma unroll
-            for (int u = 0; u < 4; ++u)
-                if (k4 + u + 1 < W) w[k4 + u] = fmaf(-t2, vv[u], w[k4 + u + 1]);
+        for (int u = 0; u < 4; ++u) {
+            const float4 q = *reinterpret_cast<const float4*>(Q + (m4 + u) * ldq + 4 * tj);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                acc[h][0] = fmaf(av[h][u], q.x, acc[h][0]);
+                acc[h][1] = fmaf(av[h][u], q.y, acc[h][1]);
+                acc[h][2] = fmaf(av[h][u], q.z, acc[h][2]);
+                acc[h][3] = fmaf(av[h][u], q.w, acc[h][3]);
+            }
         }
-        w[W - 1] = 0.0f;
     }
 }
+
+__device__ __forceinline__ void zero_acc(float (&acc)[2][4]) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc[h][q] = 0.0f;
+}
+
+// the (bi, bj) block pair number q of the trailing lower blocks k+1 <= bj <= bi < 4
+__device__ __forceinline__ void trailing_pair(int k, int q, int& bi, int& bj) {
+    for (bj = k + 1; bj < pd::NSB; ++bj) {
+        const int n = pd::NSB - bj;
+        if (q < n) {
+            bi = bj + q;
+            return;
+        }
+        q -= n;
+    }
+    bi = bj = -1;
+}
+
+// inverse, round r: updates W_ij += L_im X_mj (m = j + r, i > m), listed as i | j << 2 | m << 4
+__constant__ unsigned char c_inv_upd[10] = {
+    1 | 0 << 2 | 0 << 4, 2 | 0 << 2 | 0 << 4, 3 | 0 << 2 | 0 << 4, 2 | 1 << 2 | 1 << 4,
+    3 | 1 << 2 | 1 << 4, 3 | 2 << 2 | 2 << 4,                                   // round 0
+    2 | 0 << 2 | 1 << 4, 3 | 0 << 2 | 1 << 4, 3 | 1 << 2 | 2 << 4,             // round 1
+    3 | 0 << 2 | 2 << 4};                                                       // round 2
 
 __global__ void __launch_bounds__(pd::THREADS, 1) potrf_diag_kernel(float* __restrict__ A, int d,
                                                                    int k0, int nbc,
@@ -293,70 +340,149 @@ __global__ void __launch_bounds__(pd::THREADS, 1) potrf_diag_kernel(float* __res
     pdl_wait();
     if (status_bad(status)) return;
     extern __shared__ __align__(16) float sm[];
-    float* Lsh = sm;                          // [NB][LS]
-    float* cb = Lsh + pd::NB * pd::LS;        // [NBUF][CB]
-    float* rs = cb + pd::NBUF * pd::CB;       // [NB]
-    uint64_t* mb = reinterpret_cast<uint64_t*>(rs + pd::NB);   // [NBUF], 128 arrivals each
-    const int i = threadIdx.x, warp = i >> 5;
+    float* S = sm;                            // [NB][LD]
+    float* X = S + pd::NB * pd::LD;           // [NB][LD]
+    float* LT = X + pd::NB * pd::LD;          // [SB][LD]
+    float* IkT = LT + pd::SB * pd::LD;        // [SB][ILD]
+    float* lbuf = IkT + pd::SB * pd::ILD;     // [2][SB]
+    uint64_t* mb = reinterpret_cast<uint64_t*>(lbuf + 2 * pd::SB);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    // block-product tile of this thread: 128 threads per 32 x 32 block
+    const int grp = tid >> 7, gw = (tid >> 5) & 3;
+    const int ti = (lane >> 3) + 4 * gw, tj = lane & 7;
 
-    for (int e = i; e < (pd::NB * pd::LS + pd::NBUF * pd::CB) / 4; e += pd::THREADS)
-        reinterpret_cast<float4*>(sm)[e] = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (i == 0) {
-        for (int b = 0; b < pd::NBUF; ++b) mbar_init(&mb[b], pd::THREADS);
-        mbar_init(&mb[pd::NBUF], 1);
-        fence_mbar_init();
-    }
-
-    // row i of the block's lower triangle (zeros above the diagonal; identity past the edge)
-    float w[pd::NB];
-    const float* arow = A + static_cast<int64_t>(k0 + i) * d + k0;
-#pragma unroll
-    for (int p4 = 0; p4 < pd::NB; p4 += 4) {
+    // S = the block's lower triangle (identity past the edge); X = 0
+#pragma unroll 2
+    for (int e = tid; e < pd::NB * (pd::NB / 4); e += pd::THREADS) {
+        const int r = e >> 5, c4 = (e & 31) * 4;
         float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (i < nbc && p4 <= i && p4 < nbc) v = *reinterpret_cast<const float4*>(arow + p4);
+        if (r < nbc && c4 <= r && c4 < nbc)
+            v = *reinterpret_cast<const float4*>(A + static_cast<int64_t>(k0 + r) * d + k0 + c4);
         const float vv[4] = {v.x, v.y, v.z, v.w};
+        float o[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u)
-            w[p4 + u] = (i < nbc) ? (p4 + u <= i ? vv[u] : 0.0f) : (p4 + u == i ? 1.0f : 0.0f);
+            o[u] = (r < nbc) ? (c4 + u <= r ? vv[u] : 0.0f) : (c4 + u == r ? 1.0f : 0.0f);
+        *reinterpret_cast<float4*>(S + r * pd::LD + c4) = make_float4(o[0], o[1], o[2], o[3]);
+        *reinterpret_cast<float4*>(X + r * pd::LD + c4) = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    if (tid == 0) {
+        mbar_init(mb, 1);
+        fence_mbar_init();
     }
     __syncthreads();
-    // step 0's column: every thread publishes a_i0
-    cb[i + 3] = w[0];
-    mbar_arrive(&mb[0]);
+    if (*(volatile int*)&g_factor_stall) {
+        const bool ok = mbar_wait_cycles(mb, 0, pd::STALL_LIMIT_CYCLES);
+        if (!ok && tid == 0) set_status(status, GPTQ_ERR_TIMEOUT);
+        if (__syncthreads_or(!ok)) return;
+    }
 
     bool bad = false;
-    bool ok = true;
-    if (*(volatile int*)&g_factor_stall) ok = mbar_wait_cycles(&mb[pd::NBUF], 0, pd::STALL_LIMIT_CYCLES);
-    ok = ok && potrf_factor_phase<128>(w, 0, i, Lsh, cb, mb, rs, bad);
-    ok = ok && potrf_factor_phase<112>(w, 1, i, Lsh, cb, mb, rs, bad);
-    ok = ok && potrf_factor_phase<96>(w, 2, i, Lsh, cb, mb, rs, bad);
-    ok = ok && potrf_factor_phase<80>(w, 3, i, Lsh, cb, mb, rs, bad);
-    ok = ok && potrf_factor_phase<64>(w, 4, i, Lsh, cb, mb, rs, bad);
-    ok = ok && potrf_factor_phase<48>(w, 5, i, Lsh, cb, mb, rs, bad);
-    ok = ok && potrf_factor_phase<32>(w, 6, i, Lsh, cb, mb, rs, bad);
-    ok = ok && potrf_factor_phase<16>(w, 7, i, Lsh, cb, mb, rs, bad);
-    if (!ok) set_status(status, GPTQ_ERR_TIMEOUT);
-    if (__syncthreads_or(bad) && i == 0) set_status(status, GPTQ_ERR_NOT_PD);
-    if (__syncthreads_or(!ok)) return;
-
-    // L back into A: thread i writes column i (row segments stay coalesced across threads)
-    for (int m = i; m < nbc; ++m)
-        if (i < nbc) A[static_cast<int64_t>(k0 + m) * d + k0 + i] = Lsh[i * pd::LS + m - i + 3];
-
-    // pass 2: column i of L^-1. Warp w's columns are zero above row 32w, so it starts at step
-    // 32w with x_i = 1 at window position i - 32w, and writes zeros for the earlier steps.
-    for (int c = 0; c < 32 * warp; ++c) Dinv[c * pd::NB + i] = 0.0f;
+    float acc[2][4];
+#pragma unroll 1
+    for (int k = 0; k < pd::NSB; ++k) {
+        const int b = k * pd::SB;
+        if (warp == 0) bad = potrf32_warp(S, X, IkT, lbuf, b, lane) || bad;
+        __syncthreads();
+        if (k + 1 == pd::NSB) break;
+        // solve: L_rk = A_rk I_kk^T for the row blocks below (rows b + 32 + 32 grp + ...)
+        const int nrb = pd::NSB - 1 - k;
+        const bool solver = grp < nrb;
+        const int rb = b + pd::SB + pd::SB * grp;
+        if (solver) {
+            zero_acc(acc);
+            block_mma32(S + rb * pd::LD + b, pd::LD, IkT, pd::ILD, ti, tj, acc);
+        }
+        __syncthreads();                      // every row block read before it is overwritten
+        if (solver) {
 #pragma unroll
-    for (int p = 0; p < pd::NB; ++p) w[p] = (p == i - 32 * warp) ? 1.0f : 0.0f;
-    const int q0 = 2 * warp;
-    if (q0 <= 0) potrf_inverse_phase<128>(w, 0, i, nbc, Lsh, rs, Dinv);
-    if (q0 <= 1) potrf_inverse_phase<112>(w, 1, i, nbc, Lsh, rs, Dinv);
-    if (q0 <= 2) potrf_inverse_phase<96>(w, 2, i, nbc, Lsh, rs, Dinv);
-    if (q0 <= 3) potrf_inverse_phase<80>(w, 3, i, nbc, Lsh, rs, Dinv);
-    if (q0 <= 4) potrf_inverse_phase<64>(w, 4, i, nbc, Lsh, rs, Dinv);
-    if (q0 <= 5) potrf_inverse_phase<48>(w, 5, i, nbc, Lsh, rs, Dinv);
-    if (q0 <= 6) potrf_inverse_phase<32>(w, 6, i, nbc, Lsh, rs, Dinv);
-    potrf_inverse_phase<16>(w, 7, i, nbc, Lsh, rs, Dinv);
+            for (int h = 0; h < 2; ++h) {
+                const int r = rb + ti + 16 * h;
+                *reinterpret_cast<float4*>(S + r * pd::LD + b + 4 * tj) =
+                    make_float4(acc[h][0], acc[h][1], acc[h][2], acc[h][3]);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) LT[(4 * tj + q) * pd::LD + (r - b - pd::SB)] = acc[h][q];
+            }
+        }
+        __syncthreads();
+        // update: A_ij -= L_ik L_jk^T over the trailing lower block pairs
+        const int npairs = nrb * (nrb + 1) / 2;
+#pragma unroll 1
+        for (int q = grp; q < npairs; q += pd::THREADS / 128) {
+            int bi, bj;
+            trailing_pair(k, q, bi, bj);
+            zero_acc(acc);
+            block_mma32(S + (pd::SB * bi) * pd::LD + b, pd::LD,
+                        LT + (pd::SB * bj - b - pd::SB), pd::LD, ti, tj, acc);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                float4* o = reinterpret_cast<float4*>(S + (pd::SB * bi + ti + 16 * h) * pd::LD +
+                                                      pd::SB * bj + 4 * tj);
+                float4 v = *o;
+                v.x -= acc[h][0]; v.y -= acc[h][1]; v.z -= acc[h][2]; v.w -= acc[h][3];
+                *o = v;
+            }
+        }
+        __syncthreads();
+    }
+    if (__syncthreads_or(bad) && tid == 0) set_status(status, GPTQ_ERR_NOT_PD);
+
+    // inverse: three rounds over the column blocks
+#pragma unroll 1
+    for (int r = 0, u0 = 0; r < pd::NSB - 1; ++r) {
+        const int nupd = (pd::NSB - 1 - r) * (pd::NSB - r) / 2;
+#pragma unroll 1
+        for (int q = grp; q < nupd; q += pd::THREADS / 128) {
+            const int t = c_inv_upd[u0 + q], i = t & 3, j = (t >> 2) & 3, m = t >> 4;
+            zero_acc(acc);
+            block_mma32(S + (pd::SB * i) * pd::LD + pd::SB * m, pd::LD,
+                        X + (pd::SB * m) * pd::LD + pd::SB * j, pd::LD, ti, tj, acc);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                float4* o = reinterpret_cast<float4*>(X + (pd::SB * i + ti + 16 * h) * pd::LD +
+                                                      pd::SB * j + 4 * tj);
+                float4 v = *o;
+                v.x += acc[h][0]; v.y += acc[h][1]; v.z += acc[h][2]; v.w += acc[h][3];
+                *o = v;
+            }
+        }
+        u0 += nupd;
+        __syncthreads();
+        // X_ij = -I_ii W_ij for i = j + r + 1
+        const int nfin = pd::NSB - 1 - r;
+        const bool fin = grp < nfin;
+        const int j = grp, i = grp + r + 1;
+        if (fin) {
+            zero_acc(acc);
+            block_mma32(X + (pd::SB * i) * pd::LD + pd::SB * i, pd::LD,
+                        X + (pd::SB * i) * pd::LD + pd::SB * j, pd::LD, ti, tj, acc);
+        }
+        __syncthreads();                      // W_ij read before it is overwritten
+        if (fin) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+                *reinterpret_cast<float4*>(X + (pd::SB * i + ti + 16 * h) * pd::LD + pd::SB * j +
+                                           4 * tj) =
+                    make_float4(-acc[h][0], -acc[h][1], -acc[h][2], -acc[h][3]);
+        }
+        __syncthreads();
+    }
+
+    // L back into A (lower triangle of the valid block) and Dinv = X (zero past the edge)
+#pragma unroll 4
+    for (int e = tid; e < pd::NB * pd::NB; e += pd::THREADS) {
+        const int m = e >> 7, i = e & 127;
+        if (m < nbc && i <= m) A[static_cast<int64_t>(k0 + m) * d + k0 + i] = S[m * pd::LD + i];
+    }
+#pragma unroll 2
+    for (int e = tid; e < pd::NB * (pd::NB / 4); e += pd::THREADS) {
+        const int c = e >> 5, i4 = (e & 31) * 4;
+        const float4 v = *reinterpret_cast<const float4*>(X + c * pd::LD + i4);
+        const bool rowok = c < nbc;
+        reinterpret_cast<float4*>(Dinv)[e] =
+            make_float4(rowok && i4 < nbc ? v.x : 0.f, rowok && i4 + 1 < nbc ? v.y : 0.f,
+                        rowok && i4 + 2 < nbc ? v.z : 0.f, rowok && i4 + 3 < nbc ? v.w : 0.f);
+    }
 }
 
 static int g_potrf_smem = 0;
