@@ -106,27 +106,6 @@ __global__ void __launch_bounds__(256) rtn_kernel(const T* __restrict__ W, int64
     }
 }
 
-// fp16 weights, power-of-two groups of 32..256: 32 weights per thread (four 16-byte loads),
-// TPG = group_size / 32 threads per group. Codes stay integer-valued floats until they are
-// packed with byte permutes, so no float-to-int conversions are issued.
-// One chunk of 32 fp16 weights on the exact path (quant_codef), packed and stored like the
-// fast path does. Kept out of line: the fast path reaches it rarely.
-__device__ __noinline__ void rtn_chunk_exact(const __half* w, QParams p, int bits,
-                                             uint8_t* __restrict__ out, int64_t t) {
-    constexpr int E = 32;
-    const float maxqf = static_cast<float>((1 << bits) - 1);
-    if (bits == 4) {
-        for (int b = 0; b < E / 2; ++b) {
-            const float lo = quant_codef(__half2float(w[2 * b]), p, maxqf);
-            const float hi = quant_codef(__half2float(w[2 * b + 1]), p, maxqf);
-            out[(E / 2) * t + b] = static_cast<uint8_t>(small_int_bits(fmaf(hi, 16.0f, lo)));
-        }
-    } else {
-        for (int i = 0; i < E; ++i)
-            out[E * t + i] = static_cast<uint8_t>(small_int_bits(quant_codef(__half2float(w[i]), p, maxqf)));
-    }
-}
-
 namespace rp {
 constexpr int WARPS = 8, THREADS = WARPS * 32;
 constexpr int E = 32;                          // weights per lane
@@ -178,6 +157,65 @@ __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23: integers up to 2^22 sit in the low bits
+
+// 32 codes held as kMagic + code, packed (INT4: two per byte, the even index in the low
+// nibble; else one per byte) and stored with streaming 16-byte stores at chunk t.
+template <bool INT4>
+__device__ __forceinline__ void store_codes(const float (&m)[32], uint8_t* __restrict__ out,
+                                            int t) {
+    if (INT4) {
+        // byte b holds codes 2b (low nibble) and 2b+1: the bit pattern of kMagic + q is
+        // 0x4B400000 + q, so 16 bits(m_2b+1) + bits(m_2b) has q_2b + 16 q_2b+1 in its low byte
+        uint32_t by[16];
+#pragma unroll
+        for (int b = 0; b < 16; ++b)
+            by[b] = (__float_as_uint(m[2 * b + 1]) << 4) + __float_as_uint(m[2 * b]);
+        uint32_t word[4];
+#pragma unroll
+        for (int w4 = 0; w4 < 4; ++w4)
+            word[w4] = __byte_perm(__byte_perm(by[4 * w4], by[4 * w4 + 1], 0x0040),
+                                   __byte_perm(by[4 * w4 + 2], by[4 * w4 + 3], 0x0040), 0x5410);
+        __stcs(reinterpret_cast<uint4*>(out) + t, make_uint4(word[0], word[1], word[2], word[3]));
+    } else {
+        // one code per byte: the low byte of the magic-added pattern is the code
+        uint32_t word[8];
+#pragma unroll
+        for (int w4 = 0; w4 < 8; ++w4)
+            word[w4] = __byte_perm(__byte_perm(__float_as_uint(m[4 * w4]), __float_as_uint(m[4 * w4 + 1]), 0x0040),
+                                   __byte_perm(__float_as_uint(m[4 * w4 + 2]), __float_as_uint(m[4 * w4 + 3]), 0x0040), 0x5410);
+        __stcs(reinterpret_cast<uint4*>(out) + 2 * t, make_uint4(word[0], word[1], word[2], word[3]));
+        __stcs(reinterpret_cast<uint4*>(out) + 2 * t + 1, make_uint4(word[4], word[5], word[6], word[7]));
+    }
+}
+
+// 1/s bracketed by two fp32 values, inv_lo < 1/s < inv_hi, each within 1.5 ulp of it:
+// r = RN(1/s), and the sign of 1 - s r (exact in one fma: s has 11 significant bits, r 24, and
+// |1 - s r| <= 2^-24 on a grid of 2^-34) says on which side of 1/s r lies. An infinite s
+// (range above the fp16 grid) gives 0 for both, the quotient quant_code uses there.
+__device__ __forceinline__ void reciprocal_bracket(float s, float& inv_lo, float& inv_hi) {
+    const float r = __frcp_rn(s);
+    const float e = fmaf(-s, r, 1.0f);
+    const uint32_t rb = __float_as_uint(r);
+    inv_lo = (e > 0.0f) ? r : __uint_as_float(rb - 1u);
+    inv_hi = (e < 0.0f) ? r : __uint_as_float(rb + 1u);
+    if (isinf(s)) inv_lo = inv_hi = 0.0f;
+}
+
+// kMagic + rint(w/s) + z, rint rounding half to even, for fp16 w and s with |w/s| <= 2^8:
+// m1 and m2 round w inv_lo + C and w inv_hi + C (C = z + kMagic, ulp 1) once each. The two
+// products bracket w/s within 4.6e-5, and a w/s that is not a half-integer lies at least
+// 1.2e-4 from every half-integer (w and s are multiples of 2^(e-10) and 2^(e'-10) with |w| >=
+// s/2 near a boundary), so m1 = m2 = the nearest integer, except at an exact tie, where m1
+// and m2 are its two neighbours and the one whose w/s part k = m - C is even is taken (the
+// parity of k is the low bit of bits(m) ^ bits(C): both lie on the ulp-1 grid).
+__device__ __forceinline__ float round_code(float w, float inv_lo, float inv_hi, float C,
+                                            uint32_t Cb) {
+    const float m1 = fmaf(w, inv_lo, C);
+    const float m2 = fmaf(w, inv_hi, C);
+    return ((__float_as_uint(m1) ^ Cb) & 1u) ? m2 : m1;
+}
 
 // fp16 weights, power-of-two groups of 32..256: a lane quantizes 32 consecutive weights
 // (TPG = group_size / 32 lanes per group). Each warp streams its 2 KB per iteration through a
@@ -241,52 +279,27 @@ __global__ void __launch_bounds__(rp::THREADS, 3) rtn_f16_kernel(const __half* _
         }
         if (t >= n_chunks) continue;
         const QParams p = sym ? group_params_sym(mn, mx, maxq) : group_params_stream(mn, mx, maxq);
-        // m = fma(w, 1/scale, zero + 1.5 * 2^23): the product is exact inside the fma and the
-        // single rounding (ulp 1 at 1.5 * 2^23) rounds w/scale + zero to the nearest integer,
-        // half to even, leaving it in the low mantissa bits. Every w lies inside the group's
-        // range, so the rounded value is within 3.1e-5 of the exact w/scale + zero (1/scale is
-        // within 2^-23). A second fma gives the residual r = w/scale + zero - code; if every |r|
-        // stays 6e-5 clear of 1/2, every code is the exact rounding and lies in [0, maxq] (no
-        // clamp); otherwise the chunk is redone on the exact path.
-        constexpr float kMagic = 12582912.0f;                  // 1.5 * 2^23
+        // every code in one rounding per bracket end (round_code), so ties need no second path
+        float inv_lo, inv_hi;
+        reciprocal_bracket(p.scale, inv_lo, inv_hi);
         const float C = p.zero + kMagic;                         // exact: zero is an integer
+        const uint32_t Cb = __float_as_uint(C);
         float m[32];
-        float dev = 0.0f;
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
             const float2 f = __half22float2(hp[i]);
-            m[2 * i] = fmaf(f.x, p.inv_scale, C);
-            m[2 * i + 1] = fmaf(f.y, p.inv_scale, C);
-            const float r0 = fmaf(f.x, p.inv_scale, C - m[2 * i]);      // C - m is exact
-            const float r1 = fmaf(f.y, p.inv_scale, C - m[2 * i + 1]);
-            dev = fmaxf(dev, fmaxf(fabsf(r0), fabsf(r1)));
+            m[2 * i] = round_code(f.x, inv_lo, inv_hi, C, Cb);
+            m[2 * i + 1] = round_code(f.y, inv_lo, inv_hi, C, Cb);
         }
-        if (dev > 0.5f - 6.0e-5f) {
-            // rare: a code within 6e-5 of a rounding boundary; redo the chunk on the exact path
-            rtn_chunk_exact(reinterpret_cast<const __half*>(mine), p, bits, out, t);
-        } else if (INT4) {
-            // byte b holds codes 2b (low nibble) and 2b+1: (M + q0) + 16 q1 has q0 + 16 q1 in its
-            // low byte (exact: all values are integers below 2^24)
-            uint32_t by[16];
+        // codes are monotone in w: only a tie at the group's extremes can land one step past
+        // [0, maxq] (rint(hi/s) + z <= maxq + 1), and then every lane of the group clamps
+        const float maxqf = static_cast<float>(maxq);
+        if (round_code(mx, inv_lo, inv_hi, C, Cb) > kMagic + maxqf ||
+            round_code(mn, inv_lo, inv_hi, C, Cb) < kMagic) {
 #pragma unroll
-            for (int b = 0; b < 16; ++b)
-                by[b] = __float_as_uint(fmaf(m[2 * b + 1] - kMagic, 16.0f, m[2 * b]));
-            uint32_t word[4];
-#pragma unroll
-            for (int w4 = 0; w4 < 4; ++w4)
-                word[w4] = __byte_perm(__byte_perm(by[4 * w4], by[4 * w4 + 1], 0x0040),
-                                       __byte_perm(by[4 * w4 + 2], by[4 * w4 + 3], 0x0040), 0x5410);
-            __stcs(reinterpret_cast<uint4*>(out) + t, make_uint4(word[0], word[1], word[2], word[3]));
-        } else {
-            // one code per byte: the low byte of the magic-added pattern is the code
-            uint32_t word[8];
-#pragma unroll
-            for (int w4 = 0; w4 < 8; ++w4)
-                word[w4] = __byte_perm(__byte_perm(__float_as_uint(m[4 * w4]), __float_as_uint(m[4 * w4 + 1]), 0x0040),
-                                       __byte_perm(__float_as_uint(m[4 * w4 + 2]), __float_as_uint(m[4 * w4 + 3]), 0x0040), 0x5410);
-            __stcs(reinterpret_cast<uint4*>(out) + 2 * t, make_uint4(word[0], word[1], word[2], word[3]));
-            __stcs(reinterpret_cast<uint4*>(out) + 2 * t + 1, make_uint4(word[4], word[5], word[6], word[7]));
+            for (int i = 0; i < 32; ++i) m[i] = fminf(fmaxf(m[i], kMagic), kMagic + maxqf);
         }
+        store_codes<INT4>(m, out, t);
         if ((t & (TPG - 1)) == 0) {
             scales[t / TPG] = half_bits(p.scale);
             zeros[t / TPG] = half_bits(p.zero);
