@@ -183,32 +183,32 @@ gptq_status gather_w_launch(const void* W, int w_dtype, int d_out, int d_in, con
 // ---------------------------------------------------------------------------------------
 // blocked Cholesky
 // ---------------------------------------------------------------------------------------
-// ---- diagonal block: one CTA of 512 threads factors the 128 x 128 block A[k0:, k0:] and
+// ---- diagonal block: one CTA of 384 threads factors the 128 x 128 block A[k0:, k0:] and
 // inverts its factor, blocked in four sub-panels of 32 columns (right-looking):
 //   for k = 0..3 (b = 32k):
-//     factor   one warp: L_kk = chol(A_kk) and I_kk = L_kk^-1, 32 steps in registers
-//     solve    L_rk = A_rk I_kk^T for the row blocks r below (all threads)
+//     factor   warp 0: L_kk = chol(A_kk), 32 steps in registers
+//     solve    one thread per row below: L_rk = A_rk L_kk^-T by forward substitution;
+//              at the same time one more warp forms I_kk = L_kk^-1 (one column per lane)
 //     update   A_ij -= L_ik L_jk^T for the trailing lower blocks (all threads)
 //   inverse    X = L^-1 by block forward substitution, column blocks in parallel:
 //              W_ij = sum_{m<i} L_im X_mj accumulated right-looking, X_ij = -I_ii W_ij
-// In the factor warp, lane i holds row i of A_kk and column i of I_kk. At step c the pivot
-// a_cc is broadcast, lane i forms L[i][c] = a_ic / sqrt(a_cc) and its inverse column entry
-// y_c = w_c / L_cc, then applies the rank-1 update to its row (a_im -= L[i][c] L[m][c]) and
-// the substitution update to its inverse column (w_m -= L[m][c] y_c); both updates take the
-// same broadcast L[m][c]. Lane c+1 computes the next pivot first, so the chain from one
-// pivot to the next is a reciprocal square root, two multiply-adds and one shuffle.
-// The block products run on 2 x 4 register tiles per thread, 128 threads per 32 x 32 block.
+// In the factor warp, lane i holds row i of A_kk. At step c the pivot a_cc is broadcast by
+// shuffle, lane i forms L[i][c] = a_ic / sqrt(a_cc), publishes it in row c of LkT (L_kk
+// transposed, the exchange buffer), and applies the rank-1 update a_im -= L[i][c] L[m][c] to
+// its row. Lane c+1 computes the next pivot before the exchange, so the chain from one pivot
+// to the next is a reciprocal square root, two multiply-adds and one shuffle.
+// Each 32 x 32 block product is one warp's, on 4 x 8 register tiles (12 operand values per 32
+// multiply-adds: the products are bound by shared-memory bandwidth, not by the FMA pipe).
 // Rows and columns beyond the matrix edge are padded with the identity.
 namespace pd {
-constexpr int NB = 128, SB = 32, NSB = NB / SB, THREADS = 512;
+constexpr int NB = 128, SB = 32, NSB = NB / SB, THREADS = 384, NWARPS = THREADS / 32;
 constexpr int LD = NB + 4;          // row stride (floats) of S, X and LT: 16-byte rows, and
                                     // consecutive rows start four banks apart
-constexpr int ILD = SB + 4;         // row stride of IkT
+constexpr int KLD = SB + 4;         // row stride of LkT
 // S [NB][LD]: the block, overwritten by L; X [NB][LD]: L^-1 (its blocks below the diagonal
 // hold the partial sums W until they are final); LT [SB][LD]: the current sub-panel's L_rk,
-// transposed; IkT [SB][ILD]: I_kk transposed; lbuf [2][SB]: the factor warp's column
-// exchange; then the stall-test mbarrier
-constexpr int SMEM_FLOATS = 2 * NB * LD + SB * LD + SB * ILD + 2 * SB;
+// transposed; LkT [SB][KLD]: L_kk transposed; rinv [SB]: 1 / L_cc; then the stall-test mbarrier
+constexpr int SMEM_FLOATS = 2 * NB * LD + SB * LD + SB * KLD + SB;
 constexpr int SMEM = SMEM_FLOATS * 4 + 16;
 constexpr long long STALL_LIMIT_CYCLES = 2000000;   // about 1 ms
 }  // namespace pd
@@ -228,23 +228,19 @@ __device__ __forceinline__ float rsqrt_nr(float x) {
     return fmaf(0.5f * r, e, r);
 }
 
-// One warp: L_kk and I_kk of the 32 x 32 block at S[b:, b:]. Writes L_kk (zeros above the
-// diagonal) back into S, I_kk into X's diagonal block and, transposed, into IkT. Returns
-// true on a pivot that is not a positive normal number. Each step's column L[:, c] is
-// exchanged through lbuf (two buffers: a lane writes step c+2's column only after every lane
-// has passed step c+1's __syncwarp, so after it has read step c's); the pivot goes by shuffle.
-__device__ __forceinline__ bool potrf32_warp(float* S, float* X, float* IkT, float* lbuf, int b,
-                                            int lane) {
+// One warp: L_kk of the 32 x 32 block at S[b:, b:], written back into S (zeros above the
+// diagonal) and, transposed, into LkT; rinv[c] = 1 / L_cc. Returns true on a pivot that is
+// not a positive normal number. Each row c of LkT is written once (at step c) and read after
+// the step's __syncwarp, so it is also the exchange buffer.
+__device__ __forceinline__ bool potrf32_warp(float* S, float* LkT, float* rinv, int b, int lane) {
     constexpr unsigned FULL = 0xffffffffu;
-    float dr[pd::SB], w[pd::SB];
+    float dr[pd::SB];
     const float4* src = reinterpret_cast<const float4*>(S + (b + lane) * pd::LD + b);
 #pragma unroll
     for (int q = 0; q < pd::SB / 4; ++q) {
         const float4 v = src[q];
         dr[4 * q] = v.x; dr[4 * q + 1] = v.y; dr[4 * q + 2] = v.z; dr[4 * q + 3] = v.w;
     }
-#pragma unroll
-    for (int m = 0; m < pd::SB; ++m) w[m] = (m == lane) ? 1.0f : 0.0f;
     bool bad = false;
     float p = __shfl_sync(FULL, dr[0], 0);
 #pragma unroll
@@ -252,65 +248,98 @@ __device__ __forceinline__ bool potrf32_warp(float* S, float* X, float* IkT, flo
         bad = bad || !(p >= 1.17549435e-38f && p <= 3.40282347e38f);
         const float r = rsqrt_nr(p);                       // 1 / L_cc
         const float l = (lane >= c) ? dr[c] * r : 0.0f;     // L[lane][c]
-        const float y = w[c] * r;                           // I_kk[c][lane]
         dr[c] = l;
-        w[c] = y;
+        float* lk = LkT + c * pd::KLD;
+        lk[lane] = l;
+        if (lane == 0) rinv[c] = r;
         if (c + 1 == pd::SB) break;
-        float* lb = lbuf + (c & 1) * pd::SB;
-        lb[lane] = l;
         p = __shfl_sync(FULL, fmaf(-l, l, dr[c + 1]), c + 1);
         __syncwarp();
 #pragma unroll
         for (int m4 = (c + 1) & ~3; m4 < pd::SB; m4 += 4) {
-            const float4 v = *reinterpret_cast<const float4*>(lb + m4);   // L[m4 .. m4+3][c]
+            const float4 v = *reinterpret_cast<const float4*>(lk + m4);   // L[m4 .. m4+3][c]
             const float lv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                if (m4 + u <= c) continue;
-                dr[m4 + u] = fmaf(-l, lv[u], dr[m4 + u]);
-                w[m4 + u] = fmaf(-lv[u], y, w[m4 + u]);
-            }
+            for (int u = 0; u < 4; ++u)
+                if (m4 + u > c) dr[m4 + u] = fmaf(-l, lv[u], dr[m4 + u]);
         }
     }
     float4* dst = reinterpret_cast<float4*>(S + (b + lane) * pd::LD + b);
-    float4* idst = reinterpret_cast<float4*>(IkT + lane * pd::ILD);
 #pragma unroll
-    for (int q = 0; q < pd::SB / 4; ++q) {
+    for (int q = 0; q < pd::SB / 4; ++q)
         dst[q] = make_float4(dr[4 * q], dr[4 * q + 1], dr[4 * q + 2], dr[4 * q + 3]);
-        idst[q] = make_float4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
-    }
-#pragma unroll
-    for (int c = 0; c < pd::SB; ++c) X[(b + c) * pd::LD + b + lane] = w[c];
     return bad;
 }
 
-// acc[h][q] += sum_m P[ti + 16h][m] Q[m][4 tj + q], m < 32 (P, Q row-major, 16-byte rows)
-__device__ __forceinline__ void block_mma32(const float* P, int ldp, const float* Q, int ldq,
-                                            int ti, int tj, float (&acc)[2][4]) {
+// One thread: v[0..31] <- v L_kk^-T in place (solve x L_kk^T = v by forward substitution:
+// x_c = v_c / L_cc, then v_m -= x_c L[m][c] for m > c), with L_kk from LkT and rinv.
+__device__ __forceinline__ void trsv32(float (&v)[pd::SB], const float* LkT, const float* rinv) {
 #pragma unroll
-    for (int m4 = 0; m4 < pd::SB; m4 += 4) {
-        const float4 a0 = *reinterpret_cast<const float4*>(P + ti * ldp + m4);
-        const float4 a1 = *reinterpret_cast<const float4*>(P + (ti + 16) * ldp + m4);
-        const float av[2][4] = {{a0.x, a0.y, a0.z, a0.w}, {a1.x, a1.y, a1.z, a1.w}};
+    for (int c = 0; c < pd::SB; ++c) {
+        const float x = v[c] * rinv[c];
+        v[c] = x;
+        const float* lk = LkT + c * pd::KLD;
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const float4 q = *reinterpret_cast<const float4*>(Q + (m4 + u) * ldq + 4 * tj);
+        for (int m4 = (c + 1) & ~3; m4 < pd::SB; m4 += 4) {
+            const float4 q = *reinterpret_cast<const float4*>(lk + m4);
+            const float lv[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                acc[h][0] = fmaf(av[h][u], q.x, acc[h][0]);
-                acc[h][1] = fmaf(av[h][u], q.y, acc[h][1]);
-                acc[h][2] = fmaf(av[h][u], q.z, acc[h][2]);
-                acc[h][3] = fmaf(av[h][u], q.w, acc[h][3]);
-            }
+            for (int u = 0; u < 4; ++u)
+                if (m4 + u > c) v[m4 + u] = fmaf(-x, lv[u], v[m4 + u]);
         }
     }
 }
 
-__device__ __forceinline__ void zero_acc(float (&acc)[2][4]) {
+// One warp, one 32 x 32 block: acc[h][q] += sum_m P[ti + 8h][m] Q[m][col(q)], m < 32, with
+// ti = lane / 4, tj = lane % 4, col(q) = 4 tj + q (q < 4) and 16 + 4 tj + q - 4 (q >= 4).
+// P and Q are row-major with 16-byte rows; a P load is shared by the four lanes of a row
+// group, a Q load by the eight lanes of a column group.
+__device__ __forceinline__ void block_mma32(const float* P, int ldp, const float* Q, int ldq,
+                                            int lane, float (&acc)[4][8]) {
+    const int ti = lane >> 2, tj = lane & 3;
 #pragma unroll
-    for (int h = 0; h < 2; ++h)
+    for (int h = 0; h < 4; ++h)
 #pragma unroll
-        for (int q = 0; q < 4; ++q) acc[h][q] = 0.0f;
+        for (int q = 0; q < 8; ++q) acc[h][q] = 0.0f;
+#pragma unroll 2
+    for (int m4 = 0; m4 < pd::SB; m4 += 4) {
+        float a[4][4];
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+            const float4 v = *reinterpret_cast<const float4*>(P + (ti + 8 * h) * ldp + m4);
+            a[h][0] = v.x; a[h][1] = v.y; a[h][2] = v.z; a[h][3] = v.w;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const float* qr = Q + (m4 + u) * ldq + 4 * tj;
+            const float4 q0 = *reinterpret_cast<const float4*>(qr);
+            const float4 q1 = *reinterpret_cast<const float4*>(qr + 16);
+            const float qv[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+#pragma unroll
+            for (int h = 0; h < 4; ++h)
+#pragma unroll
+                for (int q = 0; q < 8; ++q) acc[h][q] = fmaf(a[h][u], qv[q], acc[h][q]);
+        }
+    }
+}
+
+// The 4 x 8 tile of block_mma32 in a row-major block C: op(C[r][c], acc) for each entry.
+template <typename Op>
+__device__ __forceinline__ void block_tile_apply(float* C, int ldc, int lane,
+                                                 const float (&acc)[4][8], Op op) {
+    const int ti = lane >> 2, tj = lane & 3;
+#pragma unroll
+    for (int h = 0; h < 4; ++h)
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            float4* o = reinterpret_cast<float4*>(C + (ti + 8 * h) * ldc + 16 * half + 4 * tj);
+            float4 v = *o;
+            v.x = op(v.x, acc[h][4 * half]);
+            v.y = op(v.y, acc[h][4 * half + 1]);
+            v.z = op(v.z, acc[h][4 * half + 2]);
+            v.w = op(v.w, acc[h][4 * half + 3]);
+            *o = v;
+        }
 }
 
 // the (bi, bj) block pair number q of the trailing lower blocks k+1 <= bj <= bi < 4
@@ -343,33 +372,37 @@ __global__ void __launch_bounds__(pd::THREADS, 1) potrf_diag_kernel(float* __res
     float* S = sm;                            // [NB][LD]
     float* X = S + pd::NB * pd::LD;           // [NB][LD]
     float* LT = X + pd::NB * pd::LD;          // [SB][LD]
-    float* IkT = LT + pd::SB * pd::LD;        // [SB][ILD]
-    float* lbuf = IkT + pd::SB * pd::ILD;     // [2][SB]
-    uint64_t* mb = reinterpret_cast<uint64_t*>(lbuf + 2 * pd::SB);
+    float* LkT = LT + pd::SB * pd::LD;        // [SB][KLD]
+    float* rinv = LkT + pd::SB * pd::KLD;     // [SB]
+    uint64_t* mb = reinterpret_cast<uint64_t*>(rinv + pd::SB);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    // block-product tile of this thread: 128 threads per 32 x 32 block
-    const int grp = tid >> 7, gw = (tid >> 5) & 3;
-    const int ti = (lane >> 3) + 4 * gw, tj = lane & 7;
 
-    // S = the block's lower triangle (identity past the edge); X = 0
-#pragma unroll 2
+    // S = the block's lower triangle (rows below nbc: 16-byte async copies of the chunks that
+    // reach the lower triangle; rows from nbc on: the identity); X = 0
     for (int e = tid; e < pd::NB * (pd::NB / 4); e += pd::THREADS) {
         const int r = e >> 5, c4 = (e & 31) * 4;
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (r < nbc && c4 <= r && c4 < nbc)
-            v = *reinterpret_cast<const float4*>(A + static_cast<int64_t>(k0 + r) * d + k0 + c4);
-        const float vv[4] = {v.x, v.y, v.z, v.w};
-        float o[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-            o[u] = (r < nbc) ? (c4 + u <= r ? vv[u] : 0.0f) : (c4 + u == r ? 1.0f : 0.0f);
-        *reinterpret_cast<float4*>(S + r * pd::LD + c4) = make_float4(o[0], o[1], o[2], o[3]);
+        float* dst = S + r * pd::LD + c4;
+        if (r < nbc && c4 <= r) {
+            cp_async16(dst, A + static_cast<int64_t>(k0 + r) * d + k0 + c4);
+        } else {
+            const bool eye = r >= nbc && (r >> 2) == (c4 >> 2);
+            const int u = r & 3;
+            *reinterpret_cast<float4*>(dst) =
+                make_float4(eye && u == 0 ? 1.f : 0.f, eye && u == 1 ? 1.f : 0.f,
+                            eye && u == 2 ? 1.f : 0.f, eye && u == 3 ? 1.f : 0.f);
+        }
         *reinterpret_cast<float4*>(X + r * pd::LD + c4) = make_float4(0.f, 0.f, 0.f, 0.f);
     }
+    cp_async_commit();
     if (tid == 0) {
         mbar_init(mb, 1);
         fence_mbar_init();
     }
+    cp_async_wait<0>();
+    __syncthreads();
+    // the copied diagonal chunks also brought up to three entries above the diagonal
+    if (tid < nbc)
+        for (int c = tid + 1; c <= (tid | 3); ++c) S[tid * pd::LD + c] = 0.0f;
     __syncthreads();
     if (*(volatile int*)&g_factor_stall) {
         const bool ok = mbar_wait_cycles(mb, 0, pd::STALL_LIMIT_CYCLES);
@@ -378,50 +411,49 @@ __global__ void __launch_bounds__(pd::THREADS, 1) potrf_diag_kernel(float* __res
     }
 
     bool bad = false;
-    float acc[2][4];
+    float acc[4][8];
 #pragma unroll 1
     for (int k = 0; k < pd::NSB; ++k) {
         const int b = k * pd::SB;
-        if (warp == 0) bad = potrf32_warp(S, X, IkT, lbuf, b, lane) || bad;
+        if (warp == 0) bad = potrf32_warp(S, LkT, rinv, b, lane) || bad;
+        __syncthreads();
+        // solve (warps 1 .. nrb, one row each lane) and I_kk (the next warp, one column each)
+        const int nrb = pd::NSB - 1 - k;
+        float v[pd::SB];
+        if (warp >= 1 && warp <= nrb) {
+            const int r = b + pd::SB * warp + lane;
+            float4* row = reinterpret_cast<float4*>(S + r * pd::LD + b);
+#pragma unroll
+            for (int q = 0; q < pd::SB / 4; ++q) {
+                const float4 t = row[q];
+                v[4 * q] = t.x; v[4 * q + 1] = t.y; v[4 * q + 2] = t.z; v[4 * q + 3] = t.w;
+            }
+            trsv32(v, LkT, rinv);
+#pragma unroll
+            for (int q = 0; q < pd::SB / 4; ++q)
+                row[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+#pragma unroll
+            for (int c = 0; c < pd::SB; ++c) LT[c * pd::LD + (r - b - pd::SB)] = v[c];
+        } else if (warp == nrb + 1) {
+            // column `lane` of I_kk: solve L_kk y = e_lane; as rows, y^T = e_lane^T L_kk^-T
+#pragma unroll
+            for (int m = 0; m < pd::SB; ++m) v[m] = (m == lane) ? 1.0f : 0.0f;
+            trsv32(v, LkT, rinv);
+#pragma unroll
+            for (int c = 0; c < pd::SB; ++c) X[(b + c) * pd::LD + b + lane] = v[c];
+        }
         __syncthreads();
         if (k + 1 == pd::NSB) break;
-        // solve: L_rk = A_rk I_kk^T for the row blocks below (rows b + 32 + 32 grp + ...)
-        const int nrb = pd::NSB - 1 - k;
-        const bool solver = grp < nrb;
-        const int rb = b + pd::SB + pd::SB * grp;
-        if (solver) {
-            zero_acc(acc);
-            block_mma32(S + rb * pd::LD + b, pd::LD, IkT, pd::ILD, ti, tj, acc);
-        }
-        __syncthreads();                      // every row block read before it is overwritten
-        if (solver) {
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int r = rb + ti + 16 * h;
-                *reinterpret_cast<float4*>(S + r * pd::LD + b + 4 * tj) =
-                    make_float4(acc[h][0], acc[h][1], acc[h][2], acc[h][3]);
-#pragma unroll
-                for (int q = 0; q < 4; ++q) LT[(4 * tj + q) * pd::LD + (r - b - pd::SB)] = acc[h][q];
-            }
-        }
-        __syncthreads();
-        // update: A_ij -= L_ik L_jk^T over the trailing lower block pairs
+        // update: A_ij -= L_ik L_jk^T over the trailing lower block pairs, one warp each
         const int npairs = nrb * (nrb + 1) / 2;
 #pragma unroll 1
-        for (int q = grp; q < npairs; q += pd::THREADS / 128) {
+        for (int q = warp; q < npairs; q += pd::NWARPS) {
             int bi, bj;
             trailing_pair(k, q, bi, bj);
-            zero_acc(acc);
             block_mma32(S + (pd::SB * bi) * pd::LD + b, pd::LD,
-                        LT + (pd::SB * bj - b - pd::SB), pd::LD, ti, tj, acc);
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                float4* o = reinterpret_cast<float4*>(S + (pd::SB * bi + ti + 16 * h) * pd::LD +
-                                                      pd::SB * bj + 4 * tj);
-                float4 v = *o;
-                v.x -= acc[h][0]; v.y -= acc[h][1]; v.z -= acc[h][2]; v.w -= acc[h][3];
-                *o = v;
-            }
+                        LT + (pd::SB * bj - b - pd::SB), pd::LD, lane, acc);
+            block_tile_apply(S + (pd::SB * bi) * pd::LD + pd::SB * bj, pd::LD, lane, acc,
+                             [](float c, float a) { return c - a; });
         }
         __syncthreads();
     }
@@ -432,49 +464,42 @@ __global__ void __launch_bounds__(pd::THREADS, 1) potrf_diag_kernel(float* __res
     for (int r = 0, u0 = 0; r < pd::NSB - 1; ++r) {
         const int nupd = (pd::NSB - 1 - r) * (pd::NSB - r) / 2;
 #pragma unroll 1
-        for (int q = grp; q < nupd; q += pd::THREADS / 128) {
+        for (int q = warp; q < nupd; q += pd::NWARPS) {
             const int t = c_inv_upd[u0 + q], i = t & 3, j = (t >> 2) & 3, m = t >> 4;
-            zero_acc(acc);
             block_mma32(S + (pd::SB * i) * pd::LD + pd::SB * m, pd::LD,
-                        X + (pd::SB * m) * pd::LD + pd::SB * j, pd::LD, ti, tj, acc);
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                float4* o = reinterpret_cast<float4*>(X + (pd::SB * i + ti + 16 * h) * pd::LD +
-                                                      pd::SB * j + 4 * tj);
-                float4 v = *o;
-                v.x += acc[h][0]; v.y += acc[h][1]; v.z += acc[h][2]; v.w += acc[h][3];
-                *o = v;
-            }
+                        X + (pd::SB * m) * pd::LD + pd::SB * j, pd::LD, lane, acc);
+            block_tile_apply(X + (pd::SB * i) * pd::LD + pd::SB * j, pd::LD, lane, acc,
+                             [](float c, float a) { return c + a; });
         }
         u0 += nupd;
         __syncthreads();
-        // X_ij = -I_ii W_ij for i = j + r + 1
+        // X_ij = -I_ii W_ij for i = j + r + 1 (warp j)
         const int nfin = pd::NSB - 1 - r;
-        const bool fin = grp < nfin;
-        const int j = grp, i = grp + r + 1;
-        if (fin) {
-            zero_acc(acc);
+        const bool fin = warp < nfin;
+        const int j = warp, i = warp + r + 1;
+        if (fin)
             block_mma32(X + (pd::SB * i) * pd::LD + pd::SB * i, pd::LD,
-                        X + (pd::SB * i) * pd::LD + pd::SB * j, pd::LD, ti, tj, acc);
-        }
+                        X + (pd::SB * i) * pd::LD + pd::SB * j, pd::LD, lane, acc);
         __syncthreads();                      // W_ij read before it is overwritten
-        if (fin) {
-#pragma unroll
-            for (int h = 0; h < 2; ++h)
-                *reinterpret_cast<float4*>(X + (pd::SB * i + ti + 16 * h) * pd::LD + pd::SB * j +
-                                           4 * tj) =
-                    make_float4(-acc[h][0], -acc[h][1], -acc[h][2], -acc[h][3]);
-        }
+        if (fin)
+            block_tile_apply(X + (pd::SB * i) * pd::LD + pd::SB * j, pd::LD, lane, acc,
+                             [](float, float a) { return -a; });
         __syncthreads();
     }
 
-    // L back into A (lower triangle of the valid block) and Dinv = X (zero past the edge)
-#pragma unroll 4
-    for (int e = tid; e < pd::NB * pd::NB; e += pd::THREADS) {
-        const int m = e >> 7, i = e & 127;
-        if (m < nbc && i <= m) A[static_cast<int64_t>(k0 + m) * d + k0 + i] = S[m * pd::LD + i];
+    // L back into A (lower triangle of the valid block; 16-byte stores below the diagonal
+    // chunk) and Dinv = X (zero past the edge)
+    for (int e = tid; e < pd::NB * (pd::NB / 4); e += pd::THREADS) {
+        const int m = e >> 5, c4 = (e & 31) * 4;
+        if (m >= nbc || c4 > m) continue;
+        float* dst = A + static_cast<int64_t>(k0 + m) * d + k0 + c4;
+        const float* src = S + m * pd::LD + c4;
+        if (c4 + 3 <= m) {
+            *reinterpret_cast<float4*>(dst) = *reinterpret_cast<const float4*>(src);
+        } else {
+            for (int c = 0; c <= m - c4; ++c) dst[c] = src[c];
+        }
     }
-#pragma unroll 2
     for (int e = tid; e < pd::NB * (pd::NB / 4); e += pd::THREADS) {
         const int c = e >> 5, i4 = (e & 31) * 4;
         const float4 v = *reinterpret_cast<const float4*>(X + c * pd::LD + i4);

@@ -150,14 +150,6 @@ __device__ __forceinline__ QParams group_params_stream(float xmin, float xmax, i
     return p;
 }
 
-__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
-
 constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23: integers up to 2^22 sit in the low bits
 
 // 32 codes held as kMagic + code, packed (INT4: two per byte, the even index in the low
