@@ -185,23 +185,27 @@ gptq_status gather_w_launch(const void* W, int w_dtype, int d_out, int d_in, con
 // ---------------------------------------------------------------------------------------
 // ---- diagonal block: one CTA of 384 threads factors the 128 x 128 block A[k0:, k0:] and
 // inverts its factor, blocked in four sub-panels of 32 columns (right-looking):
-//   for k = 0..3 (b = 32k):
-//     factor   warp 0: L_kk = chol(A_kk), 32 steps in registers
-//     solve    one thread per row below: L_rk = A_rk L_kk^-T by forward substitution;
-//              at the same time one more warp forms I_kk = L_kk^-1 (one column per lane)
-//     update   A_ij -= L_ik L_jk^T for the trailing lower blocks (all threads)
-//   inverse    X = L^-1 by block forward substitution, column blocks in parallel:
-//              W_ij = sum_{m<i} L_im X_mj accumulated right-looking, X_ij = -I_ii W_ij
-// In the factor warp, lane i holds row i of A_kk. At step c the pivot a_cc is broadcast by
-// shuffle, lane i forms L[i][c] = a_ic / sqrt(a_cc), publishes it in row c of LkT (L_kk
-// transposed, the exchange buffer), and applies the rank-1 update a_im -= L[i][c] L[m][c] to
-// its row. Lane c+1 computes the next pivot before the exchange, so the chain from one pivot
-// to the next is a reciprocal square root, two multiply-adds and one shuffle.
+//   for k = 0..3 (b = 32k), three phases separated by block barriers:
+//     A(k)  warp 0 factors L_kk = chol(A_kk), 32 steps in registers, while other warps run
+//           the block products that are ready: the rest of the previous sub-panel's trailing
+//           update and the inverse's partial sums W_ij += L_im X_mj
+//     B(k)  one thread per row below solves L_rk = A_rk L_kk^-T (forward substitution),
+//           and one more warp forms I_kk = L_kk^-1 (one column per lane)
+//     C(k)  the trailing update of block column k+1 (what A(k+1) and B(k+1) read) and the
+//           inverse blocks that I_kk completes, X_kj = -I_kk W_kj
+// so the inverse X = L^-1 (block forward substitution, accumulated right-looking) is done
+// with the factorisation. In the factor warp, lane i holds row i of A_kk. At step c the pivot
+// a_cc is broadcast by shuffle, lane i forms L[i][c] = a_ic / sqrt(a_cc), publishes it in row c
+// of LkT (L_kk transposed, the exchange buffer), and applies the rank-1 update a_im -= L[i][c]
+// L[m][c] to its row. Lane c+1 computes the next pivot before the exchange, so the chain from
+// one pivot to the next is a reciprocal square root, two multiply-adds and one shuffle.
 // Each 32 x 32 block product is one warp's, on 4 x 8 register tiles (12 operand values per 32
 // multiply-adds: the products are bound by shared-memory bandwidth, not by the FMA pipe).
+// Dinv is written block by block as blocks become final (the blocks above the diagonal, all
+// zero, first); L itself is not written back: nothing reads the diagonal block afterwards.
 // Rows and columns beyond the matrix edge are padded with the identity.
 namespace pd {
-constexpr int NB = 128, SB = 32, NSB = NB / SB, THREADS = 384, NWARPS = THREADS / 32;
+constexpr int NB = 128, SB = 32, NSB = NB / SB, THREADS = 384;
 constexpr int LD = NB + 4;          // row stride (floats) of S, X and LT: 16-byte rows, and
                                     // consecutive rows start four banks apart
 constexpr int KLD = SB + 4;         // row stride of LkT
@@ -213,12 +217,12 @@ constexpr int SMEM = SMEM_FLOATS * 4 + 16;
 constexpr long long STALL_LIMIT_CYCLES = 2000000;   // about 1 ms
 }  // namespace pd
 
-// Test switch for the bounded-wait path (set by gptq_test_stall_factor): when nonzero, every
-// thread of the diagonal-block kernel first waits on an mbarrier that nothing arrives at. The
-// wait gives up after STALL_LIMIT_CYCLES, the kernel records GPTQ_ERR_TIMEOUT and returns, and
-// the rest of the factorisation skips its work on the status word. No copy or MMA is in
-// flight when it gives up.
-__device__ int g_factor_stall = 0;
+// Test switch for the bounded-wait path (set by gptq_test_stall_factor, passed to each launch):
+// when nonzero, every thread of the diagonal-block kernel first waits on an mbarrier that
+// nothing arrives at. The wait gives up after STALL_LIMIT_CYCLES, the kernel records
+// GPTQ_ERR_TIMEOUT and returns, and the rest of the factorisation skips its work on the status
+// word. No copy or MMA is in flight when it gives up.
+static int g_factor_stall = 0;
 
 // 1/sqrt(x): the hardware estimate refined by one Newton-Raphson step r' = r (1 + (1 - x r^2)/2)
 __device__ __forceinline__ float rsqrt_nr(float x) {
@@ -290,22 +294,23 @@ __device__ __forceinline__ void trsv32(float (&v)[pd::SB], const float* LkT, con
     }
 }
 
-// One warp, one 32 x 32 block: acc[h][q] += sum_m P[ti + 8h][m] Q[m][col(q)], m < 32, with
-// ti = lane / 4, tj = lane % 4, col(q) = 4 tj + q (q < 4) and 16 + 4 tj + q - 4 (q >= 4).
-// P and Q are row-major with 16-byte rows; a P load is shared by the four lanes of a row
-// group, a Q load by the eight lanes of a column group.
+// One warp, H x 8 rows of a 32 x 32 block (H = 4: the whole block): acc[h][q] = sum_m
+// P[ti + 8h][m] Q[m][col(q)], m < 32, with ti = lane / 4, tj = lane % 4, col(q) = 4 tj + q
+// (q < 4) and 16 + 4 tj + q - 4 (q >= 4). P and Q are row-major with 16-byte rows; a P load is
+// shared by the four lanes of a row group, a Q load by the eight lanes of a column group.
+template <int H>
 __device__ __forceinline__ void block_mma32(const float* P, int ldp, const float* Q, int ldq,
-                                            int lane, float (&acc)[4][8]) {
+                                            int lane, float (&acc)[H][8]) {
     const int ti = lane >> 2, tj = lane & 3;
 #pragma unroll
-    for (int h = 0; h < 4; ++h)
+    for (int h = 0; h < H; ++h)
 #pragma unroll
         for (int q = 0; q < 8; ++q) acc[h][q] = 0.0f;
 #pragma unroll 2
     for (int m4 = 0; m4 < pd::SB; m4 += 4) {
-        float a[4][4];
+        float a[H][4];
 #pragma unroll
-        for (int h = 0; h < 4; ++h) {
+        for (int h = 0; h < H; ++h) {
             const float4 v = *reinterpret_cast<const float4*>(P + (ti + 8 * h) * ldp + m4);
             a[h][0] = v.x; a[h][1] = v.y; a[h][2] = v.z; a[h][3] = v.w;
         }
@@ -316,20 +321,20 @@ __device__ __forceinline__ void block_mma32(const float* P, int ldp, const float
             const float4 q1 = *reinterpret_cast<const float4*>(qr + 16);
             const float qv[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
 #pragma unroll
-            for (int h = 0; h < 4; ++h)
+            for (int h = 0; h < H; ++h)
 #pragma unroll
                 for (int q = 0; q < 8; ++q) acc[h][q] = fmaf(a[h][u], qv[q], acc[h][q]);
         }
     }
 }
 
-// The 4 x 8 tile of block_mma32 in a row-major block C: op(C[r][c], acc) for each entry.
-template <typename Op>
+// The H x 8 tile of block_mma32 in a row-major block C: op(C[r][c], acc) for each entry.
+template <int H, typename Op>
 __device__ __forceinline__ void block_tile_apply(float* C, int ldc, int lane,
-                                                 const float (&acc)[4][8], Op op) {
+                                                 const float (&acc)[H][8], Op op) {
     const int ti = lane >> 2, tj = lane & 3;
 #pragma unroll
-    for (int h = 0; h < 4; ++h)
+    for (int h = 0; h < H; ++h)
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
             float4* o = reinterpret_cast<float4*>(C + (ti + 8 * h) * ldc + 16 * half + 4 * tj);
@@ -342,32 +347,112 @@ __device__ __forceinline__ void block_tile_apply(float* C, int ldc, int lane,
         }
 }
 
-// the (bi, bj) block pair number q of the trailing lower blocks k+1 <= bj <= bi < 4
-__device__ __forceinline__ void trailing_pair(int k, int q, int& bi, int& bj) {
-    for (bj = k + 1; bj < pd::NSB; ++bj) {
-        const int n = pd::NSB - bj;
-        if (q < n) {
-            bi = bj + q;
-            return;
+// Block-product tasks of phases A(k) and C(k), one warp each, coded kind << 6 | i << 4 |
+// j << 2 | m:
+//   U  S_ij -= L_im L_jm^T   (trailing update with sub-panel m, its L_rm transposed in LT)
+//   W  X_ij += L_im X_mj     (inverse partial sum)
+//   F  X_ij = -X_ii X_ij     (inverse block final; also stored to Dinv)
+namespace pt {
+constexpr int U = 0, W = 1, F = 2;
+constexpr unsigned char T(int kind, int i, int j, int m) {
+    return static_cast<unsigned char>(kind << 6 | i << 4 | j << 2 | m);
+}
+}  // namespace pt
+__constant__ unsigned char c_tasks[26] = {
+    // C(0): block column 1 of sub-panel 0's update
+    pt::T(pt::U, 1, 1, 0), pt::T(pt::U, 2, 1, 0), pt::T(pt::U, 3, 1, 0),
+    // A(1): the rest of sub-panel 0's update; W_i0 += L_i0 X_00
+    pt::T(pt::U, 2, 2, 0), pt::T(pt::U, 3, 2, 0), pt::T(pt::U, 3, 3, 0),
+    pt::T(pt::W, 1, 0, 0), pt::T(pt::W, 2, 0, 0), pt::T(pt::W, 3, 0, 0),
+    // C(1): block column 2 of sub-panel 1's update; X_10
+    pt::T(pt::U, 2, 2, 1), pt::T(pt::U, 3, 2, 1), pt::T(pt::F, 1, 0, 0),
+    // A(2): the rest of sub-panel 1's update; W_i1 += L_i1 X_11, W_i0 += L_i1 X_10
+    pt::T(pt::U, 3, 3, 1), pt::T(pt::W, 2, 1, 1), pt::T(pt::W, 3, 1, 1),
+    pt::T(pt::W, 2, 0, 1), pt::T(pt::W, 3, 0, 1),
+    // C(2): block column 3 of sub-panel 2's update; X_20, X_21
+    pt::T(pt::U, 3, 3, 2), pt::T(pt::F, 2, 0, 0), pt::T(pt::F, 2, 1, 0),
+    // A(3): W_3j += L_32 X_2j
+    pt::T(pt::W, 3, 0, 2), pt::T(pt::W, 3, 1, 2), pt::T(pt::W, 3, 2, 2),
+    // C(3): X_30, X_31, X_32
+    pt::T(pt::F, 3, 0, 0), pt::T(pt::F, 3, 1, 0), pt::T(pt::F, 3, 2, 0)};
+// tasks of phase p (A(k) = 2k, C(k) = 2k + 1): c_tasks[c_task_off[p] .. c_task_off[p + 1])
+__constant__ unsigned char c_task_off[9] = {0, 0, 3, 9, 12, 17, 20, 23, 26};
+
+// Rows r0 + ti + 8h (h < H) of the 32 x 32 block (i, j) of X into Dinv, zero past the edge;
+// lane tile as in block_mma32
+template <int H>
+__device__ __forceinline__ void dinv_store_tile(float* Dinv, int i, int j, int r0, int nbc,
+                                                int lane, const float (&v)[H][8]) {
+    const int ti = lane >> 2, tj = lane & 3;
+#pragma unroll
+    for (int h = 0; h < H; ++h) {
+        const int r = pd::SB * i + r0 + ti + 8 * h;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            const int c = pd::SB * j + 16 * half + 4 * tj;
+            const bool ok = r < nbc;
+            *reinterpret_cast<float4*>(Dinv + r * pd::NB + c) = make_float4(
+                ok && c < nbc ? v[h][4 * half] : 0.f, ok && c + 1 < nbc ? v[h][4 * half + 1] : 0.f,
+                ok && c + 2 < nbc ? v[h][4 * half + 2] : 0.f,
+                ok && c + 3 < nbc ? v[h][4 * half + 3] : 0.f);
         }
-        q -= n;
     }
-    bi = bj = -1;
 }
 
-// inverse, round r: updates W_ij += L_im X_mj (m = j + r, i > m), listed as i | j << 2 | m << 4
-__constant__ unsigned char c_inv_upd[10] = {
-    1 | 0 << 2 | 0 << 4, 2 | 0 << 2 | 0 << 4, 3 | 0 << 2 | 0 << 4, 2 | 1 << 2 | 1 << 4,
-    3 | 1 << 2 | 1 << 4, 3 | 2 << 2 | 2 << 4,                                   // round 0
-    2 | 0 << 2 | 1 << 4, 3 | 0 << 2 | 1 << 4, 3 | 1 << 2 | 2 << 4,             // round 1
-    3 | 0 << 2 | 2 << 4};                                                       // round 2
+// Named barrier for the `count` threads (whole warps) of one task.
+__device__ __forceinline__ void bar_sync_named(int id, int count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
 
-__global__ void __launch_bounds__(pd::THREADS, 1) potrf_diag_kernel(float* __restrict__ A, int d,
-                                                                   int k0, int nbc,
+// One task of c_tasks, shared by 4 / H warps: this warp (part `part`) takes rows
+// 8 H part .. 8 H (part + 1) - 1 of the block. bar_id names the barrier of the task's warps
+// (an F task reads all of W_ij before any part of X_ij is written).
+template <int H>
+__device__ __forceinline__ void run_task(unsigned char t, float* S, float* X, const float* LT,
+                                         float* Dinv, int nbc, int lane, int part, int bar_id) {
+    const int kind = t >> 6, i = (t >> 4) & 3, j = (t >> 2) & 3, m = t & 3;
+    const int r0 = 8 * H * part;
+    float acc[H][8];
+    if (kind == pt::U) {
+        block_mma32<H>(S + (pd::SB * i + r0) * pd::LD + pd::SB * m, pd::LD,
+                       LT + (pd::SB * j - pd::SB * m - pd::SB), pd::LD, lane, acc);
+        block_tile_apply<H>(S + (pd::SB * i + r0) * pd::LD + pd::SB * j, pd::LD, lane, acc,
+                            [](float c, float a) { return c - a; });
+    } else if (kind == pt::W) {
+        block_mma32<H>(S + (pd::SB * i + r0) * pd::LD + pd::SB * m, pd::LD,
+                       X + (pd::SB * m) * pd::LD + pd::SB * j, pd::LD, lane, acc);
+        block_tile_apply<H>(X + (pd::SB * i + r0) * pd::LD + pd::SB * j, pd::LD, lane, acc,
+                            [](float c, float a) { return c + a; });
+    } else {
+        block_mma32<H>(X + (pd::SB * i + r0) * pd::LD + pd::SB * i, pd::LD,
+                       X + (pd::SB * i) * pd::LD + pd::SB * j, pd::LD, lane, acc);
+        if (H == 4) __syncwarp();         // every lane has read W_ij before it is overwritten
+        else bar_sync_named(bar_id, 32 * (4 / H));
+#pragma unroll
+        for (int h = 0; h < H; ++h)
+#pragma unroll
+            for (int q = 0; q < 8; ++q) acc[h][q] = -acc[h][q];
+        block_tile_apply<H>(X + (pd::SB * i + r0) * pd::LD + pd::SB * j, pd::LD, lane, acc,
+                            [](float, float a) { return a; });
+        dinv_store_tile<H>(Dinv, i, j, r0, nbc, lane, acc);
+    }
+}
+
+// The two task shapes, out of line (each phase runs one of them once per warp)
+__device__ __noinline__ void run_task_whole(unsigned char t, float* S, float* X, const float* LT,
+                                            float* Dinv, int nbc, int lane) {
+    run_task<4>(t, S, X, LT, Dinv, nbc, lane, 0, 0);
+}
+__device__ __noinline__ void run_task_quarter(unsigned char t, float* S, float* X,
+                                              const float* LT, float* Dinv, int nbc, int lane,
+                                              int part, int bar_id) {
+    run_task<1>(t, S, X, LT, Dinv, nbc, lane, part, bar_id);
+}
+
+__global__ void __launch_bounds__(pd::THREADS, 1) potrf_diag_kernel(const float* __restrict__ A,
+                                                                   int d, int k0, int nbc,
                                                                    float* __restrict__ Dinv,
-                                                                   int* status) {
-    pdl_wait();
-    if (status_bad(status)) return;
+                                                                   int* status, int stall) {
     extern __shared__ __align__(16) float sm[];
     float* S = sm;                            // [NB][LD]
     float* X = S + pd::NB * pd::LD;           // [NB][LD]
@@ -377,47 +462,67 @@ __global__ void __launch_bounds__(pd::THREADS, 1) potrf_diag_kernel(float* __res
     uint64_t* mb = reinterpret_cast<uint64_t*>(rinv + pd::SB);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-    // S = the block's lower triangle (rows below nbc: 16-byte async copies of the chunks that
-    // reach the lower triangle; rows from nbc on: the identity); X = 0
+    // Before the wait on the previous kernel (none of this reads what it writes): X = 0, the
+    // identity in S's rows from nbc on, zeros in S's chunks above the diagonal, and Dinv's six
+    // blocks above the block diagonal (zero)
     for (int e = tid; e < pd::NB * (pd::NB / 4); e += pd::THREADS) {
         const int r = e >> 5, c4 = (e & 31) * 4;
-        float* dst = S + r * pd::LD + c4;
-        if (r < nbc && c4 <= r) {
-            cp_async16(dst, A + static_cast<int64_t>(k0 + r) * d + k0 + c4);
-        } else {
+        if (r >= nbc || c4 > r) {
             const bool eye = r >= nbc && (r >> 2) == (c4 >> 2);
             const int u = r & 3;
-            *reinterpret_cast<float4*>(dst) =
+            *reinterpret_cast<float4*>(S + r * pd::LD + c4) =
                 make_float4(eye && u == 0 ? 1.f : 0.f, eye && u == 1 ? 1.f : 0.f,
                             eye && u == 2 ? 1.f : 0.f, eye && u == 3 ? 1.f : 0.f);
         }
         *reinterpret_cast<float4*>(X + r * pd::LD + c4) = make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    cp_async_commit();
+    for (int e = tid; e < 6 * pd::SB * (pd::SB / 4); e += pd::THREADS) {
+        const int blk = e >> 8, row = (e >> 3) & 31, c4 = (e & 7) * 4;
+        const int bi = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
+        const int bj = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
+        *reinterpret_cast<float4*>(Dinv + (pd::SB * bi + row) * pd::NB + pd::SB * bj + c4) =
+            make_float4(0.f, 0.f, 0.f, 0.f);
+    }
     if (tid == 0) {
         mbar_init(mb, 1);
         fence_mbar_init();
     }
+
+    pdl_wait();
+    // the block's lower triangle, rows below nbc: 16-byte async copies of the chunks that
+    // reach it
+    for (int e = tid; e < pd::NB * (pd::NB / 4); e += pd::THREADS) {
+        const int r = e >> 5, c4 = (e & 31) * 4;
+        if (r < nbc && c4 <= r)
+            cp_async16(S + r * pd::LD + c4, A + static_cast<int64_t>(k0 + r) * d + k0 + c4);
+    }
+    cp_async_commit();
+    const bool skip = status_bad(status);     // read while the copies are in flight
     cp_async_wait<0>();
-    __syncthreads();
+    if (__syncthreads_or(skip)) return;
     // the copied diagonal chunks also brought up to three entries above the diagonal
     if (tid < nbc)
         for (int c = tid + 1; c <= (tid | 3); ++c) S[tid * pd::LD + c] = 0.0f;
     __syncthreads();
-    if (*(volatile int*)&g_factor_stall) {
+    if (stall) {
         const bool ok = mbar_wait_cycles(mb, 0, pd::STALL_LIMIT_CYCLES);
         if (!ok && tid == 0) set_status(status, GPTQ_ERR_TIMEOUT);
         if (__syncthreads_or(!ok)) return;
     }
 
     bool bad = false;
-    float acc[4][8];
 #pragma unroll 1
     for (int k = 0; k < pd::NSB; ++k) {
         const int b = k * pd::SB;
-        if (warp == 0) bad = potrf32_warp(S, LkT, rinv, b, lane) || bad;
+        // A(k): the factor warp, and the block products that are ready
+        if (warp == 0) {
+            bad = potrf32_warp(S, LkT, rinv, b, lane) || bad;
+        } else {
+            const int t = c_task_off[2 * k] + warp - 1;
+            if (t < c_task_off[2 * k + 1]) run_task_whole(c_tasks[t], S, X, LT, Dinv, nbc, lane);
+        }
         __syncthreads();
-        // solve (warps 1 .. nrb, one row each lane) and I_kk (the next warp, one column each)
+        // B(k): solve (warps 1 .. nrb, one row each lane) and I_kk (the next warp)
         const int nrb = pd::NSB - 1 - k;
         float v[pd::SB];
         if (warp >= 1 && warp <= nrb) {
@@ -439,82 +544,30 @@ __global__ void __launch_bounds__(pd::THREADS, 1) potrf_diag_kernel(float* __res
 #pragma unroll
             for (int m = 0; m < pd::SB; ++m) v[m] = (m == lane) ? 1.0f : 0.0f;
             trsv32(v, LkT, rinv);
+            const bool colok = b + lane < nbc;
 #pragma unroll
-            for (int c = 0; c < pd::SB; ++c) X[(b + c) * pd::LD + b + lane] = v[c];
+            for (int c = 0; c < pd::SB; ++c) {
+                X[(b + c) * pd::LD + b + lane] = v[c];
+                Dinv[(b + c) * pd::NB + b + lane] = (colok && b + c < nbc) ? v[c] : 0.0f;
+            }
         }
         __syncthreads();
-        if (k + 1 == pd::NSB) break;
-        // update: A_ij -= L_ik L_jk^T over the trailing lower block pairs, one warp each
-        const int npairs = nrb * (nrb + 1) / 2;
-#pragma unroll 1
-        for (int q = warp; q < npairs; q += pd::NWARPS) {
-            int bi, bj;
-            trailing_pair(k, q, bi, bj);
-            block_mma32(S + (pd::SB * bi) * pd::LD + b, pd::LD,
-                        LT + (pd::SB * bj - b - pd::SB), pd::LD, lane, acc);
-            block_tile_apply(S + (pd::SB * bi) * pd::LD + pd::SB * bj, pd::LD, lane, acc,
-                             [](float c, float a) { return c - a; });
+        // C(k): block column k+1 of the update, and the inverse blocks I_kk completes; four
+        // warps per task (these products are on the chain)
+        {
+            const int t = c_task_off[2 * k + 1] + (warp >> 2);
+            if (t < c_task_off[2 * k + 2])
+                run_task_quarter(c_tasks[t], S, X, LT, Dinv, nbc, lane, warp & 3, 1 + (warp >> 2));
         }
         __syncthreads();
     }
     if (__syncthreads_or(bad) && tid == 0) set_status(status, GPTQ_ERR_NOT_PD);
-
-    // inverse: three rounds over the column blocks
-#pragma unroll 1
-    for (int r = 0, u0 = 0; r < pd::NSB - 1; ++r) {
-        const int nupd = (pd::NSB - 1 - r) * (pd::NSB - r) / 2;
-#pragma unroll 1
-        for (int q = warp; q < nupd; q += pd::NWARPS) {
-            const int t = c_inv_upd[u0 + q], i = t & 3, j = (t >> 2) & 3, m = t >> 4;
-            block_mma32(S + (pd::SB * i) * pd::LD + pd::SB * m, pd::LD,
-                        X + (pd::SB * m) * pd::LD + pd::SB * j, pd::LD, lane, acc);
-            block_tile_apply(X + (pd::SB * i) * pd::LD + pd::SB * j, pd::LD, lane, acc,
-                             [](float c, float a) { return c + a; });
-        }
-        u0 += nupd;
-        __syncthreads();
-        // X_ij = -I_ii W_ij for i = j + r + 1 (warp j)
-        const int nfin = pd::NSB - 1 - r;
-        const bool fin = warp < nfin;
-        const int j = warp, i = warp + r + 1;
-        if (fin)
-            block_mma32(X + (pd::SB * i) * pd::LD + pd::SB * i, pd::LD,
-                        X + (pd::SB * i) * pd::LD + pd::SB * j, pd::LD, lane, acc);
-        __syncthreads();                      // W_ij read before it is overwritten
-        if (fin)
-            block_tile_apply(X + (pd::SB * i) * pd::LD + pd::SB * j, pd::LD, lane, acc,
-                             [](float, float a) { return -a; });
-        __syncthreads();
-    }
-
-    // L back into A (lower triangle of the valid block; 16-byte stores below the diagonal
-    // chunk) and Dinv = X (zero past the edge)
-    for (int e = tid; e < pd::NB * (pd::NB / 4); e += pd::THREADS) {
-        const int m = e >> 5, c4 = (e & 31) * 4;
-        if (m >= nbc || c4 > m) continue;
-        float* dst = A + static_cast<int64_t>(k0 + m) * d + k0 + c4;
-        const float* src = S + m * pd::LD + c4;
-        if (c4 + 3 <= m) {
-            *reinterpret_cast<float4*>(dst) = *reinterpret_cast<const float4*>(src);
-        } else {
-            for (int c = 0; c <= m - c4; ++c) dst[c] = src[c];
-        }
-    }
-    for (int e = tid; e < pd::NB * (pd::NB / 4); e += pd::THREADS) {
-        const int c = e >> 5, i4 = (e & 31) * 4;
-        const float4 v = *reinterpret_cast<const float4*>(X + c * pd::LD + i4);
-        const bool rowok = c < nbc;
-        reinterpret_cast<float4*>(Dinv)[e] =
-            make_float4(rowok && i4 < nbc ? v.x : 0.f, rowok && i4 + 1 < nbc ? v.y : 0.f,
-                        rowok && i4 + 2 < nbc ? v.z : 0.f, rowok && i4 + 3 < nbc ? v.w : 0.f);
-    }
 }
 
 static int g_potrf_smem = 0;
 
 gptq_status factor_stall_set(int on) {
-    const int v = on ? 1 : 0;
-    GPTQ_CUDA_TRY(cudaMemcpyToSymbol(g_factor_stall, &v, sizeof(int)));
+    g_factor_stall = on ? 1 : 0;
     return GPTQ_OK;
 }
 
@@ -629,8 +682,9 @@ gptq_status factor_inverse_launch(float* A, int d, float* Dinv, float* X, float*
             const int reserve =
                 std::min(sms / GPTQ_FACTOR_RESERVE_DIV, std::max(1, (rem + nb - 1) / nb));
             const int side_ctas = std::max(1, sms - reserve);
-            GPTQ_CUDA_TRY(launch_pdl(potrf_diag_kernel, dim3(1), dim3(pd::THREADS), smem, s, A, d,
-                                     k0, nbc, Dm, status));
+            GPTQ_CUDA_TRY(launch_pdl(potrf_diag_kernel, dim3(1), dim3(pd::THREADS), smem, s,
+                                     static_cast<const float*>(A), d, k0, nbc, Dm, status,
+                                     g_factor_stall));
             GPTQ_LAUNCHED();
             if (rem > 0) {
                 TcGemmArgs t{};  // A21 = A21 * Dinv_m^T
@@ -716,7 +770,8 @@ gptq_status factor_inverse_launch(float* A, int d, float* Dinv, float* X, float*
                 float* Dm = Dinv + static_cast<int64_t>(m) * nb * nb;
                 float* A21 = A + static_cast<int64_t>(e) * d + k0;
                 GPTQ_CUDA_TRY(launch_pdl(potrf_diag_kernel, dim3(1), dim3(pd::THREADS), smem, s,
-                                         A, d, k0, nbc, Dm, status));
+                                         static_cast<const float*>(A), d, k0, nbc, Dm, status,
+                                         g_factor_stall));
                 GPTQ_LAUNCHED();
                 if (rem == 0) continue;
                 TcGemmArgs t{};  // A21 = A21 * Dinv_m^T
