@@ -399,8 +399,9 @@ unsigned long long gptq_launch_count(void);
  * mbarrier that nothing arrives at, with a limit of about 1 ms, so the next
  * gptq_quantize_layer / gptq_inverse_factor on the current device returns GPTQ_ERR_TIMEOUT;
  * the kernels after it skip their work on the status word and the CUDA context stays usable.
- * on = 0 restores normal operation. The switch is per device (current device) and process-wide;
- * it is for tests only. Errors: CUDA, UNSUPPORTED.
+ * on = 0 restores normal operation. The switch is process-wide (every device) and is read when
+ * a factorisation is enqueued; it is for tests only. Errors: CUDA, UNSUPPORTED (no usable
+ * device).
  * ------------------------------------------------------------------------------------------ */
 gptq_status gptq_test_stall_factor(int on);
 

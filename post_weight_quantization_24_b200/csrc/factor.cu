@@ -12,6 +12,7 @@
 // U^T U = H_d^-1 (the unique upper Cholesky factor of the inverse). The permutation and the
 // reversal are folded into one gather of H.
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 
 #include "internal.cuh"
@@ -222,7 +223,7 @@ constexpr long long STALL_LIMIT_CYCLES = 2000000;   // about 1 ms
 // nothing arrives at. The wait gives up after STALL_LIMIT_CYCLES, the kernel records
 // GPTQ_ERR_TIMEOUT and returns, and the rest of the factorisation skips its work on the status
 // word. No copy or MMA is in flight when it gives up.
-static int g_factor_stall = 0;
+static std::atomic<int> g_factor_stall{0};
 
 // 1/sqrt(x): the hardware estimate refined by one Newton-Raphson step r' = r (1 + (1 - x r^2)/2)
 __device__ __forceinline__ float rsqrt_nr(float x) {
@@ -567,7 +568,7 @@ __global__ void __launch_bounds__(pd::THREADS, 1) potrf_diag_kernel(const float*
 static int g_potrf_smem = 0;
 
 gptq_status factor_stall_set(int on) {
-    g_factor_stall = on ? 1 : 0;
+    g_factor_stall.store(on ? 1 : 0);
     return GPTQ_OK;
 }
 
@@ -684,7 +685,7 @@ gptq_status factor_inverse_launch(float* A, int d, float* Dinv, float* X, float*
             const int side_ctas = std::max(1, sms - reserve);
             GPTQ_CUDA_TRY(launch_pdl(potrf_diag_kernel, dim3(1), dim3(pd::THREADS), smem, s,
                                      static_cast<const float*>(A), d, k0, nbc, Dm, status,
-                                     g_factor_stall));
+                                     g_factor_stall.load()));
             GPTQ_LAUNCHED();
             if (rem > 0) {
                 TcGemmArgs t{};  // A21 = A21 * Dinv_m^T
@@ -771,7 +772,7 @@ gptq_status factor_inverse_launch(float* A, int d, float* Dinv, float* X, float*
                 float* A21 = A + static_cast<int64_t>(e) * d + k0;
                 GPTQ_CUDA_TRY(launch_pdl(potrf_diag_kernel, dim3(1), dim3(pd::THREADS), smem, s,
                                          static_cast<const float*>(A), d, k0, nbc, Dm, status,
-                                         g_factor_stall));
+                                         g_factor_stall.load()));
                 GPTQ_LAUNCHED();
                 if (rem == 0) continue;
                 TcGemmArgs t{};  // A21 = A21 * Dinv_m^T
