@@ -200,8 +200,8 @@ gptq_status gather_w_launch(const void* W, int w_dtype, int d_out, int d_in, con
 // of LkT (L_kk transposed, the exchange buffer), and applies the rank-1 update a_im -= L[i][c]
 // L[m][c] to its row. Lane c+1 computes the next pivot before the exchange, so the chain from
 // one pivot to the next is a reciprocal square root, two multiply-adds and one shuffle.
-// Each 32 x 32 block product is one warp's, on 4 x 8 register tiles (12 operand values per 32
-// multiply-adds: the products are bound by shared-memory bandwidth, not by the FMA pipe).
+// A 32 x 32 block product is one warp's (4 x 8 register tiles) in phase A, where it runs
+// beside the factor warp, and four warps' (8 rows each) in phase C, where it is on the chain.
 // Dinv is written block by block as blocks become final (the blocks above the diagonal, all
 // zero, first); L itself is not written back: nothing reads the diagonal block afterwards.
 // Rows and columns beyond the matrix edge are padded with the identity.
