@@ -485,26 +485,32 @@ def sequential_measure(gptq, device, peaks, n_blocks=2, n_tokens=65536, d=4096, 
         blocks.append((f(d_ff, d), f(d_ff, d), f(d, d_ff)))
     X0 = workloads.make_activations(workloads.WORKLOADS["mlp_up_7b"].replace(
         d_in=d, n_tokens=n_tokens, seed=78), device=device)
-    sequential.quantize_mlp_stack(X0, blocks[:1])            # warm-up (one block)
+    sequential.quantize_mlp_stack(X0, blocks)                # warm-up (the whole stack)
     torch.cuda.synchronize()
-    timings = {}
-    a, b = _events()
-    a.record()
-    _, recs = sequential.quantize_mlp_stack(X0, blocks, timings=timings)
-    b.record()
-    torch.cuda.synchronize()
-    ms = a.elapsed_time(b)
+    passes = []                                              # (ms, stage timings, records)
+    for _ in range(3):
+        timings = {}
+        a, b = _events()
+        a.record()
+        _, recs = sequential.quantize_mlp_stack(X0, blocks, timings=timings)
+        b.record()
+        torch.cuda.synchronize()
+        passes.append((a.elapsed_time(b), timings, recs))
+    passes.sort(key=lambda x: x[0])
+    ms, timings, recs = passes[1]                            # the median pass
     w4_flops = n_blocks * 2.0 * n_tokens * (2 * d_ff * d + d * d_ff)
     h_flops = n_blocks * float(n_tokens) * (d * (d + 1) + d_ff * (d_ff + 1))
     out = {"blocks": n_blocks, "tokens": n_tokens, "ms": ms,
+           "ms_passes": [x[0] for x in passes],
            "layers_per_s": 2 * n_blocks / (ms / 1e3),
            "weights_per_s": n_blocks * 3 * d * d_ff / (ms / 1e3),
            "stage_ms": timings,
            "w4a16_frac": w4_flops / (timings.get("w4a16", 1e-9) / 1e3) / 1e12 / peaks["bf16_tflops"],
            "hessian_frac": h_flops / (timings.get("hessian", 1e-9) / 1e3) / 1e12 / peaks["bf16_tflops"],
            "losses": {r["name"]: r["loss"] for r in recs},
-           "workload": f"{n_blocks} gated-MLP blocks d={d} d_ff={d_ff}, {n_tokens} tokens, INT4 g128"}
-    del blocks, X0, recs
+           "workload": f"{n_blocks} gated-MLP blocks d={d} d_ff={d_ff}, {n_tokens} tokens, INT4 g128",
+           "timing": "median of 3 passes after one untimed pass of the whole stack"}
+    del blocks, X0, recs, passes
     torch.cuda.empty_cache()
     return out
 
