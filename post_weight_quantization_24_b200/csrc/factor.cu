@@ -626,7 +626,7 @@ gptq_status side_streams(SideStreams** out) {
 // inverse X = L^-1, then U = reverse(X).
 //
 // Main stream, panel m (columns k0 .. e-1, e = k0 + nbc; rem = d - e rows below):
-//   diag(m)   L11 and its inverse Dinv_m (one CTA)
+//   diag(m)   Dinv_m = L11^-1 (one CTA factors the diagonal block; L11 itself is not kept)
 //   trsm(m)   L21 = A21 Dinv_m^T, in place (each output tile is the input tile it reads)
 //   next(m)   the trailing update of panel m+1's columns only: A[e:, e:e+128] -= L21 L21^T
 // Side stream, after trsm(m):
